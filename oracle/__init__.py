@@ -1,0 +1,9 @@
+"""fp64 CPU oracle for split-K sparse MLA decode -- test infrastructure only.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The CUDA library never uses it.
+"""
+from .oracle import DC, DR, PAGE_SIZE, build, combine, decode, max_threads, partial, set_threads
+
+__all__ = ["DC", "DR", "PAGE_SIZE", "build", "combine", "decode", "max_threads",
+           "partial", "set_threads"]
