@@ -1,0 +1,464 @@
+#!/usr/bin/env python
+"""Benchmark of split-K sparse MLA decode on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--nsplit S] [--impl ours|reference]
+
+One step = one whole decode (partial pass + LSE combine, through the C ABI)
+over one batch of the named synthetic workload, inputs resident in HBM.  L2
+is flushed before every step; each step is timed with CUDA events on the
+launching stream.  Rank 0 prints one JSON line.  Under torchrun every rank
+runs an independent replica (its own seed), so per-GPU work is fixed
+(weak scaling) and the step time is the max over ranks.
+
+The metric (query tokens per second, us per call and achieved HBM GB/s,
+against NSPLIT) follows "The Occupancy Hypothesis ..." (section "The
+Experiment": decode throughput measured against NSPLIT) and "The Moment of
+Truth ..." (section "The Split-K Imperative": the C=1 single-request case).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "sparse MLA decode query-tokens/s, µs/call and achieved HBM GB/s vs NSPLIT"
+UNIT = "query-tokens/s"
+DEFAULT_WORKLOAD = "single_request"
+L2_FLUSH_BYTES = 256 << 20
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawTextHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--nsplit", type=int, default=0, help="0 = the library's heuristic")
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-sweep", action="store_true", help="skip the NSPLIT sweep")
+    ap.add_argument("--cpu-seconds", type=float, default=6.0,
+                    help="time budget of the oracle CPU baseline sample")
+    return ap.parse_args(argv)
+
+
+# ----------------------------------------------------------------------------- workload facts
+def workload_bytes(w):
+    """Algorithmic bytes of one step.
+
+    partial pass, per query token: every valid selected row once (1152 B),
+    its page-table entry (4 B), the K index entries (4 B each) and q
+    (H * 1152 B); the combine adds o (H * 1024 B) and lse (H * 4 B).
+    """
+    valid = w.n_valid()
+    BT = w.B * w.T
+    partial = valid * (1152 + 4) + BT * w.K * 4 + BT * w.H * 1152
+    step = partial + BT * w.H * (1024 + 4)
+    return partial, step
+
+
+def workload_flops(w):
+    """2 * H * valid * (576 + 512): QK^T over 576 dims and PV over 512."""
+    return 2 * w.H * w.n_valid() * (576 + 512)
+
+
+def describe(w):
+    return (f"B{w.B} T{w.T} H{w.H} K{w.K} dc512+dr64 bf16, paged cache page64, "
+            f"{w.num_pages} pages, ctx {min(w.ctx_lens)}..{max(w.ctx_lens)}")
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    HW = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
+          "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
+
+    def __init__(self, device_index: int, period_s: float = 0.002):
+        self.period = period_s
+        self.samples = []
+        self.reasons = 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:  # NVML missing: no clock record
+            self._nv = None
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                self.reasons |= nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self._nv is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join()
+        if self._nv is not None and not self.samples:
+            try:
+                self.samples.append(self._nv.nvmlDeviceGetClockInfo(self._h, self._nv.NVML_CLOCK_SM))
+            except Exception:
+                pass
+
+    def summary(self):
+        if self._nv is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        names = [k for k, bit in self.HW.items() if self.reasons & bit]
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------------------- distributed
+def dist_init():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    dev = torch.device("cuda", torch.cuda.current_device()) if torch.cuda.is_available() else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    dev = torch.device("cuda", torch.cuda.current_device()) if torch.cuda.is_available() else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------- oracle baseline
+def cpu_baseline(w, budget_s: float):
+    """The fp64 oracle as it stands, on this host's cores, over whole steps of
+    the same workload (or the first query tokens of one step when a step alone
+    exceeds the budget)."""
+    import numpy as np
+    import oracle
+    bits = lambda t: t.contiguous().view(__import__("torch").int16).numpy().view(np.uint16)
+    q, cache = bits(w.q), bits(w.cache)
+    pt, idx = w.page_table.numpy(), w.idx.numpy()
+    threads = oracle.max_threads()
+    units = w.B * w.T * w.H
+    # one query token first, to size the sample
+    t0 = time.perf_counter()
+    oracle.decode(q[:1, :1], cache, pt[:1], idx[:1, :1], w.scale)
+    per_token = time.perf_counter() - t0
+    n_tok = max(1, min(w.B * w.T, int(budget_s / max(per_token, 1e-9))))
+    bt = [(b, t) for b in range(w.B) for t in range(w.T)][:n_tok]
+    reps = 0
+    t0 = time.perf_counter()
+    while True:
+        for b, t in bt:
+            oracle.decode(q[b:b + 1, t:t + 1], cache, pt[b:b + 1], idx[b:b + 1, t:t + 1], w.scale)
+        reps += 1
+        if time.perf_counter() - t0 >= budget_s * 0.5 or reps >= 50:
+            break
+    el = time.perf_counter() - t0
+    tokens = reps * len(bt)
+    sample = (f"{len(bt)} of {w.B * w.T} query tokens of one step (all {w.H} heads, "
+              f"K={w.K}) x {reps} repeats")
+    return {"value": tokens / el, "unit": UNIT, "cores": min(threads, w.H), "kind": "oracle",
+            "sample": sample, "threads_available": threads, "us_per_token": el / tokens * 1e6}
+
+
+# ----------------------------------------------------------------------------- GPU arm
+def run_ours(args, world, rank, local):
+    import torch
+    from sparse_mla_decode_partial_b200 import binding, build, workloads
+
+    build.build()
+    lib = binding.lib()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    builder = workloads.WORKLOADS[args.workload]
+    seed_kw = {}
+    if world > 1:
+        import inspect
+        base_seed = inspect.signature(builder).parameters["seed"].default
+        seed_kw = {"seed": base_seed + 1000 * rank}
+    w_host = builder(**seed_kw)
+    w = w_host.to(dev)
+    B, T, H, K = w.B, w.T, w.H, w.K
+    nsplit = args.nsplit or binding.choose_nsplit(B, T, H, K, 0)
+    stream = torch.cuda.current_stream(dev)
+    sptr = stream.cuda_stream
+
+    part_bytes, step_bytes = workload_bytes(w_host)
+    flops = workload_flops(w_host)
+    hbm_peak, tc_peak, peak_src = load_peaks()
+
+    flush_w = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    flush_r = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    sink = torch.empty(1, dtype=torch.float32, device=dev)
+
+    def flush():
+        flush_w.fill_(1.0)
+        torch.sum(flush_r, dim=0, out=sink[0])
+
+    def make_step(S):
+        n = B * T * H * S
+        po = torch.empty(max(n * 512, 4), dtype=torch.float32, device=dev)
+        pm = torch.empty(max(n, 1), dtype=torch.float32, device=dev)
+        pl = torch.empty(max(n, 1), dtype=torch.float32, device=dev)
+        o = torch.empty((B, T, H, 512), dtype=torch.bfloat16, device=dev)
+        lse = torch.empty((B, T, H), dtype=torch.float32, device=dev)
+        args_common = (w.q.data_ptr(), w.cache.data_ptr(), w.num_pages, w.page_table.data_ptr(),
+                       w.pt_stride, w.idx.data_ptr(), B, T, H, K, 64, w.scale)
+
+        def step(mid_event):
+            """One decode: partial pass, event, LSE combine (S = 1: one direct pass)."""
+            if S == 1:
+                st = lib.smla_decode(*args_common, 1, None, 0, o.data_ptr(), lse.data_ptr(), sptr)
+                mid_event.record(stream)
+                return st, 1
+            st = lib.smla_decode_partial(*args_common, S, po.data_ptr(), pm.data_ptr(),
+                                         pl.data_ptr(), sptr)
+            mid_event.record(stream)
+            st2 = lib.smla_lse_combine(po.data_ptr(), pm.data_ptr(), pl.data_ptr(), B, T, H, S,
+                                       o.data_ptr(), lse.data_ptr(), sptr)
+            return st or st2, 2
+        return step, (o, lse)
+
+    def timed(step, n):
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n)]
+        launches = 0
+        for i in range(n):
+            flush()
+            ev[i][0].record(stream)
+            st, nl = step(ev[i][1])
+            ev[i][2].record(stream)
+            if st != 0:
+                raise RuntimeError(binding.status_string(st))
+            launches += nl
+        torch.cuda.synchronize(dev)
+        tot = [e[0].elapsed_time(e[2]) for e in ev]
+        part = [e[0].elapsed_time(e[1]) for e in ev]
+        return tot, part, launches
+
+    step, _ = make_step(nsplit)
+    for _ in range(max(3, args.warmup)):
+        flush()
+        step(torch.cuda.Event())
+    torch.cuda.synchronize(dev)
+
+    sampler = ClockSampler(dev.index)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    with sampler:
+        tot, part, launches = timed(step, args.steps)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+
+    ms_step = statistics.fmean(tot)
+    ms_part = statistics.fmean(part)
+    ms_step_max = max_over_ranks(ms_step, world)
+    tokens_all = sum_over_ranks(float(B * T), world)
+    value = tokens_all / (ms_step_max * 1e-3)
+
+    # e2e: host buffers through the C ABI, copies inside the timed region
+    e2e = None
+    if True:
+        q_h = w_host.q.pin_memory()
+        idx_h = w_host.idx.pin_memory()
+        pt_h = w_host.page_table.pin_memory()
+        o_h = torch.empty((B, T, H, 512), dtype=torch.bfloat16).pin_memory()
+        lse_h = torch.empty((B, T, H), dtype=torch.float32).pin_memory()
+        q_d, idx_d, pt_d = torch.empty_like(w.q), torch.empty_like(w.idx), torch.empty_like(w.page_table)
+        o_d = torch.empty((B, T, H, 512), dtype=torch.bfloat16, device=dev)
+        lse_d = torch.empty((B, T, H), dtype=torch.float32, device=dev)
+        ws = torch.empty(max(16, binding.workspace_bytes(B, T, H, nsplit)), dtype=torch.uint8,
+                         device=dev)
+        h2d = q_h.numel() * 2 + idx_h.numel() * 4 + pt_h.numel() * 4
+        d2h = o_h.numel() * 2 + lse_h.numel() * 4
+
+        def e2e_step():
+            q_d.copy_(q_h, non_blocking=True)
+            idx_d.copy_(idx_h, non_blocking=True)
+            pt_d.copy_(pt_h, non_blocking=True)
+            st = lib.smla_decode(q_d.data_ptr(), w.cache.data_ptr(), w.num_pages, pt_d.data_ptr(),
+                                 w.pt_stride, idx_d.data_ptr(), B, T, H, K, 64, w.scale, nsplit,
+                                 ws.data_ptr(), ws.numel(), o_d.data_ptr(), lse_d.data_ptr(), sptr)
+            o_h.copy_(o_d, non_blocking=True)
+            lse_h.copy_(lse_d, non_blocking=True)
+            return st
+
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        n_e2e = max(10, min(args.steps, 200))
+        times = []
+        for _ in range(n_e2e):
+            flush()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            st = e2e_step()
+            e1.record(stream)
+            stream.synchronize()
+            if st != 0:
+                raise RuntimeError(binding.status_string(st))
+            times.append(e0.elapsed_time(e1))
+        e2e_ms = max_over_ranks(statistics.fmean(times), world)
+        e2e = {"value": tokens_all / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+               "note": "q, top-k indices and page table copied in from pinned host memory and "
+                       "o, lse copied out every step; the latent cache stays resident"}
+
+    # NSPLIT sweep (rank 0 only, after the timed region)
+    sweep = []
+    if rank == 0 and not args.no_sweep:
+        cands = list(w_host.nsplit_sweep) or sorted({1, 2, 4, 8, 16, 32, 64, nsplit})
+        for S in sorted(set(cands) | {nsplit}):
+            st_fn, _ = make_step(S)
+            for _ in range(5):
+                flush()
+                st_fn(torch.cuda.Event())
+            t, p_, _ = timed(st_fn, max(20, min(args.steps, 200)))
+            us = statistics.fmean(t) * 1e3
+            sweep.append({"nsplit": S, "us_per_call": round(us, 3),
+                          "partial_us": round(statistics.fmean(p_) * 1e3, 3),
+                          "q_tok_s": round(B * T / (us * 1e-6), 1),
+                          "hbm_gbs": round(step_bytes / (us * 1e-6) / 1e9, 1)})
+
+    if rank != 0:
+        return None
+
+    part_us = ms_part * 1e3
+    achieved = part_bytes / (part_us * 1e-6) / 1e9
+    tc_achieved = flops / (part_us * 1e-6) / 1e12
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step_max, 6),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1)*0.5 bf16 q and cache, distinct random top-k indices)",
+        "config": {"workload": args.workload, "shape": describe(w_host), "nsplit": nsplit,
+                   "nsplit_policy": "explicit" if args.nsplit else "heuristic",
+                   "batch": B, "q_len": T, "heads": H, "topk": K,
+                   "l2": "flushed before every step: 256 MB write then 256 MB read",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "us_per_call": round(ms_step_max * 1e3, 3),
+        "hbm_gbs_step": round(step_bytes / (ms_step * 1e-3) / 1e9, 1),
+        "kernel_us": {"partial": round(part_us, 3), "combine": round((ms_step - ms_part) * 1e3, 3)},
+        "roofline": {"bound": "hbm", "kernel": "smla_partial_mma_kernel", "achieved": round(achieved, 1),
+                     "peak": hbm_peak, "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),
+                     "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured" else "fallback",
+                     "traffic": None, "algorithmic_bytes_per_launch": part_bytes,
+                     "tensor_tflops": round(tc_achieved, 2),
+                     "tensor_frac_of_bf16_peak": round(tc_achieved / tc_peak, 4)},
+        "gpu_launches": launches,
+        "clocks": sampler.summary(),
+        "e2e": e2e,
+        "nsplit_sweep": sweep,
+    }
+    return line
+
+
+def run_reference(args, world, rank):
+    """The oracle (CPU, fp64) as the reference arm, on this host's cores."""
+    if rank != 0:
+        return None
+    from sparse_mla_decode_partial_b200 import workloads
+    w = workloads.WORKLOADS[args.workload]()
+    budget = max(2.0, args.cpu_seconds)
+    t_all = time.perf_counter()
+    res = cpu_baseline(w, budget)
+    value = res["value"]
+    nsplit = args.nsplit or None
+    return {
+        "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(w.B * w.T / value * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded N(0,1)*0.5 bf16 q and cache, distinct random top-k indices)",
+        "config": {"workload": args.workload, "shape": describe(w), "nsplit": nsplit,
+                   "batch": w.B, "q_len": w.T, "heads": w.H, "topk": w.K},
+        "impl": "reference",
+        "cpu_baseline": res,
+        "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "wall_s": round(time.perf_counter() - t_all, 2),
+    }
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    world, rank, local = dist_init()
+    if args.impl == "reference":
+        line = run_reference(args, world, rank)
+    else:
+        line = run_ours(args, world, rank, local)
+        if rank == 0 and line is not None:
+            from sparse_mla_decode_partial_b200 import workloads
+            line["cpu_baseline"] = cpu_baseline(workloads.WORKLOADS[args.workload](),
+                                                args.cpu_seconds)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0 and line is not None:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,181 @@
+/*
+ * smla.h -- C ABI of the split-K sparse MLA decode library (libsmla.so).
+ *
+ * The operation.  For every query token (b, t) and head h, attend over the
+ * top-k latent KV rows that idx[b, t, :] selects from a paged cache:
+ *
+ *   row r        = [ c_r (512 bf16) | k_pe_r (64 bf16) ]        (576 bf16, 1152 B)
+ *   q[b,t,h]     = [ q_nope (512 bf16) | q_pe (64 bf16) ]
+ *   s_j          = scale * ( q_nope . c_r + q_pe . k_pe_r )       r = row of idx[b,t,j]
+ *   o[b,t,h]     = sum_j softmax(s)_j * c_r                       (512 values)
+ *   lse[b,t,h]   = ln sum_j exp(s_j)
+ *
+ * Sources.  "The Moment of Truth: Validating Split-K Parallelization for
+ * Blackwell MLA Decode", section "The Split-K Imperative": the sparse MLA
+ * decode kernel attends over top-k candidate tokens retrieved from the KV
+ * cache; split-K partitions that top-k axis across thread blocks, each block
+ * computing a partial attention output, and a log-sum-exp combine kernel
+ * merges them.  "The Occupancy Hypothesis: How One Kernel Parameter Unlocked
+ * 1.8x Decode Speedup on Blackwell", sections "The Occupancy Insight" and
+ * "The Broader Context": NSPLIT multiplies the grid; its best value depends
+ * on SM count, heads, batch and query length.  The pages print no formula,
+ * dimension or index convention; the definition above is the standard
+ * absorbed-MLA decode reading, and the conventions below are this library's.
+ *
+ * Index convention.  idx holds logical token positions of sequence b.  A
+ * position i maps to physical cache row
+ *     page_table[b * pt_stride + i / 64] * 64 + i % 64.
+ * -1 is padding and contributes nothing.  Any other entry with i < 0,
+ * i >= pt_stride * 64, or whose page entry is outside [0, num_pages), is also
+ * treated as padding and counted in a device-side counter that
+ * smla_check_device() reports as SMLA_ERR_INDEX_RANGE.  Duplicate entries
+ * each count once.  A token with no valid entry gets o = 0, lse = -inf.
+ *
+ * Split convention.  With S = nsplit, Kc = ceil(K / S): split s covers index
+ * positions [s*Kc, min(K, (s+1)*Kc)).  Trailing splits may be short or empty.
+ *
+ * Common rules for every entry point:
+ *  - All pointers are DEVICE pointers on the current device, owned by the
+ *    caller.  The library allocates no device memory; it keeps only a small
+ *    host-side cache of per-device kernel attributes.
+ *  - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL is
+ *    the legacy default stream).  Arguments are checked on the host before
+ *    anything is launched; a failed check launches nothing.
+ *  - q, kv_cache, part_o, o and workspace must be 16-byte aligned; int32 and
+ *    fp32 arrays 4-byte aligned.  Otherwise SMLA_ERR_MISALIGNED.
+ *  - Dimensions are fixed at 512 + 64 and page_size must be 64; heads per
+ *    query token at most 64.  Otherwise SMLA_ERR_UNSUPPORTED.
+ *  - B, T, H or K equal to 0 are legal (K = 0: every o = 0, lse = -inf).
+ *  - A CUDA error at launch returns SMLA_ERR_CUDA; smla_last_error() gives
+ *    its text.  No entry point throws, aborts or exits.
+ *  - Entry points may be called from several host threads on different
+ *    streams at once.
+ */
+#ifndef SMLA_H_
+#define SMLA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define SMLA_DC 512        /* latent (value) width */
+#define SMLA_DR 64         /* shared RoPE key width */
+#define SMLA_D 576         /* cache row width in bf16 elements */
+#define SMLA_PAGE_SIZE 64  /* tokens per cache page */
+#define SMLA_MAX_HEADS 64
+#define SMLA_MAX_NSPLIT 1024
+
+typedef enum {
+    SMLA_OK = 0,
+    SMLA_ERR_INVALID_ARG = 1,
+    SMLA_ERR_UNSUPPORTED = 2,
+    SMLA_ERR_MISALIGNED = 3,
+    SMLA_ERR_WORKSPACE_TOO_SMALL = 4,
+    SMLA_ERR_INDEX_RANGE = 5,
+    SMLA_ERR_CUDA = 6,
+    SMLA_ERR_TIMEOUT = 7
+} smla_status;
+
+/*
+ * NSPLIT heuristic (host only, no CUDA call unless sm_count <= 0).
+ * "The Occupancy Hypothesis ...", section "The Broader Context": the right
+ * NSPLIT depends on SM count, heads per rank, batch size and query length;
+ * section "The Occupancy Insight": more blocks in flight hide memory latency.
+ * One CTA serves all heads of one (b, t, split), so the grid is B*T*NSPLIT
+ * CTAs.  The heuristic picks the NSPLIT in [1, min(SMLA_MAX_NSPLIT-bound, K/32)]
+ * that minimises a model of wave count x rows per CTA plus per-CTA overhead
+ * and the split-K scratch traffic.  sm_count <= 0 queries the current
+ * device.  If the environment variable SMLA_NSPLIT holds a positive integer,
+ * that value is returned instead (clamped to [1, SMLA_MAX_NSPLIT]).
+ * Returns >= 1; returns 1 for degenerate sizes.
+ */
+int smla_choose_nsplit(int B, int T, int H, int K, int sm_count);
+
+/*
+ * Bytes of workspace smla_decode needs for this shape and nsplit (>= 1):
+ * part_o, part_m and part_lse, each rounded up to 256 bytes.
+ * Returns 0 for invalid arguments.
+ */
+size_t smla_workspace_bytes(int B, int T, int H, int nsplit);
+
+/*
+ * Split-K partial pass ("The Split-K Imperative": each block computes a
+ * partial attention output over its chunk of the top-k axis).
+ *
+ *   q          bf16  [B, T, H, 576]                 device, 16-B aligned
+ *   kv_cache   bf16  [num_pages, 64, 576]           device, 16-B aligned
+ *   page_table int32 [B, pt_stride]                 device
+ *   topk_idx   int32 [B, T, K], -1 = padding        device
+ *   scale      softmax scale applied to the full 576-wide dot product
+ *   nsplit     S in [1, SMLA_MAX_NSPLIT]
+ * Outputs (fp32, device, caller-owned):
+ *   part_o   [B, T, H, S, 512]  sum_j exp(s_j - part_m) c_j   (unnormalised)
+ *   part_m   [B, T, H, S]       the reference point part_o is scaled by: the
+ *                               split's maximum score (-inf for a split with
+ *                               no valid entry)
+ *   part_lse [B, T, H, S]       ln sum_j exp(s_j) over the split (-inf if empty)
+ * so part_o * exp(part_m - part_lse) is the split's normalised output.
+ * An empty split writes part_o = 0, part_m = part_lse = -inf.
+ */
+smla_status smla_decode_partial(const void *q, const void *kv_cache, int64_t num_pages,
+                                const int32_t *page_table, int pt_stride,
+                                const int32_t *topk_idx, int B, int T, int H, int K,
+                                int page_size, float scale, int nsplit, float *part_o,
+                                float *part_m, float *part_lse, void *stream);
+
+/*
+ * LSE combine ("The Split-K Imperative": partial outputs merged by a
+ * log-sum-exp combine kernel).  Per (b, t, h):
+ *   M = max_s part_m,  L = sum_s exp(part_lse_s - M)
+ *   o = sum_s exp(part_m_s - M) part_o_s / L     -> bf16 [B, T, H, 512]
+ *   lse = M + ln L                               -> fp32 [B, T, H]
+ * All splits empty: o = 0, lse = -inf.  Inputs as written by
+ * smla_decode_partial with the same B, T, H, nsplit.
+ */
+smla_status smla_lse_combine(const float *part_o, const float *part_m, const float *part_lse,
+                             int B, int T, int H, int nsplit, void *o, float *lse,
+                             void *stream);
+
+/*
+ * Whole decode: partial pass then combine, on one stream.  nsplit = 0 picks
+ * smla_choose_nsplit(B, T, H, K, <current device SMs>).  The workspace holds
+ * the partials; it must be at least smla_workspace_bytes(B, T, H, S) for the
+ * S actually used (size it with the value smla_choose_nsplit returns), else
+ * SMLA_ERR_WORKSPACE_TOO_SMALL.  With S = 1 the partial pass writes o and
+ * lse directly and the workspace is not touched (it may then be NULL).
+ *   o   bf16 [B, T, H, 512] device, 16-B aligned
+ *   lse fp32 [B, T, H]      device
+ */
+smla_status smla_decode(const void *q, const void *kv_cache, int64_t num_pages,
+                        const int32_t *page_table, int pt_stride, const int32_t *topk_idx,
+                        int B, int T, int H, int K, int page_size, float scale, int nsplit,
+                        void *workspace, size_t workspace_bytes, void *o, float *lse,
+                        void *stream);
+
+/*
+ * Checked mode: synchronises `stream`, then reads the current device's
+ * sticky error state, optionally clearing it.  *n_bad_index (may be NULL)
+ * receives the number of out-of-range index entries seen since the last
+ * clear (each counted once per query token).  Returns SMLA_ERR_TIMEOUT if a
+ * kernel gave up a bounded wait, else SMLA_ERR_INDEX_RANGE if any entry was
+ * out of range, else SMLA_OK (or SMLA_ERR_CUDA).
+ */
+smla_status smla_check_device(int clear, unsigned long long *n_bad_index, void *stream);
+
+/* Static text for a status code. */
+const char *smla_status_string(smla_status status);
+
+/* Text of the last CUDA error seen by this host thread ("" if none). */
+const char *smla_last_error(void);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int smla_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SMLA_H_ */

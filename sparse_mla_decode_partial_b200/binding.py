@@ -1,0 +1,203 @@
+"""ctypes binding of libsmla.so (the C ABI in include/smla.h).
+
+Argument marshalling only: every step of the decode runs in the library's
+CUDA kernels.  torch tensors supply device memory and the current stream.
+If the library is missing, calls raise -- there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libsmla.so")
+
+DC, DR, D, PAGE_SIZE = 512, 64, 576, 64
+MAX_HEADS, MAX_NSPLIT = 64, 1024
+
+STATUS = {
+    0: "SMLA_OK", 1: "SMLA_ERR_INVALID_ARG", 2: "SMLA_ERR_UNSUPPORTED", 3: "SMLA_ERR_MISALIGNED",
+    4: "SMLA_ERR_WORKSPACE_TOO_SMALL", 5: "SMLA_ERR_INDEX_RANGE", 6: "SMLA_ERR_CUDA",
+    7: "SMLA_ERR_TIMEOUT",
+}
+
+# exported symbol -> (restype, argtypes)
+_P, _I, _I64, _F, _SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+SIGNATURES = {
+    "smla_choose_nsplit": (_I, [_I, _I, _I, _I, _I]),
+    "smla_workspace_bytes": (_SZ, [_I, _I, _I, _I]),
+    "smla_decode_partial": (_I, [_P, _P, _I64, _P, _I, _P, _I, _I, _I, _I, _I, _F, _I, _P, _P, _P,
+                                 _P]),
+    "smla_lse_combine": (_I, [_P, _P, _P, _I, _I, _I, _I, _P, _P, _P]),
+    "smla_decode": (_I, [_P, _P, _I64, _P, _I, _P, _I, _I, _I, _I, _I, _F, _I, _P, _SZ, _P, _P,
+                         _P]),
+    "smla_check_device": (_I, [_I, ctypes.POINTER(ctypes.c_ulonglong), _P]),
+    "smla_status_string": (ctypes.c_char_p, [_I]),
+    "smla_last_error": (ctypes.c_char_p, []),
+    "smla_version": (_I, []),
+}
+
+
+class SmlaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = f"{where}: {STATUS.get(status, status)}"
+        if status == 6:
+            msg += f" ({lib().smla_last_error().decode()})"
+        super().__init__(msg)
+
+
+_lib = None
+
+
+def lib():
+    """Load libsmla.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m sparse_mla_decode_partial_b200.build`")
+        handle = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(handle, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = handle
+    return _lib
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise SmlaError(status, where)
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else t.data_ptr()
+
+
+def _need(t, dtype, name, device=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if not t.is_cuda or (device is not None and t.device != device):
+        raise ValueError(f"{name} must be a CUDA tensor on {device}")
+
+
+def choose_nsplit(B: int, T: int, H: int, K: int, sm_count: int = 0) -> int:
+    return int(lib().smla_choose_nsplit(B, T, H, K, sm_count))
+
+
+def workspace_bytes(B: int, T: int, H: int, nsplit: int) -> int:
+    return int(lib().smla_workspace_bytes(B, T, H, nsplit))
+
+
+def _decode_args(q, cache, page_table, idx):
+    _need(q, torch.bfloat16, "q")
+    dev = q.device
+    _need(cache, torch.bfloat16, "cache", dev)
+    _need(page_table, torch.int32, "page_table", dev)
+    _need(idx, torch.int32, "idx", dev)
+    if q.dim() != 4 or q.shape[-1] != D:
+        raise ValueError(f"q must be [B,T,H,{D}]")
+    B, T, H, _ = q.shape
+    if idx.dim() != 3 or tuple(idx.shape[:2]) != (B, T):
+        raise ValueError("idx must be [B,T,K]")
+    if page_table.dim() != 2 or page_table.shape[0] != B:
+        raise ValueError("page_table must be [B, pt_stride]")
+    if cache.numel() % (PAGE_SIZE * D):
+        raise ValueError("cache must be [num_pages, 64, 576]")
+    num_pages = cache.numel() // (PAGE_SIZE * D)
+    return B, T, H, idx.shape[2], page_table.shape[1], num_pages
+
+
+def decode_partial(q, cache, page_table, idx, scale: float, nsplit: int, *, part_o=None,
+                   part_m=None, part_lse=None, stream=None):
+    """Partial pass; returns (part_o [B,T,H,S,512], part_m [B,T,H,S], part_lse [B,T,H,S])."""
+    B, T, H, K, pt_stride, num_pages = _decode_args(q, cache, page_table, idx)
+    dev = q.device
+    if part_o is None:
+        part_o = torch.empty((B, T, H, nsplit, DC), dtype=torch.float32, device=dev)
+    if part_m is None:
+        part_m = torch.empty((B, T, H, nsplit), dtype=torch.float32, device=dev)
+    if part_lse is None:
+        part_lse = torch.empty((B, T, H, nsplit), dtype=torch.float32, device=dev)
+    for t, n in ((part_o, "part_o"), (part_m, "part_m"), (part_lse, "part_lse")):
+        _need(t, torch.float32, n, dev)
+    _check(lib().smla_decode_partial(_ptr(q), _ptr(cache), num_pages, _ptr(page_table), pt_stride,
+                                     _ptr(idx), B, T, H, K, PAGE_SIZE, float(scale), int(nsplit),
+                                     _ptr(part_o), _ptr(part_m), _ptr(part_lse),
+                                     _stream(stream)), "smla_decode_partial")
+    return part_o, part_m, part_lse
+
+
+def lse_combine(part_o, part_m, part_lse, *, o=None, lse=None, stream=None):
+    """LSE combine; returns (o bf16 [B,T,H,512], lse fp32 [B,T,H])."""
+    _need(part_m, torch.float32, "part_m")
+    dev = part_m.device
+    _need(part_o, torch.float32, "part_o", dev)
+    _need(part_lse, torch.float32, "part_lse", dev)
+    if part_m.dim() != 4:
+        raise ValueError("part_m must be [B,T,H,S]")
+    B, T, H, S = part_m.shape
+    if tuple(part_o.shape) != (B, T, H, S, DC) or part_lse.shape != part_m.shape:
+        raise ValueError("partial shapes disagree")
+    if o is None:
+        o = torch.empty((B, T, H, DC), dtype=torch.bfloat16, device=dev)
+    if lse is None:
+        lse = torch.empty((B, T, H), dtype=torch.float32, device=dev)
+    _need(o, torch.bfloat16, "o", dev)
+    _need(lse, torch.float32, "lse", dev)
+    _check(lib().smla_lse_combine(_ptr(part_o), _ptr(part_m), _ptr(part_lse), B, T, H, S, _ptr(o),
+                                  _ptr(lse), _stream(stream)), "smla_lse_combine")
+    return o, lse
+
+
+def decode(q, cache, page_table, idx, scale: float, nsplit: int = 0, *, workspace=None,
+           o=None, lse=None, stream=None):
+    """Whole decode (partial + combine); returns (o bf16 [B,T,H,512], lse fp32 [B,T,H]).
+
+    nsplit = 0 uses the library's heuristic.  A workspace (uint8 CUDA tensor)
+    is allocated here when not given.
+    """
+    B, T, H, K, pt_stride, num_pages = _decode_args(q, cache, page_table, idx)
+    dev = q.device
+    if nsplit == 0:
+        nsplit = choose_nsplit(B, T, H, K, 0)
+    need = workspace_bytes(B, T, H, nsplit) if nsplit > 1 else 0
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    _need(workspace, torch.uint8, "workspace", dev)
+    if o is None:
+        o = torch.empty((B, T, H, DC), dtype=torch.bfloat16, device=dev)
+    if lse is None:
+        lse = torch.empty((B, T, H), dtype=torch.float32, device=dev)
+    _need(o, torch.bfloat16, "o", dev)
+    _need(lse, torch.float32, "lse", dev)
+    _check(lib().smla_decode(_ptr(q), _ptr(cache), num_pages, _ptr(page_table), pt_stride,
+                             _ptr(idx), B, T, H, K, PAGE_SIZE, float(scale), int(nsplit),
+                             _ptr(workspace), workspace.numel(), _ptr(o), _ptr(lse),
+                             _stream(stream)), "smla_decode")
+    return o, lse
+
+
+def check_device(clear: bool = True, stream=None):
+    """Synchronise and read the sticky device status: (status, n_bad_index)."""
+    n = ctypes.c_ulonglong(0)
+    st = lib().smla_check_device(1 if clear else 0, ctypes.byref(n), _stream(stream))
+    return int(st), int(n.value)
+
+
+def status_string(status: int) -> str:
+    return lib().smla_status_string(status).decode()

@@ -1,0 +1,298 @@
+// smla_api.cu -- host side of the C ABI declared in include/smla.h: argument
+// checks, the NSPLIT heuristic, workspace carving and kernel launches.
+// Every entry point returns a status; nothing throws across the ABI.
+#include <cuda_runtime.h>
+
+#include <climits>
+#include <cmath>
+#include <cstdint>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <set>
+#include <utility>
+
+#include "smla.h"
+#include "smla_combine.cuh"
+#include "smla_partial_mma.cuh"
+
+namespace {
+
+using smla::PartialParams;
+
+thread_local char g_last_error[256] = "";
+
+smla_status cuda_fail(cudaError_t e) {
+    std::snprintf(g_last_error, sizeof g_last_error, "%s: %s", cudaGetErrorName(e),
+                  cudaGetErrorString(e));
+    return SMLA_ERR_CUDA;
+}
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Per (device, kernel) one-time opt-in to large dynamic shared memory.
+cudaError_t ensure_smem_attr(const void *kernel, int bytes) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    static std::mutex mu;
+    static std::set<std::pair<int, const void *>> done;
+    std::lock_guard<std::mutex> lock(mu);
+    const auto key = std::make_pair(dev, kernel);
+    if (done.count(key)) return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) done.insert(key);
+    return e;
+}
+
+int current_device_sms() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+        return 148;
+    return n;
+}
+
+// NSPLIT model ("The Occupancy Hypothesis ...", sections "The Occupancy
+// Insight" and "The Broader Context": more blocks in flight hide memory
+// latency, and the best NSPLIT depends on SMs, heads, batch and query
+// length).  Cost in units of "one CTA gathering one 1152-B row at its share
+// of HBM bandwidth":
+//     waves(S) * (kFixedRows + ceil(K / S))     wave-quantised gather time
+//   + scratch(S)                                partials written, re-read
+// S is capped so that every split keeps at least kMinRowsPerSplit rows.
+constexpr double kFixedRows = 48.0;     // per-CTA latency: launch, Q load, index chase
+constexpr double kScratchWeight = 0.5;  // partials mostly stay in L2
+constexpr int kMinRowsPerSplit = 32;
+constexpr double kPartialBytesPerHead = (smla::kDc + 2) * 4.0;
+
+int nsplit_model(int B, int T, int H, int K, int sm_count) {
+    const long long base = (long long)B * T;
+    int s_max = (K + kMinRowsPerSplit - 1) / kMinRowsPerSplit;
+    if (s_max < 1) s_max = 1;
+    if (s_max > SMLA_MAX_NSPLIT) s_max = SMLA_MAX_NSPLIT;
+    while (s_max > 1 && base * s_max > INT_MAX) --s_max;
+    const double slots = (double)sm_count;  // one partial CTA per SM (shared-memory bound)
+    double best = 0.0;
+    int best_s = 1;
+    for (int s = 1; s <= s_max; ++s) {
+        const double ctas = (double)base * s;
+        const double waves = std::ceil(ctas / slots);
+        const double rows = std::ceil((double)K / s);
+        double t = waves * (kFixedRows + rows);
+        if (s > 1) t += kScratchWeight * ctas * H * kPartialBytesPerHead * 2.0 / smla::kRowBytes / slots;
+        if (s == 1 || t < best * (1.0 - 1e-9)) {
+            best = t;
+            best_s = s;
+        }
+    }
+    return best_s;
+}
+
+smla_status check_decode_args(const void *q, const void *kv_cache, int64_t num_pages,
+                              const int32_t *page_table, int pt_stride, const int32_t *idx,
+                              int B, int T, int H, int K, int page_size, float scale) {
+    if (B < 0 || T < 0 || H < 0 || K < 0) return SMLA_ERR_INVALID_ARG;
+    if (page_size != SMLA_PAGE_SIZE) return SMLA_ERR_UNSUPPORTED;
+    if (H > SMLA_MAX_HEADS) return SMLA_ERR_UNSUPPORTED;
+    if (!std::isfinite(scale)) return SMLA_ERR_INVALID_ARG;
+    if (B == 0 || T == 0 || H == 0) return SMLA_OK;
+    if (q == nullptr) return SMLA_ERR_INVALID_ARG;
+    if (!aligned(q, 16)) return SMLA_ERR_MISALIGNED;
+    if (K > 0) {
+        if (kv_cache == nullptr || page_table == nullptr || idx == nullptr) return SMLA_ERR_INVALID_ARG;
+        if (num_pages < 1 || pt_stride < 1) return SMLA_ERR_INVALID_ARG;
+        if (num_pages > (int64_t)1 << 40) return SMLA_ERR_INVALID_ARG;
+        if (!aligned(kv_cache, 16) || !aligned(page_table, 4) || !aligned(idx, 4))
+            return SMLA_ERR_MISALIGNED;
+    }
+    if ((long long)B * T * H > INT_MAX) return SMLA_ERR_INVALID_ARG;
+    return SMLA_OK;
+}
+
+template <int HG, int NT, int NS, bool DIRECT>
+smla_status launch_mma(const PartialParams &p, int grid, cudaStream_t st) {
+    using C = smla::MmaCfg<HG, NT, NS>;
+    const void *fn = reinterpret_cast<const void *>(&smla::smla_partial_mma_kernel<HG, NT, NS, DIRECT>);
+    cudaError_t e = ensure_smem_attr(fn, C::kSmemBytes);
+    if (e != cudaSuccess) return cuda_fail(e);
+    smla::smla_partial_mma_kernel<HG, NT, NS, DIRECT><<<grid, C::kThreads, C::kSmemBytes, st>>>(p);
+    e = cudaGetLastError();
+    return e == cudaSuccess ? SMLA_OK : cuda_fail(e);
+}
+
+template <bool DIRECT>
+smla_status launch_partial(const PartialParams &p, cudaStream_t st) {
+    const long long grid = (long long)p.B * p.T * p.nsplit;
+    if (grid > INT_MAX) return SMLA_ERR_INVALID_ARG;
+    switch ((p.H + 15) / 16) {
+        case 1: return launch_mma<1, 32, 4, DIRECT>(p, (int)grid, st);
+        case 2: return launch_mma<2, 32, 4, DIRECT>(p, (int)grid, st);
+        case 3: return launch_mma<3, 32, 4, DIRECT>(p, (int)grid, st);
+        case 4: return launch_mma<4, 32, 4, DIRECT>(p, (int)grid, st);
+        default: return SMLA_ERR_UNSUPPORTED;
+    }
+}
+
+PartialParams make_params(const void *q, const void *kv_cache, int64_t num_pages,
+                          const int32_t *page_table, int pt_stride, const int32_t *idx, int B,
+                          int T, int H, int K, float scale, int nsplit) {
+    PartialParams p{};
+    p.q = static_cast<const __nv_bfloat16 *>(q);
+    p.cache = static_cast<const __nv_bfloat16 *>(kv_cache);
+    p.num_pages = num_pages;
+    p.page_table = page_table;
+    p.pt_stride = pt_stride;
+    p.idx = idx;
+    p.B = B;
+    p.T = T;
+    p.H = H;
+    p.K = K;
+    p.scale_log2 = scale * smla::kLog2e;
+    p.nsplit = nsplit;
+    p.kc = (K + nsplit - 1) / nsplit;
+    return p;
+}
+
+smla_status launch_combine(const float *part_o, const float *part_m, const float *part_lse, int B,
+                           int T, int H, int nsplit, void *o, float *lse, cudaStream_t st) {
+    const long long units = (long long)B * T * H;
+    if (units == 0) return SMLA_OK;
+    if (units > INT_MAX) return SMLA_ERR_INVALID_ARG;
+    smla::smla_combine_kernel<<<(int)units, smla::kCombineThreads, nsplit * sizeof(float), st>>>(
+        part_o, part_m, part_lse, nsplit, static_cast<__nv_bfloat16 *>(o), lse);
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? SMLA_OK : cuda_fail(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+int smla_version(void) { return 100; }
+
+const char *smla_last_error(void) { return g_last_error; }
+
+const char *smla_status_string(smla_status status) {
+    switch (status) {
+        case SMLA_OK: return "SMLA_OK";
+        case SMLA_ERR_INVALID_ARG: return "SMLA_ERR_INVALID_ARG: invalid argument";
+        case SMLA_ERR_UNSUPPORTED: return "SMLA_ERR_UNSUPPORTED: unsupported shape or page size";
+        case SMLA_ERR_MISALIGNED: return "SMLA_ERR_MISALIGNED: pointer alignment";
+        case SMLA_ERR_WORKSPACE_TOO_SMALL: return "SMLA_ERR_WORKSPACE_TOO_SMALL: workspace too small";
+        case SMLA_ERR_INDEX_RANGE: return "SMLA_ERR_INDEX_RANGE: index entry out of range";
+        case SMLA_ERR_CUDA: return "SMLA_ERR_CUDA: CUDA error (see smla_last_error)";
+        case SMLA_ERR_TIMEOUT: return "SMLA_ERR_TIMEOUT: a kernel wait timed out";
+    }
+    return "unknown smla_status";
+}
+
+int smla_choose_nsplit(int B, int T, int H, int K, int sm_count) {
+    if (const char *env = std::getenv("SMLA_NSPLIT")) {
+        char *end = nullptr;
+        const long v = std::strtol(env, &end, 10);
+        if (end != env && v > 0) return (int)(v > SMLA_MAX_NSPLIT ? SMLA_MAX_NSPLIT : v);
+    }
+    if (B <= 0 || T <= 0 || H <= 0 || K <= 0) return 1;
+    if (sm_count <= 0) sm_count = current_device_sms();
+    return nsplit_model(B, T, H, K, sm_count);
+}
+
+size_t smla_workspace_bytes(int B, int T, int H, int nsplit) {
+    if (B < 0 || T < 0 || H < 0 || nsplit < 1 || nsplit > SMLA_MAX_NSPLIT) return 0;
+    const size_t n = (size_t)B * T * H * nsplit;
+    return round256(n * smla::kDc * sizeof(float)) + 2 * round256(n * sizeof(float));
+}
+
+smla_status smla_decode_partial(const void *q, const void *kv_cache, int64_t num_pages,
+                                const int32_t *page_table, int pt_stride, const int32_t *topk_idx,
+                                int B, int T, int H, int K, int page_size, float scale, int nsplit,
+                                float *part_o, float *part_m, float *part_lse, void *stream) {
+    smla_status st = check_decode_args(q, kv_cache, num_pages, page_table, pt_stride, topk_idx, B,
+                                       T, H, K, page_size, scale);
+    if (st != SMLA_OK) return st;
+    if (nsplit < 1 || nsplit > SMLA_MAX_NSPLIT) return SMLA_ERR_INVALID_ARG;
+    if (B == 0 || T == 0 || H == 0) return SMLA_OK;
+    if (part_o == nullptr || part_m == nullptr || part_lse == nullptr) return SMLA_ERR_INVALID_ARG;
+    if (!aligned(part_o, 16) || !aligned(part_m, 4) || !aligned(part_lse, 4))
+        return SMLA_ERR_MISALIGNED;
+    PartialParams p = make_params(q, kv_cache, num_pages, page_table, pt_stride, topk_idx, B, T, H,
+                                  K, scale, nsplit);
+    p.part_o = part_o;
+    p.part_m = part_m;
+    p.part_lse = part_lse;
+    return launch_partial<false>(p, static_cast<cudaStream_t>(stream));
+}
+
+smla_status smla_lse_combine(const float *part_o, const float *part_m, const float *part_lse,
+                             int B, int T, int H, int nsplit, void *o, float *lse, void *stream) {
+    if (B < 0 || T < 0 || H < 0) return SMLA_ERR_INVALID_ARG;
+    if (nsplit < 1 || nsplit > SMLA_MAX_NSPLIT) return SMLA_ERR_INVALID_ARG;
+    if (B == 0 || T == 0 || H == 0) return SMLA_OK;
+    if (!part_o || !part_m || !part_lse || !o || !lse) return SMLA_ERR_INVALID_ARG;
+    if (!aligned(part_o, 16) || !aligned(part_m, 4) || !aligned(part_lse, 4) || !aligned(o, 16) ||
+        !aligned(lse, 4))
+        return SMLA_ERR_MISALIGNED;
+    return launch_combine(part_o, part_m, part_lse, B, T, H, nsplit, o, lse,
+                          static_cast<cudaStream_t>(stream));
+}
+
+smla_status smla_decode(const void *q, const void *kv_cache, int64_t num_pages,
+                        const int32_t *page_table, int pt_stride, const int32_t *topk_idx, int B,
+                        int T, int H, int K, int page_size, float scale, int nsplit,
+                        void *workspace, size_t workspace_bytes, void *o, float *lse,
+                        void *stream) {
+    smla_status st = check_decode_args(q, kv_cache, num_pages, page_table, pt_stride, topk_idx, B,
+                                       T, H, K, page_size, scale);
+    if (st != SMLA_OK) return st;
+    if (nsplit < 0 || nsplit > SMLA_MAX_NSPLIT) return SMLA_ERR_INVALID_ARG;
+    if (B == 0 || T == 0 || H == 0) return SMLA_OK;
+    if (o == nullptr || lse == nullptr) return SMLA_ERR_INVALID_ARG;
+    if (!aligned(o, 16) || !aligned(lse, 4)) return SMLA_ERR_MISALIGNED;
+    if (nsplit == 0) nsplit = smla_choose_nsplit(B, T, H, K, 0);
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    PartialParams p = make_params(q, kv_cache, num_pages, page_table, pt_stride, topk_idx, B, T, H,
+                                  K, scale, nsplit);
+    if (nsplit == 1) {
+        p.o = static_cast<__nv_bfloat16 *>(o);
+        p.lse = lse;
+        return launch_partial<true>(p, s);
+    }
+    if (workspace_bytes < smla_workspace_bytes(B, T, H, nsplit)) return SMLA_ERR_WORKSPACE_TOO_SMALL;
+    if (workspace == nullptr) return SMLA_ERR_INVALID_ARG;
+    if (!aligned(workspace, 16)) return SMLA_ERR_MISALIGNED;
+    const size_t n = (size_t)B * T * H * nsplit;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    p.part_o = reinterpret_cast<float *>(ws);
+    p.part_m = reinterpret_cast<float *>(ws + round256(n * smla::kDc * sizeof(float)));
+    p.part_lse = reinterpret_cast<float *>(ws + round256(n * smla::kDc * sizeof(float)) +
+                                           round256(n * sizeof(float)));
+    st = launch_partial<false>(p, s);
+    if (st != SMLA_OK) return st;
+    return launch_combine(p.part_o, p.part_m, p.part_lse, B, T, H, nsplit, o, lse, s);
+}
+
+smla_status smla_check_device(int clear, unsigned long long *n_bad_index, void *stream) {
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e);
+    unsigned int flags = 0;
+    unsigned long long count = 0;
+    e = cudaMemcpyFromSymbol(&flags, smla::g_status_flags, sizeof flags);
+    if (e == cudaSuccess) e = cudaMemcpyFromSymbol(&count, smla::g_bad_index_count, sizeof count);
+    if (e == cudaSuccess && clear) {
+        const unsigned int zf = 0;
+        const unsigned long long zc = 0;
+        e = cudaMemcpyToSymbol(smla::g_status_flags, &zf, sizeof zf);
+        if (e == cudaSuccess) e = cudaMemcpyToSymbol(smla::g_bad_index_count, &zc, sizeof zc);
+    }
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (n_bad_index) *n_bad_index = count;
+    if (flags & smla::kFlagTimeout) return SMLA_ERR_TIMEOUT;
+    if (flags & smla::kFlagIndexRange) return SMLA_ERR_INDEX_RANGE;
+    return SMLA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,252 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle.
+
+Every case feeds the same seeded inputs to both sides.  Tolerances are the
+problem statement's: o max-abs <= 1e-2 and relative L2 <= 5e-3, lse <= 1e-3
+(see parity_util).  Small cases compare every output; the full-size batched
+and mixed-length workloads, run in the launch configuration the benchmark
+times (heuristic NSPLIT), compare sampled query tokens.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from parity_util import (bits, check_o_lse, normalised_partials, oracle_decode, sample_bt)
+from sparse_mla_decode_partial_b200 import binding, build, workloads
+
+pytestmark = pytest.mark.gpu
+
+DEV = torch.device("cuda:0")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    build.build()
+    binding.lib()
+    binding.check_device(clear=True)
+    yield
+    st, n = binding.check_device(clear=True)
+    assert st in (0, 5), binding.status_string(st)
+
+
+def run_decode(w, nsplit, **kw):
+    wd = w.to(DEV)
+    o, lse = binding.decode(wd.q, wd.cache, wd.page_table, wd.idx, w.scale, nsplit, **kw)
+    torch.cuda.synchronize()
+    return o, lse
+
+
+def small(name="s", seed=5, B=2, T=2, H=16, K=300, ctx=2000, **kw):
+    return workloads.make_workload(name, B=B, T=T, H=H, K=K, ctx_lens=[ctx] * B, seed=seed, **kw)
+
+
+# ------------------------------------------------------------------ the five configurations
+@pytest.mark.parametrize("nsplit", [4, 1, 0])
+def test_tiny(nsplit):
+    w = workloads.tiny()
+    o, lse = run_decode(w, nsplit)
+    o_ref, lse_ref, _ = oracle_decode(w)
+    check_o_lse(o, lse, o_ref, lse_ref, f"tiny S={nsplit}")
+
+
+@pytest.fixture(scope="module")
+def single_request():
+    return workloads.single_request()
+
+
+@pytest.mark.parametrize("nsplit", [1, 4, 16, 32, 64, 0])
+def test_single_request_nsplit_sweep(single_request, nsplit):
+    w = single_request
+    o, lse = run_decode(w, nsplit)
+    o_ref, lse_ref, _ = oracle_decode(w)
+    check_o_lse(o, lse, o_ref, lse_ref, f"single_request S={nsplit}")
+
+
+@pytest.mark.parametrize("nsplit", [16, 64, 0])
+def test_spec_verify(nsplit):
+    w = workloads.spec_verify()
+    o, lse = run_decode(w, nsplit)
+    o_ref, lse_ref, _ = oracle_decode(w)
+    check_o_lse(o, lse, o_ref, lse_ref, f"spec_verify S={nsplit}")
+
+
+def test_batched_full_size_sampled():
+    w = workloads.batched()
+    o, lse = run_decode(w, 0)
+    sample = sample_bt(w, 10, seed=1)
+    o_ref, lse_ref, _ = oracle_decode(w, sample)
+    bi = [b for b, _ in sample]
+    ti = [t for _, t in sample]
+    check_o_lse(o[bi, ti], lse[bi, ti], o_ref, lse_ref, "batched sampled")
+    assert torch.isfinite(o.float()).all() and torch.isfinite(lse).all()
+
+
+def test_mixed_full_size_sampled():
+    w = workloads.mixed()
+    o, lse = run_decode(w, 0)
+    short = [b for b, c in enumerate(w.ctx_lens) if c < 2048][:3]
+    sample = sorted(set([(b, 0) for b in short] + sample_bt(w, 5, seed=2)))
+    o_ref, lse_ref, _ = oracle_decode(w, sample)
+    bi = [b for b, _ in sample]
+    ti = [t for _, t in sample]
+    check_o_lse(o[bi, ti], lse[bi, ti], o_ref, lse_ref, "mixed sampled")
+    assert torch.isfinite(o.float()).all() and torch.isfinite(lse).all()
+
+
+def test_batched_reduced_full_compare():
+    w = workloads.batched(B=6)
+    for nsplit in (0, 2, 8):
+        o, lse = run_decode(w, nsplit)
+        o_ref, lse_ref, _ = oracle_decode(w)
+        check_o_lse(o, lse, o_ref, lse_ref, f"batched B=6 S={nsplit}")
+
+
+def test_mixed_reduced_full_compare():
+    w = workloads.mixed(B=5)
+    for nsplit in (0, 3, 8):
+        o, lse = run_decode(w, nsplit)
+        o_ref, lse_ref, _ = oracle_decode(w)
+        check_o_lse(o, lse, o_ref, lse_ref, f"mixed B=5 S={nsplit}")
+
+
+# ------------------------------------------------------------------ the two passes separately
+@pytest.mark.parametrize("H", [8, 16, 64])
+def test_partial_pass_against_oracle_partials(H):
+    w = small(H=H, K=200, B=1, T=2)
+    w.idx[0, 1, 64:128] = -1          # one whole split (Kc = 50) of padding and more
+    nsplit = 4
+    wd = w.to(DEV)
+    po, pm, pl = binding.decode_partial(wd.q, wd.cache, wd.page_table, wd.idx, w.scale, nsplit)
+    torch.cuda.synchronize()
+    rpo, rpm, rpl, _ = oracle.partial(bits(w.q), bits(w.cache), w.page_table.numpy(),
+                                      w.idx.numpy(), w.scale, nsplit)
+    got = normalised_partials(po.cpu().numpy(), pm.cpu().numpy(), pl.cpu().numpy())
+    ref = normalised_partials(rpo, rpm, rpl)
+    assert np.abs(got - ref).max() <= 1e-2
+    assert np.linalg.norm(got - ref) / np.linalg.norm(ref) <= 5e-3
+    plg = pl.cpu().numpy()
+    assert np.array_equal(np.isneginf(plg), np.isneginf(rpl))
+    fin = ~np.isneginf(rpl)
+    assert np.abs(plg[fin] - rpl[fin]).max() <= 1e-3
+
+
+def test_combine_pass_against_oracle_combine():
+    w = small(H=16, K=256, B=2, T=1)
+    w.idx[1, 0, 100:] = -1
+    nsplit = 8
+    rpo, rpm, rpl, _ = oracle.partial(bits(w.q), bits(w.cache), w.page_table.numpy(),
+                                      w.idx.numpy(), w.scale, nsplit)
+    o_ref, lse_ref = oracle.combine(rpo, rpm, rpl)
+    t = lambda a: torch.tensor(a, dtype=torch.float32, device=DEV).contiguous()
+    o, lse = binding.lse_combine(t(rpo), t(rpm), t(rpl))
+    torch.cuda.synchronize()
+    check_o_lse(o, lse, o_ref, lse_ref, "combine")
+
+
+# ------------------------------------------------------------------ edge cases
+@pytest.mark.parametrize("H", [1, 5, 16, 17, 33, 48, 64])
+@pytest.mark.parametrize("K", [1, 31, 33, 100])
+def test_ragged_heads_and_topk(H, K):
+    w = small(H=H, K=K, B=2, T=1, ctx=500, seed=H * 131 + K)
+    for nsplit in (1, 3, K + 3):
+        o, lse = run_decode(w, nsplit)
+        o_ref, lse_ref, _ = oracle_decode(w)
+        check_o_lse(o, lse, o_ref, lse_ref, f"H={H} K={K} S={nsplit}")
+
+
+@pytest.mark.parametrize("pattern", ["trailing", "interleaved", "whole_split", "all", "leading"])
+def test_padding_placements(pattern):
+    w = small(H=16, K=256, B=2, T=2, seed=9)
+    if pattern == "trailing":
+        w.idx[:, :, 200:] = -1
+    elif pattern == "interleaved":
+        w.idx[:, :, ::3] = -1
+    elif pattern == "whole_split":
+        w.idx[:, :, 64:128] = -1      # S = 4 -> split 1 is entirely padding
+    elif pattern == "leading":
+        w.idx[:, :, :130] = -1
+    else:
+        w.idx[0, 1, :] = -1
+        w.idx[1, 0, :] = -1
+    for nsplit in (1, 4, 7):
+        o, lse = run_decode(w, nsplit)
+        o_ref, lse_ref, _ = oracle_decode(w)
+        check_o_lse(o, lse, o_ref, lse_ref, f"{pattern} S={nsplit}")
+    if pattern == "all":
+        assert torch.all(o[0, 1] == 0) and torch.all(torch.isneginf(lse[0, 1]))
+
+
+def test_empty_topk():
+    w = small(H=16, K=0, B=2, T=1)
+    o, lse = run_decode(w, 1)
+    assert torch.all(o == 0) and torch.all(torch.isneginf(lse))
+
+
+def test_out_of_range_entries_masked_and_counted():
+    w = small(H=16, K=128, B=1, T=1)
+    w.idx[0, 0, 3] = -5
+    w.idx[0, 0, 10] = w.pt_stride * 64 + 1
+    w.page_table[0, 0] = 10 ** 6                      # every index on logical page 0 goes bad
+    n_page0 = int(((w.idx[0, 0] >= 0) & (w.idx[0, 0] < 64)).sum())
+    binding.check_device(clear=True)
+    o, lse = run_decode(w, 4)
+    st, n = binding.check_device(clear=True)
+    o_ref, lse_ref, bad = oracle_decode(w)
+    check_o_lse(o, lse, o_ref, lse_ref, "out of range")
+    assert st == 5, binding.status_string(st)
+    assert n == 2 + n_page0 == bad // w.H
+
+
+def test_deterministic():
+    w = workloads.single_request()
+    o1, l1 = run_decode(w, 16)
+    o2, l2 = run_decode(w, 16)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_output_guards_untouched():
+    w = small(H=16, K=300, B=2, T=3)
+    wd = w.to(DEV)
+    n_o, n_l = w.B * w.T * w.H * 512, w.B * w.T * w.H
+    o_buf = torch.full((n_o + 4096,), 7.0, dtype=torch.bfloat16, device=DEV)
+    l_buf = torch.full((n_l + 2048,), 7.0, dtype=torch.float32, device=DEV)
+    o = o_buf[2048:2048 + n_o].view(w.B, w.T, w.H, 512)
+    lse = l_buf[1024:1024 + n_l].view(w.B, w.T, w.H)
+    for nsplit in (1, 5):
+        binding.decode(wd.q, wd.cache, wd.page_table, wd.idx, w.scale, nsplit, o=o, lse=lse)
+        torch.cuda.synchronize()
+        assert torch.all(o_buf[:2048] == 7) and torch.all(o_buf[2048 + n_o:] == 7)
+        assert torch.all(l_buf[:1024] == 7) and torch.all(l_buf[1024 + n_l:] == 7)
+    o_ref, lse_ref, _ = oracle_decode(w)
+    check_o_lse(o, lse, o_ref, lse_ref, "guarded")
+
+
+def test_side_stream_and_reused_workspace():
+    w = small(H=16, K=512, B=3, T=1)
+    wd = w.to(DEV)
+    s = torch.cuda.Stream()
+    ws = torch.empty(binding.workspace_bytes(3, 1, 16, 8), dtype=torch.uint8, device=DEV)
+    with torch.cuda.stream(s):
+        o, lse = binding.decode(wd.q, wd.cache, wd.page_table, wd.idx, w.scale, 8, workspace=ws,
+                                stream=s)
+    s.synchronize()
+    o_ref, lse_ref, _ = oracle_decode(w)
+    check_o_lse(o, lse, o_ref, lse_ref, "side stream")
+
+
+def test_device_error_paths():
+    w = small(H=16, K=64, B=1, T=1).to(DEV)
+    lib = binding.lib()
+    o = torch.empty((1, 1, 16, 512), dtype=torch.bfloat16, device=DEV)
+    lse = torch.empty((1, 1, 16), dtype=torch.float32, device=DEV)
+    qbytes = torch.empty(w.q.numel() * 2 + 64, dtype=torch.uint8, device=DEV)
+    mis = qbytes.data_ptr() + 2                      # 2-byte aligned, not 16
+    st = lib.smla_decode(mis, w.cache.data_ptr(), w.num_pages, w.page_table.data_ptr(),
+                         w.pt_stride, w.idx.data_ptr(), 1, 1, 16, 64, 64, w.scale, 1, None, 0,
+                         o.data_ptr(), lse.data_ptr(), None)
+    assert st == 3
+    st = lib.smla_decode(w.q.data_ptr(), w.cache.data_ptr(), w.num_pages, w.page_table.data_ptr(),
+                         w.pt_stride, w.idx.data_ptr(), 1, 1, 16, 64, 64, w.scale, 4, None, 100,
+                         o.data_ptr(), lse.data_ptr(), None)
+    assert st == 4

@@ -1,0 +1,164 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every function include/smla.h declares, rejects bad arguments before any CUDA
+call, sizes workspaces as documented, and the NSPLIT heuristic behaves as
+its model says."""
+import ctypes
+import math
+import os
+import re
+
+import pytest
+
+from sparse_mla_decode_partial_b200 import binding, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER_DIR = os.path.join(ROOT, "include")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return binding.lib()
+
+
+def declared_functions():
+    names = set()
+    for fn in os.listdir(HEADER_DIR):
+        if fn.endswith(".h"):
+            text = open(os.path.join(HEADER_DIR, fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names |= set(re.findall(r"\b(smla_\w+)\s*\(", text))
+    return sorted(names)
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert "smla_decode" in names and "smla_decode_partial" in names
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared but not exported"
+        assert n in binding.SIGNATURES, f"{n} has no binding signature"
+
+
+def test_status_strings(lib):
+    for code, name in binding.STATUS.items():
+        assert binding.status_string(code).startswith(name)
+    assert lib.smla_version() >= 100
+
+
+def test_workspace_bytes_formula(lib):
+    r = lambda x: (x + 255) // 256 * 256
+    for B, T, H, S in [(1, 1, 16, 64), (64, 1, 16, 8), (60, 1, 64, 3), (1, 9, 8, 16), (2, 3, 5, 7)]:
+        n = B * T * H * S
+        assert binding.workspace_bytes(B, T, H, S) == r(n * 512 * 4) + 2 * r(n * 4)
+    assert binding.workspace_bytes(1, 1, 1, 0) == 0
+    assert binding.workspace_bytes(-1, 1, 1, 1) == 0
+    assert binding.workspace_bytes(1, 1, 1, 1025) == 0
+
+
+FAKE = 0x10000000  # an aligned address that is never dereferenced: every call
+                   # below fails its host-side argument check before any CUDA call
+
+
+def call_partial(lib, q=FAKE, cache=FAKE, num_pages=10, pt=FAKE, pt_stride=4, idx=FAKE, B=1, T=1,
+                 H=16, K=64, ps=64, scale=0.1, nsplit=2, po=FAKE, pm=FAKE, pl=FAKE):
+    return lib.smla_decode_partial(q, cache, num_pages, pt, pt_stride, idx, B, T, H, K, ps, scale,
+                                   nsplit, po, pm, pl, None)
+
+
+def call_decode(lib, q=FAKE, cache=FAKE, num_pages=10, pt=FAKE, pt_stride=4, idx=FAKE, B=1, T=1,
+                H=16, K=64, ps=64, scale=0.1, nsplit=2, ws=FAKE, ws_bytes=1 << 30, o=FAKE,
+                lse=FAKE):
+    return lib.smla_decode(q, cache, num_pages, pt, pt_stride, idx, B, T, H, K, ps, scale, nsplit,
+                           ws, ws_bytes, o, lse, None)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(ps=32), 2), (dict(H=65), 2), (dict(B=-1), 1), (dict(K=-2), 1), (dict(nsplit=0), 1),
+    (dict(nsplit=1025), 1), (dict(q=0), 1), (dict(q=FAKE + 8), 3), (dict(cache=FAKE + 4), 3),
+    (dict(idx=FAKE + 2), 3), (dict(po=FAKE + 4), 3), (dict(pm=FAKE + 2), 3), (dict(po=0), 1),
+    (dict(num_pages=0), 1), (dict(pt_stride=0), 1), (dict(scale=math.inf), 1),
+    (dict(scale=math.nan), 1), (dict(cache=0), 1), (dict(pt=0), 1),
+])
+def test_partial_rejects_bad_arguments(lib, kw, expect):
+    assert call_partial(lib, **kw) == expect
+
+
+@pytest.mark.parametrize("kw", [dict(B=0), dict(T=0), dict(H=0)])
+def test_empty_problem_is_a_noop(lib, kw):
+    assert call_partial(lib, **kw) == 0
+    assert call_decode(lib, **kw) == 0
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(ws_bytes=100), 4), (dict(ws=0), 1), (dict(ws=FAKE + 8), 3), (dict(o=FAKE + 8), 3),
+    (dict(lse=FAKE + 2), 3), (dict(o=0), 1), (dict(nsplit=-1), 1), (dict(ps=16), 2),
+])
+def test_decode_rejects_bad_arguments(lib, kw, expect):
+    assert call_decode(lib, **kw) == expect
+
+
+def test_combine_rejects_bad_arguments(lib):
+    c = lambda **kw: lib.smla_lse_combine(kw.get("po", FAKE), kw.get("pm", FAKE),
+                                          kw.get("pl", FAKE), kw.get("B", 1), 1, 16,
+                                          kw.get("S", 4), kw.get("o", FAKE), kw.get("lse", FAKE),
+                                          None)
+    assert c(S=0) == 1 and c(S=2000) == 1 and c(B=-1) == 1 and c(po=0) == 1
+    assert c(po=FAKE + 4) == 3 and c(o=FAKE + 8) == 3 and c(B=0) == 0
+
+
+# ------------------------------------------------------------------ NSPLIT heuristic
+def model(B, T, H, K, sms):
+    """The cost model the library documents, restated for a table check."""
+    base = B * T
+    s_max = max(1, min(1024, -(-K // 32)))
+    best, best_s = None, 1
+    for s in range(1, s_max + 1):
+        ctas = base * s
+        t = math.ceil(ctas / sms) * (48.0 + math.ceil(K / s))
+        if s > 1:
+            t += 0.5 * ctas * H * (514 * 4.0) * 2.0 / 1152 / sms
+        if best is None or t < best * (1 - 1e-9):
+            best, best_s = t, s
+    return best_s
+
+
+@pytest.mark.parametrize("shape", [(1, 1, 16, 2048), (1, 9, 8, 2048), (64, 1, 16, 2048),
+                                   (60, 1, 64, 2048), (1, 1, 8, 256), (4, 1, 16, 100),
+                                   (128, 1, 16, 2048), (1, 1, 16, 31)])
+def test_nsplit_heuristic_matches_model(lib, shape, monkeypatch):
+    monkeypatch.delenv("SMLA_NSPLIT", raising=False)
+    B, T, H, K = shape
+    assert binding.choose_nsplit(B, T, H, K, 148) == model(B, T, H, K, 148)
+
+
+def test_nsplit_heuristic_properties(lib, monkeypatch):
+    monkeypatch.delenv("SMLA_NSPLIT", raising=False)
+    # one query token on an idle GPU: split as far as the 32-rows floor allows
+    assert binding.choose_nsplit(1, 1, 16, 2048, 148) == 64
+    # the split count never drops a split below 32 rows (except a single split)
+    for K in (1, 20, 33, 64, 65, 1000):
+        s = binding.choose_nsplit(1, 1, 16, K, 148)
+        assert s == 1 or math.ceil(K / s) >= 32 or s <= -(-K // 32)
+    # a batch that already fills the GPU is not split
+    assert binding.choose_nsplit(148, 1, 16, 2048, 148) == 1
+    # degenerate sizes
+    assert binding.choose_nsplit(0, 1, 16, 2048, 148) == 1
+    assert binding.choose_nsplit(1, 1, 16, 0, 148) == 1
+
+
+def test_nsplit_env_override(lib, monkeypatch):
+    monkeypatch.setenv("SMLA_NSPLIT", "37")
+    assert binding.choose_nsplit(64, 1, 16, 2048, 148) == 37
+    monkeypatch.setenv("SMLA_NSPLIT", "99999")
+    assert binding.choose_nsplit(64, 1, 16, 2048, 148) == 1024
+    monkeypatch.setenv("SMLA_NSPLIT", "junk")
+    assert binding.choose_nsplit(1, 1, 16, 2048, 148) == 64
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    q = torch.zeros((1, 1, 16, 576), dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        binding.decode(q, torch.zeros((1, 64, 576), dtype=torch.bfloat16),
+                       torch.zeros((1, 1), dtype=torch.int32), torch.zeros((1, 1, 4), dtype=torch.int32),
+                       0.1, 1)
