@@ -44,7 +44,8 @@
  *  - q, kv_cache, part_o, o and workspace must be 16-byte aligned; int32 and
  *    fp32 arrays 4-byte aligned.  Otherwise SMLA_ERR_MISALIGNED.
  *  - Dimensions are fixed at 512 + 64 and page_size must be 64; heads per
- *    query token at most 64.  Otherwise SMLA_ERR_UNSUPPORTED.
+ *    query token at most 64; num_pages at most SMLA_MAX_PAGES.  Otherwise
+ *    SMLA_ERR_UNSUPPORTED.
  *  - B, T, H or K equal to 0 are legal (K = 0: every o = 0, lse = -inf).
  *  - A CUDA error at launch returns SMLA_ERR_CUDA; smla_last_error() gives
  *    its text.  No entry point throws, aborts or exits.
@@ -67,6 +68,7 @@ extern "C" {
 #define SMLA_PAGE_SIZE 64  /* tokens per cache page */
 #define SMLA_MAX_HEADS 64
 #define SMLA_MAX_NSPLIT 1024
+#define SMLA_MAX_PAGES 33554431 /* cache rows must be addressable as int32 */
 
 typedef enum {
     SMLA_OK = 0,
@@ -85,9 +87,10 @@ typedef enum {
  * NSPLIT depends on SM count, heads per rank, batch size and query length;
  * section "The Occupancy Insight": more blocks in flight hide memory latency.
  * One CTA serves all heads of one (b, t, split), so the grid is B*T*NSPLIT
- * CTAs.  The heuristic picks the NSPLIT in [1, min(SMLA_MAX_NSPLIT-bound, K/32)]
+ * CTAs.  The heuristic picks the NSPLIT in [1, min(SMLA_MAX_NSPLIT, ceil(K/32))]
  * that minimises a model of wave count x rows per CTA plus per-CTA overhead
- * and the split-K scratch traffic.  sm_count <= 0 queries the current
+ * and the split-K scratch traffic, with two resident CTAs per SM for H <= 16
+ * and one otherwise.  sm_count <= 0 queries the current
  * device.  If the environment variable SMLA_NSPLIT holds a positive integer,
  * that value is returned instead (clamped to [1, SMLA_MAX_NSPLIT]).
  * Returns >= 1; returns 1 for degenerate sizes.

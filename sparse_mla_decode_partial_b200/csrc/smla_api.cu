@@ -1,6 +1,8 @@
 // smla_api.cu -- host side of the C ABI declared in include/smla.h: argument
 // checks, the NSPLIT heuristic, workspace carving and kernel launches.
 // Every entry point returns a status; nothing throws across the ABI.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <climits>
@@ -16,6 +18,7 @@
 #include "smla.h"
 #include "smla_combine.cuh"
 #include "smla_partial_mma.cuh"
+#include "smla_partial_tc.cuh"
 
 namespace {
 
@@ -75,7 +78,9 @@ int nsplit_model(int B, int T, int H, int K, int sm_count) {
     if (s_max < 1) s_max = 1;
     if (s_max > SMLA_MAX_NSPLIT) s_max = SMLA_MAX_NSPLIT;
     while (s_max > 1 && base * s_max > INT_MAX) --s_max;
-    const double slots = (double)sm_count;  // one partial CTA per SM (shared-memory bound)
+    // partial CTAs resident per SM: two for H <= 16 (the mma kernel's 2-stage
+    // form fits twice), one otherwise (shared memory)
+    const double slots = (double)sm_count * (H <= 16 ? 2.0 : 1.0);
     double best = 0.0;
     int best_s = 1;
     for (int s = 1; s <= s_max; ++s) {
@@ -105,7 +110,7 @@ smla_status check_decode_args(const void *q, const void *kv_cache, int64_t num_p
     if (K > 0) {
         if (kv_cache == nullptr || page_table == nullptr || idx == nullptr) return SMLA_ERR_INVALID_ARG;
         if (num_pages < 1 || pt_stride < 1) return SMLA_ERR_INVALID_ARG;
-        if (num_pages > (int64_t)1 << 40) return SMLA_ERR_INVALID_ARG;
+        if (num_pages > SMLA_MAX_PAGES) return SMLA_ERR_UNSUPPORTED;
         if (!aligned(kv_cache, 16) || !aligned(page_table, 4) || !aligned(idx, 4))
             return SMLA_ERR_MISALIGNED;
     }
@@ -124,17 +129,68 @@ smla_status launch_mma(const PartialParams &p, int grid, cudaStream_t st) {
     return e == cudaSuccess ? SMLA_OK : cuda_fail(e);
 }
 
+// cuTensorMapEncodeTiled from the driver, without linking libcuda.
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    });
+    return fn;
+}
+
+// 2-D view of the cache for the row gather: [num_pages * 64 rows, 576 bf16],
+// 1152-byte row stride, boxes of 64 columns x 1 row, 128-byte swizzle; rows
+// outside the tensor read as zeros.
+smla_status encode_cache_map(const PartialParams &p, CUtensorMap *out) {
+    auto enc = tensor_map_encoder();
+    if (enc == nullptr) {
+        std::snprintf(g_last_error, sizeof g_last_error, "cuTensorMapEncodeTiled unavailable");
+        return SMLA_ERR_CUDA;
+    }
+    cuuint64_t dims[2] = {(cuuint64_t)smla::kD, (cuuint64_t)p.num_pages * smla::kPage};
+    cuuint64_t strides[1] = {(cuuint64_t)smla::kRowBytes};
+    cuuint32_t box[2] = {64, 1};
+    cuuint32_t estride[2] = {1, 1};
+    const CUresult r = enc(out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<__nv_bfloat16 *>(p.cache),
+                           dims, strides, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        std::snprintf(g_last_error, sizeof g_last_error, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+        return SMLA_ERR_CUDA;
+    }
+    return SMLA_OK;
+}
+
+template <bool DIRECT>
+smla_status launch_tc(const PartialParams &p, int grid, cudaStream_t st) {
+    CUtensorMap tmap{};  // unused when there is nothing to gather (K == 0)
+    if (p.K > 0) {
+        const smla_status s = encode_cache_map(p, &tmap);
+        if (s != SMLA_OK) return s;
+    }
+    const void *fn = reinterpret_cast<const void *>(&smla::smla_partial_tc_kernel<DIRECT>);
+    cudaError_t e = ensure_smem_attr(fn, smla::TcCfg::kSmemBytes);
+    if (e != cudaSuccess) return cuda_fail(e);
+    smla::smla_partial_tc_kernel<DIRECT><<<grid, smla::TcCfg::kThreads, smla::TcCfg::kSmemBytes, st>>>(
+        p, tmap);
+    e = cudaGetLastError();
+    return e == cudaSuccess ? SMLA_OK : cuda_fail(e);
+}
+
 template <bool DIRECT>
 smla_status launch_partial(const PartialParams &p, cudaStream_t st) {
     const long long grid = (long long)p.B * p.T * p.nsplit;
     if (grid > INT_MAX) return SMLA_ERR_INVALID_ARG;
-    switch ((p.H + 15) / 16) {
-        case 1: return launch_mma<1, 32, 4, DIRECT>(p, (int)grid, st);
-        case 2: return launch_mma<2, 32, 4, DIRECT>(p, (int)grid, st);
-        case 3: return launch_mma<3, 32, 4, DIRECT>(p, (int)grid, st);
-        case 4: return launch_mma<4, 32, 4, DIRECT>(p, (int)grid, st);
-        default: return SMLA_ERR_UNSUPPORTED;
-    }
+    if (p.H > 32) return launch_tc<DIRECT>(p, (int)grid, st);
+    if (p.H > 16) return launch_mma<2, 32, 4, DIRECT>(p, (int)grid, st);
+    return launch_mma<1, 32, 2, DIRECT>(p, (int)grid, st);
 }
 
 PartialParams make_params(const void *q, const void *kv_cache, int64_t num_pages,
@@ -162,9 +218,40 @@ smla_status launch_combine(const float *part_o, const float *part_m, const float
     const long long units = (long long)B * T * H;
     if (units == 0) return SMLA_OK;
     if (units > INT_MAX) return SMLA_ERR_INVALID_ARG;
-    smla::smla_combine_kernel<<<(int)units, smla::kCombineThreads, nsplit * sizeof(float), st>>>(
-        part_o, part_m, part_lse, nsplit, static_cast<__nv_bfloat16 *>(o), lse);
-    const cudaError_t e = cudaGetLastError();
+    // Programmatic dependent launch: the combine grid may be scheduled while
+    // the partial pass still runs; the kernel waits (griddepcontrol.wait) for
+    // its predecessor to complete before reading anything.
+    cudaLaunchConfig_t cfg = {};
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    __nv_bfloat16 *ob = static_cast<__nv_bfloat16 *>(o);
+    cudaError_t e;
+    if (nsplit <= 8) {
+        // one warp per (b, t, h), every load in flight at once
+        cfg.gridDim = dim3((unsigned)((units + smla::kCombineWarpUnits - 1) / smla::kCombineWarpUnits));
+        cfg.blockDim = dim3(32 * smla::kCombineWarpUnits);
+        const int n = (int)units;
+        if (nsplit <= 2)
+            e = cudaLaunchKernelEx(&cfg, smla::smla_combine_warp_kernel<2>, part_o, part_m, part_lse,
+                                   nsplit, n, ob, lse);
+        else if (nsplit <= 4)
+            e = cudaLaunchKernelEx(&cfg, smla::smla_combine_warp_kernel<4>, part_o, part_m, part_lse,
+                                   nsplit, n, ob, lse);
+        else
+            e = cudaLaunchKernelEx(&cfg, smla::smla_combine_warp_kernel<8>, part_o, part_m, part_lse,
+                                   nsplit, n, ob, lse);
+    } else {
+        cfg.gridDim = dim3((unsigned)units);
+        cfg.blockDim = dim3(smla::kCombineThreads);
+        e = cudaLaunchKernelEx(&cfg, smla::smla_combine_kernel, part_o, part_m, part_lse, nsplit, ob,
+                               lse);
+    }
+    if (e == cudaSuccess) e = cudaGetLastError();
     return e == cudaSuccess ? SMLA_OK : cuda_fail(e);
 }
 

@@ -6,8 +6,20 @@
 // (b, t, h), with m_s the reference point of split s and lse_s its log-sum-exp:
 //   M = max_s m_s,  L = sum_s exp(lse_s - M),
 //   o = sum_s exp(m_s - M) O_s / L,  lse = M + ln L;  every split empty: 0, -inf.
-// One 128-thread CTA per (b, t, h); thread i owns output columns 4i..4i+3 and
-// streams the S partial rows with 16-byte loads.
+//
+// One 512-thread CTA per (b, t, h): 4 groups of 128 threads, thread c of a
+// group owning output columns 4c..4c+3.  Splits are taken in batches of
+// 4 x kCombineDepth; in a batch every thread issues all its loads (partial
+// rows, m, lse) before using any, so a batch costs one memory round trip.
+// A running maximum rescales the accumulators between batches.
+//
+// For few splits (S <= 8) a second form gives each (b, t, h) one warp: lane l
+// owns columns 4l + 128j (j < 4, coalesced float4 rows) and issues every load
+// of every split at once, so thousands of units finish in one wave.
+//
+// Both are launched as programmatic dependents of the partial pass: they may
+// be scheduled while that grid still runs, and wait on griddepcontrol before
+// touching memory.
 #pragma once
 
 #include <cstdint>
@@ -15,88 +27,164 @@
 
 namespace smla {
 
-constexpr int kCombineThreads = 128;
-
-__device__ __forceinline__ float block_reduce_max_128(float v, float *red) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-    __syncthreads();
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
-    __syncthreads();
-    return fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
-}
-
-__device__ __forceinline__ float block_reduce_sum_128(float v, float *red) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    __syncthreads();
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
-    __syncthreads();
-    return (red[0] + red[1]) + (red[2] + red[3]);
-}
+constexpr int kCombineThreads = 512;
+constexpr int kCombineGroups = 4;
+constexpr int kCombineDepth = 16;  // splits per group per batch
 
 __global__ void __launch_bounds__(kCombineThreads)
     smla_combine_kernel(const float *__restrict__ part_o, const float *__restrict__ part_m,
                         const float *__restrict__ part_lse, int nsplit,
                         __nv_bfloat16 *__restrict__ o, float *__restrict__ lse) {
-    extern __shared__ float w_s[];  // [nsplit] combine weights
-    __shared__ float red[4];
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    __shared__ float red_m[kCombineGroups];
+    __shared__ float red_l[kCombineGroups];
+    __shared__ float4 red_acc[kCombineGroups - 1][128];
+
     const size_t u = blockIdx.x;
-    const int tid = threadIdx.x;
+    const int g = threadIdx.x >> 7;
+    const int c = threadIdx.x & 127;
     const float *pm = part_m + u * nsplit;
     const float *pl = part_lse + u * nsplit;
+    const float4 *po = reinterpret_cast<const float4 *>(part_o + u * (size_t)nsplit * 512) + c;
 
-    float M = -INFINITY;
-    for (int s = tid; s < nsplit; s += kCombineThreads) M = fmaxf(M, pm[s]);
-    M = block_reduce_max_128(M, red);
-
-    uint2 *dst = reinterpret_cast<uint2 *>(o + u * 512) + tid;
-    if (M == -INFINITY) {
-        *dst = make_uint2(0u, 0u);
-        if (tid == 0) lse[u] = -INFINITY;
-        return;
-    }
-    float L = 0.f;
-    for (int s = tid; s < nsplit; s += kCombineThreads) {
-        const float v = pl[s];
-        if (v != -INFINITY) L += expf(v - M);
-    }
-    L = block_reduce_sum_128(L, red);
-    const float invL = 1.f / L;
-    for (int s = tid; s < nsplit; s += kCombineThreads) {
-        const float m = pm[s];
-        w_s[s] = (m == -INFINITY) ? 0.f : expf(m - M) * invL;
-    }
-    __syncthreads();
-
-    const float4 *src = reinterpret_cast<const float4 *>(part_o + u * (size_t)nsplit * 512) + tid;
+    float M = -INFINITY;  // running max over all batches (identical in every thread)
+    float L = 0.f;        // this group's sum of exp(lse_s - M)
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    int s = 0;
-    for (; s + 4 <= nsplit; s += 4) {
-        float4 v[4];
+
+    for (int s0 = 0; s0 < nsplit; s0 += kCombineGroups * kCombineDepth) {
+        float mv[kCombineDepth], lv[kCombineDepth];
+        float4 v[kCombineDepth];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) v[k] = __ldg(src + (size_t)(s + k) * 128);
+        for (int k = 0; k < kCombineDepth; ++k) {
+            const int s = s0 + g * kCombineDepth + k;
+            if (s < nsplit) {
+                mv[k] = __ldg(pm + s);
+                lv[k] = __ldg(pl + s);
+                v[k] = __ldg(po + (size_t)s * 128);
+            } else {
+                mv[k] = -INFINITY;
+                lv[k] = -INFINITY;
+                v[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+        }
+        float mb = -INFINITY;
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const float w = w_s[s + k];
+        for (int k = 0; k < kCombineDepth; ++k) mb = fmaxf(mb, mv[k]);
+        if (c == 0) red_m[g] = mb;
+        __syncthreads();
+        mb = fmaxf(fmaxf(red_m[0], red_m[1]), fmaxf(red_m[2], red_m[3]));
+        __syncthreads();  // red_m is rewritten by the next batch
+        const float Mn = fmaxf(M, mb);
+        if (Mn == -INFINITY) continue;  // nothing valid so far
+        const float r = (M == -INFINITY) ? 0.f : expf(M - Mn);
+        acc.x *= r;
+        acc.y *= r;
+        acc.z *= r;
+        acc.w *= r;
+        L *= r;
+#pragma unroll
+        for (int k = 0; k < kCombineDepth; ++k) {
+            const float w = (mv[k] == -INFINITY) ? 0.f : expf(mv[k] - Mn);
             acc.x = fmaf(w, v[k].x, acc.x);
             acc.y = fmaf(w, v[k].y, acc.y);
             acc.z = fmaf(w, v[k].z, acc.z);
             acc.w = fmaf(w, v[k].w, acc.w);
+            if (lv[k] != -INFINITY) L += expf(lv[k] - Mn);
+        }
+        M = Mn;
+    }
+
+    if (g > 0) red_acc[g - 1][c] = acc;
+    if (c == 0) red_l[g] = L;
+    __syncthreads();
+    if (g != 0) return;
+    uint2 *dst = reinterpret_cast<uint2 *>(o + u * 512) + c;
+    if (M == -INFINITY) {
+        *dst = make_uint2(0u, 0u);
+        if (c == 0) lse[u] = -INFINITY;
+        return;
+    }
+#pragma unroll
+    for (int k = 0; k < kCombineGroups - 1; ++k) {
+        const float4 a = red_acc[k][c];
+        acc.x += a.x;
+        acc.y += a.y;
+        acc.z += a.z;
+        acc.w += a.w;
+    }
+    const float Lt = (red_l[0] + red_l[1]) + (red_l[2] + red_l[3]);
+    const float inv = 1.f / Lt;
+    __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+    __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+    *dst = make_uint2(*reinterpret_cast<uint32_t *>(&lo), *reinterpret_cast<uint32_t *>(&hi));
+    if (c == 0) lse[u] = M + logf(Lt);
+}
+
+constexpr int kCombineWarpUnits = 4;  // units (warps) per CTA of the warp form
+
+template <int SMAX>
+__global__ void __launch_bounds__(32 * kCombineWarpUnits)
+    smla_combine_warp_kernel(const float *__restrict__ part_o, const float *__restrict__ part_m,
+                             const float *__restrict__ part_lse, int nsplit, int n_units,
+                             __nv_bfloat16 *__restrict__ o, float *__restrict__ lse) {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    const int lane = threadIdx.x & 31;
+    const long long u = (long long)blockIdx.x * kCombineWarpUnits + (threadIdx.x >> 5);
+    if (u >= n_units) return;
+    const float *pm = part_m + u * nsplit;
+    const float *pl = part_lse + u * nsplit;
+    const float4 *po = reinterpret_cast<const float4 *>(part_o + u * (long long)nsplit * 512) + lane;
+
+    float mv[SMAX], lv[SMAX];
+    float4 v[SMAX][4];
+#pragma unroll
+    for (int s = 0; s < SMAX; ++s) {
+        if (s < nsplit) {
+            mv[s] = __ldg(pm + s);
+            lv[s] = __ldg(pl + s);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) v[s][j] = __ldg(po + s * 128 + j * 32);
+        } else {
+            mv[s] = -INFINITY;
+            lv[s] = -INFINITY;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) v[s][j] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
     }
-    for (; s < nsplit; ++s) {
-        const float4 v = __ldg(src + (size_t)s * 128);
-        const float w = w_s[s];
-        acc.x = fmaf(w, v.x, acc.x);
-        acc.y = fmaf(w, v.y, acc.y);
-        acc.z = fmaf(w, v.z, acc.z);
-        acc.w = fmaf(w, v.w, acc.w);
+    float M = -INFINITY;
+#pragma unroll
+    for (int s = 0; s < SMAX; ++s) M = fmaxf(M, mv[s]);
+    uint2 *dst = reinterpret_cast<uint2 *>(o + u * 512) + lane;
+    if (M == -INFINITY) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) dst[j * 32] = make_uint2(0u, 0u);
+        if (lane == 0) lse[u] = -INFINITY;
+        return;
     }
-    __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
-    __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
-    *dst = make_uint2(*reinterpret_cast<uint32_t *>(&lo), *reinterpret_cast<uint32_t *>(&hi));
-    if (tid == 0) lse[u] = M + logf(L);
+    float L = 0.f;
+    float4 acc[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int s = 0; s < SMAX; ++s) {
+        if (lv[s] != -INFINITY) L += expf(lv[s] - M);
+        const float w = (mv[s] == -INFINITY) ? 0.f : expf(mv[s] - M);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            acc[j].x = fmaf(w, v[s][j].x, acc[j].x);
+            acc[j].y = fmaf(w, v[s][j].y, acc[j].y);
+            acc[j].z = fmaf(w, v[s][j].z, acc[j].z);
+            acc[j].w = fmaf(w, v[s][j].w, acc[j].w);
+        }
+    }
+    const float inv = 1.f / L;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        __nv_bfloat162 lo = __floats2bfloat162_rn(acc[j].x * inv, acc[j].y * inv);
+        __nv_bfloat162 hi = __floats2bfloat162_rn(acc[j].z * inv, acc[j].w * inv);
+        dst[j * 32] = make_uint2(*reinterpret_cast<uint32_t *>(&lo), *reinterpret_cast<uint32_t *>(&hi));
+    }
+    if (lane == 0) lse[u] = M + logf(L);
 }
 
 }  // namespace smla

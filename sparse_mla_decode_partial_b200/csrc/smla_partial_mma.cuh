@@ -11,14 +11,21 @@
 // CTA is what keeps the pass at one HBM read per selected row.
 //
 // Warp roles (HG = head groups of 16 rows, the mma M dimension):
-//   warp 4*HG      producer: resolves index -> page -> row, issues one 1-D
+//   warp 4*HG      producer: first resolves the split's index entries to
+//                  physical rows (index loads, then page-table loads, 32 per
+//                  lane in flight) into shared memory, then issues one 1-D
 //                  bulk async copy (TMA engine, 1152 B) per row into a ring of
-//                  NSTAGE tiles of NT rows, completes on an mbarrier.
-//   warps 0..4HG-1 consumers, 4 per head group: S = Q K^T over 576 dims
-//                  (each warp NT/4 columns), masked online softmax in fp32
-//                  (exp2 domain, quad shuffles + one smem exchange per tile),
-//                  P to smem as bf16, O += P C (each warp 128 of the 512
-//                  output columns, fp32 registers).
+//                  NSTAGE tiles of NT rows, each completing on an mbarrier.
+//   warps 0..4HG-1 consumers, 4 per head group.  Each warp keeps the Q
+//                  fragments of one quarter of the 576 dims in registers and
+//                  computes that quarter's partial S = Q K^T for all NT rows
+//                  of a tile (independent accumulators per n8 tile); the four
+//                  partials meet once per tile in shared memory (double
+//                  buffered: one named barrier per tile).  Every warp then
+//                  holds the full S of its 16 heads, runs the masked online
+//                  softmax in fp32 (exp2 domain, quad shuffles), turns P into
+//                  A fragments in registers and accumulates O += P C for its
+//                  128 of the 512 output columns in fp32 registers.
 // Shared-memory rows are 1168 B apart (1152 + 16) so that the 8 row addresses
 // of every ldmatrix phase fall in distinct 16-byte bank groups.
 #pragma once
@@ -38,6 +45,7 @@ constexpr int kRowBytes = kD * 2;                 // 1152
 constexpr int kSmemRowBytes = kRowBytes + 16;     // 1168
 constexpr float kLog2e = 1.4426950408889634f;     // log2(e)
 constexpr float kLn2 = 0.69314718055994531f;      // ln(2)
+constexpr int kResolveChunk = 2048;  // index entries resolved to rows ahead of the copies
 
 // Source of the bulk copy for a padding slot: a row of zeros, so that masked
 // slots hold finite values (their probability is 0, and 0 * finite = 0).
@@ -67,21 +75,24 @@ struct MmaCfg {
     static constexpr int kHeads = 16 * HG;
     static constexpr int kComputeWarps = 4 * HG;
     static constexpr int kThreads = (kComputeWarps + 1) * 32;
-    static constexpr int kPStride = NT * 2 + 16;  // bytes per P row (conflict-free ldmatrix)
+    static constexpr int kSRow = NT + 8;  // floats per S-partial row (32-byte pad: conflict-free float2)
     static constexpr int kStageBytes = NT * kSmemRowBytes;
-    static constexpr int kOffQ = 0;
-    static constexpr int kOffKV = kOffQ + kHeads * kSmemRowBytes;
-    static constexpr int kOffP = kOffKV + NSTAGE * kStageBytes;
-    static constexpr int kOffRed = kOffP + HG * 16 * kPStride;   // float [HG][4][16]
-    static constexpr int kOffL = kOffRed + HG * 4 * 16 * 4;       // float [HG][4][16]
-    static constexpr int kOffHdr = kOffL + HG * 4 * 16 * 4;       // u64 [NSTAGE]
-    static constexpr int kOffBar = kOffHdr + NSTAGE * 8;          // u64 full[], empty[], q
-    static constexpr int kSmemBytes = kOffBar + (2 * NSTAGE + 1) * 8;
+    static constexpr int kQBytes = kHeads * kSmemRowBytes;
+    static constexpr int kSPartBytes = HG * 2 * 4 * 16 * kSRow * 4;
+    static constexpr int kOffQ = 0;  // Q rows, then (after Q is in registers) the S partials
+    static constexpr int kOffKV = kOffQ + ((kQBytes > kSPartBytes ? kQBytes : kSPartBytes) + 127) / 128 * 128;
+    static constexpr int kOffHdr = kOffKV + NSTAGE * kStageBytes;  // u64 [NSTAGE]
+    static constexpr int kOffBar = kOffHdr + NSTAGE * 8;            // u64 full[], empty[]
+    static constexpr int kOffRows = kOffBar + 2 * NSTAGE * 8;       // int [kResolveChunk]
+    static constexpr int kSmemBytes = kOffRows + kResolveChunk * 4;
     static_assert(kSmemBytes <= 232448, "shared memory per CTA");
+    // CTAs per SM the launch bounds ask for: two when a pair fits (more
+    // producers per SM keep more row gathers in flight).
+    static constexpr int kMinBlocks = (2 * (kSmemBytes + 1024) <= 233472 && kThreads <= 192) ? 2 : 1;
 };
 
 template <int HG, int NT, int NSTAGE, bool DIRECT>
-__global__ void __launch_bounds__(MmaCfg<HG, NT, NSTAGE>::kThreads, 1)
+__global__ void __launch_bounds__(MmaCfg<HG, NT, NSTAGE>::kThreads, MmaCfg<HG, NT, NSTAGE>::kMinBlocks)
     smla_partial_mma_kernel(const PartialParams p) {
     using C = MmaCfg<HG, NT, NSTAGE>;
     extern __shared__ __align__(128) uint8_t smem[];
@@ -100,7 +111,6 @@ __global__ void __launch_bounds__(MmaCfg<HG, NT, NSTAGE>::kThreads, 1)
 
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::kOffBar);
     uint64_t *empty = full + NSTAGE;
-    uint64_t *qbar = full + 2 * NSTAGE;
     volatile uint64_t *hdr = reinterpret_cast<volatile uint64_t *>(smem + C::kOffHdr);
 
     if (threadIdx.x == 0) {
@@ -108,93 +118,87 @@ __global__ void __launch_bounds__(MmaCfg<HG, NT, NSTAGE>::kThreads, 1)
             mbar_init(&full[i], 1);
             mbar_init(&empty[i], C::kComputeWarps);
         }
-        mbar_init(qbar, 1);
         fence_mbar_init();
     }
-    // Head rows beyond H are zero (they are never written by a copy).
-    {
-        constexpr int kChunks = kSmemRowBytes / 16;
-        const int n = (C::kHeads - p.H) * kChunks;
-        for (int i = threadIdx.x; i < n; i += blockDim.x) {
-            const int r = p.H + i / kChunks;
-            *reinterpret_cast<uint4 *>(smem + C::kOffQ + r * kSmemRowBytes + (i % kChunks) * 16) =
-                make_uint4(0u, 0u, 0u, 0u);
-        }
-    }
+    // The combine kernel is launched as a programmatic dependent: let it be
+    // scheduled now; it waits for this grid's completion before reading.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     __syncthreads();
 
     if (warp == C::kComputeWarps) {
         // ============================================================ producer
-        const __nv_bfloat16 *qsrc = p.q + (size_t)bt * p.H * kD;
-        if (lane == 0) {
-            mbar_expect_tx(qbar, (uint32_t)(p.H * kRowBytes));
-            mbar_arrive(qbar);
-        }
-        __syncwarp();
-        for (int h = lane; h < p.H; h += 32)
-            bulk_g2s(smem + C::kOffQ + h * kSmemRowBytes, qsrc + (size_t)h * kD, kRowBytes, qbar);
-
-        const int *idx_bt = p.idx + (size_t)bt * p.K;
+        const int *idx_bt = p.idx + (size_t)bt * p.K + j0;
         const int *pt_b = p.page_table + (size_t)b * p.pt_stride;
         const long long max_pos = (long long)p.pt_stride * kPage;
         const uint64_t policy = l2_policy_evict_first();
-        constexpr int kSlots = NT / 32;
-        const uint8_t *src[kSlots];
-        bool valid[kSlots];
-
-        auto resolve = [&](int tile) {
-            int iv[kSlots];
+        int *rows_s = reinterpret_cast<int *>(smem + C::kOffRows);
+        constexpr int kResolveBatch = HG <= 2 ? 32 : 16;  // loads in flight per lane
+        const int len = j1 - j0;
+        int it = 0;  // tile counter over the whole split
+        for (int base = 0; base < len; base += kResolveChunk) {
+            const int n = min(kResolveChunk, len - base);
+            // Resolve the whole chunk before the first copy: index loads, then
+            // page-table loads, each batch of 32 per lane in flight at once.
+            for (int b0 = 0; b0 < n; b0 += 32 * kResolveBatch) {
+                int iv[kResolveBatch];
 #pragma unroll
-            for (int k = 0; k < kSlots; ++k) {
-                const int j = j0 + tile * NT + k * 32 + lane;
-                iv[k] = (j < j1) ? __ldg(idx_bt + j) : -1;
-            }
+                for (int k = 0; k < kResolveBatch; ++k) {
+                    const int j = b0 + k * 32 + lane;
+                    iv[k] = (j < n) ? __ldg(idx_bt + base + j) : -1;
+                }
+                int pg[kResolveBatch];
 #pragma unroll
-            for (int k = 0; k < kSlots; ++k) {
-                const int i = iv[k];
-                valid[k] = false;
-                src[k] = reinterpret_cast<const uint8_t *>(g_zero_row);
-                if (i != -1) {
-                    bool bad = (i < 0) || ((long long)i >= max_pos);
-                    if (!bad) {
-                        const int page = __ldg(pt_b + (i >> 6));
-                        bad = (page < 0) || ((long long)page >= p.num_pages);
-                        if (!bad) {
-                            valid[k] = true;
-                            src[k] = reinterpret_cast<const uint8_t *>(p.cache) +
-                                     ((size_t)page * kPage + (size_t)(i & (kPage - 1))) * kRowBytes;
+                for (int k = 0; k < kResolveBatch; ++k) {
+                    const int i = iv[k];
+                    pg[k] = (i >= 0 && (long long)i < max_pos) ? __ldg(pt_b + (i >> 6)) : -1;
+                }
+#pragma unroll
+                for (int k = 0; k < kResolveBatch; ++k) {
+                    const int j = b0 + k * 32 + lane;
+                    const int i = iv[k];
+                    int row = -1;
+                    if (i != -1) {
+                        const bool ok = (i >= 0) && ((long long)i < max_pos) && (pg[k] >= 0) &&
+                                        ((long long)pg[k] < p.num_pages);
+                        if (ok) {
+                            row = pg[k] * kPage + (i & (kPage - 1));
+                        } else if (j < n) {
+                            atomicOr(&g_status_flags, kFlagIndexRange);
+                            atomicAdd(&g_bad_index_count, 1ull);
                         }
                     }
-                    if (bad) {
-                        atomicOr(&g_status_flags, kFlagIndexRange);
-                        atomicAdd(&g_bad_index_count, 1ull);
-                    }
+                    if (j < n) rows_s[j] = row;
                 }
             }
-        };
-
-        if (n_tiles > 0) resolve(0);
-        for (int it = 0; it < n_tiles; ++it) {
-            const int stage = it % NSTAGE;
-            if (it >= NSTAGE) mbar_wait(&empty[stage], ((it / NSTAGE) - 1) & 1, dead);
-            if (lane == 0) mbar_expect_tx(&full[stage], (uint32_t)(NT * kRowBytes));
             __syncwarp();
-            uint8_t *dst = smem + C::kOffKV + stage * C::kStageBytes;
-            uint64_t mask = 0;
+            // Issue one bulk copy per row (or per padding slot, from the zero row).
+            const int chunk_tiles = (n + NT - 1) / NT;
+            for (int t = 0; t < chunk_tiles; ++t, ++it) {
+                const int stage = it % NSTAGE;
+                if (it >= NSTAGE) mbar_wait(&empty[stage], ((it / NSTAGE) - 1) & 1, dead);
+                if (lane == 0) mbar_expect_tx(&full[stage], (uint32_t)(NT * kRowBytes));
+                __syncwarp();
+                uint8_t *dst = smem + C::kOffKV + stage * C::kStageBytes;
+                uint64_t mask = 0;
 #pragma unroll
-            for (int k = 0; k < kSlots; ++k) {
-                uint8_t *d = dst + (k * 32 + lane) * kSmemRowBytes;
-                if (valid[k])
-                    bulk_g2s_hint(d, src[k], kRowBytes, &full[stage], policy);
-                else
-                    bulk_g2s(d, src[k], kRowBytes, &full[stage]);
-                mask |= (uint64_t)__ballot_sync(0xffffffffu, valid[k]) << (32 * k);
+                for (int k = 0; k < NT / 32; ++k) {
+                    const int r = t * NT + k * 32 + lane;
+                    const int row = (r < n) ? rows_s[r] : -1;
+                    uint8_t *d = dst + (k * 32 + lane) * kSmemRowBytes;
+                    if (row >= 0)
+                        bulk_g2s_hint(d, reinterpret_cast<const uint8_t *>(p.cache) +
+                                             (size_t)row * kRowBytes,
+                                      kRowBytes, &full[stage], policy);
+                    else
+                        bulk_g2s(d, g_zero_row, kRowBytes, &full[stage]);
+                    mask |= (uint64_t)__ballot_sync(0xffffffffu, row >= 0) << (32 * k);
+                }
+                if (lane == 0) {
+                    hdr[stage] = mask;
+                    mbar_arrive(&full[stage]);  // release: hdr is visible to the waiters
+                }
             }
-            if (lane == 0) {
-                hdr[stage] = mask;
-                mbar_arrive(&full[stage]);  // release: hdr is visible to the waiters
-            }
-            if (it + 1 < n_tiles) resolve(it + 1);
+            __syncwarp();  // rows_s is rewritten by the next chunk
         }
         // Copies still in flight must land before the CTA may exit.
         for (int it = (n_tiles > NSTAGE ? n_tiles - NSTAGE : 0); it < n_tiles; ++it)
@@ -204,11 +208,44 @@ __global__ void __launch_bounds__(MmaCfg<HG, NT, NSTAGE>::kThreads, 1)
 
     // ================================================================ consumers
     const int g = warp >> 2;   // head group
-    const int qw = warp & 3;   // quarter: S columns and O columns owned
+    const int qw = warp & 3;   // quarter: k range of S, and 128 output columns
     const int r0 = lane >> 2;  // fragment row (and r0 + 8)
     const int cq = lane & 3;   // fragment column pair
-    constexpr int NTW = NT / 32;  // n8 tiles of S per warp
-    const int col0 = qw * (NT / 4);
+    constexpr int NTS = NT / 8;  // n8 tiles of S (all NT columns, every warp)
+    constexpr int KQ = kD / 16 / 4;  // k16 steps of S per warp (576 / 16 / 4 = 9)
+    const uint32_t bar_grp = 1 + g;
+    const uint32_t bar_all = 1 + HG;
+
+    // Q fragments of this warp's k quarter stay in registers for the whole split.
+    // Each warp loads its own 16 heads x 144 dims with plain 16-byte loads (rows
+    // beyond H are zero), parks them in shared memory and ldmatrix-es them out;
+    // the TMA engine stays free for the gathered rows.
+    uint32_t qa[KQ][4];
+    {
+        const uint4 *qsrc = reinterpret_cast<const uint4 *>(p.q + (size_t)bt * p.H * kD);
+        uint4 qv[9];
+#pragma unroll
+        for (int i = 0; i < 9; ++i) {
+            const int c = lane + 32 * i;          // 16 rows x 18 chunks of 8 dims
+            const int h = 16 * g + c / 18;
+            qv[i] = (h < p.H) ? __ldg(qsrc + (size_t)h * (kD / 8) + KQ * 2 * qw + c % 18)
+                              : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int i = 0; i < 9; ++i) {
+            const int c = lane + 32 * i;
+            *reinterpret_cast<uint4 *>(smem + C::kOffQ + (16 * g + c / 18) * kSmemRowBytes +
+                                       (KQ * 2 * qw + c % 18) * 16) = qv[i];
+        }
+        __syncwarp();
+        const uint32_t q_base = smem_addr(smem + C::kOffQ) +
+                                (16 * g + (lane & 15)) * kSmemRowBytes + (lane >> 4) * 16;
+#pragma unroll
+        for (int kk = 0; kk < KQ; ++kk)
+            ldsm_x4(q_base + (KQ * qw + kk) * 32, qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3]);
+    }
+    // The Q region is reused for the split-k score exchange from here on.
+    named_bar_sync(bar_all, 128 * HG);
 
     float m_run0 = -INFINITY, m_run1 = -INFINITY;
     float l0 = 0.f, l1 = 0.f;
@@ -216,14 +253,8 @@ __global__ void __launch_bounds__(MmaCfg<HG, NT, NSTAGE>::kThreads, 1)
 #pragma unroll
     for (int n = 0; n < 16; ++n) oacc[n][0] = oacc[n][1] = oacc[n][2] = oacc[n][3] = 0.f;
 
-    const uint32_t q_base = smem_addr(smem + C::kOffQ) +
-                            (16 * g + (lane & 15)) * kSmemRowBytes + (lane >> 4) * 16;
-    uint8_t *pbuf = smem + C::kOffP + g * 16 * C::kPStride;
-    const uint32_t p_base = smem_addr(pbuf) + (lane & 15) * C::kPStride + (lane >> 4) * 16;
-    float *red = reinterpret_cast<float *>(smem + C::kOffRed) + g * 64;
-    const uint32_t bar_id = 1 + g;
-
-    mbar_wait(qbar, 0, dead);
+    // S partials: [group][buffer][warp][16 rows][NT cols] fp32, rows padded by 32 B.
+    float *spart = reinterpret_cast<float *>(smem + C::kOffQ) + g * 2 * 4 * 16 * C::kSRow;
 
     for (int it = 0; it < n_tiles; ++it) {
         const int stage = it % NSTAGE;
@@ -231,61 +262,61 @@ __global__ void __launch_bounds__(MmaCfg<HG, NT, NSTAGE>::kThreads, 1)
         const uint64_t vmask = hdr[stage];
         const uint32_t kv = smem_addr(smem + C::kOffKV + stage * C::kStageBytes);
 
-        // ---- S = Q K^T, columns [col0, col0 + NT/4)
-        float sacc[NTW][4];
+        // ---- partial S = Q K^T over this warp's 144 dims, all NT columns
+        float sacc[NTS][4];
 #pragma unroll
-        for (int n = 0; n < NTW; ++n) sacc[n][0] = sacc[n][1] = sacc[n][2] = sacc[n][3] = 0.f;
-        uint32_t b_base;
-        if (NTW == 2)
-            b_base = kv + (col0 + (lane & 7) + ((lane >> 4) << 3)) * kSmemRowBytes +
-                     ((lane >> 3) & 1) * 16;
-        else
-            b_base = kv + (col0 + (lane & 7)) * kSmemRowBytes + ((lane >> 3) & 1) * 16;
-#pragma unroll 6
-        for (int kk = 0; kk < kD / 16; ++kk) {
-            uint32_t a0, a1, a2, a3;
-            ldsm_x4(q_base + kk * 32, a0, a1, a2, a3);
-            if (NTW == 2) {
+        for (int n = 0; n < NTS; ++n) sacc[n][0] = sacc[n][1] = sacc[n][2] = sacc[n][3] = 0.f;
+        const uint32_t b_base = kv + ((lane & 7) + ((lane >> 4) << 3)) * kSmemRowBytes +
+                                ((lane >> 3) & 1) * 16 + KQ * qw * 32;
+#pragma unroll
+        for (int kk = 0; kk < KQ; ++kk) {
+#pragma unroll
+            for (int np = 0; np < NTS / 2; ++np) {
                 uint32_t b0, b1, b2, b3;
-                ldsm_x4(b_base + kk * 32, b0, b1, b2, b3);
-                mma_bf16_16816(sacc[0], a0, a1, a2, a3, b0, b1);
-                mma_bf16_16816(sacc[NTW - 1], a0, a1, a2, a3, b2, b3);
-            } else {
-                uint32_t b0, b1;
-                ldsm_x2(b_base + kk * 32, b0, b1);
-                mma_bf16_16816(sacc[0], a0, a1, a2, a3, b0, b1);
+                ldsm_x4(b_base + np * 16 * kSmemRowBytes + kk * 32, b0, b1, b2, b3);
+                mma_bf16_16816(sacc[2 * np], qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3], b0, b1);
+                mma_bf16_16816(sacc[2 * np + 1], qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3], b2, b3);
             }
         }
+        float *sp = spart + (it & 1) * 4 * 16 * C::kSRow;
+#pragma unroll
+        for (int n = 0; n < NTS; ++n) {
+            float *d = sp + qw * 16 * C::kSRow + 8 * n + 2 * cq;
+            *reinterpret_cast<float2 *>(d + r0 * C::kSRow) = make_float2(sacc[n][0], sacc[n][1]);
+            *reinterpret_cast<float2 *>(d + (r0 + 8) * C::kSRow) = make_float2(sacc[n][2], sacc[n][3]);
+        }
+        named_bar_sync(bar_grp, 128);
 
-        // ---- scale into the log2 domain, mask, row max of this warp's columns
+        // ---- full S (sum of the four k quarters), scaled to log2 units, masked
         float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
-        for (int n = 0; n < NTW; ++n) {
+        for (int n = 0; n < NTS; ++n) {
+            float2 a = make_float2(0.f, 0.f), c = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const int col = col0 + 8 * n + 2 * cq + e;
-                const bool ok = (vmask >> col) & 1ull;
-                const float v0 = ok ? sacc[n][e] * p.scale_log2 : -INFINITY;
-                const float v1 = ok ? sacc[n][2 + e] * p.scale_log2 : -INFINITY;
-                sacc[n][e] = v0;
-                sacc[n][2 + e] = v1;
-                mx0 = fmaxf(mx0, v0);
-                mx1 = fmaxf(mx1, v1);
+            for (int w = 0; w < 4; ++w) {
+                const float *src = sp + w * 16 * C::kSRow + 8 * n + 2 * cq;
+                const float2 x = *reinterpret_cast<const float2 *>(src + r0 * C::kSRow);
+                const float2 y = *reinterpret_cast<const float2 *>(src + (r0 + 8) * C::kSRow);
+                a.x += x.x;
+                a.y += x.y;
+                c.x += y.x;
+                c.y += y.y;
             }
+            const int col = 8 * n + 2 * cq;
+            const bool ok0 = (vmask >> col) & 1ull, ok1 = (vmask >> (col + 1)) & 1ull;
+            sacc[n][0] = ok0 ? a.x * p.scale_log2 : -INFINITY;
+            sacc[n][1] = ok1 ? a.y * p.scale_log2 : -INFINITY;
+            sacc[n][2] = ok0 ? c.x * p.scale_log2 : -INFINITY;
+            sacc[n][3] = ok1 ? c.y * p.scale_log2 : -INFINITY;
+            mx0 = fmaxf(mx0, fmaxf(sacc[n][0], sacc[n][1]));
+            mx1 = fmaxf(mx1, fmaxf(sacc[n][2], sacc[n][3]));
         }
         mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
         mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
         mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
         mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-        if (cq == 0) {
-            red[qw * 16 + r0] = mx0;
-            red[qw * 16 + r0 + 8] = mx1;
-        }
-        named_bar_sync(bar_id, 128);
-        const float t0 = fmaxf(fmaxf(red[r0], red[16 + r0]), fmaxf(red[32 + r0], red[48 + r0]));
-        const float t1 = fmaxf(fmaxf(red[8 + r0], red[24 + r0]), fmaxf(red[40 + r0], red[56 + r0]));
-        const float mn0 = fmaxf(m_run0, t0);
-        const float mn1 = fmaxf(m_run1, t1);
+        const float mn0 = fmaxf(m_run0, mx0);
+        const float mn1 = fmaxf(m_run1, mx1);
         const float mu0 = (mn0 == -INFINITY) ? 0.f : mn0;
         const float mu1 = (mn1 == -INFINITY) ? 0.f : mn1;
         const float al0 = exp2f(m_run0 - mu0);
@@ -293,18 +324,17 @@ __global__ void __launch_bounds__(MmaCfg<HG, NT, NSTAGE>::kThreads, 1)
         m_run0 = mn0;
         m_run1 = mn1;
 
-        // ---- P = exp2(s - m), row sums, P -> smem (bf16)
+        // ---- P = exp2(s - m) straight into A fragments (k16 step j = n8 tiles 2j, 2j+1)
+        uint32_t pa[NT / 16][4];
         float ps0 = 0.f, ps1 = 0.f;
 #pragma unroll
-        for (int n = 0; n < NTW; ++n) {
+        for (int n = 0; n < NTS; ++n) {
             const float p00 = exp2f(sacc[n][0] - mu0), p01 = exp2f(sacc[n][1] - mu0);
             const float p10 = exp2f(sacc[n][2] - mu1), p11 = exp2f(sacc[n][3] - mu1);
             ps0 += p00 + p01;
             ps1 += p10 + p11;
-            const int col = col0 + 8 * n + 2 * cq;
-            *reinterpret_cast<uint32_t *>(pbuf + r0 * C::kPStride + col * 2) = pack_bf16x2(p00, p01);
-            *reinterpret_cast<uint32_t *>(pbuf + (r0 + 8) * C::kPStride + col * 2) =
-                pack_bf16x2(p10, p11);
+            pa[n >> 1][(n & 1) * 2 + 0] = pack_bf16x2(p00, p01);
+            pa[n >> 1][(n & 1) * 2 + 1] = pack_bf16x2(p10, p11);
         }
         l0 = l0 * al0 + ps0;
         l1 = l1 * al1 + ps1;
@@ -315,46 +345,35 @@ __global__ void __launch_bounds__(MmaCfg<HG, NT, NSTAGE>::kThreads, 1)
             oacc[n][2] *= al1;
             oacc[n][3] *= al1;
         }
-        named_bar_sync(bar_id, 128);
 
         // ---- O[:, qw*128 .. +128] += P C
         const uint32_t v_base = kv + ((lane & 7) + ((lane >> 3) & 1) * 8) * kSmemRowBytes +
                                 (qw * 128 + (lane >> 4) * 8) * 2;
 #pragma unroll
-        for (int kk = 0; kk < NT / 16; ++kk) {
-            uint32_t a0, a1, a2, a3;
-            ldsm_x4(p_base + kk * 32, a0, a1, a2, a3);
+        for (int j = 0; j < NT / 16; ++j) {
 #pragma unroll
             for (int np = 0; np < 8; ++np) {
                 uint32_t b0, b1, b2, b3;
-                ldsm_x4_t(v_base + kk * 16 * kSmemRowBytes + np * 32, b0, b1, b2, b3);
-                mma_bf16_16816(oacc[2 * np], a0, a1, a2, a3, b0, b1);
-                mma_bf16_16816(oacc[2 * np + 1], a0, a1, a2, a3, b2, b3);
+                ldsm_x4_t(v_base + j * 16 * kSmemRowBytes + np * 32, b0, b1, b2, b3);
+                mma_bf16_16816(oacc[2 * np], pa[j][0], pa[j][1], pa[j][2], pa[j][3], b0, b1);
+                mma_bf16_16816(oacc[2 * np + 1], pa[j][0], pa[j][1], pa[j][2], pa[j][3], b2, b3);
             }
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[stage]);
     }
 
-    // ---- epilogue: full row sums, then partial (or final) outputs
+    // ---- epilogue: row sums (every warp of the group holds the same full sums)
     l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
     l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
     l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
     l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
-    float *lred = reinterpret_cast<float *>(smem + C::kOffL) + g * 64;
-    if (cq == 0) {
-        lred[qw * 16 + r0] = l0;
-        lred[qw * 16 + r0 + 8] = l1;
-    }
-    named_bar_sync(bar_id, 128);
-    const float lt0 = lred[r0] + lred[16 + r0] + lred[32 + r0] + lred[48 + r0];
-    const float lt1 = lred[8 + r0] + lred[24 + r0] + lred[40 + r0] + lred[56 + r0];
 
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
         const int h = 16 * g + r0 + 8 * half;
         if (h >= p.H) continue;
-        const float lt = half ? lt1 : lt0;
+        const float lt = half ? l1 : l0;
         const float mr = half ? m_run1 : m_run0;
         const size_t row = (size_t)bt * p.H + h;
         if (!DIRECT) {

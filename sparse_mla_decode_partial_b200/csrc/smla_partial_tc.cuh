@@ -1,0 +1,420 @@
+// smla_partial_tc.cuh -- split-K partial pass on the 5th-generation tensor
+// core (tcgen05 + TMEM) for query tokens with up to 64 heads.
+//
+// "The Moment of Truth: Validating Split-K Parallelization for Blackwell MLA
+// Decode", section "The Split-K Imperative": tensor-core (MMA) attention over
+// the top-k candidate rows, split-K over that axis, partials merged by LSE.
+//
+// One CTA = one (query token, split), all heads (M = 64 rows of the MMA;
+// heads >= H are zero rows of Q and are never written out).  192 threads:
+//   warps 0-3  softmax warpgroup: stages Q (128B-swizzled) once, then per
+//              PAIR of 32-row tiles reads S from TMEM (tcgen05.ld), masks,
+//              keeps a running max per head with lazy rescaling (O is only
+//              rescaled when the max grows by more than 2^8), writes P as bf16
+//              into the tile's spent k_pe box, and finally drains O.
+//   warp 4     producer: resolves the split's indices to rows (as the mma
+//              kernel does) and gathers each 32-row tile with 72 TMA
+//              tile::gather4 copies (4 rows x 64 columns, 128B swizzle) into a
+//              4-stage ring; padding slots gather row 0 and are masked.
+//   warp 5     TMEM owner + MMA issuer (one thread):
+//                QK(t):  S[64 x 32] = Q[64 x 576] K_t^T        36 x (M64 N32 K16)
+//                PV(t):  O[64 x 512] += P_t[64 x 32] C_t[32 x 512]  2 x 2 x (M64 N256 K16)
+//              QK of pair p+1 is issued before PV of pair p so the softmax
+//              of one pair overlaps the scores of the next.
+// TMEM (512 columns; M = 64 accumulators occupy lanes 0-15 of each 32-lane
+// sub-partition, or 16-31 when addressed at lane offset 16):
+//   cols [0,256)   lane off 0: O[:, 0:256]     lane off 16: O[:, 256:512]
+//   cols 256+32b   lane off 0: S of the pair's first tile, 16: second tile
+//                  (b = pair parity, double buffered)
+// So thread (warp q, lane l) of the softmax warpgroup owns head 16q + l%16,
+// the first (l < 16) or second (l >= 16) tile of a pair, and one half of O.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "smla_partial_mma.cuh"
+#include "smla_tc_ptx.cuh"
+
+namespace smla {
+
+struct TcCfg {
+    static constexpr int kThreads = 192;
+    static constexpr int kTileRows = 32;
+    static constexpr int kStages = 4;
+    static constexpr int kBoxBytes = kTileRows * 128;       // 4096: 32 rows x 64 bf16
+    static constexpr int kStageBytes = 9 * kBoxBytes;       // 36864
+    static constexpr int kQBoxBytes = 64 * 128;             // 8192
+    static constexpr int kOffQ = 0;                         // 9 x 8192
+    static constexpr int kOffKV = 9 * kQBoxBytes;           // 73728
+    static constexpr int kOffRows = kOffKV + kStages * kStageBytes;  // 221184
+    static constexpr int kOffBar = kOffRows + kResolveChunk * 4;     // 229376
+    // barriers: kv_full[4], kv_empty[4], s_full[2], p_full[2], o_done, q_ready
+    static constexpr int kNumBars = 4 + 4 + 2 + 2 + 1 + 1;
+    static constexpr int kOffTmem = kOffBar + kNumBars * 8;
+    static constexpr int kOffHdr = kOffTmem + 16;           // u32 [4]
+    static constexpr int kBytes = kOffHdr + 16;
+    static constexpr int kSmemBytes = kBytes + 1024;        // + alignment slack for 1024-B atoms
+    static constexpr uint32_t kTmemCols = 512;
+    static constexpr uint32_t kSCol = 256;
+    static constexpr float kTau = 8.0f;                     // lazy-rescale threshold (log2 units)
+};
+static_assert(TcCfg::kSmemBytes <= 232448, "shared memory per CTA");
+
+template <bool DIRECT>
+__global__ void __launch_bounds__(TcCfg::kThreads, 1)
+    smla_partial_tc_kernel(const PartialParams p, const __grid_constant__ CUtensorMap tmap) {
+    using C = TcCfg;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    // 1024-byte aligned base (128B-swizzle atoms are 8 rows x 128 B).
+    uint8_t *smem = smem_raw + ((1024 - (smem_addr(smem_raw) & 1023)) & 1023);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int unit = blockIdx.x;  // (b * T + t) * S + s
+    const int s = unit % p.nsplit;
+    const int bt = unit / p.nsplit;
+    const int b = bt / p.T;
+    const long long j0l = (long long)s * p.kc;
+    const int j0 = (int)(j0l < p.K ? j0l : p.K);
+    const int j1 = (int)((long long)j0 + p.kc < p.K ? (long long)j0 + p.kc : p.K);
+    const int n_tiles = (j1 - j0 + C::kTileRows - 1) / C::kTileRows;
+    const int n_pairs = (n_tiles + 1) / 2;
+    bool dead = false;
+
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::kOffBar);
+    uint64_t *kv_full = bars;
+    uint64_t *kv_empty = bars + 4;
+    uint64_t *s_full = bars + 8;
+    uint64_t *p_full = bars + 10;
+    uint64_t *o_done = bars + 12;
+    uint64_t *q_ready = bars + 13;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::kOffTmem);
+    volatile uint32_t *hdr = reinterpret_cast<volatile uint32_t *>(smem + C::kOffHdr);
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < 4; ++i) {
+            mbar_init(&kv_full[i], 1);
+            mbar_init(&kv_empty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&s_full[i], 1);
+            mbar_init(&p_full[i], 4);
+        }
+        mbar_init(o_done, 1);
+        mbar_init(q_ready, 4);
+        fence_mbar_init();
+    }
+    if (warp == 5) {
+        tmem_alloc(tmem_slot, C::kTmemCols);
+        tmem_relinquish();
+    }
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(tmem_slot);
+    const uint32_t sbase = smem_addr(smem);
+
+    if (warp == 4) {
+        // ============================================================ producer
+        const int *idx_bt = p.idx + (size_t)bt * p.K + j0;
+        const int *pt_b = p.page_table + (size_t)b * p.pt_stride;
+        const long long max_pos = (long long)p.pt_stride * kPage;
+        // Padding slots gather cache row 0 (always in range) and are masked to
+        // probability 0 by the softmax, so they add 0 * row 0 to O.
+        constexpr int kPadRow = 0;
+        const uint64_t policy = l2_policy_evict_first();
+        int *rows_s = reinterpret_cast<int *>(smem + C::kOffRows);
+        const int len = j1 - j0;
+        int it = 0;
+        for (int base = 0; base < len; base += kResolveChunk) {
+            const int n = min(kResolveChunk, len - base);
+            for (int b0 = 0; b0 < n; b0 += 32 * 16) {
+                int iv[16];
+#pragma unroll
+                for (int k = 0; k < 16; ++k) {
+                    const int j = b0 + k * 32 + lane;
+                    iv[k] = (j < n) ? __ldg(idx_bt + base + j) : -1;
+                }
+                int pg[16];
+#pragma unroll
+                for (int k = 0; k < 16; ++k) {
+                    const int i = iv[k];
+                    pg[k] = (i >= 0 && (long long)i < max_pos) ? __ldg(pt_b + (i >> 6)) : -1;
+                }
+#pragma unroll
+                for (int k = 0; k < 16; ++k) {
+                    const int j = b0 + k * 32 + lane;
+                    const int i = iv[k];
+                    int row = -1;
+                    if (i != -1) {
+                        const bool ok = (i >= 0) && ((long long)i < max_pos) && (pg[k] >= 0) &&
+                                        ((long long)pg[k] < p.num_pages);
+                        if (ok) {
+                            row = pg[k] * kPage + (i & (kPage - 1));
+                        } else if (j < n) {
+                            atomicOr(&g_status_flags, kFlagIndexRange);
+                            atomicAdd(&g_bad_index_count, 1ull);
+                        }
+                    }
+                    if (j < n) rows_s[j] = row;
+                }
+            }
+            __syncwarp();
+            const int chunk_tiles = (n + C::kTileRows - 1) / C::kTileRows;
+            for (int t = 0; t < chunk_tiles; ++t, ++it) {
+                const int stage = it % C::kStages;
+                if (it >= C::kStages) mbar_wait(&kv_empty[stage], ((it / C::kStages) - 1) & 1, dead);
+                if (lane == 0) mbar_expect_tx(&kv_full[stage], (uint32_t)C::kStageBytes);
+                __syncwarp();
+                const int r = t * C::kTileRows + lane;
+                const int my_row = (r < n) ? rows_s[r] : -1;
+                const uint32_t vmask = __ballot_sync(0xffffffffu, my_row >= 0);
+                uint8_t *dst = smem + C::kOffKV + stage * C::kStageBytes;
+                // 8 groups of 4 rows x 9 column boxes = 72 gathers, spread over the
+                // warp; the trip count is uniform so every shuffle has all 32 lanes.
+#pragma unroll
+                for (int i0 = 0; i0 < 96; i0 += 32) {
+                    const int i = i0 + lane;
+                    const int grp = (i / 9) & 7, box = i % 9;
+                    int rr[4];
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const int v = __shfl_sync(0xffffffffu, my_row, 4 * grp + k);
+                        rr[k] = v >= 0 ? v : kPadRow;
+                    }
+                    if (i < 72)
+                        tma_gather4(dst + box * C::kBoxBytes + grp * 512, &tmap, box * 64, rr[0],
+                                    rr[1], rr[2], rr[3], &kv_full[stage], policy);
+                }
+                if (lane == 0) {
+                    hdr[stage] = vmask;
+                    mbar_arrive(&kv_full[stage]);  // release: hdr is visible to the waiters
+                }
+            }
+            __syncwarp();
+        }
+        // Copies still in flight must land before the CTA may exit.
+        for (int t2 = (n_tiles > C::kStages ? n_tiles - C::kStages : 0); t2 < n_tiles; ++t2)
+            mbar_wait(&kv_full[t2 % C::kStages], (t2 / C::kStages) & 1, dead);
+    } else if (warp == 5) {
+        // ============================================================ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t kIdescQK = idesc_bf16_f32(64, 32, false, false);
+            constexpr uint32_t kIdescPV = idesc_bf16_f32(64, 256, false, true);
+            const uint32_t q_addr = sbase + C::kOffQ;
+            mbar_wait(q_ready, 0, dead);
+            tc_fence_after();
+            for (int pr = 0; pr <= n_pairs; ++pr) {
+                if (pr < n_pairs) {
+                    const uint32_t s_col = C::kSCol + 32 * (pr & 1);
+                    for (int t = 2 * pr; t < 2 * pr + 2 && t < n_tiles; ++t) {
+                        const int stage = t % C::kStages;
+                        mbar_wait(&kv_full[stage], (t / C::kStages) & 1, dead);
+                        tc_fence_after();
+                        const uint32_t kv_addr = sbase + C::kOffKV + stage * C::kStageBytes;
+                        const uint32_t d = tmem + ((uint32_t)(16 * (t & 1)) << 16) + s_col;
+#pragma unroll 4
+                        for (int kk = 0; kk < 36; ++kk) {
+                            const uint32_t koff = (kk & 3) * 32;  // 16-element step inside the 128-B row
+                            const uint64_t a = smem_desc(q_addr + (kk >> 2) * C::kQBoxBytes + koff, 16,
+                                                         1024, kSwizzle128B);
+                            const uint64_t bd = smem_desc(kv_addr + (kk >> 2) * C::kBoxBytes + koff,
+                                                          16, 1024, kSwizzle128B);
+                            umma_bf16(d, a, bd, kIdescQK, kk > 0 ? 1u : 0u);
+                        }
+                    }
+                    umma_commit(&s_full[pr & 1]);
+                }
+                if (pr >= 1) {
+                    const int pp = pr - 1;
+                    mbar_wait(&p_full[pp & 1], (pp >> 1) & 1, dead);
+                    tc_fence_after();
+                    for (int t = 2 * pp; t < 2 * pp + 2 && t < n_tiles; ++t) {
+                        const int stage = t % C::kStages;
+                        const uint32_t kv_addr = sbase + C::kOffKV + stage * C::kStageBytes;
+                        const uint32_t p_addr = kv_addr + 8 * C::kBoxBytes;
+#pragma unroll
+                        for (int kk = 0; kk < 2; ++kk) {
+                            const uint32_t acc = (t > 0 || kk > 0) ? 1u : 0u;
+                            const uint64_t a = smem_desc(p_addr + kk * 32, 16, 512, kSwizzle64B);
+                            const uint64_t blo = smem_desc(kv_addr + kk * 2048, C::kBoxBytes, 1024,
+                                                           kSwizzle128B);
+                            const uint64_t bhi = smem_desc(kv_addr + 4 * C::kBoxBytes + kk * 2048,
+                                                           C::kBoxBytes, 1024, kSwizzle128B);
+                            umma_bf16(tmem, a, blo, kIdescPV, acc);
+                            umma_bf16(tmem + (16u << 16), a, bhi, kIdescPV, acc);
+                        }
+                        umma_commit(&kv_empty[stage]);
+                    }
+                    umma_commit(o_done);
+                }
+            }
+        }
+        __syncwarp();
+    } else {
+        // ============================================================ softmax warpgroup
+        const int tid = threadIdx.x;  // 0..127
+        const int q4 = warp;          // TMEM sub-partition (lanes 32*q4 .. +31)
+        const int hrow = 16 * q4 + (lane & 15);
+        const int half = lane >> 4;
+
+        // ---- stage Q (heads x 576, zero rows beyond H) as 9 swizzled 64-column boxes
+        {
+            const uint4 *qsrc = reinterpret_cast<const uint4 *>(p.q + (size_t)bt * p.H * kD);
+            for (int c0 = 0; c0 < 64 * 72; c0 += 128 * 12) {
+                uint4 v[12];
+#pragma unroll
+                for (int k = 0; k < 12; ++k) {
+                    const int c = c0 + k * 128 + tid;
+                    const int h = c / 72;
+                    v[k] = (c < 64 * 72 && h < p.H) ? __ldg(qsrc + (size_t)h * 72 + (c % 72))
+                                                     : make_uint4(0u, 0u, 0u, 0u);
+                }
+#pragma unroll
+                for (int k = 0; k < 12; ++k) {
+                    const int c = c0 + k * 128 + tid;
+                    if (c < 64 * 72) {
+                        const int h = c / 72, k16 = c % 72;
+                        const int box = k16 >> 3, ch = k16 & 7;
+                        *reinterpret_cast<uint4 *>(smem + C::kOffQ + box * C::kQBoxBytes + h * 128 +
+                                                   ((ch ^ (h & 7)) << 4)) = v[k];
+                    }
+                }
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(q_ready);
+        }
+
+        float m_ref = -INFINITY;  // running reference max of head hrow (log2 units)
+        float l_acc = 0.f;        // sum of P over this thread's tiles, relative to m_ref
+        const uint32_t t_lane = tmem + ((uint32_t)(32 * q4) << 16);
+
+        for (int pr = 0; pr < n_pairs; ++pr) {
+            const int t = 2 * pr + half;
+            const bool exists = t < n_tiles;
+            mbar_wait(&s_full[pr & 1], (pr >> 1) & 1, dead);
+            if (pr >= 1) mbar_wait(o_done, (pr - 1) & 1, dead);
+            tc_fence_after();
+            uint32_t sr[32];
+            tmem_ld32(t_lane + C::kSCol + 32 * (pr & 1), sr);
+            tmem_ld_wait();
+            uint32_t vmask = 0;
+            if (exists) {
+                mbar_wait(&kv_full[t % C::kStages], (t / C::kStages) & 1, dead);
+                vmask = hdr[t % C::kStages];
+            }
+            float sv[32];
+            float mt = -INFINITY;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                sv[j] = ((vmask >> j) & 1u) ? __uint_as_float(sr[j]) * p.scale_log2 : -INFINITY;
+                mt = fmaxf(mt, sv[j]);
+            }
+            mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 16));
+            float alpha = 1.f;
+            if (mt > m_ref + C::kTau) {
+                alpha = (m_ref == -INFINITY) ? 0.f : exp2f(m_ref - mt);
+                m_ref = mt;
+            }
+            // Rescale this thread's half row of O when its head's max jumped
+            // (warp-collective TMEM access; alpha = 1 for the other threads).
+            const bool need = (pr >= 1) && (alpha != 1.f);
+            if (__any_sync(0xffffffffu, need)) {
+#pragma unroll 1
+                for (int c = 0; c < 256; c += 32) {
+                    uint32_t orr[32];
+                    tmem_ld32(t_lane + c, orr);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) orr[j] = __float_as_uint(__uint_as_float(orr[j]) * alpha);
+                    tmem_st32(t_lane + c, orr);
+                }
+                tmem_st_wait();
+            }
+            const float mu = (m_ref == -INFINITY) ? 0.f : m_ref;
+            float ps = 0.f;
+            uint32_t pk[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const float a0 = exp2f(sv[2 * j] - mu), a1 = exp2f(sv[2 * j + 1] - mu);
+                ps += a0 + a1;
+                pk[j] = pack_bf16x2(a0, a1);
+            }
+            l_acc = l_acc * alpha + ps;
+            if (exists) {
+                // P tile (64 heads x 32 rows, bf16) in the spent k_pe box, K-major 64B swizzle
+                uint8_t *pbase = smem + C::kOffKV + (t % C::kStages) * C::kStageBytes + 8 * C::kBoxBytes;
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+                    *reinterpret_cast<uint4 *>(pbase + hrow * 64 + ((c ^ ((hrow >> 1) & 3)) << 4)) =
+                        make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&p_full[pr & 1]);
+        }
+
+        // ---- epilogue: O (unnormalised) and m, lse of head hrow
+        const float l_tot = l_acc + __shfl_xor_sync(0xffffffffu, l_acc, 16);
+        if (n_pairs > 0) {
+            mbar_wait(o_done, (n_pairs - 1) & 1, dead);
+            tc_fence_after();
+        }
+        const bool write = hrow < p.H;
+        const size_t row = (size_t)bt * p.H + hrow;
+#pragma unroll 1
+        for (int c = 0; c < 256; c += 32) {
+            uint32_t orr[32];
+            if (n_pairs > 0) {
+                tmem_ld32(t_lane + c, orr);
+                tmem_ld_wait();
+            } else {
+#pragma unroll
+                for (int j = 0; j < 32; ++j) orr[j] = 0u;
+            }
+            if (!write) continue;
+            const int col = 256 * half + c;
+            if (!DIRECT) {
+                float4 *dst = reinterpret_cast<float4 *>(p.part_o + (row * p.nsplit + s) * kDc + col);
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                    dst[j] = make_float4(__uint_as_float(orr[4 * j]), __uint_as_float(orr[4 * j + 1]),
+                                         __uint_as_float(orr[4 * j + 2]), __uint_as_float(orr[4 * j + 3]));
+            } else {
+                const float inv = (l_tot > 0.f) ? 1.f / l_tot : 0.f;
+                uint4 *dst = reinterpret_cast<uint4 *>(p.o + row * kDc + col);
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    dst[j] = make_uint4(
+                        pack_bf16x2(__uint_as_float(orr[8 * j]) * inv, __uint_as_float(orr[8 * j + 1]) * inv),
+                        pack_bf16x2(__uint_as_float(orr[8 * j + 2]) * inv, __uint_as_float(orr[8 * j + 3]) * inv),
+                        pack_bf16x2(__uint_as_float(orr[8 * j + 4]) * inv, __uint_as_float(orr[8 * j + 5]) * inv),
+                        pack_bf16x2(__uint_as_float(orr[8 * j + 6]) * inv, __uint_as_float(orr[8 * j + 7]) * inv));
+            }
+        }
+        if (write && half == 0) {
+            const float lse_v = (l_tot > 0.f) ? (m_ref + log2f(l_tot)) * kLn2 : -INFINITY;
+            if (!DIRECT) {
+                const size_t k = row * p.nsplit + s;
+                p.part_m[k] = (l_tot > 0.f) ? m_ref * kLn2 : -INFINITY;
+                p.part_lse[k] = lse_v;
+            } else {
+                p.lse[row] = lse_v;
+            }
+        }
+        tc_fence_before();
+    }
+
+    __syncthreads();
+    if (warp == 5) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::kTmemCols);
+    }
+}
+
+}  // namespace smla

@@ -131,17 +131,17 @@ def test_partial_pass_against_oracle_partials(H):
     assert np.abs(plg[fin] - rpl[fin]).max() <= 1e-3
 
 
-def test_combine_pass_against_oracle_combine():
+@pytest.mark.parametrize("nsplit", [2, 5, 8, 16, 70])
+def test_combine_pass_against_oracle_combine(nsplit):
     w = small(H=16, K=256, B=2, T=1)
     w.idx[1, 0, 100:] = -1
-    nsplit = 8
     rpo, rpm, rpl, _ = oracle.partial(bits(w.q), bits(w.cache), w.page_table.numpy(),
                                       w.idx.numpy(), w.scale, nsplit)
     o_ref, lse_ref = oracle.combine(rpo, rpm, rpl)
     t = lambda a: torch.tensor(a, dtype=torch.float32, device=DEV).contiguous()
     o, lse = binding.lse_combine(t(rpo), t(rpm), t(rpl))
     torch.cuda.synchronize()
-    check_o_lse(o, lse, o_ref, lse_ref, "combine")
+    check_o_lse(o, lse, o_ref, lse_ref, f"combine S={nsplit}")
 
 
 # ------------------------------------------------------------------ edge cases

@@ -110,13 +110,14 @@ def test_combine_rejects_bad_arguments(lib):
 def model(B, T, H, K, sms):
     """The cost model the library documents, restated for a table check."""
     base = B * T
+    slots = sms * (2 if H <= 16 else 1)
     s_max = max(1, min(1024, -(-K // 32)))
     best, best_s = None, 1
     for s in range(1, s_max + 1):
         ctas = base * s
-        t = math.ceil(ctas / sms) * (48.0 + math.ceil(K / s))
+        t = math.ceil(ctas / slots) * (48.0 + math.ceil(K / s))
         if s > 1:
-            t += 0.5 * ctas * H * (514 * 4.0) * 2.0 / 1152 / sms
+            t += 0.5 * ctas * H * (514 * 4.0) * 2.0 / 1152 / slots
         if best is None or t < best * (1 - 1e-9):
             best, best_s = t, s
     return best_s
@@ -140,7 +141,8 @@ def test_nsplit_heuristic_properties(lib, monkeypatch):
         s = binding.choose_nsplit(1, 1, 16, K, 148)
         assert s == 1 or math.ceil(K / s) >= 32 or s <= -(-K // 32)
     # a batch that already fills the GPU is not split
-    assert binding.choose_nsplit(148, 1, 16, 2048, 148) == 1
+    assert binding.choose_nsplit(296, 1, 16, 2048, 148) == 1
+    assert binding.choose_nsplit(148, 1, 64, 2048, 148) == 1
     # degenerate sizes
     assert binding.choose_nsplit(0, 1, 16, 2048, 148) == 1
     assert binding.choose_nsplit(1, 1, 16, 0, 148) == 1
