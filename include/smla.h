@@ -168,6 +168,42 @@ smla_status smla_decode(const void *q, const void *kv_cache, int64_t num_pages,
  */
 smla_status smla_check_device(int clear, unsigned long long *n_bad_index, void *stream);
 
+/*
+ * Whole decode with no caller-provided workspace and no allocation.
+ *
+ * The pages have no counterpart to this entry point; it exists for callers
+ * that cannot allocate device memory at the moment they decode: code running
+ * inside a region that must not call cudaMalloc (an allocator that is itself
+ * being serviced, a memory pool that is locked or exhausted, a host process
+ * that only ever receives device pointers from someone else), or plain C
+ * callers with no allocator of their own.  It behaves like smla_decode with
+ * the same arguments minus the workspace: the split-K partials live instead in
+ * one scratch array of SMLA_NOALLOC_SCRATCH_BYTES that the library itself
+ * holds in device memory on every GPU that loads it, until the process exits.
+ *
+ *  - q, kv_cache, page_table, topk_idx, o, lse: as for smla_decode (device,
+ *    caller-owned).  nsplit = 0 picks the heuristic's value.
+ *  - If smla_workspace_bytes(B, T, H, S) for the split count actually used is
+ *    larger than SMLA_NOALLOC_SCRATCH_BYTES, the call launches nothing and
+ *    returns SMLA_ERR_WORKSPACE_TOO_SMALL (smla_last_error() says how many
+ *    bytes were needed); pass a smaller nsplit or use smla_decode.
+ *  - The first call on each device looks up that device's copy of the scratch
+ *    array (cudaGetSymbolAddress, with the device current); make that first
+ *    call before starting any stream capture.  It allocates nothing and calls
+ *    no allocating CUDA or library routine, then or later.
+ *  - All calls on a device share the one array and it keeps whatever the last
+ *    call left in it; nothing in it has to start at zero, because every split
+ *    the combine reads is written first by the same call.  Calls whose work
+ *    overlaps on the GPU (different streams, or host threads racing on one
+ *    device) race on the array and produce wrong results: serialise them.
+ */
+#define SMLA_NOALLOC_SCRATCH_BYTES (16u << 20)
+smla_status smla_decode_noalloc(const void *q, const void *kv_cache, int64_t num_pages,
+                                const int32_t *page_table, int pt_stride,
+                                const int32_t *topk_idx, int B, int T, int H, int K,
+                                int page_size, float scale, int nsplit, void *o, float *lse,
+                                void *stream);
+
 /* Static text for a status code. */
 const char *smla_status_string(smla_status status);
 

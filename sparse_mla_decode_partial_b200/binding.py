@@ -17,6 +17,7 @@ LIB_PATH = os.path.join(_PKG, "libsmla.so")
 
 DC, DR, D, PAGE_SIZE = 512, 64, 576, 64
 MAX_HEADS, MAX_NSPLIT = 64, 1024
+NOALLOC_SCRATCH_BYTES = 16 << 20
 
 STATUS = {
     0: "SMLA_OK", 1: "SMLA_ERR_INVALID_ARG", 2: "SMLA_ERR_UNSUPPORTED", 3: "SMLA_ERR_MISALIGNED",
@@ -34,6 +35,8 @@ SIGNATURES = {
     "smla_lse_combine": (_I, [_P, _P, _P, _I, _I, _I, _I, _P, _P, _P]),
     "smla_decode": (_I, [_P, _P, _I64, _P, _I, _P, _I, _I, _I, _I, _I, _F, _I, _P, _SZ, _P, _P,
                          _P]),
+    "smla_decode_noalloc": (_I, [_P, _P, _I64, _P, _I, _P, _I, _I, _I, _I, _I, _F, _I, _P, _P,
+                                 _P]),
     "smla_check_device": (_I, [_I, ctypes.POINTER(ctypes.c_ulonglong), _P]),
     "smla_status_string": (ctypes.c_char_p, [_I]),
     "smla_last_error": (ctypes.c_char_p, []),
@@ -189,6 +192,23 @@ def decode(q, cache, page_table, idx, scale: float, nsplit: int = 0, *, workspac
                              _ptr(idx), B, T, H, K, PAGE_SIZE, float(scale), int(nsplit),
                              _ptr(workspace), workspace.numel(), _ptr(o), _ptr(lse),
                              _stream(stream)), "smla_decode")
+    return o, lse
+
+
+def decode_noalloc(q, cache, page_table, idx, scale: float, nsplit: int = 0, *, o, lse,
+                   stream=None):
+    """Whole decode through smla_decode_noalloc: no workspace argument and no
+    allocation anywhere (the split-K partials use the library's own device
+    scratch array).  For callers that cannot allocate device memory while they
+    decode, so o and lse must be given.  Calls that overlap on the GPU race on
+    the shared scratch."""
+    B, T, H, K, pt_stride, num_pages = _decode_args(q, cache, page_table, idx)
+    _need(o, torch.bfloat16, "o", q.device)
+    _need(lse, torch.float32, "lse", q.device)
+    _check(lib().smla_decode_noalloc(_ptr(q), _ptr(cache), num_pages, _ptr(page_table),
+                                     pt_stride, _ptr(idx), B, T, H, K, PAGE_SIZE, float(scale),
+                                     int(nsplit), _ptr(o), _ptr(lse), _stream(stream)),
+           "smla_decode_noalloc")
     return o, lse
 
 

@@ -362,6 +362,64 @@ smla_status smla_decode(const void *q, const void *kv_cache, int64_t num_pages,
     return launch_combine(p.part_o, p.part_m, p.part_lse, B, T, H, nsplit, o, lse, s);
 }
 
+// ---------------------------------------------------------------------------
+// Allocation-free decode.  The split-K partials go to a scratch array that the
+// library owns in device memory (one copy per device that loads this module).
+// In host code `g_noalloc_scratch` names a host-side stand-in, not a device
+// address, so each device's real address is looked up once with
+// cudaGetSymbolAddress while that device is current, and only that address is
+// handed to the kernels.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[SMLA_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void *g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of this device's scratch array (set up on first use).
+smla_status noalloc_scratch(void **out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (dev < 0 || dev >= kMaxDevices) return SMLA_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (g_noalloc_ptr[dev] == nullptr) {
+        void *ptr = nullptr;
+        e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+        if (e != cudaSuccess) return cuda_fail(e);
+        g_noalloc_ptr[dev] = ptr;
+    }
+    *out = g_noalloc_ptr[dev];
+    return SMLA_OK;
+}
+}  // namespace
+
+smla_status smla_decode_noalloc(const void *q, const void *kv_cache, int64_t num_pages,
+                                const int32_t *page_table, int pt_stride, const int32_t *topk_idx,
+                                int B, int T, int H, int K, int page_size, float scale, int nsplit,
+                                void *o, float *lse, void *stream) {
+    smla_status st = check_decode_args(q, kv_cache, num_pages, page_table, pt_stride, topk_idx, B,
+                                       T, H, K, page_size, scale);
+    if (st != SMLA_OK) return st;
+    if (nsplit < 0 || nsplit > SMLA_MAX_NSPLIT) return SMLA_ERR_INVALID_ARG;
+    if (B == 0 || T == 0 || H == 0) return SMLA_OK;
+    if (nsplit == 0) nsplit = smla_choose_nsplit(B, T, H, K, 0);
+    const size_t need = nsplit > 1 ? smla_workspace_bytes(B, T, H, nsplit) : 0;
+    if (need > SMLA_NOALLOC_SCRATCH_BYTES) {
+        std::snprintf(g_last_error, sizeof g_last_error,
+                      "smla_decode_noalloc: %zu bytes of split-K scratch needed for nsplit=%d, "
+                      "the built-in scratch holds %u",
+                      need, nsplit, (unsigned)SMLA_NOALLOC_SCRATCH_BYTES);
+        return SMLA_ERR_WORKSPACE_TOO_SMALL;
+    }
+    void *scratch = nullptr;
+    st = noalloc_scratch(&scratch);
+    if (st != SMLA_OK) return st;
+    return smla_decode(q, kv_cache, num_pages, page_table, pt_stride, topk_idx, B, T, H, K,
+                       page_size, scale, nsplit, scratch, SMLA_NOALLOC_SCRATCH_BYTES, o, lse,
+                       stream);
+}
+
 smla_status smla_check_device(int clear, unsigned long long *n_bad_index, void *stream) {
     cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e);
