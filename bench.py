@@ -77,6 +77,24 @@ def describe(w):
             f"{w.num_pages} pages, ctx {min(w.ctx_lens)}..{max(w.ctx_lens)}")
 
 
+def measured_traffic(workload: str):
+    """DRAM bytes (read + write) per launch of the partial kernel for this
+    workload from the committed ncu capture, or None when no capture exists
+    or the kernel sources changed since it was taken."""
+    import glob
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "ncu_traffic.json")) as f:
+            rec = json.load(f)[workload]
+    except (OSError, KeyError, ValueError):
+        return None
+    h = hashlib.sha256()
+    for fn in sorted(glob.glob(os.path.join(ROOT, "sparse_mla_decode_partial_b200", "csrc", "*"))):
+        with open(fn, "rb") as f:
+            h.update(f.read())
+    return rec["traffic_bytes_per_launch"] if h.hexdigest()[:16] == rec["sources_sha256_16"] else None
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -160,6 +178,27 @@ def dist_init():
     return world, rank, local
 
 
+def replica_workload(name: str, rank: int, world: int):
+    """The workload one rank runs: rank r of an N-rank job draws an independent
+    replica of the named workload (seed offset 1000 * r), so every GPU has the
+    same amount of work (weak scaling) and no data crosses ranks."""
+    import inspect
+    from sparse_mla_decode_partial_b200 import workloads
+    builder = workloads.WORKLOADS[name]
+    if world == 1:
+        return builder()
+    base_seed = inspect.signature(builder).parameters["seed"].default
+    return builder(seed=base_seed + 1000 * rank)
+
+
+def aggregate(tokens_local: float, ms_local: float, world: int):
+    """Whole-job throughput: query tokens of all ranks / the slowest rank's
+    step time.  Returns (tokens_all, ms_max, tokens per second)."""
+    ms_max = max_over_ranks(ms_local, world)
+    tokens_all = sum_over_ranks(tokens_local, world)
+    return tokens_all, ms_max, tokens_all / (ms_max * 1e-3)
+
+
 def barrier(world):
     if world > 1:
         import torch.distributed as dist
@@ -231,13 +270,7 @@ def run_ours(args, world, rank, local):
     lib = binding.lib()
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    builder = workloads.WORKLOADS[args.workload]
-    seed_kw = {}
-    if world > 1:
-        import inspect
-        base_seed = inspect.signature(builder).parameters["seed"].default
-        seed_kw = {"seed": base_seed + 1000 * rank}
-    w_host = builder(**seed_kw)
+    w_host = replica_workload(args.workload, rank, world)
     w = w_host.to(dev)
     B, T, H, K = w.B, w.T, w.H, w.K
     nsplit = args.nsplit or binding.choose_nsplit(B, T, H, K, 0)
@@ -315,9 +348,7 @@ def run_ours(args, world, rank, local):
 
     ms_step = statistics.fmean(tot)
     ms_part = statistics.fmean(part)
-    ms_step_max = max_over_ranks(ms_step, world)
-    tokens_all = sum_over_ranks(float(B * T), world)
-    value = tokens_all / (ms_step_max * 1e-3)
+    tokens_all, ms_step_max, value = aggregate(float(B * T), ms_step, world)
 
     # e2e: host buffers through the C ABI, copies inside the timed region
     e2e = None
@@ -407,10 +438,14 @@ def run_ours(args, world, rank, local):
         "kernel_us": {"partial": round(part_us, 3),
                       "note": "partial pass timed alone in a second loop of the same length; "
                               "the step runs it and the combine through one smla_decode call"},
-        "roofline": {"bound": "hbm", "kernel": "smla_partial_mma_kernel", "achieved": round(achieved, 1),
+        "roofline": {"bound": "hbm",
+                     "kernel": "smla_partial_tc_kernel" if H > 32 else "smla_partial_mma_kernel", "achieved": round(achieved, 1),
                      "peak": hbm_peak, "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),
                      "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured" else "fallback",
-                     "traffic": None, "algorithmic_bytes_per_launch": part_bytes,
+                     "traffic": measured_traffic(args.workload),
+                     "traffic_source": "profiles/ncu_traffic.json (ncu dram__bytes_read.sum + "
+                                       "dram__bytes_write.sum of one capture of this kernel)",
+                     "algorithmic_bytes_per_launch": part_bytes,
                      "tensor_tflops": round(tc_achieved, 2),
                      "tensor_frac_of_bf16_peak": round(tc_achieved / tc_peak, 4)},
         "gpu_launches": launches,
@@ -450,15 +485,21 @@ def run_reference(args, world, rank):
 
 def main(argv=None):
     args = parse_args(argv)
-    world, rank, local = dist_init()
     if args.impl == "reference":
-        line = run_reference(args, world, rank)
-    else:
-        line = run_ours(args, world, rank, local)
-        if rank == 0 and line is not None:
-            from sparse_mla_decode_partial_b200 import workloads
-            line["cpu_baseline"] = cpu_baseline(workloads.WORKLOADS[args.workload](),
-                                                args.cpu_seconds)
+        # The CPU oracle as the reference arm: rank 0 alone runs and prints;
+        # under torchrun the other ranks exit at once, with no process group.
+        rank = int(os.environ.get("RANK", "0"))
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        line = run_reference(args, world, rank) if rank == 0 else None
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return 0
+    world, rank, local = dist_init()
+    line = run_ours(args, world, rank, local)
+    if rank == 0 and line is not None:
+        from sparse_mla_decode_partial_b200 import workloads
+        line["cpu_baseline"] = cpu_baseline(workloads.WORKLOADS[args.workload](),
+                                            args.cpu_seconds)
     if world > 1:
         import torch.distributed as dist
         dist.barrier()

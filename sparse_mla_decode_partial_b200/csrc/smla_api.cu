@@ -16,6 +16,12 @@
 #include <utility>
 
 #include "smla.h"
+
+// Tile shape of the mma kernel for H <= 16 (two CTAs per SM either way).
+#ifndef SMLA_MMA_TILE_ROWS
+#define SMLA_MMA_TILE_ROWS 32
+#define SMLA_MMA_STAGES 2
+#endif
 #include "smla_combine.cuh"
 #include "smla_partial_mma.cuh"
 #include "smla_partial_tc.cuh"
@@ -190,7 +196,7 @@ smla_status launch_partial(const PartialParams &p, cudaStream_t st) {
     if (grid > INT_MAX) return SMLA_ERR_INVALID_ARG;
     if (p.H > 32) return launch_tc<DIRECT>(p, (int)grid, st);
     if (p.H > 16) return launch_mma<2, 32, 4, DIRECT>(p, (int)grid, st);
-    return launch_mma<1, 32, 2, DIRECT>(p, (int)grid, st);
+    return launch_mma<1, SMLA_MMA_TILE_ROWS, SMLA_MMA_STAGES, DIRECT>(p, (int)grid, st);
 }
 
 PartialParams make_params(const void *q, const void *kv_cache, int64_t num_pages,

@@ -71,7 +71,7 @@ struct PartialParams {
 
 template <int HG, int NT, int NSTAGE>
 struct MmaCfg {
-    static_assert(NT == 32 || NT == 64, "tile rows");
+    static_assert(NT == 16 || NT == 32 || NT == 64, "tile rows");
     static constexpr int kHeads = 16 * HG;
     static constexpr int kComputeWarps = 4 * HG;
     static constexpr int kThreads = (kComputeWarps + 1) * 32;
@@ -181,16 +181,19 @@ __global__ void __launch_bounds__(MmaCfg<HG, NT, NSTAGE>::kThreads, MmaCfg<HG, N
                 uint8_t *dst = smem + C::kOffKV + stage * C::kStageBytes;
                 uint64_t mask = 0;
 #pragma unroll
-                for (int k = 0; k < NT / 32; ++k) {
-                    const int r = t * NT + k * 32 + lane;
-                    const int row = (r < n) ? rows_s[r] : -1;
-                    uint8_t *d = dst + (k * 32 + lane) * kSmemRowBytes;
-                    if (row >= 0)
-                        bulk_g2s_hint(d, reinterpret_cast<const uint8_t *>(p.cache) +
-                                             (size_t)row * kRowBytes,
-                                      kRowBytes, &full[stage], policy);
-                    else
-                        bulk_g2s(d, g_zero_row, kRowBytes, &full[stage]);
+                for (int k = 0; k < (NT + 31) / 32; ++k) {
+                    const int slot = k * 32 + lane;
+                    const int r = t * NT + slot;
+                    const int row = (slot < NT && r < n) ? rows_s[r] : -1;
+                    uint8_t *d = dst + slot * kSmemRowBytes;
+                    if (slot < NT) {
+                        if (row >= 0)
+                            bulk_g2s_hint(d, reinterpret_cast<const uint8_t *>(p.cache) +
+                                                 (size_t)row * kRowBytes,
+                                          kRowBytes, &full[stage], policy);
+                        else
+                            bulk_g2s(d, g_zero_row, kRowBytes, &full[stage]);
+                    }
                     mask |= (uint64_t)__ballot_sync(0xffffffffu, row >= 0) << (32 * k);
                 }
                 if (lane == 0) {

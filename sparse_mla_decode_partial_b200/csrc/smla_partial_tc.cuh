@@ -6,21 +6,28 @@
 // the top-k candidate rows, split-K over that axis, partials merged by LSE.
 //
 // One CTA = one (query token, split), all heads (M = 64 rows of the MMA;
-// heads >= H are zero rows of Q and are never written out).  192 threads:
+// heads >= H are zero rows of Q and are never written out).  288 threads:
 //   warps 0-3  softmax warpgroup: stages Q (128B-swizzled) once, then per
 //              PAIR of 32-row tiles reads S from TMEM (tcgen05.ld), masks,
 //              keeps a running max per head with lazy rescaling (O is only
 //              rescaled when the max grows by more than 2^8), writes P as bf16
 //              into the tile's spent k_pe box, and finally drains O.
-//   warp 4     producer: resolves the split's indices to rows (as the mma
-//              kernel does) and gathers each 32-row tile with 72 TMA
-//              tile::gather4 copies (4 rows x 64 columns, 128B swizzle) into a
-//              4-stage ring; padding slots gather row 0 and are masked.
-//   warp 5     TMEM owner + MMA issuer (one thread):
+//   warps 4-7  producers: resolve the split's indices to rows (as the mma
+//              kernel does), then gather each 32-row tile with 16-byte
+//              cp.async copies written straight into the 128B-swizzled
+//              K-major layout (each warp instruction moves 4 rows x 128 B,
+//              coalesced); completion reaches the stage's mbarrier through
+//              cp.async.mbarrier.arrive.  Four warps keep enough copies in
+//              flight; the TMA engine would cap this at one 512-B gather4 or
+//              one 1152-B row per operation.  Padding slots copy row 0 and
+//              are masked.
+//   warp 8     TMEM owner + MMA issuer (one thread):
 //                QK(t):  S[64 x 32] = Q[64 x 576] K_t^T        36 x (M64 N32 K16)
 //                PV(t):  O[64 x 512] += P_t[64 x 32] C_t[32 x 512]  2 x 2 x (M64 N256 K16)
-//              QK of pair p+1 is issued before PV of pair p so the softmax
-//              of one pair overlaps the scores of the next.
+//              The issuer polls: a tile's QK goes out as soon as the tile
+//              has landed, a pair's PV as soon as its P is ready, so the
+//              softmax of one pair overlaps the scores of the next and a
+//              finished pair frees its stages without waiting for new loads.
 // TMEM (512 columns; M = 64 accumulators occupy lanes 0-15 of each 32-lane
 // sub-partition, or 16-31 when addressed at lane offset 16):
 //   cols [0,256)   lane off 0: O[:, 0:256]     lane off 16: O[:, 256:512]
@@ -40,7 +47,12 @@
 namespace smla {
 
 struct TcCfg {
-    static constexpr int kThreads = 192;
+#ifndef SMLA_TC_PRODUCER_WARPS
+#define SMLA_TC_PRODUCER_WARPS 4
+#endif
+    static constexpr int kProducerWarps = SMLA_TC_PRODUCER_WARPS;
+    static constexpr int kMmaWarp = 4 + kProducerWarps;
+    static constexpr int kThreads = 32 * (kMmaWarp + 1);
     static constexpr int kTileRows = 32;
     static constexpr int kStages = 4;
     static constexpr int kBoxBytes = kTileRows * 128;       // 4096: 32 rows x 64 bf16
@@ -50,8 +62,8 @@ struct TcCfg {
     static constexpr int kOffKV = 9 * kQBoxBytes;           // 73728
     static constexpr int kOffRows = kOffKV + kStages * kStageBytes;  // 221184
     static constexpr int kOffBar = kOffRows + kResolveChunk * 4;     // 229376
-    // barriers: kv_full[4], kv_empty[4], s_full[2], p_full[2], o_done, q_ready
-    static constexpr int kNumBars = 4 + 4 + 2 + 2 + 1 + 1;
+    // barriers: kv_full[4], kv_empty[4], s_full[2], p_full[2], o_done[2], q_ready
+    static constexpr int kNumBars = 4 + 4 + 2 + 2 + 2 + 1;
     static constexpr int kOffTmem = kOffBar + kNumBars * 8;
     static constexpr int kOffHdr = kOffTmem + 16;           // u32 [4]
     static constexpr int kBytes = kOffHdr + 16;
@@ -88,25 +100,28 @@ __global__ void __launch_bounds__(TcCfg::kThreads, 1)
     uint64_t *kv_empty = bars + 4;
     uint64_t *s_full = bars + 8;
     uint64_t *p_full = bars + 10;
-    uint64_t *o_done = bars + 12;
-    uint64_t *q_ready = bars + 13;
+    uint64_t *o_done = bars + 12;  // [pair parity]: PV of that pair complete
+    uint64_t *q_ready = bars + 14;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::kOffTmem);
     volatile uint32_t *hdr = reinterpret_cast<volatile uint32_t *>(smem + C::kOffHdr);
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < 4; ++i) {
-            mbar_init(&kv_full[i], 1);
+            // 32 cp.async arrivals per producer warp + one plain arrive that
+            // publishes the tile's validity mask
+            mbar_init(&kv_full[i], 32 * C::kProducerWarps + 1);
             mbar_init(&kv_empty[i], 1);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&s_full[i], 1);
             mbar_init(&p_full[i], 4);
         }
-        mbar_init(o_done, 1);
+        mbar_init(&o_done[0], 1);
+        mbar_init(&o_done[1], 1);
         mbar_init(q_ready, 4);
         fence_mbar_init();
     }
-    if (warp == 5) {
+    if (warp == C::kMmaWarp) {
         tmem_alloc(tmem_slot, C::kTmemCols);
         tmem_relinquish();
     }
@@ -117,25 +132,30 @@ __global__ void __launch_bounds__(TcCfg::kThreads, 1)
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(tmem_slot);
     const uint32_t sbase = smem_addr(smem);
 
-    if (warp == 4) {
-        // ============================================================ producer
+    if (warp >= 4 && warp < 4 + C::kProducerWarps) {
+        // ============================================================ producers
+        const int pw = warp - 4;
+        const int ptid = threadIdx.x - 128;  // 0 .. 32 * kProducerWarps - 1
+        constexpr int kPT = 32 * C::kProducerWarps;
         const int *idx_bt = p.idx + (size_t)bt * p.K + j0;
         const int *pt_b = p.page_table + (size_t)b * p.pt_stride;
         const long long max_pos = (long long)p.pt_stride * kPage;
-        // Padding slots gather cache row 0 (always in range) and are masked to
+        // Padding slots copy cache row 0 (always in range) and are masked to
         // probability 0 by the softmax, so they add 0 * row 0 to O.
         constexpr int kPadRow = 0;
-        const uint64_t policy = l2_policy_evict_first();
         int *rows_s = reinterpret_cast<int *>(smem + C::kOffRows);
+        const uint8_t *cache = reinterpret_cast<const uint8_t *>(p.cache);
+        const uint32_t bar_prod = 1;  // named barrier of the 4 producer warps
         const int len = j1 - j0;
         int it = 0;
         for (int base = 0; base < len; base += kResolveChunk) {
             const int n = min(kResolveChunk, len - base);
-            for (int b0 = 0; b0 < n; b0 += 32 * 16) {
+            named_bar_sync(bar_prod, 32 * C::kProducerWarps);  // rows_s free for rewriting
+            for (int b0 = 0; b0 < n; b0 += kPT * 16) {
                 int iv[16];
 #pragma unroll
                 for (int k = 0; k < 16; ++k) {
-                    const int j = b0 + k * 32 + lane;
+                    const int j = b0 + k * kPT + ptid;
                     iv[k] = (j < n) ? __ldg(idx_bt + base + j) : -1;
                 }
                 int pg[16];
@@ -146,7 +166,7 @@ __global__ void __launch_bounds__(TcCfg::kThreads, 1)
                 }
 #pragma unroll
                 for (int k = 0; k < 16; ++k) {
-                    const int j = b0 + k * 32 + lane;
+                    const int j = b0 + k * kPT + ptid;
                     const int i = iv[k];
                     int row = -1;
                     if (i != -1) {
@@ -162,44 +182,40 @@ __global__ void __launch_bounds__(TcCfg::kThreads, 1)
                     if (j < n) rows_s[j] = row;
                 }
             }
-            __syncwarp();
+            named_bar_sync(bar_prod, 32 * C::kProducerWarps);  // rows_s complete
             const int chunk_tiles = (n + C::kTileRows - 1) / C::kTileRows;
             for (int t = 0; t < chunk_tiles; ++t, ++it) {
                 const int stage = it % C::kStages;
                 if (it >= C::kStages) mbar_wait(&kv_empty[stage], ((it / C::kStages) - 1) & 1, dead);
-                if (lane == 0) mbar_expect_tx(&kv_full[stage], (uint32_t)C::kStageBytes);
-                __syncwarp();
-                const int r = t * C::kTileRows + lane;
-                const int my_row = (r < n) ? rows_s[r] : -1;
-                const uint32_t vmask = __ballot_sync(0xffffffffu, my_row >= 0);
                 uint8_t *dst = smem + C::kOffKV + stage * C::kStageBytes;
-                // 8 groups of 4 rows x 9 column boxes = 72 gathers, spread over the
-                // warp; the trip count is uniform so every shuffle has all 32 lanes.
-#pragma unroll
-                for (int i0 = 0; i0 < 96; i0 += 32) {
-                    const int i = i0 + lane;
-                    const int grp = (i / 9) & 7, box = i % 9;
-                    int rr[4];
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const int v = __shfl_sync(0xffffffffu, my_row, 4 * grp + k);
-                        rr[k] = v >= 0 ? v : kPadRow;
-                    }
-                    if (i < 72)
-                        tma_gather4(dst + box * C::kBoxBytes + grp * 512, &tmap, box * 64, rr[0],
-                                    rr[1], rr[2], rr[3], &kv_full[stage], policy);
+                // 72 warp instructions per tile, each 4 rows x 128 B; warp pw takes i = pw mod 4
+#pragma unroll 2
+                for (int i = pw; i < 72; i += C::kProducerWarps) {
+                    const int seg = 4 * i + (lane >> 3);  // 0..287: row r, column box
+                    const int r = seg / 9, box = seg - 9 * r, ch = lane & 7;
+                    const int j = t * C::kTileRows + r;
+                    const int row = (j < n) ? rows_s[j] : -1;
+                    const uint8_t *src = cache + (size_t)(row >= 0 ? row : kPadRow) * kRowBytes +
+                                         box * 128 + ch * 16;
+                    const uint32_t d = smem_addr(dst + box * C::kBoxBytes + r * 128 + ((ch ^ (r & 7)) << 4));
+                    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(src) : "memory");
                 }
-                if (lane == 0) {
-                    hdr[stage] = vmask;
-                    mbar_arrive(&kv_full[stage]);  // release: hdr is visible to the waiters
+                asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(
+                                 smem_addr(&kv_full[stage]))
+                             : "memory");
+                if (pw == 0) {
+                    const int j = t * C::kTileRows + lane;
+                    const uint32_t vmask = __ballot_sync(0xffffffffu, j < n && rows_s[j] >= 0);
+                    if (lane == 0) {
+                        hdr[stage] = vmask;
+                        mbar_arrive(&kv_full[stage]);  // release: hdr is visible to the waiters
+                    }
                 }
             }
-            __syncwarp();
         }
         // Copies still in flight must land before the CTA may exit.
-        for (int t2 = (n_tiles > C::kStages ? n_tiles - C::kStages : 0); t2 < n_tiles; ++t2)
-            mbar_wait(&kv_full[t2 % C::kStages], (t2 / C::kStages) & 1, dead);
-    } else if (warp == 5) {
+        asm volatile("cp.async.wait_all;" ::: "memory");
+    } else if (warp == C::kMmaWarp) {
         // ============================================================ MMA issuer
         if (lane == 0) {
             constexpr uint32_t kIdescQK = idesc_bf16_f32(64, 32, false, false);
@@ -207,15 +223,27 @@ __global__ void __launch_bounds__(TcCfg::kThreads, 1)
             const uint32_t q_addr = sbase + C::kOffQ;
             mbar_wait(q_ready, 0, dead);
             tc_fence_after();
-            for (int pr = 0; pr <= n_pairs; ++pr) {
-                if (pr < n_pairs) {
-                    const uint32_t s_col = C::kSCol + 32 * (pr & 1);
-                    for (int t = 2 * pr; t < 2 * pr + 2 && t < n_tiles; ++t) {
-                        const int stage = t % C::kStages;
-                        mbar_wait(&kv_full[stage], (t / C::kStages) & 1, dead);
+            // Issue whatever is ready: the next tile's QK as soon as it has landed
+            // (and its S buffer is free), a pair's PV as soon as its P is written.
+            // PV never waits behind the next tiles' loads, so a finished pair
+            // frees its stages immediately.
+            int qk_next = 0, qk_tile = 0, pv_next = 0;
+            bool idle = false;
+            uint64_t idle_since = 0;
+            while (pv_next < n_pairs && !dead) {
+                bool progressed = false;
+                if (qk_next < n_pairs && qk_next < pv_next + 2) {
+                    const int tiles_in_pair = min(2, n_tiles - 2 * qk_next);
+                    const int t = 2 * qk_next + qk_tile;
+                    const int stage = t % C::kStages;
+                    if (qk_tile < tiles_in_pair && mbar_test_wait(&kv_full[stage], (t / C::kStages) & 1)) {
+                        // the tile was written by cp.async (generic proxy); the MMA
+                        // reads it through the async proxy
+                        fence_proxy_async_smem();
                         tc_fence_after();
                         const uint32_t kv_addr = sbase + C::kOffKV + stage * C::kStageBytes;
-                        const uint32_t d = tmem + ((uint32_t)(16 * (t & 1)) << 16) + s_col;
+                        const uint32_t d = tmem + ((uint32_t)(16 * (t & 1)) << 16) + C::kSCol +
+                                           32 * (qk_next & 1);
 #pragma unroll 4
                         for (int kk = 0; kk < 36; ++kk) {
                             const uint32_t koff = (kk & 3) * 32;  // 16-element step inside the 128-B row
@@ -225,13 +253,19 @@ __global__ void __launch_bounds__(TcCfg::kThreads, 1)
                                                           16, 1024, kSwizzle128B);
                             umma_bf16(d, a, bd, kIdescQK, kk > 0 ? 1u : 0u);
                         }
+                        ++qk_tile;
+                        progressed = true;
                     }
-                    umma_commit(&s_full[pr & 1]);
+                    if (qk_tile == tiles_in_pair) {
+                        umma_commit(&s_full[qk_next & 1]);
+                        ++qk_next;
+                        qk_tile = 0;
+                        progressed = true;
+                    }
                 }
-                if (pr >= 1) {
-                    const int pp = pr - 1;
-                    mbar_wait(&p_full[pp & 1], (pp >> 1) & 1, dead);
+                if (pv_next < qk_next && mbar_test_wait(&p_full[pv_next & 1], (pv_next >> 1) & 1)) {
                     tc_fence_after();
+                    const int pp = pv_next;
                     for (int t = 2 * pp; t < 2 * pp + 2 && t < n_tiles; ++t) {
                         const int stage = t % C::kStages;
                         const uint32_t kv_addr = sbase + C::kOffKV + stage * C::kStageBytes;
@@ -249,7 +283,18 @@ __global__ void __launch_bounds__(TcCfg::kThreads, 1)
                         }
                         umma_commit(&kv_empty[stage]);
                     }
-                    umma_commit(o_done);
+                    umma_commit(&o_done[pp & 1]);
+                    ++pv_next;
+                    progressed = true;
+                }
+                if (progressed) {
+                    idle = false;
+                } else if (!idle) {
+                    idle = true;
+                    idle_since = global_timer_ns();
+                } else if (global_timer_ns() - idle_since > kWaitLimitNs) {
+                    atomicOr(&g_status_flags, kFlagTimeout);  // give up: every other wait is bounded too
+                    dead = true;
                 }
             }
         }
@@ -297,7 +342,6 @@ __global__ void __launch_bounds__(TcCfg::kThreads, 1)
             const int t = 2 * pr + half;
             const bool exists = t < n_tiles;
             mbar_wait(&s_full[pr & 1], (pr >> 1) & 1, dead);
-            if (pr >= 1) mbar_wait(o_done, (pr - 1) & 1, dead);
             tc_fence_after();
             uint32_t sr[32];
             tmem_ld32(t_lane + C::kSCol + 32 * (pr & 1), sr);
@@ -324,6 +368,11 @@ __global__ void __launch_bounds__(TcCfg::kThreads, 1)
             // (warp-collective TMEM access; alpha = 1 for the other threads).
             const bool need = (pr >= 1) && (alpha != 1.f);
             if (__any_sync(0xffffffffu, need)) {
+                // O must hold PV of pair pr-1 before it is rescaled.  The tensor
+                // pipe runs in issue order and QK(pr) went out after PV(pr-2), so
+                // PV(pr-3) is done and this parity wait cannot alias.
+                mbar_wait(&o_done[(pr - 1) & 1], ((pr - 1) >> 1) & 1, dead);
+                tc_fence_after();
 #pragma unroll 1
                 for (int c = 0; c < 256; c += 32) {
                     uint32_t orr[32];
@@ -362,7 +411,7 @@ __global__ void __launch_bounds__(TcCfg::kThreads, 1)
         // ---- epilogue: O (unnormalised) and m, lse of head hrow
         const float l_tot = l_acc + __shfl_xor_sync(0xffffffffu, l_acc, 16);
         if (n_pairs > 0) {
-            mbar_wait(o_done, (n_pairs - 1) & 1, dead);
+            mbar_wait(&o_done[(n_pairs - 1) & 1], ((n_pairs - 1) >> 1) & 1, dead);
             tc_fence_after();
         }
         const bool write = hrow < p.H;
@@ -411,7 +460,7 @@ __global__ void __launch_bounds__(TcCfg::kThreads, 1)
     }
 
     __syncthreads();
-    if (warp == 5) {
+    if (warp == C::kMmaWarp) {
         tc_fence_after();
         tmem_dealloc(tmem, C::kTmemCols);
     }

@@ -1,0 +1,90 @@
+"""Multi-rank host logic of bench.py on CPU: two gloo ranks (world_size 2).
+
+The decode path shards into independent query tokens with no exchange step,
+so N GPUs run N independent replicas; the only cross-rank traffic is the
+benchmark's own bookkeeping (max of step times, sum of tokens, barriers).
+These tests run that bookkeeping over gloo with no GPU.
+"""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, out_dir):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    sys.path.insert(0, ROOT)
+    import bench
+    w, r, _ = bench.dist_init()
+    assert (w, r) == (world, rank)
+    wl = bench.replica_workload("tiny", rank, world)
+    # rank-dependent step times: the job is as slow as its slowest rank
+    ms_local = 1.0 + rank
+    tokens_all, ms_max, value = bench.aggregate(float(wl.B * wl.T), ms_local, world)
+    bench.barrier(world)
+    digest = float(wl.q.float().sum())
+    with open(os.path.join(out_dir, f"rank{rank}.json"), "w") as f:
+        json.dump({"tokens_all": tokens_all, "ms_max": ms_max, "value": value,
+                   "digest": digest, "idx_first": int(wl.idx[0, 0, 0])}, f)
+    import torch.distributed as dist
+    dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_aggregate_weak_scaling(tmp_path):
+    port = free_port()
+    mp.start_processes(_rank_main, args=(2, port, str(tmp_path)), nprocs=2, join=True,
+                       start_method="spawn")
+    r0 = json.load(open(tmp_path / "rank0.json"))
+    r1 = json.load(open(tmp_path / "rank1.json"))
+    for r in (r0, r1):
+        assert r["tokens_all"] == 2.0            # one query token per tiny replica
+        assert r["ms_max"] == 2.0                # max over ranks, not the local time
+        assert abs(r["value"] - 2.0 / 2e-3) < 1e-6
+    assert r0["digest"] != r1["digest"]          # independent replicas (own seeds)
+
+
+def test_single_rank_replica_is_the_canonical_workload():
+    sys.path.insert(0, ROOT)
+    import bench
+    from sparse_mla_decode_partial_b200 import workloads
+    a = bench.replica_workload("tiny", 0, 1)
+    b = workloads.tiny()
+    assert torch.equal(a.q, b.q) and torch.equal(a.idx, b.idx)
+    tokens_all, ms_max, value = bench.aggregate(1.0, 4.0, 1)
+    assert (tokens_all, ms_max) == (1.0, 4.0) and abs(value - 250.0) < 1e-9
+
+
+def test_reference_arm_other_ranks_exit_without_work():
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1", MASTER_ADDR="127.0.0.1",
+               MASTER_PORT=str(free_port()))
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference"],
+                       env=env, capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0 and r.stdout.strip() == ""
+
+
+def test_reference_arm_rank0_prints_one_line():
+    env = dict(os.environ, RANK="0", WORLD_SIZE="1")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--workload", "tiny", "--cpu-seconds", "0.5"],
+                       env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr
+    lines = [l for l in r.stdout.splitlines() if l.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["cpu_baseline"]["kind"] == "oracle"
+    assert d["unit"] == "query-tokens/s" and d["value"] > 0
+    assert d["e2e"]["h2d_bytes_per_step"] == 0
