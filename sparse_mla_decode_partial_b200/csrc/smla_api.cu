@@ -190,10 +190,27 @@ smla_status launch_tc(const PartialParams &p, int grid, cudaStream_t st) {
     return e == cudaSuccess ? SMLA_OK : cuda_fail(e);
 }
 
+template <int HG, bool DIRECT>
+smla_status launch_small(const PartialParams &p, int grid, cudaStream_t st) {
+    using C = smla::SmallCfg<HG>;
+    const void *fn = reinterpret_cast<const void *>(&smla::smla_partial_small_kernel<HG, DIRECT>);
+    cudaError_t e = ensure_smem_attr(fn, C::kMaxSmemBytes);
+    if (e != cudaSuccess) return cuda_fail(e);
+    smla::smla_partial_small_kernel<HG, DIRECT>
+        <<<grid, C::kThreads, C::smem_bytes(p.pt_stride), st>>>(p);
+    e = cudaGetLastError();
+    return e == cudaSuccess ? SMLA_OK : cuda_fail(e);
+}
+
 template <bool DIRECT>
 smla_status launch_partial(const PartialParams &p, cudaStream_t st) {
     const long long grid = (long long)p.B * p.T * p.nsplit;
     if (grid > INT_MAX) return SMLA_ERR_INVALID_ARG;
+    // one tile per split: the latency path (see smla_partial_small_kernel)
+    if (p.H <= 32 && p.K > 0 && p.kc <= 32 && p.pt_stride <= smla::kSmallMaxPt) {
+        if (p.H <= 16) return launch_small<1, DIRECT>(p, (int)grid, st);
+        return launch_small<2, DIRECT>(p, (int)grid, st);
+    }
     if (p.H > 32) return launch_tc<DIRECT>(p, (int)grid, st);
     if (p.H > 16) return launch_mma<2, 32, 4, DIRECT>(p, (int)grid, st);
     return launch_mma<1, SMLA_MMA_TILE_ROWS, SMLA_MMA_STAGES, DIRECT>(p, (int)grid, st);
@@ -359,10 +376,11 @@ smla_status smla_decode(const void *q, const void *kv_cache, int64_t num_pages,
     if (!aligned(workspace, 16)) return SMLA_ERR_MISALIGNED;
     const size_t n = (size_t)B * T * H * nsplit;
     uint8_t *ws = static_cast<uint8_t *>(workspace);
+    const size_t off_m = round256(n * smla::kDc * sizeof(float));
+    const size_t off_l = off_m + round256(n * sizeof(float));
     p.part_o = reinterpret_cast<float *>(ws);
-    p.part_m = reinterpret_cast<float *>(ws + round256(n * smla::kDc * sizeof(float)));
-    p.part_lse = reinterpret_cast<float *>(ws + round256(n * smla::kDc * sizeof(float)) +
-                                           round256(n * sizeof(float)));
+    p.part_m = reinterpret_cast<float *>(ws + off_m);
+    p.part_lse = reinterpret_cast<float *>(ws + off_l);
     st = launch_partial<false>(p, s);
     if (st != SMLA_OK) return st;
     return launch_combine(p.part_o, p.part_m, p.part_lse, B, T, H, nsplit, o, lse, s);

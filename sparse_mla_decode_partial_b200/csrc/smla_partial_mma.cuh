@@ -65,8 +65,8 @@ struct PartialParams {
     float *part_o;                // [B, T, H, S, 512]
     float *part_m;                // [B, T, H, S]
     float *part_lse;              // [B, T, H, S]
-    __nv_bfloat16 *o;             // direct mode (S == 1): [B, T, H, 512]
-    float *lse;                   // direct mode: [B, T, H]
+    __nv_bfloat16 *o;             // direct / single-launch mode: [B, T, H, 512]
+    float *lse;                   // direct / single-launch mode: [B, T, H]
 };
 
 template <int HG, int NT, int NSTAGE>
@@ -89,6 +89,205 @@ struct MmaCfg {
     // CTAs per SM the launch bounds ask for: two when a pair fits (more
     // producers per SM keep more row gathers in flight).
     static constexpr int kMinBlocks = (2 * (kSmemBytes + 1024) <= 233472 && kThreads <= 192) ? 2 : 1;
+};
+
+// Per-thread state and work of one consumer warp (4 warps per head group of
+// 16 heads).  Each warp keeps the Q fragments of one quarter of the 576 dims
+// in registers and computes that quarter's partial S for all NT rows of a tile
+// (independent accumulators per n8 tile); the four partials meet once per tile
+// in shared memory.  Every warp then holds the full S of its 16 heads, runs the
+// masked online softmax in fp32 (exp2 domain, quad shuffles), turns P into A
+// fragments in registers and accumulates O += P C for its 128 of the 512
+// output columns in fp32 registers.
+template <int NT, int HG>
+struct MmaConsumer {
+    static constexpr int NTS = NT / 8;          // n8 tiles of S (all NT columns)
+    static constexpr int KQ = kD / 16 / 4;      // k16 steps of S per warp (9)
+    static constexpr int kSRow = NT + 8;        // floats per S-partial row (32-B pad)
+    int g, qw, lane, r0, cq;
+    uint32_t qa[KQ][4];
+    float oacc[16][4];
+    float m_run0, m_run1, l0, l1;
+
+    __device__ __forceinline__ void init(int warp, int lane_) {
+        g = warp >> 2;     // head group
+        qw = warp & 3;     // quarter: k range of S, and 128 output columns
+        lane = lane_;
+        r0 = lane >> 2;    // fragment row (and r0 + 8)
+        cq = lane & 3;     // fragment column pair
+        m_run0 = m_run1 = -INFINITY;
+        l0 = l1 = 0.f;
+#pragma unroll
+        for (int n = 0; n < 16; ++n) oacc[n][0] = oacc[n][1] = oacc[n][2] = oacc[n][3] = 0.f;
+    }
+
+    // This warp's 16 heads x 144 dims of Q with plain 16-byte loads (rows beyond
+    // H are zero), parked in shared memory (rows 1168 B apart) and ldmatrix-ed
+    // into A fragments.
+    __device__ __forceinline__ void load_q(uint8_t *q_smem, const PartialParams &p, int bt) {
+        const uint4 *qsrc = reinterpret_cast<const uint4 *>(p.q + (size_t)bt * p.H * kD);
+        uint4 qv[9];
+#pragma unroll
+        for (int i = 0; i < 9; ++i) {
+            const int c = lane + 32 * i;  // 16 rows x 18 chunks of 8 dims
+            const int h = 16 * g + c / 18;
+            qv[i] = (h < p.H) ? __ldg(qsrc + (size_t)h * (kD / 8) + KQ * 2 * qw + c % 18)
+                              : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int i = 0; i < 9; ++i) {
+            const int c = lane + 32 * i;
+            *reinterpret_cast<uint4 *>(q_smem + (16 * g + c / 18) * kSmemRowBytes +
+                                       (KQ * 2 * qw + c % 18) * 16) = qv[i];
+        }
+        __syncwarp();
+        const uint32_t q_base =
+            smem_addr(q_smem) + (16 * g + (lane & 15)) * kSmemRowBytes + (lane >> 4) * 16;
+#pragma unroll
+        for (int kk = 0; kk < KQ; ++kk)
+            ldsm_x4(q_base + (KQ * qw + kk) * 32, qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3]);
+    }
+
+    // One tile of NT rows (1168-B rows at shared address kv); vmask bit j = row j
+    // valid; sp = this group's S-partial buffer for the tile (double buffered by
+    // the caller so one named barrier per tile suffices).
+    __device__ __forceinline__ void tile(uint32_t kv, uint64_t vmask, float *sp, float scale_log2) {
+        // ---- partial S = Q K^T over this warp's 144 dims, all NT columns
+        float sacc[NTS][4];
+#pragma unroll
+        for (int n = 0; n < NTS; ++n) sacc[n][0] = sacc[n][1] = sacc[n][2] = sacc[n][3] = 0.f;
+        const uint32_t b_base = kv + ((lane & 7) + ((lane >> 4) << 3)) * kSmemRowBytes +
+                                ((lane >> 3) & 1) * 16 + KQ * qw * 32;
+#pragma unroll
+        for (int kk = 0; kk < KQ; ++kk) {
+#pragma unroll
+            for (int np = 0; np < NTS / 2; ++np) {
+                uint32_t b0, b1, b2, b3;
+                ldsm_x4(b_base + np * 16 * kSmemRowBytes + kk * 32, b0, b1, b2, b3);
+                mma_bf16_16816(sacc[2 * np], qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3], b0, b1);
+                mma_bf16_16816(sacc[2 * np + 1], qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3], b2, b3);
+            }
+        }
+#pragma unroll
+        for (int n = 0; n < NTS; ++n) {
+            float *d = sp + qw * 16 * kSRow + 8 * n + 2 * cq;
+            *reinterpret_cast<float2 *>(d + r0 * kSRow) = make_float2(sacc[n][0], sacc[n][1]);
+            *reinterpret_cast<float2 *>(d + (r0 + 8) * kSRow) = make_float2(sacc[n][2], sacc[n][3]);
+        }
+        named_bar_sync(1 + g, 128);
+
+        // ---- full S (sum of the four k quarters), scaled to log2 units, masked
+        float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+        for (int n = 0; n < NTS; ++n) {
+            float2 a = make_float2(0.f, 0.f), c = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+                const float *src = sp + w * 16 * kSRow + 8 * n + 2 * cq;
+                const float2 x = *reinterpret_cast<const float2 *>(src + r0 * kSRow);
+                const float2 y = *reinterpret_cast<const float2 *>(src + (r0 + 8) * kSRow);
+                a.x += x.x;
+                a.y += x.y;
+                c.x += y.x;
+                c.y += y.y;
+            }
+            const int col = 8 * n + 2 * cq;
+            const bool ok0 = (vmask >> col) & 1ull, ok1 = (vmask >> (col + 1)) & 1ull;
+            sacc[n][0] = ok0 ? a.x * scale_log2 : -INFINITY;
+            sacc[n][1] = ok1 ? a.y * scale_log2 : -INFINITY;
+            sacc[n][2] = ok0 ? c.x * scale_log2 : -INFINITY;
+            sacc[n][3] = ok1 ? c.y * scale_log2 : -INFINITY;
+            mx0 = fmaxf(mx0, fmaxf(sacc[n][0], sacc[n][1]));
+            mx1 = fmaxf(mx1, fmaxf(sacc[n][2], sacc[n][3]));
+        }
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+        const float mn0 = fmaxf(m_run0, mx0);
+        const float mn1 = fmaxf(m_run1, mx1);
+        const float mu0 = (mn0 == -INFINITY) ? 0.f : mn0;
+        const float mu1 = (mn1 == -INFINITY) ? 0.f : mn1;
+        const float al0 = exp2f(m_run0 - mu0);
+        const float al1 = exp2f(m_run1 - mu1);
+        m_run0 = mn0;
+        m_run1 = mn1;
+
+        // ---- P = exp2(s - m) straight into A fragments (k16 step j = n8 tiles 2j, 2j+1)
+        uint32_t pa[NT / 16][4];
+        float ps0 = 0.f, ps1 = 0.f;
+#pragma unroll
+        for (int n = 0; n < NTS; ++n) {
+            const float p00 = exp2f(sacc[n][0] - mu0), p01 = exp2f(sacc[n][1] - mu0);
+            const float p10 = exp2f(sacc[n][2] - mu1), p11 = exp2f(sacc[n][3] - mu1);
+            ps0 += p00 + p01;
+            ps1 += p10 + p11;
+            pa[n >> 1][(n & 1) * 2 + 0] = pack_bf16x2(p00, p01);
+            pa[n >> 1][(n & 1) * 2 + 1] = pack_bf16x2(p10, p11);
+        }
+        l0 = l0 * al0 + ps0;
+        l1 = l1 * al1 + ps1;
+#pragma unroll
+        for (int n = 0; n < 16; ++n) {
+            oacc[n][0] *= al0;
+            oacc[n][1] *= al0;
+            oacc[n][2] *= al1;
+            oacc[n][3] *= al1;
+        }
+
+        // ---- O[:, qw*128 .. +128] += P C
+        const uint32_t v_base = kv + ((lane & 7) + ((lane >> 3) & 1) * 8) * kSmemRowBytes +
+                                (qw * 128 + (lane >> 4) * 8) * 2;
+#pragma unroll
+        for (int j = 0; j < NT / 16; ++j) {
+#pragma unroll
+            for (int np = 0; np < 8; ++np) {
+                uint32_t b0, b1, b2, b3;
+                ldsm_x4_t(v_base + j * 16 * kSmemRowBytes + np * 32, b0, b1, b2, b3);
+                mma_bf16_16816(oacc[2 * np], pa[j][0], pa[j][1], pa[j][2], pa[j][3], b0, b1);
+                mma_bf16_16816(oacc[2 * np + 1], pa[j][0], pa[j][1], pa[j][2], pa[j][3], b2, b3);
+            }
+        }
+    }
+
+    // Row sums (every warp of the group holds the same full sums), then the
+    // unnormalised partial with m and lse, or (DIRECT) the final o and lse.
+    template <bool DIRECT>
+    __device__ __forceinline__ void epilogue(const PartialParams &p, int bt, int s) {
+        l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+        l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+        l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+        l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            const int h = 16 * g + r0 + 8 * half;
+            if (h >= p.H) continue;
+            const float lt = half ? l1 : l0;
+            const float mr = half ? m_run1 : m_run0;
+            const size_t row = (size_t)bt * p.H + h;
+            if (!DIRECT) {
+                float *dst = p.part_o + (row * p.nsplit + s) * kDc + qw * 128 + 2 * cq;
+#pragma unroll
+                for (int n = 0; n < 16; ++n)
+                    *reinterpret_cast<float2 *>(dst + 8 * n) =
+                        make_float2(oacc[n][2 * half], oacc[n][2 * half + 1]);
+                if (qw == 0 && cq == 0) {
+                    const size_t k = row * p.nsplit + s;
+                    p.part_m[k] = (lt > 0.f) ? mr * kLn2 : -INFINITY;
+                    p.part_lse[k] = (lt > 0.f) ? (mr + log2f(lt)) * kLn2 : -INFINITY;
+                }
+            } else {
+                const float inv = (lt > 0.f) ? 1.f / lt : 0.f;
+                __nv_bfloat16 *dst = p.o + row * kDc + qw * 128 + 2 * cq;
+#pragma unroll
+                for (int n = 0; n < 16; ++n)
+                    *reinterpret_cast<uint32_t *>(dst + 8 * n) =
+                        pack_bf16x2(oacc[n][2 * half] * inv, oacc[n][2 * half + 1] * inv);
+                if (qw == 0 && cq == 0)
+                    p.lse[row] = (lt > 0.f) ? (mr + log2f(lt)) * kLn2 : -INFINITY;
+            }
+        }
+    }
 };
 
 template <int HG, int NT, int NSTAGE, bool DIRECT>
@@ -210,196 +409,135 @@ __global__ void __launch_bounds__(MmaCfg<HG, NT, NSTAGE>::kThreads, MmaCfg<HG, N
     }
 
     // ================================================================ consumers
-    const int g = warp >> 2;   // head group
-    const int qw = warp & 3;   // quarter: k range of S, and 128 output columns
-    const int r0 = lane >> 2;  // fragment row (and r0 + 8)
-    const int cq = lane & 3;   // fragment column pair
-    constexpr int NTS = NT / 8;  // n8 tiles of S (all NT columns, every warp)
-    constexpr int KQ = kD / 16 / 4;  // k16 steps of S per warp (576 / 16 / 4 = 9)
-    const uint32_t bar_grp = 1 + g;
-    const uint32_t bar_all = 1 + HG;
-
-    // Q fragments of this warp's k quarter stay in registers for the whole split.
-    // Each warp loads its own 16 heads x 144 dims with plain 16-byte loads (rows
-    // beyond H are zero), parks them in shared memory and ldmatrix-es them out;
-    // the TMA engine stays free for the gathered rows.
-    uint32_t qa[KQ][4];
-    {
-        const uint4 *qsrc = reinterpret_cast<const uint4 *>(p.q + (size_t)bt * p.H * kD);
-        uint4 qv[9];
-#pragma unroll
-        for (int i = 0; i < 9; ++i) {
-            const int c = lane + 32 * i;          // 16 rows x 18 chunks of 8 dims
-            const int h = 16 * g + c / 18;
-            qv[i] = (h < p.H) ? __ldg(qsrc + (size_t)h * (kD / 8) + KQ * 2 * qw + c % 18)
-                              : make_uint4(0u, 0u, 0u, 0u);
-        }
-#pragma unroll
-        for (int i = 0; i < 9; ++i) {
-            const int c = lane + 32 * i;
-            *reinterpret_cast<uint4 *>(smem + C::kOffQ + (16 * g + c / 18) * kSmemRowBytes +
-                                       (KQ * 2 * qw + c % 18) * 16) = qv[i];
-        }
-        __syncwarp();
-        const uint32_t q_base = smem_addr(smem + C::kOffQ) +
-                                (16 * g + (lane & 15)) * kSmemRowBytes + (lane >> 4) * 16;
-#pragma unroll
-        for (int kk = 0; kk < KQ; ++kk)
-            ldsm_x4(q_base + (KQ * qw + kk) * 32, qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3]);
-    }
+    MmaConsumer<NT, HG> cons;
+    cons.init(warp, lane);
+    cons.load_q(smem + C::kOffQ, p, bt);
     // The Q region is reused for the split-k score exchange from here on.
-    named_bar_sync(bar_all, 128 * HG);
-
-    float m_run0 = -INFINITY, m_run1 = -INFINITY;
-    float l0 = 0.f, l1 = 0.f;
-    float oacc[16][4];
-#pragma unroll
-    for (int n = 0; n < 16; ++n) oacc[n][0] = oacc[n][1] = oacc[n][2] = oacc[n][3] = 0.f;
-
-    // S partials: [group][buffer][warp][16 rows][NT cols] fp32, rows padded by 32 B.
-    float *spart = reinterpret_cast<float *>(smem + C::kOffQ) + g * 2 * 4 * 16 * C::kSRow;
-
+    named_bar_sync(1 + HG, 128 * HG);
+    float *spart = reinterpret_cast<float *>(smem + C::kOffQ) + cons.g * 2 * 4 * 16 * C::kSRow;
     for (int it = 0; it < n_tiles; ++it) {
         const int stage = it % NSTAGE;
         mbar_wait(&full[stage], (it / NSTAGE) & 1, dead);
-        const uint64_t vmask = hdr[stage];
-        const uint32_t kv = smem_addr(smem + C::kOffKV + stage * C::kStageBytes);
-
-        // ---- partial S = Q K^T over this warp's 144 dims, all NT columns
-        float sacc[NTS][4];
-#pragma unroll
-        for (int n = 0; n < NTS; ++n) sacc[n][0] = sacc[n][1] = sacc[n][2] = sacc[n][3] = 0.f;
-        const uint32_t b_base = kv + ((lane & 7) + ((lane >> 4) << 3)) * kSmemRowBytes +
-                                ((lane >> 3) & 1) * 16 + KQ * qw * 32;
-#pragma unroll
-        for (int kk = 0; kk < KQ; ++kk) {
-#pragma unroll
-            for (int np = 0; np < NTS / 2; ++np) {
-                uint32_t b0, b1, b2, b3;
-                ldsm_x4(b_base + np * 16 * kSmemRowBytes + kk * 32, b0, b1, b2, b3);
-                mma_bf16_16816(sacc[2 * np], qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3], b0, b1);
-                mma_bf16_16816(sacc[2 * np + 1], qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3], b2, b3);
-            }
-        }
-        float *sp = spart + (it & 1) * 4 * 16 * C::kSRow;
-#pragma unroll
-        for (int n = 0; n < NTS; ++n) {
-            float *d = sp + qw * 16 * C::kSRow + 8 * n + 2 * cq;
-            *reinterpret_cast<float2 *>(d + r0 * C::kSRow) = make_float2(sacc[n][0], sacc[n][1]);
-            *reinterpret_cast<float2 *>(d + (r0 + 8) * C::kSRow) = make_float2(sacc[n][2], sacc[n][3]);
-        }
-        named_bar_sync(bar_grp, 128);
-
-        // ---- full S (sum of the four k quarters), scaled to log2 units, masked
-        float mx0 = -INFINITY, mx1 = -INFINITY;
-#pragma unroll
-        for (int n = 0; n < NTS; ++n) {
-            float2 a = make_float2(0.f, 0.f), c = make_float2(0.f, 0.f);
-#pragma unroll
-            for (int w = 0; w < 4; ++w) {
-                const float *src = sp + w * 16 * C::kSRow + 8 * n + 2 * cq;
-                const float2 x = *reinterpret_cast<const float2 *>(src + r0 * C::kSRow);
-                const float2 y = *reinterpret_cast<const float2 *>(src + (r0 + 8) * C::kSRow);
-                a.x += x.x;
-                a.y += x.y;
-                c.x += y.x;
-                c.y += y.y;
-            }
-            const int col = 8 * n + 2 * cq;
-            const bool ok0 = (vmask >> col) & 1ull, ok1 = (vmask >> (col + 1)) & 1ull;
-            sacc[n][0] = ok0 ? a.x * p.scale_log2 : -INFINITY;
-            sacc[n][1] = ok1 ? a.y * p.scale_log2 : -INFINITY;
-            sacc[n][2] = ok0 ? c.x * p.scale_log2 : -INFINITY;
-            sacc[n][3] = ok1 ? c.y * p.scale_log2 : -INFINITY;
-            mx0 = fmaxf(mx0, fmaxf(sacc[n][0], sacc[n][1]));
-            mx1 = fmaxf(mx1, fmaxf(sacc[n][2], sacc[n][3]));
-        }
-        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
-        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-        const float mn0 = fmaxf(m_run0, mx0);
-        const float mn1 = fmaxf(m_run1, mx1);
-        const float mu0 = (mn0 == -INFINITY) ? 0.f : mn0;
-        const float mu1 = (mn1 == -INFINITY) ? 0.f : mn1;
-        const float al0 = exp2f(m_run0 - mu0);
-        const float al1 = exp2f(m_run1 - mu1);
-        m_run0 = mn0;
-        m_run1 = mn1;
-
-        // ---- P = exp2(s - m) straight into A fragments (k16 step j = n8 tiles 2j, 2j+1)
-        uint32_t pa[NT / 16][4];
-        float ps0 = 0.f, ps1 = 0.f;
-#pragma unroll
-        for (int n = 0; n < NTS; ++n) {
-            const float p00 = exp2f(sacc[n][0] - mu0), p01 = exp2f(sacc[n][1] - mu0);
-            const float p10 = exp2f(sacc[n][2] - mu1), p11 = exp2f(sacc[n][3] - mu1);
-            ps0 += p00 + p01;
-            ps1 += p10 + p11;
-            pa[n >> 1][(n & 1) * 2 + 0] = pack_bf16x2(p00, p01);
-            pa[n >> 1][(n & 1) * 2 + 1] = pack_bf16x2(p10, p11);
-        }
-        l0 = l0 * al0 + ps0;
-        l1 = l1 * al1 + ps1;
-#pragma unroll
-        for (int n = 0; n < 16; ++n) {
-            oacc[n][0] *= al0;
-            oacc[n][1] *= al0;
-            oacc[n][2] *= al1;
-            oacc[n][3] *= al1;
-        }
-
-        // ---- O[:, qw*128 .. +128] += P C
-        const uint32_t v_base = kv + ((lane & 7) + ((lane >> 3) & 1) * 8) * kSmemRowBytes +
-                                (qw * 128 + (lane >> 4) * 8) * 2;
-#pragma unroll
-        for (int j = 0; j < NT / 16; ++j) {
-#pragma unroll
-            for (int np = 0; np < 8; ++np) {
-                uint32_t b0, b1, b2, b3;
-                ldsm_x4_t(v_base + j * 16 * kSmemRowBytes + np * 32, b0, b1, b2, b3);
-                mma_bf16_16816(oacc[2 * np], pa[j][0], pa[j][1], pa[j][2], pa[j][3], b0, b1);
-                mma_bf16_16816(oacc[2 * np + 1], pa[j][0], pa[j][1], pa[j][2], pa[j][3], b2, b3);
-            }
-        }
+        cons.tile(smem_addr(smem + C::kOffKV + stage * C::kStageBytes), hdr[stage],
+                  spart + (it & 1) * 4 * 16 * C::kSRow, p.scale_log2);
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[stage]);
     }
+    cons.template epilogue<DIRECT>(p, bt, s);
+}
 
-    // ---- epilogue: row sums (every warp of the group holds the same full sums)
-    l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
-    l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
-    l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
-    l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+// ----------------------------------------------------------------------------
+// Latency path: a split of at most 32 rows (one tile), as in single-request
+// decode with a large NSPLIT.  There the pipelined kernel's chain -- index
+// load, then page-table load, then 32 TMA row copies issued one after another,
+// then the math -- is the whole cost.  This kernel instead loads the
+// sequence's entire page-table row together with the indices and Q (one
+// memory round trip), resolves the rows from shared memory, gathers the tile
+// with 16-byte cp.async copies issued by every thread (one more round trip,
+// no serial TMA queue) and runs the same consumer math on it.
+constexpr int kSmallMaxPt = 8192;  // page-table entries kept in shared memory
 
+
+template <int HG>
+struct SmallCfg {
+    static constexpr int NT = 32;
+    static constexpr int kThreads = 128 * HG;
+    static constexpr int kQBytes = 16 * HG * kSmemRowBytes;
+    static constexpr int kSPartBytes = HG * 2 * 4 * 16 * (NT + 8) * 4;
+    static constexpr int kOffQ = 0;  // Q rows, then the S partials
+    static constexpr int kOffKV = ((kQBytes > kSPartBytes ? kQBytes : kSPartBytes) + 127) / 128 * 128;
+    static constexpr int kOffRows = kOffKV + NT * kSmemRowBytes;  // int [32] rows, u32 mask
+    static constexpr int kOffPt = kOffRows + 36 * 4;             // int [pt_stride]
+    static constexpr int kMaxSmemBytes = kOffPt + kSmallMaxPt * 4;
+    static int smem_bytes(int pt_stride) { return kOffPt + pt_stride * 4; }
+};
+
+template <int HG, bool DIRECT>
+__global__ void __launch_bounds__(SmallCfg<HG>::kThreads)
+    smla_partial_small_kernel(const PartialParams p) {
+    using C = SmallCfg<HG>;
+    constexpr int NT = C::NT;
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int tid = threadIdx.x;
+    const int unit = blockIdx.x;  // (b * T + t) * S + s
+    const int s = unit % p.nsplit;
+    const int bt = unit / p.nsplit;
+    const int b = bt / p.T;
+    const long long j0l = (long long)s * p.kc;
+    const int j0 = (int)(j0l < p.K ? j0l : p.K);
+    const int j1 = (int)((long long)j0 + p.kc < p.K ? (long long)j0 + p.kc : p.K);
+    int *rows_s = reinterpret_cast<int *>(smem + C::kOffRows);
+    int *pt_s = reinterpret_cast<int *>(smem + C::kOffPt);
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
+    // 1. page-table row, this split's indices and Q: all loads in flight at once
+    const int *pt_b = p.page_table + (size_t)b * p.pt_stride;
+    for (int i0 = 0; i0 < p.pt_stride; i0 += C::kThreads * 8) {
+        int v[8];
 #pragma unroll
-    for (int half = 0; half < 2; ++half) {
-        const int h = 16 * g + r0 + 8 * half;
-        if (h >= p.H) continue;
-        const float lt = half ? l1 : l0;
-        const float mr = half ? m_run1 : m_run0;
-        const size_t row = (size_t)bt * p.H + h;
-        if (!DIRECT) {
-            float *dst = p.part_o + (row * p.nsplit + s) * kDc + qw * 128 + 2 * cq;
+        for (int k = 0; k < 8; ++k) {
+            const int i = i0 + k * C::kThreads + tid;
+            v[k] = (i < p.pt_stride) ? __ldg(pt_b + i) : -1;
+        }
 #pragma unroll
-            for (int n = 0; n < 16; ++n)
-                *reinterpret_cast<float2 *>(dst + 8 * n) =
-                    make_float2(oacc[n][2 * half], oacc[n][2 * half + 1]);
-            if (qw == 0 && cq == 0) {
-                const size_t k = row * p.nsplit + s;
-                p.part_m[k] = (lt > 0.f) ? mr * kLn2 : -INFINITY;
-                p.part_lse[k] = (lt > 0.f) ? (mr + log2f(lt)) * kLn2 : -INFINITY;
-            }
-        } else {
-            const float inv = (lt > 0.f) ? 1.f / lt : 0.f;
-            __nv_bfloat16 *dst = p.o + row * kDc + qw * 128 + 2 * cq;
-#pragma unroll
-            for (int n = 0; n < 16; ++n)
-                *reinterpret_cast<uint32_t *>(dst + 8 * n) =
-                    pack_bf16x2(oacc[n][2 * half] * inv, oacc[n][2 * half + 1] * inv);
-            if (qw == 0 && cq == 0) p.lse[row] = (lt > 0.f) ? (mr + log2f(lt)) * kLn2 : -INFINITY;
+        for (int k = 0; k < 8; ++k) {
+            const int i = i0 + k * C::kThreads + tid;
+            if (i < p.pt_stride) pt_s[i] = v[k];
         }
     }
+    int my_idx = -1;
+    if (tid < NT && j0 + tid < j1) my_idx = __ldg(p.idx + (size_t)bt * p.K + j0 + tid);
+    MmaConsumer<NT, HG> cons;
+    cons.init(warp, lane);
+    cons.load_q(smem + C::kOffQ, p, bt);
+    __syncthreads();
+
+    // 2. rows of the tile (warp 0); out-of-range entries are masked and counted
+    if (warp == 0) {
+        const int i = my_idx;
+        int row = -1;
+        if (i != -1) {
+            const long long max_pos = (long long)p.pt_stride * kPage;
+            bool ok = (i >= 0) && ((long long)i < max_pos);
+            const int pg = ok ? pt_s[i >> 6] : -1;
+            ok = ok && (pg >= 0) && ((long long)pg < p.num_pages);
+            if (ok) {
+                row = pg * kPage + (i & (kPage - 1));
+            } else {
+                atomicOr(&g_status_flags, kFlagIndexRange);
+                atomicAdd(&g_bad_index_count, 1ull);
+            }
+        }
+        rows_s[lane] = row;
+        const uint32_t m = __ballot_sync(0xffffffffu, row >= 0);
+        if (lane == 0) rows_s[32] = (int)m;
+    }
+    __syncthreads();
+
+    // 3. gather: 32 rows x 72 chunks of 16 B, cp.async from every thread
+    const uint8_t *cache = reinterpret_cast<const uint8_t *>(p.cache);
+    const uint8_t *zero = reinterpret_cast<const uint8_t *>(g_zero_row);
+    uint8_t *kv = smem + C::kOffKV;
+    for (int c = tid; c < NT * 72; c += C::kThreads) {
+        const int r = c / 72, k = c - 72 * (c / 72);
+        const int row = rows_s[r];
+        const uint8_t *src = (row >= 0 ? cache + (size_t)row * kRowBytes : zero) + k * 16;
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                         smem_addr(kv + r * kSmemRowBytes + k * 16)),
+                     "l"(src)
+                     : "memory");
+    }
+    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+    const uint32_t vmask = (uint32_t)rows_s[32];
+    __syncthreads();
+
+    // 4. the tile and the epilogue (the Q region now holds the S partials)
+    cons.tile(smem_addr(kv), vmask,
+              reinterpret_cast<float *>(smem + C::kOffQ) + cons.g * 2 * 4 * 16 * (NT + 8),
+              p.scale_log2);
+    cons.template epilogue<DIRECT>(p, bt, s);
 }
 
 }  // namespace smla

@@ -250,3 +250,42 @@ def test_device_error_paths():
                          w.pt_stride, w.idx.data_ptr(), 1, 1, 16, 64, 64, w.scale, 4, None, 100,
                          o.data_ptr(), lse.data_ptr(), None)
     assert st == 4
+
+
+# ------------------------------------------------------------------ one-tile splits
+# When every split holds at most 32 entries (H <= 32) the partial pass runs the
+# latency form of the kernel (one CTA per split, every load in flight at once).
+# Whatever a reused workspace held before must not change the result.
+@pytest.mark.parametrize("fill", [0x00, 0xFF, 0x5A])
+def test_one_tile_splits_arbitrary_workspace_contents(fill):
+    w = small("one_tile", seed=11, B=1, T=2, H=16, K=1024, ctx=30000)
+    wd = w.to(DEV)
+    S = 32                                                # 32 rows per split
+    ws = torch.full((binding.workspace_bytes(1, 2, 16, S),), fill, dtype=torch.uint8, device=DEV)
+    o_ref, lse_ref, _ = oracle_decode(w)
+    for call in range(3):                                 # partials left by the previous call
+        o, lse = binding.decode(wd.q, wd.cache, wd.page_table, wd.idx, w.scale, S, workspace=ws)
+        torch.cuda.synchronize()
+        check_o_lse(o, lse, o_ref, lse_ref, f"fill={fill:#x} call {call}")
+    assert binding.check_device(clear=False)[0] == 0
+
+
+@pytest.mark.parametrize("H,K,S", [(16, 33, 32), (32, 64, 2), (8, 1, 4), (17, 640, 20),
+                                   (32, 2048, 64), (1, 100, 7)])
+def test_one_tile_split_shapes(H, K, S):
+    # empty splits (K=33, S=32 -> 17 one-or-two-row splits and 15 empty ones),
+    # both head groups (H <= 16, H <= 32), one row in all, odd S
+    w = small("one_tile_shapes", seed=H * 100 + K, B=2, T=1, H=H, K=K, ctx=4000)
+    o, lse = run_decode(w, S)
+    o_ref, lse_ref, _ = oracle_decode(w)
+    check_o_lse(o, lse, o_ref, lse_ref, f"one-tile H={H} K={K} S={S}")
+
+
+def test_one_tile_splits_many_waves():
+    # 64 tokens x 64 splits = 4096 blocks: many waves of the latency form
+    w = small("one_tile_big", seed=12, B=64, T=1, H=16, K=2048, ctx=8000)
+    o, lse = run_decode(w, 64)
+    sample = [(0, 0), (17, 0), (63, 0)]
+    o_ref, lse_ref, _ = oracle_decode(w, sample)
+    idx = torch.tensor([b for b, _ in sample])
+    check_o_lse(o[idx, 0], lse[idx, 0], o_ref, lse_ref, "many waves")
