@@ -106,6 +106,14 @@ def load_peaks():
 
 
 # ----------------------------------------------------------------------------- clocks
+def partial_kernel_name(H: int, K: int, nsplit: int, pt_stride: int) -> str:
+    """The partial kernel the library launches for this shape (its dispatch rule)."""
+    kc = -(-K // nsplit) if K > 0 else 0
+    if H <= 32 and K > 0 and kc <= 32 and pt_stride <= 8192:
+        return "smla_partial_small_kernel"
+    return "smla_partial_tc_kernel" if H > 32 else "smla_partial_mma_kernel"
+
+
 class ClockSampler:
     """Samples SM clock and throttle reasons through NVML while running."""
 
@@ -439,7 +447,8 @@ def run_ours(args, world, rank, local):
                       "note": "partial pass timed alone in a second loop of the same length; "
                               "the step runs it and the combine through one smla_decode call"},
         "roofline": {"bound": "hbm",
-                     "kernel": "smla_partial_tc_kernel" if H > 32 else "smla_partial_mma_kernel", "achieved": round(achieved, 1),
+                     "kernel": partial_kernel_name(H, K, nsplit, w_host.pt_stride),
+                     "achieved": round(achieved, 1),
                      "peak": hbm_peak, "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),
                      "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured" else "fallback",
                      "traffic": measured_traffic(args.workload),
