@@ -208,8 +208,8 @@ struct MmaConsumer {
         const float mn1 = fmaxf(m_run1, mx1);
         const float mu0 = (mn0 == -INFINITY) ? 0.f : mn0;
         const float mu1 = (mn1 == -INFINITY) ? 0.f : mn1;
-        const float al0 = exp2f(m_run0 - mu0);
-        const float al1 = exp2f(m_run1 - mu1);
+        const float al0 = fast_exp2(m_run0 - mu0);
+        const float al1 = fast_exp2(m_run1 - mu1);
         m_run0 = mn0;
         m_run1 = mn1;
 
@@ -218,8 +218,8 @@ struct MmaConsumer {
         float ps0 = 0.f, ps1 = 0.f;
 #pragma unroll
         for (int n = 0; n < NTS; ++n) {
-            const float p00 = exp2f(sacc[n][0] - mu0), p01 = exp2f(sacc[n][1] - mu0);
-            const float p10 = exp2f(sacc[n][2] - mu1), p11 = exp2f(sacc[n][3] - mu1);
+            const float p00 = fast_exp2(sacc[n][0] - mu0), p01 = fast_exp2(sacc[n][1] - mu0);
+            const float p10 = fast_exp2(sacc[n][2] - mu1), p11 = fast_exp2(sacc[n][3] - mu1);
             ps0 += p00 + p01;
             ps1 += p10 + p11;
             pa[n >> 1][(n & 1) * 2 + 0] = pack_bf16x2(p00, p01);

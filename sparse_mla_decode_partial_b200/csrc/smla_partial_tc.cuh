@@ -6,35 +6,37 @@
 // the top-k candidate rows, split-K over that axis, partials merged by LSE.
 //
 // One CTA = one (query token, split), all heads (M = 64 rows of the MMA;
-// heads >= H are zero rows of Q and are never written out).  288 threads:
+// heads >= H are zero rows of Q and are never written out).  416 threads:
 //   warps 0-3  softmax warpgroup: stages Q (128B-swizzled) once, then per
 //              PAIR of 32-row tiles reads S from TMEM (tcgen05.ld), masks,
 //              keeps a running max per head with lazy rescaling (O is only
 //              rescaled when the max grows by more than 2^8), writes P as bf16
-//              into the tile's spent k_pe box, and finally drains O.
-//   warps 4-7  producers: resolve the split's indices to rows (as the mma
+//              into each tile's spent k_pe box, and finally drains O.
+//   warps 4-11 producers: resolve the split's indices to rows (as the mma
 //              kernel does), then gather each 32-row tile with 16-byte
 //              cp.async copies written straight into the 128B-swizzled
 //              K-major layout (each warp instruction moves 4 rows x 128 B,
-//              coalesced); completion reaches the stage's mbarrier through
-//              cp.async.mbarrier.arrive.  Four warps keep enough copies in
-//              flight; the TMA engine would cap this at one 512-B gather4 or
-//              one 1152-B row per operation.  Padding slots copy row 0 and
-//              are masked.
-//   warp 8     TMEM owner + MMA issuer (one thread):
-//                QK(t):  S[64 x 32] = Q[64 x 576] K_t^T        36 x (M64 N32 K16)
-//                PV(t):  O[64 x 512] += P_t[64 x 32] C_t[32 x 512]  2 x 2 x (M64 N256 K16)
-//              The issuer polls: a tile's QK goes out as soon as the tile
-//              has landed, a pair's PV as soon as its P is ready, so the
-//              softmax of one pair overlaps the scores of the next and a
-//              finished pair frees its stages without waiting for new loads.
+//              coalesced); completion reaches the tile's mbarrier through
+//              cp.async.mbarrier.arrive.  Padding slots copy row 0 and are
+//              masked.
+//   warp 12    TMEM owner + MMA issuer (one thread):
+//                QK(pair): S[64 x 64] = Q[64 x 576] [K_2p K_2p+1]^T   36 x (M64 N64 K16)
+//                PV(t):    O[64 x 512] += P_t[64 x 32] C_t[32 x 512]  2 x 2 x (M64 N256 K16)
+//              A tcgen05 MMA costs at least ~46 cycles whatever its size
+//              below M64 N64 (M64 N32 costs the same as M64 N64), so the
+//              two tiles of a pair share one N = 64 score MMA per k-step: the
+//              ring keeps the pair's tiles side by side in every 64-column
+//              box.  The issuer polls: a pair's QK goes out as soon as both
+//              tiles have landed, its PV as soon as its P is ready.
+// Shared memory ring: two pair slots of 2 x 36864 B; box b (64 columns) of
+// tile h of a slot at slot + 8192 b + 4096 h, rows 128 B apart.
 // TMEM (512 columns; M = 64 accumulators occupy lanes 0-15 of each 32-lane
 // sub-partition, or 16-31 when addressed at lane offset 16):
 //   cols [0,256)   lane off 0: O[:, 0:256]     lane off 16: O[:, 256:512]
-//   cols 256+32b   lane off 0: S of the pair's first tile, 16: second tile
-//                  (b = pair parity, double buffered)
-// So thread (warp q, lane l) of the softmax warpgroup owns head 16q + l%16,
-// the first (l < 16) or second (l >= 16) tile of a pair, and one half of O.
+//   cols 256+64b   lane off 0: S of pair b (b = pair parity, double buffered),
+//                  columns 0-31 its first tile, 32-63 its second
+// Softmax thread (warp q, lane l): lanes 0-15 own head 16q + l and do the
+// pair's softmax; lane l + 16 rescales the second half of the same head's O.
 #pragma once
 
 #include <cstdint>
@@ -48,15 +50,16 @@ namespace smla {
 
 struct TcCfg {
 #ifndef SMLA_TC_PRODUCER_WARPS
-#define SMLA_TC_PRODUCER_WARPS 4
+#define SMLA_TC_PRODUCER_WARPS 8
 #endif
     static constexpr int kProducerWarps = SMLA_TC_PRODUCER_WARPS;
     static constexpr int kMmaWarp = 4 + kProducerWarps;
     static constexpr int kThreads = 32 * (kMmaWarp + 1);
     static constexpr int kTileRows = 32;
-    static constexpr int kStages = 4;
+    static constexpr int kStages = 4;                       // tiles in the ring (2 pair slots)
     static constexpr int kBoxBytes = kTileRows * 128;       // 4096: 32 rows x 64 bf16
-    static constexpr int kStageBytes = 9 * kBoxBytes;       // 36864
+    static constexpr int kBoxStride = 2 * kBoxBytes;        // 8192: the pair's two tiles per box
+    static constexpr int kStageBytes = 9 * kBoxBytes;       // 36864 per tile
     static constexpr int kQBoxBytes = 64 * 128;             // 8192
     static constexpr int kOffQ = 0;                         // 9 x 8192
     static constexpr int kOffKV = 9 * kQBoxBytes;           // 73728
@@ -70,6 +73,9 @@ struct TcCfg {
     static constexpr int kSmemBytes = kBytes + 1024;        // + alignment slack for 1024-B atoms
     static constexpr uint32_t kTmemCols = 512;
     static constexpr uint32_t kSCol = 256;
+    __host__ __device__ static constexpr int tile_off(int stage) {  // tile base inside the ring
+        return (stage >> 1) * 2 * kStageBytes + (stage & 1) * kBoxBytes;
+    }
     static constexpr float kTau = 8.0f;                     // lazy-rescale threshold (log2 units)
 };
 static_assert(TcCfg::kSmemBytes <= 232448, "shared memory per CTA");
@@ -187,7 +193,7 @@ __global__ void __launch_bounds__(TcCfg::kThreads, 1)
             for (int t = 0; t < chunk_tiles; ++t, ++it) {
                 const int stage = it % C::kStages;
                 if (it >= C::kStages) mbar_wait(&kv_empty[stage], ((it / C::kStages) - 1) & 1, dead);
-                uint8_t *dst = smem + C::kOffKV + stage * C::kStageBytes;
+                uint8_t *dst = smem + C::kOffKV + C::tile_off(stage);
                 // 72 warp instructions per tile, each 4 rows x 128 B; warp pw takes i = pw mod 4
 #pragma unroll 2
                 for (int i = pw; i < 72; i += C::kProducerWarps) {
@@ -197,7 +203,7 @@ __global__ void __launch_bounds__(TcCfg::kThreads, 1)
                     const int row = (j < n) ? rows_s[j] : -1;
                     const uint8_t *src = cache + (size_t)(row >= 0 ? row : kPadRow) * kRowBytes +
                                          box * 128 + ch * 16;
-                    const uint32_t d = smem_addr(dst + box * C::kBoxBytes + r * 128 + ((ch ^ (r & 7)) << 4));
+                    const uint32_t d = smem_addr(dst + box * C::kBoxStride + r * 128 + ((ch ^ (r & 7)) << 4));
                     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(src) : "memory");
                 }
                 asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(
@@ -218,48 +224,50 @@ __global__ void __launch_bounds__(TcCfg::kThreads, 1)
     } else if (warp == C::kMmaWarp) {
         // ============================================================ MMA issuer
         if (lane == 0) {
-            constexpr uint32_t kIdescQK = idesc_bf16_f32(64, 32, false, false);
+            constexpr uint32_t kIdescQK = idesc_bf16_f32(64, 64, false, false);
             constexpr uint32_t kIdescPV = idesc_bf16_f32(64, 256, false, true);
             const uint32_t q_addr = sbase + C::kOffQ;
             mbar_wait(q_ready, 0, dead);
             tc_fence_after();
-            // Issue whatever is ready: the next tile's QK as soon as it has landed
-            // (and its S buffer is free), a pair's PV as soon as its P is written.
-            // PV never waits behind the next tiles' loads, so a finished pair
-            // frees its stages immediately.
-            int qk_next = 0, qk_tile = 0, pv_next = 0;
+            // Issue whatever is ready: a pair's QK as soon as its tiles have
+            // landed (and its S buffer is free), a pair's PV as soon as its P
+            // is written.  PV never waits behind the next pair's loads, so a
+            // finished pair frees its slot immediately.  (Issuing blocks while
+            // the tensor pipe is busy; splitting QK into chunks so that a
+            // ready PV could slip in between measured no faster: it only moves
+            // the wait onto the other slot.)
+            int qk_next = 0, qk_landed = 0, pv_next = 0;
             bool idle = false;
             uint64_t idle_since = 0;
             while (pv_next < n_pairs && !dead) {
                 bool progressed = false;
                 if (qk_next < n_pairs && qk_next < pv_next + 2) {
                     const int tiles_in_pair = min(2, n_tiles - 2 * qk_next);
-                    const int t = 2 * qk_next + qk_tile;
-                    const int stage = t % C::kStages;
-                    if (qk_tile < tiles_in_pair && mbar_test_wait(&kv_full[stage], (t / C::kStages) & 1)) {
-                        // the tile was written by cp.async (generic proxy); the MMA
-                        // reads it through the async proxy
+                    while (qk_landed < tiles_in_pair) {
+                        const int t = 2 * qk_next + qk_landed;
+                        if (!mbar_test_wait(&kv_full[t % C::kStages], (t / C::kStages) & 1)) break;
+                        ++qk_landed;
+                    }
+                    if (qk_landed == tiles_in_pair) {
+                        // The tiles were written by cp.async (generic proxy); the
+                        // MMA reads them through the async proxy.  A pair with one
+                        // tile reads a stale second half: its scores are masked.
                         fence_proxy_async_smem();
                         tc_fence_after();
-                        const uint32_t kv_addr = sbase + C::kOffKV + stage * C::kStageBytes;
-                        const uint32_t d = tmem + ((uint32_t)(16 * (t & 1)) << 16) + C::kSCol +
-                                           32 * (qk_next & 1);
+                        const uint32_t kv_addr = sbase + C::kOffKV + C::tile_off((2 * qk_next) % C::kStages);
+                        const uint32_t d = tmem + C::kSCol + 64 * (qk_next & 1);
 #pragma unroll 4
                         for (int kk = 0; kk < 36; ++kk) {
                             const uint32_t koff = (kk & 3) * 32;  // 16-element step inside the 128-B row
                             const uint64_t a = smem_desc(q_addr + (kk >> 2) * C::kQBoxBytes + koff, 16,
                                                          1024, kSwizzle128B);
-                            const uint64_t bd = smem_desc(kv_addr + (kk >> 2) * C::kBoxBytes + koff,
+                            const uint64_t bd = smem_desc(kv_addr + (kk >> 2) * C::kBoxStride + koff,
                                                           16, 1024, kSwizzle128B);
                             umma_bf16(d, a, bd, kIdescQK, kk > 0 ? 1u : 0u);
                         }
-                        ++qk_tile;
-                        progressed = true;
-                    }
-                    if (qk_tile == tiles_in_pair) {
                         umma_commit(&s_full[qk_next & 1]);
                         ++qk_next;
-                        qk_tile = 0;
+                        qk_landed = 0;
                         progressed = true;
                     }
                 }
@@ -268,16 +276,16 @@ __global__ void __launch_bounds__(TcCfg::kThreads, 1)
                     const int pp = pv_next;
                     for (int t = 2 * pp; t < 2 * pp + 2 && t < n_tiles; ++t) {
                         const int stage = t % C::kStages;
-                        const uint32_t kv_addr = sbase + C::kOffKV + stage * C::kStageBytes;
-                        const uint32_t p_addr = kv_addr + 8 * C::kBoxBytes;
+                        const uint32_t kv_addr = sbase + C::kOffKV + C::tile_off(stage);
+                        const uint32_t p_addr = kv_addr + 8 * C::kBoxStride;
 #pragma unroll
                         for (int kk = 0; kk < 2; ++kk) {
                             const uint32_t acc = (t > 0 || kk > 0) ? 1u : 0u;
                             const uint64_t a = smem_desc(p_addr + kk * 32, 16, 512, kSwizzle64B);
-                            const uint64_t blo = smem_desc(kv_addr + kk * 2048, C::kBoxBytes, 1024,
+                            const uint64_t blo = smem_desc(kv_addr + kk * 2048, C::kBoxStride, 1024,
                                                            kSwizzle128B);
-                            const uint64_t bhi = smem_desc(kv_addr + 4 * C::kBoxBytes + kk * 2048,
-                                                           C::kBoxBytes, 1024, kSwizzle128B);
+                            const uint64_t bhi = smem_desc(kv_addr + 4 * C::kBoxStride + kk * 2048,
+                                                           C::kBoxStride, 1024, kSwizzle128B);
                             umma_bf16(tmem, a, blo, kIdescPV, acc);
                             umma_bf16(tmem + (16u << 16), a, bhi, kIdescPV, acc);
                         }
@@ -335,35 +343,46 @@ __global__ void __launch_bounds__(TcCfg::kThreads, 1)
         }
 
         float m_ref = -INFINITY;  // running reference max of head hrow (log2 units)
-        float l_acc = 0.f;        // sum of P over this thread's tiles, relative to m_ref
+        float l_acc = 0.f;        // sum of P of head hrow relative to m_ref (lanes 0-15; 0 elsewhere)
         const uint32_t t_lane = tmem + ((uint32_t)(32 * q4) << 16);
 
         for (int pr = 0; pr < n_pairs; ++pr) {
-            const int t = 2 * pr + half;
-            const bool exists = t < n_tiles;
+            const int t0 = 2 * pr;
+            const bool has1 = t0 + 1 < n_tiles;
             mbar_wait(&s_full[pr & 1], (pr >> 1) & 1, dead);
             tc_fence_after();
-            uint32_t sr[32];
-            tmem_ld32(t_lane + C::kSCol + 32 * (pr & 1), sr);
+            // S of the pair: lanes 0-15 hold head hrow, columns 0-31 tile t0,
+            // 32-63 tile t0+1 (lanes 16-31 read unused TMEM lanes, ignored)
+            uint32_t s0[32], s1[32];
+            tmem_ld32(t_lane + C::kSCol + 64 * (pr & 1), s0);
+            tmem_ld32(t_lane + C::kSCol + 64 * (pr & 1) + 32, s1);
             tmem_ld_wait();
-            uint32_t vmask = 0;
-            if (exists) {
-                mbar_wait(&kv_full[t % C::kStages], (t / C::kStages) & 1, dead);
-                vmask = hdr[t % C::kStages];
+            mbar_wait(&kv_full[t0 % C::kStages], (t0 / C::kStages) & 1, dead);
+            const uint32_t vm0 = hdr[t0 % C::kStages];
+            uint32_t vm1 = 0;
+            if (has1) {
+                mbar_wait(&kv_full[(t0 + 1) % C::kStages], ((t0 + 1) / C::kStages) & 1, dead);
+                vm1 = hdr[(t0 + 1) % C::kStages];
             }
-            float sv[32];
+            const bool owner = half == 0;  // lanes 0-15 run the softmax of head hrow
+            // scores in log2 units, padding (and an absent second tile) -> -inf;
+            // selects, not branches
             float mt = -INFINITY;
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
-                sv[j] = ((vmask >> j) & 1u) ? __uint_as_float(sr[j]) * p.scale_log2 : -INFINITY;
-                mt = fmaxf(mt, sv[j]);
+                const float x0 = ((vm0 >> j) & 1u) ? __uint_as_float(s0[j]) * p.scale_log2 : -INFINITY;
+                const float x1 = ((vm1 >> j) & 1u) ? __uint_as_float(s1[j]) * p.scale_log2 : -INFINITY;
+                s0[j] = __float_as_uint(x0);
+                s1[j] = __float_as_uint(x1);
+                mt = fmaxf(mt, fmaxf(x0, x1));
             }
-            mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 16));
+            if (!owner) mt = -INFINITY;
             float alpha = 1.f;
-            if (mt > m_ref + C::kTau) {
-                alpha = (m_ref == -INFINITY) ? 0.f : exp2f(m_ref - mt);
+            if (owner && mt > m_ref + C::kTau) {
+                alpha = (m_ref == -INFINITY) ? 0.f : fast_exp2(m_ref - mt);
                 m_ref = mt;
             }
+            alpha = __shfl_sync(0xffffffffu, alpha, lane & 15);  // lane l+16 rescales O[:, 256:512]
             // Rescale this thread's half row of O when its head's max jumped
             // (warp-collective TMEM access; alpha = 1 for the other threads).
             const bool need = (pr >= 1) && (alpha != 1.f);
@@ -384,23 +403,30 @@ __global__ void __launch_bounds__(TcCfg::kThreads, 1)
                 }
                 tmem_st_wait();
             }
-            const float mu = (m_ref == -INFINITY) ? 0.f : m_ref;
-            float ps = 0.f;
-            uint32_t pk[16];
+            if (owner) {
+                const float mu = (m_ref == -INFINITY) ? 0.f : m_ref;
+                float ps = 0.f;
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                const float a0 = exp2f(sv[2 * j] - mu), a1 = exp2f(sv[2 * j + 1] - mu);
-                ps += a0 + a1;
-                pk[j] = pack_bf16x2(a0, a1);
-            }
-            l_acc = l_acc * alpha + ps;
-            if (exists) {
-                // P tile (64 heads x 32 rows, bf16) in the spent k_pe box, K-major 64B swizzle
-                uint8_t *pbase = smem + C::kOffKV + (t % C::kStages) * C::kStageBytes + 8 * C::kBoxBytes;
+                for (int h = 0; h < 2; ++h) {
+                    uint32_t pk[16];
 #pragma unroll
-                for (int c = 0; c < 4; ++c)
-                    *reinterpret_cast<uint4 *>(pbase + hrow * 64 + ((c ^ ((hrow >> 1) & 3)) << 4)) =
-                        make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+                    for (int j = 0; j < 16; ++j) {
+                        const uint32_t r0 = h ? s1[2 * j] : s0[2 * j], r1 = h ? s1[2 * j + 1] : s0[2 * j + 1];
+                        const float a0 = fast_exp2(__uint_as_float(r0) - mu);  // exp2(-inf) = 0
+                        const float a1 = fast_exp2(__uint_as_float(r1) - mu);
+                        ps += a0 + a1;
+                        pk[j] = pack_bf16x2(a0, a1);
+                    }
+                    if (h == 1 && !has1) continue;
+                    // P tile (64 heads x 32 rows, bf16) in the tile's spent k_pe box,
+                    // K-major 64B swizzle
+                    uint8_t *pbase = smem + C::kOffKV + C::tile_off((t0 + h) % C::kStages) + 8 * C::kBoxStride;
+#pragma unroll
+                    for (int c = 0; c < 4; ++c)
+                        *reinterpret_cast<uint4 *>(pbase + hrow * 64 + ((c ^ ((hrow >> 1) & 3)) << 4)) =
+                            make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+                }
+                l_acc = l_acc * alpha + ps;
             }
             fence_proxy_async_smem();
             tc_fence_before();
