@@ -65,6 +65,11 @@ int current_device_sms() {
     return n;
 }
 
+// Kernel choice of launch_partial, as the schedule needs it.
+bool uses_latency_kernel(int H, int K, int kc, int pt_stride) {
+    return H <= 32 && K > 0 && kc <= 32 && pt_stride <= smla::kSmallMaxPt;
+}
+
 // NSPLIT model ("The Occupancy Hypothesis ...", sections "The Occupancy
 // Insight" and "The Broader Context": more blocks in flight hide memory
 // latency, and the best NSPLIT depends on SMs, heads, batch and query
@@ -76,6 +81,7 @@ int current_device_sms() {
 constexpr double kFixedRows = 48.0;     // per-CTA latency: launch, Q load, index chase
 constexpr double kScratchWeight = 0.5;  // partials mostly stay in L2
 constexpr int kMinRowsPerSplit = 32;
+constexpr double kBalancedMargin = 0.15;
 constexpr double kPartialBytesPerHead = (smla::kDc + 2) * 4.0;
 
 int nsplit_model(int B, int T, int H, int K, int sm_count) {
@@ -99,6 +105,20 @@ int nsplit_model(int B, int T, int H, int K, int sm_count) {
             best = t;
             best_s = s;
         }
+    }
+    // Balanced schedule (see use_balanced): one full wave of `slots` CTAs with
+    // equal rows, about base + slots pieces in all (each costs kFixedRows and
+    // writes one partial per head).  A CTA that moves from one token to the
+    // next stalls its pipeline, which the model does not see (measured: 5-15%
+    // of the pass), so the balanced choice must win by kBalancedMargin.
+    const long long s_bal = (long long)std::ceil((double)slots / (double)base) + 1;
+    const double units = (double)base * ((K + 31) / 32);
+    if (H <= 32 && s_bal >= 2 && s_bal <= s_max && units >= 4.0 * slots &&
+        !uses_latency_kernel(H, K, (K + (int)s_bal - 1) / (int)s_bal, 0)) {
+        const double pieces = (double)base + slots;
+        double t = kFixedRows * pieces / slots + units * 32.0 / slots;
+        t += kScratchWeight * pieces * H * kPartialBytesPerHead * 2.0 / smla::kRowBytes / slots;
+        if (t < best * (1.0 - kBalancedMargin)) best_s = (int)s_bal;
     }
     return best_s;
 }
@@ -204,7 +224,7 @@ smla_status launch_small(const PartialParams &p, int grid, cudaStream_t st) {
 
 template <bool DIRECT>
 smla_status launch_partial(const PartialParams &p, cudaStream_t st) {
-    const long long grid = (long long)p.B * p.T * p.nsplit;
+    const long long grid = p.balanced ? (long long)p.grid : (long long)p.B * p.T * p.nsplit;
     if (grid > INT_MAX) return SMLA_ERR_INVALID_ARG;
     // one tile per split: the latency path (see smla_partial_small_kernel)
     if (p.H <= 32 && p.K > 0 && p.kc <= 32 && p.pt_stride <= smla::kSmallMaxPt) {
@@ -234,6 +254,36 @@ PartialParams make_params(const void *q, const void *kv_cache, int64_t num_pages
     p.nsplit = nsplit;
     p.kc = (K + nsplit - 1) / nsplit;
     return p;
+}
+
+// Partial CTAs resident per SM for the pipelined kernels (their launch bounds).
+int resident_per_sm(int H) {
+    if (H > 32) return 1;  // tcgen05 kernel: one CTA per SM (shared memory, TMEM)
+    if (H > 16) return smla::MmaCfg<2, 32, 4>::kMinBlocks;
+    return smla::MmaCfg<1, SMLA_MMA_TILE_ROWS, SMLA_MMA_STAGES>::kMinBlocks;
+}
+
+// Balanced schedule ("The Occupancy Hypothesis ...", section "The Occupancy
+// Insight": the grid should keep every SM busy).  With S slots per token the
+// equal split launches B*T*S CTAs, which leaves a partly filled last wave
+// whenever B*T*S is not a multiple of the resident CTAs R.  The balanced
+// schedule launches exactly R CTAs, each taking an equal share of the
+// flattened (token, 32-row tile) space; a token then spans at most
+// ceil(R / (B*T)) + 1 CTAs, each writing one of its S slots.  Used when it
+// fits in S slots and each CTA gets at least 4 tiles.  The tcgen05 kernel
+// (H > 32) keeps equal splits.
+bool use_balanced(int B, int T, int H, int K, int nsplit, int pt_stride, int sms, int *grid) {
+    if (nsplit < 2 || K <= 0 || H > 32) return false;
+    const int kc = (K + nsplit - 1) / nsplit;
+    if (uses_latency_kernel(H, K, kc, pt_stride)) return false;
+    const long long bt = (long long)B * T;
+    const long long resident = (long long)sms * resident_per_sm(H);
+    const long long units = bt * ((K + 31) / 32);
+    if (bt * nsplit <= resident) return false;             // equal splits fit one wave
+    if ((long long)(nsplit - 1) * bt < resident) return false;  // a token could need > S slots
+    if (units < 4 * resident) return false;
+    *grid = (int)resident;
+    return true;
 }
 
 smla_status launch_combine(const float *part_o, const float *part_m, const float *part_lse, int B,
@@ -381,6 +431,13 @@ smla_status smla_decode(const void *q, const void *kv_cache, int64_t num_pages,
     p.part_o = reinterpret_cast<float *>(ws);
     p.part_m = reinterpret_cast<float *>(ws + off_m);
     p.part_lse = reinterpret_cast<float *>(ws + off_l);
+    int grid = 0;
+    if (use_balanced(B, T, H, K, nsplit, pt_stride, current_device_sms(), &grid)) {
+        p.balanced = 1;
+        p.grid = grid;
+        p.tpt = (K + 31) / 32;
+        p.n_units = (long long)B * T * p.tpt;
+    }
     st = launch_partial<false>(p, s);
     if (st != SMLA_OK) return st;
     return launch_combine(p.part_o, p.part_m, p.part_lse, B, T, H, nsplit, o, lse, s);

@@ -6,6 +6,8 @@
 // (b, t, h), with m_s the reference point of split s and lse_s its log-sum-exp:
 //   M = max_s m_s,  L = sum_s exp(lse_s - M),
 //   o = sum_s exp(m_s - M) O_s / L,  lse = M + ln L;  every split empty: 0, -inf.
+// A split with m_s = -inf is empty and its O_s is never used (the balanced
+// schedule of the whole decode leaves such slots unwritten).
 //
 // One 512-thread CTA per (b, t, h): 4 groups of 128 threads, thread c of a
 // group owning output columns 4c..4c+3.  Splits are taken in batches of
@@ -84,11 +86,14 @@ __global__ void __launch_bounds__(kCombineThreads)
         L *= r;
 #pragma unroll
         for (int k = 0; k < kCombineDepth; ++k) {
-            const float w = (mv[k] == -INFINITY) ? 0.f : expf(mv[k] - Mn);
-            acc.x = fmaf(w, v[k].x, acc.x);
-            acc.y = fmaf(w, v[k].y, acc.y);
-            acc.z = fmaf(w, v[k].z, acc.z);
-            acc.w = fmaf(w, v[k].w, acc.w);
+            // An empty slot (m = -inf) contributes nothing, whatever its part_o
+            // holds (selects, so that stale bits there never reach acc).
+            const bool on = mv[k] != -INFINITY;
+            const float w = on ? expf(mv[k] - Mn) : 0.f;
+            acc.x = on ? fmaf(w, v[k].x, acc.x) : acc.x;
+            acc.y = on ? fmaf(w, v[k].y, acc.y) : acc.y;
+            acc.z = on ? fmaf(w, v[k].z, acc.z) : acc.z;
+            acc.w = on ? fmaf(w, v[k].w, acc.w) : acc.w;
             if (lv[k] != -INFINITY) L += expf(lv[k] - Mn);
         }
         M = Mn;
@@ -168,13 +173,14 @@ __global__ void __launch_bounds__(32 * kCombineWarpUnits)
 #pragma unroll
     for (int s = 0; s < SMAX; ++s) {
         if (lv[s] != -INFINITY) L += expf(lv[s] - M);
-        const float w = (mv[s] == -INFINITY) ? 0.f : expf(mv[s] - M);
+        const bool on = mv[s] != -INFINITY;  // empty slot: part_o is not used
+        const float w = on ? expf(mv[s] - M) : 0.f;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-            acc[j].x = fmaf(w, v[s][j].x, acc[j].x);
-            acc[j].y = fmaf(w, v[s][j].y, acc[j].y);
-            acc[j].z = fmaf(w, v[s][j].z, acc[j].z);
-            acc[j].w = fmaf(w, v[s][j].w, acc[j].w);
+            acc[j].x = on ? fmaf(w, v[s][j].x, acc[j].x) : acc[j].x;
+            acc[j].y = on ? fmaf(w, v[s][j].y, acc[j].y) : acc[j].y;
+            acc[j].z = on ? fmaf(w, v[s][j].z, acc[j].z) : acc[j].z;
+            acc[j].w = on ? fmaf(w, v[s][j].w, acc[j].w) : acc[j].w;
         }
     }
     const float inv = 1.f / L;

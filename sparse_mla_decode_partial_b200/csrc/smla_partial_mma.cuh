@@ -65,9 +65,77 @@ struct PartialParams {
     float *part_o;                // [B, T, H, S, 512]
     float *part_m;                // [B, T, H, S]
     float *part_lse;              // [B, T, H, S]
-    __nv_bfloat16 *o;             // direct / single-launch mode: [B, T, H, 512]
-    float *lse;                   // direct / single-launch mode: [B, T, H]
+    __nv_bfloat16 *o;             // direct mode (nsplit = 1): [B, T, H, 512]
+    float *lse;                   // direct mode (nsplit = 1): [B, T, H]
+    // Balanced schedule (pipelined kernels, whole decode only): CTA c of
+    // `grid` takes tiles [c U / grid, (c+1) U / grid) of the flattened
+    // (query token, 32-row tile) space, U = B T tpt.  0 = equal splits of kc.
+    int balanced;
+    int tpt;                      // 32-row tiles per query token, ceil(K / 32)
+    int grid;
+    long long n_units;            // U
 };
+
+// One piece of a CTA's work: rows [j0, j1) of query token bt, written as
+// partial slot `slot`.  `last`: the piece ends the token (balanced schedule),
+// so its CTA also marks the token's unused slots empty.
+struct WorkItem {
+    int bt, j0, j1, slot;
+    bool last;
+};
+
+// CTA that owns flattened tile u under the balanced schedule: the c with
+// floor(c U / G) <= u < floor((c+1) U / G).
+__device__ __forceinline__ int owner_cta(const PartialParams &p, long long u) {
+    return (int)(((u + 1) * p.grid - 1) / p.n_units);
+}
+
+// Iterates the items of CTA c: start with u = item_begin(p, c).  Equal splits
+// give one item, split s = c % nsplit of token c / nsplit.
+__device__ __forceinline__ long long item_begin(const PartialParams &p, int c) {
+    return p.balanced ? (long long)c * p.n_units / p.grid : 0;
+}
+__device__ __forceinline__ bool next_item(const PartialParams &p, int c, long long &u, WorkItem &w) {
+    if (!p.balanced) {
+        if (u != 0) return false;
+        u = 1;
+        const int s = c % p.nsplit;
+        const long long j0 = (long long)s * p.kc;
+        w.bt = c / p.nsplit;
+        w.j0 = (int)(j0 < p.K ? j0 : p.K);
+        w.j1 = (int)(j0 + p.kc < p.K ? j0 + p.kc : p.K);
+        w.slot = s;
+        w.last = false;
+        return true;
+    }
+    const long long u_end = (long long)(c + 1) * p.n_units / p.grid;
+    if (u >= u_end) return false;
+    const long long bt = u / p.tpt;
+    const long long tok_end = (bt + 1) * p.tpt;
+    const long long ue = u_end < tok_end ? u_end : tok_end;
+    w.bt = (int)bt;
+    w.j0 = (int)((u - bt * p.tpt) * 32);
+    const long long j1 = (ue - bt * p.tpt) * 32;
+    w.j1 = (int)(j1 < p.K ? j1 : p.K);
+    w.slot = c - owner_cta(p, bt * p.tpt);
+    w.last = ue == tok_end;
+    u = ue;
+    return true;
+}
+
+// Balanced schedule: the CTA holding a token's last rows marks the slots no
+// CTA wrote for that token (slot + 1 .. nsplit - 1) as empty, m = lse = -inf;
+// the combine gives them weight 0 without reading their part_o.
+__device__ __forceinline__ void mark_unused_slots(const PartialParams &p, const WorkItem &w, int tid,
+                                                  int nthreads) {
+    const int spare = p.nsplit - 1 - w.slot;
+    if (!w.last || spare <= 0) return;
+    for (int i = tid; i < p.H * spare; i += nthreads) {
+        const size_t k = ((size_t)w.bt * p.H + i / spare) * p.nsplit + w.slot + 1 + i % spare;
+        p.part_m[k] = -INFINITY;
+        p.part_lse[k] = -INFINITY;
+    }
+}
 
 template <int HG, int NT, int NSTAGE>
 struct MmaCfg {
@@ -294,18 +362,12 @@ template <int HG, int NT, int NSTAGE, bool DIRECT>
 __global__ void __launch_bounds__(MmaCfg<HG, NT, NSTAGE>::kThreads, MmaCfg<HG, NT, NSTAGE>::kMinBlocks)
     smla_partial_mma_kernel(const PartialParams p) {
     using C = MmaCfg<HG, NT, NSTAGE>;
+    static_assert(NT == 32, "the balanced schedule counts 32-row tiles");
     extern __shared__ __align__(128) uint8_t smem[];
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int unit = blockIdx.x;  // (b * T + t) * S + s
-    const int s = unit % p.nsplit;
-    const int bt = unit / p.nsplit;
-    const int b = bt / p.T;
-    const long long j0l = (long long)s * p.kc;
-    const int j0 = (int)(j0l < p.K ? j0l : p.K);
-    const int j1 = (int)((long long)j0 + p.kc < p.K ? (long long)j0 + p.kc : p.K);
-    const int n_tiles = (j1 - j0 + NT - 1) / NT;
+    const int cta = blockIdx.x;
     bool dead = false;  // set once a bounded wait of this thread has timed out
 
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::kOffBar);
@@ -326,104 +388,121 @@ __global__ void __launch_bounds__(MmaCfg<HG, NT, NSTAGE>::kThreads, MmaCfg<HG, N
 
     if (warp == C::kComputeWarps) {
         // ============================================================ producer
-        const int *idx_bt = p.idx + (size_t)bt * p.K + j0;
-        const int *pt_b = p.page_table + (size_t)b * p.pt_stride;
         const long long max_pos = (long long)p.pt_stride * kPage;
         const uint64_t policy = l2_policy_evict_first();
         int *rows_s = reinterpret_cast<int *>(smem + C::kOffRows);
         constexpr int kResolveBatch = HG <= 2 ? 32 : 16;  // loads in flight per lane
-        const int len = j1 - j0;
-        int it = 0;  // tile counter over the whole split
-        for (int base = 0; base < len; base += kResolveChunk) {
-            const int n = min(kResolveChunk, len - base);
-            // Resolve the whole chunk before the first copy: index loads, then
-            // page-table loads, each batch of 32 per lane in flight at once.
-            for (int b0 = 0; b0 < n; b0 += 32 * kResolveBatch) {
-                int iv[kResolveBatch];
+        int it = 0;  // tile counter over all of this CTA's items (ring position)
+        long long u = item_begin(p, cta);
+        WorkItem w;
+        while (next_item(p, cta, u, w)) {
+            const int *idx_bt = p.idx + (size_t)w.bt * p.K + w.j0;
+            const int *pt_b = p.page_table + (size_t)(w.bt / p.T) * p.pt_stride;
+            const int len = w.j1 - w.j0;
+            for (int base = 0; base < len; base += kResolveChunk) {
+                const int n = min(kResolveChunk, len - base);
+                __syncwarp();  // rows_s is rewritten below
+                // Resolve the whole chunk before the first copy: index loads, then
+                // page-table loads, each batch of 32 per lane in flight at once.
+                for (int b0 = 0; b0 < n; b0 += 32 * kResolveBatch) {
+                    int iv[kResolveBatch];
 #pragma unroll
-                for (int k = 0; k < kResolveBatch; ++k) {
-                    const int j = b0 + k * 32 + lane;
-                    iv[k] = (j < n) ? __ldg(idx_bt + base + j) : -1;
-                }
-                int pg[kResolveBatch];
+                    for (int k = 0; k < kResolveBatch; ++k) {
+                        const int j = b0 + k * 32 + lane;
+                        iv[k] = (j < n) ? __ldg(idx_bt + base + j) : -1;
+                    }
+                    int pg[kResolveBatch];
 #pragma unroll
-                for (int k = 0; k < kResolveBatch; ++k) {
-                    const int i = iv[k];
-                    pg[k] = (i >= 0 && (long long)i < max_pos) ? __ldg(pt_b + (i >> 6)) : -1;
-                }
+                    for (int k = 0; k < kResolveBatch; ++k) {
+                        const int i = iv[k];
+                        pg[k] = (i >= 0 && (long long)i < max_pos) ? __ldg(pt_b + (i >> 6)) : -1;
+                    }
 #pragma unroll
-                for (int k = 0; k < kResolveBatch; ++k) {
-                    const int j = b0 + k * 32 + lane;
-                    const int i = iv[k];
-                    int row = -1;
-                    if (i != -1) {
-                        const bool ok = (i >= 0) && ((long long)i < max_pos) && (pg[k] >= 0) &&
-                                        ((long long)pg[k] < p.num_pages);
-                        if (ok) {
-                            row = pg[k] * kPage + (i & (kPage - 1));
-                        } else if (j < n) {
-                            atomicOr(&g_status_flags, kFlagIndexRange);
-                            atomicAdd(&g_bad_index_count, 1ull);
+                    for (int k = 0; k < kResolveBatch; ++k) {
+                        const int j = b0 + k * 32 + lane;
+                        const int i = iv[k];
+                        int row = -1;
+                        if (i != -1) {
+                            const bool ok = (i >= 0) && ((long long)i < max_pos) && (pg[k] >= 0) &&
+                                            ((long long)pg[k] < p.num_pages);
+                            if (ok) {
+                                row = pg[k] * kPage + (i & (kPage - 1));
+                            } else if (j < n) {
+                                atomicOr(&g_status_flags, kFlagIndexRange);
+                                atomicAdd(&g_bad_index_count, 1ull);
+                            }
                         }
+                        if (j < n) rows_s[j] = row;
                     }
-                    if (j < n) rows_s[j] = row;
                 }
-            }
-            __syncwarp();
-            // Issue one bulk copy per row (or per padding slot, from the zero row).
-            const int chunk_tiles = (n + NT - 1) / NT;
-            for (int t = 0; t < chunk_tiles; ++t, ++it) {
-                const int stage = it % NSTAGE;
-                if (it >= NSTAGE) mbar_wait(&empty[stage], ((it / NSTAGE) - 1) & 1, dead);
-                if (lane == 0) mbar_expect_tx(&full[stage], (uint32_t)(NT * kRowBytes));
                 __syncwarp();
-                uint8_t *dst = smem + C::kOffKV + stage * C::kStageBytes;
-                uint64_t mask = 0;
+                // Issue one bulk copy per row (or per padding slot, from the zero row).
+                const int chunk_tiles = (n + NT - 1) / NT;
+                for (int t = 0; t < chunk_tiles; ++t, ++it) {
+                    const int stage = it % NSTAGE;
+                    if (it >= NSTAGE) mbar_wait(&empty[stage], ((it / NSTAGE) - 1) & 1, dead);
+                    if (lane == 0) mbar_expect_tx(&full[stage], (uint32_t)(NT * kRowBytes));
+                    __syncwarp();
+                    uint8_t *dst = smem + C::kOffKV + stage * C::kStageBytes;
+                    uint64_t mask = 0;
 #pragma unroll
-                for (int k = 0; k < (NT + 31) / 32; ++k) {
-                    const int slot = k * 32 + lane;
-                    const int r = t * NT + slot;
-                    const int row = (slot < NT && r < n) ? rows_s[r] : -1;
-                    uint8_t *d = dst + slot * kSmemRowBytes;
-                    if (slot < NT) {
-                        if (row >= 0)
-                            bulk_g2s_hint(d, reinterpret_cast<const uint8_t *>(p.cache) +
-                                                 (size_t)row * kRowBytes,
-                                          kRowBytes, &full[stage], policy);
-                        else
-                            bulk_g2s(d, g_zero_row, kRowBytes, &full[stage]);
+                    for (int k = 0; k < (NT + 31) / 32; ++k) {
+                        const int slot = k * 32 + lane;
+                        const int r = t * NT + slot;
+                        const int row = (slot < NT && r < n) ? rows_s[r] : -1;
+                        uint8_t *d = dst + slot * kSmemRowBytes;
+                        if (slot < NT) {
+                            if (row >= 0)
+                                bulk_g2s_hint(d, reinterpret_cast<const uint8_t *>(p.cache) +
+                                                     (size_t)row * kRowBytes,
+                                              kRowBytes, &full[stage], policy);
+                            else
+                                bulk_g2s(d, g_zero_row, kRowBytes, &full[stage]);
+                        }
+                        mask |= (uint64_t)__ballot_sync(0xffffffffu, row >= 0) << (32 * k);
                     }
-                    mask |= (uint64_t)__ballot_sync(0xffffffffu, row >= 0) << (32 * k);
-                }
-                if (lane == 0) {
-                    hdr[stage] = mask;
-                    mbar_arrive(&full[stage]);  // release: hdr is visible to the waiters
+                    if (lane == 0) {
+                        hdr[stage] = mask;
+                        mbar_arrive(&full[stage]);  // release: hdr is visible to the waiters
+                    }
                 }
             }
-            __syncwarp();  // rows_s is rewritten by the next chunk
         }
         // Copies still in flight must land before the CTA may exit.
-        for (int it = (n_tiles > NSTAGE ? n_tiles - NSTAGE : 0); it < n_tiles; ++it)
-            mbar_wait(&full[it % NSTAGE], (it / NSTAGE) & 1, dead);
+        for (int k = (it > NSTAGE ? it - NSTAGE : 0); k < it; ++k)
+            mbar_wait(&full[k % NSTAGE], (k / NSTAGE) & 1, dead);
         return;
     }
 
     // ================================================================ consumers
-    MmaConsumer<NT, HG> cons;
-    cons.init(warp, lane);
-    cons.load_q(smem + C::kOffQ, p, bt);
-    // The Q region is reused for the split-k score exchange from here on.
-    named_bar_sync(1 + HG, 128 * HG);
-    float *spart = reinterpret_cast<float *>(smem + C::kOffQ) + cons.g * 2 * 4 * 16 * C::kSRow;
-    for (int it = 0; it < n_tiles; ++it) {
-        const int stage = it % NSTAGE;
-        mbar_wait(&full[stage], (it / NSTAGE) & 1, dead);
-        cons.tile(smem_addr(smem + C::kOffKV + stage * C::kStageBytes), hdr[stage],
-                  spart + (it & 1) * 4 * 16 * C::kSRow, p.scale_log2);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[stage]);
+    // The Q region doubles as the split-k score exchange of every head group
+    // (a group's exchange buffer overlaps the next group's Q rows), so Q is
+    // (re)written only when all consumer warps are past their last exchange.
+    float *spart_base = reinterpret_cast<float *>(smem + C::kOffQ);
+    int it = 0;
+    long long u = item_begin(p, cta);
+    WorkItem w;
+    bool first = true;
+    while (next_item(p, cta, u, w)) {
+        MmaConsumer<NT, HG> cons;
+        cons.init(warp, lane);
+        if (!first) named_bar_sync(1 + HG, 128 * HG);
+        first = false;
+        cons.load_q(smem + C::kOffQ, p, w.bt);
+        named_bar_sync(1 + HG, 128 * HG);  // Q is in registers: the region is free
+        float *spart = spart_base + cons.g * 2 * 4 * 16 * C::kSRow;
+        const int n_tiles = (w.j1 - w.j0 + NT - 1) / NT;
+        for (int t = 0; t < n_tiles; ++t, ++it) {
+            const int stage = it % NSTAGE;
+            mbar_wait(&full[stage], (it / NSTAGE) & 1, dead);
+            cons.tile(smem_addr(smem + C::kOffKV + stage * C::kStageBytes), hdr[stage],
+                      spart + (it & 1) * 4 * 16 * C::kSRow, p.scale_log2);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[stage]);
+        }
+        cons.template epilogue<DIRECT>(p, w.bt, w.slot);
+        if (!DIRECT && warp < 4) mark_unused_slots(p, w, threadIdx.x, 128);
     }
-    cons.template epilogue<DIRECT>(p, bt, s);
 }
 
 // ----------------------------------------------------------------------------

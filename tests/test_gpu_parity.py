@@ -289,3 +289,65 @@ def test_one_tile_splits_many_waves():
     o_ref, lse_ref, _ = oracle_decode(w, sample)
     idx = torch.tensor([b for b, _ in sample])
     check_o_lse(o[idx, 0], lse[idx, 0], o_ref, lse_ref, "many waves")
+
+
+# ------------------------------------------------------------------ balanced schedule
+# The whole decode may cover a token's top-k axis with up to nsplit pieces of
+# unequal length, one full wave of CTAs with equal work each.  These shapes
+# take that path on a 148-SM B200 (checked below with the library's rule).
+def balanced_taken(B, T, H, K, S, sms):
+    resident = sms * (2 if H <= 16 else 1)
+    bt, units = B * T, B * T * -(-K // 32)
+    return (S >= 2 and H <= 32 and not (-(-K // S) <= 32) and bt * S > resident
+            and (S - 1) * bt >= resident and units >= 4 * resident)
+
+
+def sms():
+    return torch.cuda.get_device_properties(0).multi_processor_count
+
+
+@pytest.mark.parametrize("B,T,H,K,S", [(64, 1, 16, 2048, 6), (64, 1, 16, 2048, 40),
+                                       (40, 1, 24, 1000, 8), (20, 3, 16, 777, 16),
+                                       (128, 1, 16, 2048, 4)])
+def test_balanced_schedule(B, T, H, K, S):
+    w = workloads.make_workload("balanced", B=B, T=T, H=H, K=K, ctx_lens=[6000] * B, seed=B + K)
+    S_used = S or binding.choose_nsplit(B, T, H, K, 0)
+    assert balanced_taken(B, T, H, K, S_used, sms()), "shape does not exercise the balanced path"
+    o, lse = run_decode(w, S)
+    sample = sample_bt(w, 6, seed=K)
+    o_ref, lse_ref, _ = oracle_decode(w, sample)
+    bi = [b for b, _ in sample]
+    ti = [t for _, t in sample]
+    check_o_lse(o[bi, ti], lse[bi, ti], o_ref, lse_ref, f"balanced B={B} T={T} H={H} K={K} S={S}")
+    assert torch.isfinite(o.float()).all() and torch.isfinite(lse).all()
+
+
+def test_balanced_schedule_ignores_stale_workspace():
+    # slots no CTA writes keep whatever the workspace held: NaN bit patterns
+    # (0xFF bytes) there must not reach o
+    B, T, H, K, S = 64, 1, 16, 2048, 9
+    w = workloads.make_workload("balanced_nan", B=B, T=T, H=H, K=K, ctx_lens=[5000] * B, seed=77)
+    assert balanced_taken(B, T, H, K, S, sms())
+    wd = w.to(DEV)
+    ws = torch.full((binding.workspace_bytes(B, T, H, S),), 0xFF, dtype=torch.uint8, device=DEV)
+    o, lse = binding.decode(wd.q, wd.cache, wd.page_table, wd.idx, w.scale, S, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.isfinite(o.float()).all() and torch.isfinite(lse).all()
+    sample = [(0, 0), (31, 0), (63, 0)]
+    o_ref, lse_ref, _ = oracle_decode(w, sample)
+    bi = [b for b, _ in sample]
+    check_o_lse(o[bi, 0], lse[bi, 0], o_ref, lse_ref, "balanced, 0xFF workspace")
+
+
+def test_balanced_schedule_with_padding_and_short_contexts():
+    # tokens whose whole top-k is padding, or mostly padding, spread over pieces
+    B, H, K, S = 48, 16, 2048, 8
+    ctx = [100 if b % 5 == 0 else (1500 if b % 5 == 1 else 9000) for b in range(B)]
+    w = workloads.make_workload("balanced_pad", B=B, T=1, H=H, K=K, ctx_lens=ctx, seed=5)
+    w.idx[0::7, 0, :] = -1                       # some tokens select nothing at all
+    assert balanced_taken(B, 1, H, K, S, sms())
+    o, lse = run_decode(w, S)
+    sample = [(0, 0), (1, 0), (5, 0), (7, 0), (14, 0), (46, 0), (47, 0)]
+    o_ref, lse_ref, _ = oracle_decode(w, sample)
+    bi = [b for b, _ in sample]
+    check_o_lse(o[bi, 0], lse[bi, 0], o_ref, lse_ref, "balanced with padding")

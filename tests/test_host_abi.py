@@ -120,12 +120,23 @@ def model(B, T, H, K, sms):
             t += 0.5 * ctas * H * (514 * 4.0) * 2.0 / 1152 / slots
         if best is None or t < best * (1 - 1e-9):
             best, best_s = t, s
+    # balanced schedule: one full wave of `slots` CTAs, base + slots pieces
+    s_bal = math.ceil(slots / base) + 1
+    units = base * -(-K // 32)
+    latency_kernel = H <= 32 and math.ceil(K / s_bal) <= 32
+    if H <= 32 and 2 <= s_bal <= s_max and units >= 4 * slots and not latency_kernel:
+        pieces = base + slots
+        t = 48.0 * pieces / slots + units * 32.0 / slots
+        t += 0.5 * pieces * H * (514 * 4.0) * 2.0 / 1152 / slots
+        if t < best * (1 - 0.15):
+            best_s = s_bal
     return best_s
 
 
 @pytest.mark.parametrize("shape", [(1, 1, 16, 2048), (1, 9, 8, 2048), (64, 1, 16, 2048),
                                    (60, 1, 64, 2048), (1, 1, 8, 256), (4, 1, 16, 100),
-                                   (128, 1, 16, 2048), (1, 1, 16, 31)])
+                                   (128, 1, 16, 2048), (1, 1, 16, 31), (64, 1, 24, 2048),
+                                   (8, 1, 16, 2048), (20, 3, 16, 4096)])
 def test_nsplit_heuristic_matches_model(lib, shape, monkeypatch):
     monkeypatch.delenv("SMLA_NSPLIT", raising=False)
     B, T, H, K = shape
@@ -140,6 +151,9 @@ def test_nsplit_heuristic_properties(lib, monkeypatch):
     for K in (1, 20, 33, 64, 65, 1000):
         s = binding.choose_nsplit(1, 1, 16, K, 148)
         assert s == 1 or math.ceil(K / s) >= 32 or s <= -(-K // 32)
+    # batched decode on mma.sync (2 CTAs per SM): 4 splits fill one wave well
+    # enough that the balanced schedule (6 slots) does not pay
+    assert binding.choose_nsplit(64, 1, 16, 2048, 148) == 4
     # a batch that already fills the GPU is not split
     assert binding.choose_nsplit(296, 1, 16, 2048, 148) == 1
     assert binding.choose_nsplit(148, 1, 64, 2048, 148) == 1
@@ -155,6 +169,47 @@ def test_nsplit_env_override(lib, monkeypatch):
     assert binding.choose_nsplit(64, 1, 16, 2048, 148) == 1024
     monkeypatch.setenv("SMLA_NSPLIT", "junk")
     assert binding.choose_nsplit(1, 1, 16, 2048, 148) == 64
+
+
+def balanced_items(B, T, K, grid):
+    """Work pieces of the balanced schedule, as the kernels enumerate them."""
+    tpt = -(-K // 32)
+    U = B * T * tpt
+    owner = lambda u: ((u + 1) * grid - 1) // U
+    out = []
+    for c in range(grid):
+        u, u_end = c * U // grid, (c + 1) * U // grid
+        while u < u_end:
+            bt = u // tpt
+            ue = min(u_end, (bt + 1) * tpt)
+            out.append((c, bt, (u - bt * tpt) * 32, min(K, (ue - bt * tpt) * 32),
+                        c - owner(bt * tpt), ue == (bt + 1) * tpt))
+            u = ue
+    return out
+
+
+@pytest.mark.parametrize("B,T,K,grid,S", [(64, 1, 2048, 296, 6), (60, 1, 2048, 148, 4),
+                                          (7, 3, 1000, 148, 9), (128, 1, 2048, 296, 4),
+                                          (5, 1, 33, 2, 2)])
+def test_balanced_schedule_covers_every_row_once(B, T, K, grid, S):
+    items = balanced_items(B, T, K, grid)
+    rows = {}
+    for c, bt, j0, j1, slot, last in items:
+        assert 0 <= slot < S and j0 < j1
+        for j in range(j0, j1):
+            assert (bt, j) not in rows
+            rows[(bt, j)] = slot
+    assert len(rows) == B * T * K
+    # per token: slots 0..n-1 in row order, exactly one piece marked last
+    for bt in range(B * T):
+        pieces = sorted((j0, slot, last) for c, b, j0, j1, slot, last in items if b == bt)
+        assert [sl for _, sl, _ in pieces] == list(range(len(pieces)))
+        assert [la for _, _, la in pieces] == [False] * (len(pieces) - 1) + [True]
+    # every CTA has the same number of tiles, +-1
+    per_cta = {}
+    for c, bt, j0, j1, slot, last in items:
+        per_cta[c] = per_cta.get(c, 0) + -(-(j1 - j0) // 32)
+    assert max(per_cta.values()) - min(per_cta.values()) <= 1 + (K % 32 != 0)
 
 
 def test_binding_refuses_cpu_tensors():
