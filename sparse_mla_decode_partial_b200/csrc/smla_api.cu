@@ -318,6 +318,12 @@ smla_status launch_combine(const float *part_o, const float *part_m, const float
         else
             e = cudaLaunchKernelEx(&cfg, smla::smla_combine_warp_kernel<8>, part_o, part_m, part_lse,
                                    nsplit, n, ob, lse);
+    } else if (units <= INT_MAX / 4) {
+        // four CTAs per (b, t, h), one per 128-column quarter
+        cfg.gridDim = dim3((unsigned)(units * 4));
+        cfg.blockDim = dim3(smla::kCombineThreads);
+        e = cudaLaunchKernelEx(&cfg, smla::smla_combine_quarter_kernel, part_o, part_m, part_lse,
+                               nsplit, ob, lse);
     } else {
         cfg.gridDim = dim3((unsigned)units);
         cfg.blockDim = dim3(smla::kCombineThreads);

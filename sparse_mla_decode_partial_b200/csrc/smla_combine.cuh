@@ -125,6 +125,109 @@ __global__ void __launch_bounds__(kCombineThreads)
     if (c == 0) lse[u] = M + logf(Lt);
 }
 
+// Column-quarter form (S > 8): one 512-thread CTA per (b, t, h) and 128 of
+// its 512 output columns, so a (b, t, h) is combined by four CTAs on four SMs
+// and each CTA pulls a quarter of the partial bytes.  16 groups of 32 threads;
+// thread c of a group owns columns 4c..4c+3 of the quarter; group g takes
+// splits g, g+16, ... (kCombineQDepth per batch, all loads of a batch in
+// flight at once).  Every quarter computes M and L itself (they are scalars).
+constexpr int kCombineQGroups = 16;
+constexpr int kCombineQDepth = 4;
+
+__global__ void __launch_bounds__(kCombineThreads)
+    smla_combine_quarter_kernel(const float *__restrict__ part_o, const float *__restrict__ part_m,
+                                const float *__restrict__ part_lse, int nsplit,
+                                __nv_bfloat16 *__restrict__ o, float *__restrict__ lse) {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    __shared__ float red_m[kCombineQGroups];
+    __shared__ float red_l[kCombineQGroups];
+    __shared__ float4 red_acc[kCombineQGroups - 1][32];
+
+    const size_t u = blockIdx.x >> 2;
+    const int quarter = blockIdx.x & 3;
+    const int g = threadIdx.x >> 5;
+    const int c = threadIdx.x & 31;
+    const float *pm = part_m + u * nsplit;
+    const float *pl = part_lse + u * nsplit;
+    const float4 *po = reinterpret_cast<const float4 *>(part_o + u * (size_t)nsplit * 512) + quarter * 32 + c;
+
+    float M = -INFINITY;  // running max over all batches (identical in every thread)
+    float L = 0.f;        // this group's sum of exp(lse_s - M)
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+
+    for (int s0 = 0; s0 < nsplit; s0 += kCombineQGroups * kCombineQDepth) {
+        float mv[kCombineQDepth], lv[kCombineQDepth];
+        float4 v[kCombineQDepth];
+#pragma unroll
+        for (int k = 0; k < kCombineQDepth; ++k) {
+            const int sp = s0 + g + kCombineQGroups * k;
+            if (sp < nsplit) {
+                mv[k] = __ldg(pm + sp);
+                lv[k] = __ldg(pl + sp);
+                v[k] = __ldg(po + (size_t)sp * 128);
+            } else {
+                mv[k] = -INFINITY;
+                lv[k] = -INFINITY;
+                v[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+        }
+        float mb = -INFINITY;
+#pragma unroll
+        for (int k = 0; k < kCombineQDepth; ++k) mb = fmaxf(mb, mv[k]);
+        if (c == 0) red_m[g] = mb;
+        __syncthreads();
+#pragma unroll
+        for (int k = 0; k < kCombineQGroups; ++k) mb = fmaxf(mb, red_m[k]);
+        __syncthreads();  // red_m is rewritten by the next batch
+        const float Mn = fmaxf(M, mb);
+        if (Mn == -INFINITY) continue;  // nothing valid so far
+        const float r = (M == -INFINITY) ? 0.f : expf(M - Mn);
+        acc.x *= r;
+        acc.y *= r;
+        acc.z *= r;
+        acc.w *= r;
+        L *= r;
+#pragma unroll
+        for (int k = 0; k < kCombineQDepth; ++k) {
+            const bool on = mv[k] != -INFINITY;  // empty slot: part_o is not used
+            const float w = on ? expf(mv[k] - Mn) : 0.f;
+            acc.x = on ? fmaf(w, v[k].x, acc.x) : acc.x;
+            acc.y = on ? fmaf(w, v[k].y, acc.y) : acc.y;
+            acc.z = on ? fmaf(w, v[k].z, acc.z) : acc.z;
+            acc.w = on ? fmaf(w, v[k].w, acc.w) : acc.w;
+            if (lv[k] != -INFINITY) L += expf(lv[k] - Mn);
+        }
+        M = Mn;
+    }
+
+    if (g > 0) red_acc[g - 1][c] = acc;
+    if (c == 0) red_l[g] = L;
+    __syncthreads();
+    if (g != 0) return;
+    uint2 *dst = reinterpret_cast<uint2 *>(o + u * 512 + quarter * 128) + c;
+    if (M == -INFINITY) {
+        *dst = make_uint2(0u, 0u);
+        if (quarter == 0 && c == 0) lse[u] = -INFINITY;
+        return;
+    }
+    float Lt = 0.f;
+#pragma unroll
+    for (int k = 0; k < kCombineQGroups; ++k) Lt += red_l[k];
+#pragma unroll
+    for (int k = 0; k < kCombineQGroups - 1; ++k) {
+        const float4 a = red_acc[k][c];
+        acc.x += a.x;
+        acc.y += a.y;
+        acc.z += a.z;
+        acc.w += a.w;
+    }
+    const float inv = 1.f / Lt;
+    __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+    __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+    *dst = make_uint2(*reinterpret_cast<uint32_t *>(&lo), *reinterpret_cast<uint32_t *>(&hi));
+    if (quarter == 0 && c == 0) lse[u] = M + logf(Lt);
+}
+
 constexpr int kCombineWarpUnits = 4;  // units (warps) per CTA of the warp form
 
 template <int SMAX>
