@@ -149,6 +149,13 @@ smla_status smla_lse_combine(const float *part_o, const float *part_m, const flo
  * S actually used (size it with the value smla_choose_nsplit returns), else
  * SMLA_ERR_WORKSPACE_TOO_SMALL.  With S = 1 the partial pass writes o and
  * lse directly and the workspace is not touched (it may then be NULL).
+ * S is the number of partial slots per query token.  When an equal split
+ * into S chunks would leave a partly filled last wave of CTAs (pipelined
+ * kernels, H <= 32), the call instead covers each token's top-k axis with at
+ * most S contiguous pieces of unequal length, so that exactly one wave of
+ * CTAs carries equal work; the LSE combine is exact for any partition, so
+ * only the rounding order differs from smla_decode_partial's equal split.
+ * The workspace contents on entry do not matter.
  *   o   bf16 [B, T, H, 512] device, 16-B aligned
  *   lse fp32 [B, T, H]      device
  */

@@ -1,8 +1,6 @@
 // smla_api.cu -- host side of the C ABI declared in include/smla.h: argument
 // checks, the NSPLIT heuristic, workspace carving and kernel launches.
 // Every entry point returns a status; nothing throws across the ABI.
-#include <cuda.h>
-#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <climits>
@@ -155,57 +153,12 @@ smla_status launch_mma(const PartialParams &p, int grid, cudaStream_t st) {
     return e == cudaSuccess ? SMLA_OK : cuda_fail(e);
 }
 
-// cuTensorMapEncodeTiled from the driver, without linking libcuda.
-PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void *ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-    });
-    return fn;
-}
-
-// 2-D view of the cache for the row gather: [num_pages * 64 rows, 576 bf16],
-// 1152-byte row stride, boxes of 64 columns x 1 row, 128-byte swizzle; rows
-// outside the tensor read as zeros.
-smla_status encode_cache_map(const PartialParams &p, CUtensorMap *out) {
-    auto enc = tensor_map_encoder();
-    if (enc == nullptr) {
-        std::snprintf(g_last_error, sizeof g_last_error, "cuTensorMapEncodeTiled unavailable");
-        return SMLA_ERR_CUDA;
-    }
-    cuuint64_t dims[2] = {(cuuint64_t)smla::kD, (cuuint64_t)p.num_pages * smla::kPage};
-    cuuint64_t strides[1] = {(cuuint64_t)smla::kRowBytes};
-    cuuint32_t box[2] = {64, 1};
-    cuuint32_t estride[2] = {1, 1};
-    const CUresult r = enc(out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<__nv_bfloat16 *>(p.cache),
-                           dims, strides, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) {
-        std::snprintf(g_last_error, sizeof g_last_error, "cuTensorMapEncodeTiled failed (%d)", (int)r);
-        return SMLA_ERR_CUDA;
-    }
-    return SMLA_OK;
-}
-
 template <bool DIRECT>
 smla_status launch_tc(const PartialParams &p, int grid, cudaStream_t st) {
-    CUtensorMap tmap{};  // unused when there is nothing to gather (K == 0)
-    if (p.K > 0) {
-        const smla_status s = encode_cache_map(p, &tmap);
-        if (s != SMLA_OK) return s;
-    }
     const void *fn = reinterpret_cast<const void *>(&smla::smla_partial_tc_kernel<DIRECT>);
     cudaError_t e = ensure_smem_attr(fn, smla::TcCfg::kSmemBytes);
     if (e != cudaSuccess) return cuda_fail(e);
-    smla::smla_partial_tc_kernel<DIRECT><<<grid, smla::TcCfg::kThreads, smla::TcCfg::kSmemBytes, st>>>(
-        p, tmap);
+    smla::smla_partial_tc_kernel<DIRECT><<<grid, smla::TcCfg::kThreads, smla::TcCfg::kSmemBytes, st>>>(p);
     e = cudaGetLastError();
     return e == cudaSuccess ? SMLA_OK : cuda_fail(e);
 }

@@ -40,7 +40,6 @@
 #pragma once
 
 #include <cstdint>
-#include <cuda.h>
 #include <cuda_bf16.h>
 
 #include "smla_partial_mma.cuh"
@@ -82,7 +81,7 @@ static_assert(TcCfg::kSmemBytes <= 232448, "shared memory per CTA");
 
 template <bool DIRECT>
 __global__ void __launch_bounds__(TcCfg::kThreads, 1)
-    smla_partial_tc_kernel(const PartialParams p, const __grid_constant__ CUtensorMap tmap) {
+    smla_partial_tc_kernel(const PartialParams p) {
     using C = TcCfg;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte aligned base (128B-swizzle atoms are 8 rows x 128 B).

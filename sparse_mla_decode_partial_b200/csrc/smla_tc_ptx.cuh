@@ -1,10 +1,9 @@
 // smla_tc_ptx.cuh -- inline-PTX wrappers for the 5th-generation tensor core
-// (tcgen05: TMEM allocation, MMA issue, commit, TMEM loads/stores, fences),
-// the TMA row gather (tile::gather4) and the shared-memory matrix descriptors.
+// (tcgen05: TMEM allocation, MMA issue, commit, TMEM loads/stores, fences)
+// and the shared-memory matrix descriptors.
 #pragma once
 
 #include <cstdint>
-#include <cuda.h>
 
 #include "smla_ptx.cuh"
 
@@ -89,21 +88,6 @@ __device__ __forceinline__ void tmem_st_wait() {
 // Generic-proxy shared-memory writes -> visible to the async proxy (MMA reads).
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-// ---------------------------------------------------------------- TMA gather of 4 rows
-// Four rows (row0..row3) x one 64-element box of a 2-D tensor map, into four
-// consecutive 128-byte rows at dst (swizzled by the map's swizzle mode).
-// Rows outside the tensor are filled with zeros.
-__device__ __forceinline__ void tma_gather4(void *dst_smem, const CUtensorMap *tmap, int col, int row0,
-                                            int row1, int row2, int row3, uint64_t *bar,
-                                            uint64_t policy) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-        ".L2::cache_hint [%0], [%1, {%3, %4, %5, %6, %7}], [%2], %8;" ::"r"(smem_addr(dst_smem)),
-        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(smem_addr(bar)), "r"(col), "r"(row0), "r"(row1),
-        "r"(row2), "r"(row3), "l"(policy)
-        : "memory");
 }
 
 // ---------------------------------------------------------------- descriptors
