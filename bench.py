@@ -358,31 +358,46 @@ def run_ours(args, world, rank, local):
     ms_part = statistics.fmean(part)
     tokens_all, ms_step_max, value = aggregate(float(B * T), ms_step, world)
 
-    # e2e: host buffers through the C ABI, copies inside the timed region
+    # e2e: host buffers through the C ABI, copies inside the timed region.
+    # The step's inputs (q, top-k indices, page table) sit in one pinned
+    # staging buffer and travel in one host->device copy; o and lse come back
+    # in one device->host copy (each piece 256-byte aligned inside its buffer).
     e2e = None
     if True:
-        q_h = w_host.q.pin_memory()
-        idx_h = w_host.idx.pin_memory()
-        pt_h = w_host.page_table.pin_memory()
-        o_h = torch.empty((B, T, H, 512), dtype=torch.bfloat16).pin_memory()
-        lse_h = torch.empty((B, T, H), dtype=torch.float32).pin_memory()
-        q_d, idx_d, pt_d = torch.empty_like(w.q), torch.empty_like(w.idx), torch.empty_like(w.page_table)
-        o_d = torch.empty((B, T, H, 512), dtype=torch.bfloat16, device=dev)
-        lse_d = torch.empty((B, T, H), dtype=torch.float32, device=dev)
+        def layout(parts):
+            offs, off = [], 0
+            for t in parts:
+                offs.append(off)
+                off += (t.numel() * t.element_size() + 255) // 256 * 256
+            return offs, off
+
+        def views(buf, offs, like):
+            return [buf[o:o + t.numel() * t.element_size()].view(t.dtype).view(t.shape)
+                    for o, t in zip(offs, like)]
+
+        in_parts = [w_host.q, w_host.idx, w_host.page_table]
+        in_offs, in_bytes = layout(in_parts)
+        in_h = torch.empty(in_bytes, dtype=torch.uint8).pin_memory()
+        in_d = torch.empty(in_bytes, dtype=torch.uint8, device=dev)
+        for v, t in zip(views(in_h, in_offs, in_parts), in_parts):
+            v.copy_(t)
+        q_d, idx_d, pt_d = views(in_d, in_offs, in_parts)
+        out_like = [torch.empty((B, T, H, 512), dtype=torch.bfloat16),
+                    torch.empty((B, T, H), dtype=torch.float32)]
+        out_offs, out_bytes = layout(out_like)
+        out_h = torch.empty(out_bytes, dtype=torch.uint8).pin_memory()
+        out_d = torch.empty(out_bytes, dtype=torch.uint8, device=dev)
+        o_d, lse_d = views(out_d, out_offs, out_like)
         ws = torch.empty(max(16, binding.workspace_bytes(B, T, H, nsplit)), dtype=torch.uint8,
                          device=dev)
-        h2d = q_h.numel() * 2 + idx_h.numel() * 4 + pt_h.numel() * 4
-        d2h = o_h.numel() * 2 + lse_h.numel() * 4
+        h2d, d2h = in_bytes, out_bytes
 
         def e2e_step():
-            q_d.copy_(q_h, non_blocking=True)
-            idx_d.copy_(idx_h, non_blocking=True)
-            pt_d.copy_(pt_h, non_blocking=True)
+            in_d.copy_(in_h, non_blocking=True)
             st = lib.smla_decode(q_d.data_ptr(), w.cache.data_ptr(), w.num_pages, pt_d.data_ptr(),
                                  w.pt_stride, idx_d.data_ptr(), B, T, H, K, 64, w.scale, nsplit,
                                  ws.data_ptr(), ws.numel(), o_d.data_ptr(), lse_d.data_ptr(), sptr)
-            o_h.copy_(o_d, non_blocking=True)
-            lse_h.copy_(lse_d, non_blocking=True)
+            out_h.copy_(out_d, non_blocking=True)
             return st
 
         for _ in range(3):
@@ -403,8 +418,9 @@ def run_ours(args, world, rank, local):
         e2e_ms = max_over_ranks(statistics.fmean(times), world)
         e2e = {"value": tokens_all / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
-               "note": "q, top-k indices and page table copied in from pinned host memory and "
-                       "o, lse copied out every step; the latent cache stays resident"}
+               "note": "q, top-k indices and page table copied in from one pinned host buffer "
+                       "(one copy) and o, lse copied out (one copy) every step; the latent "
+                       "cache stays resident"}
 
     # NSPLIT sweep (rank 0 only, after the timed region)
     sweep = []

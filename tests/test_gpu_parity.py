@@ -351,3 +351,40 @@ def test_balanced_schedule_with_padding_and_short_contexts():
     o_ref, lse_ref, _ = oracle_decode(w, sample)
     bi = [b for b, _ in sample]
     check_o_lse(o[bi, 0], lse[bi, 0], o_ref, lse_ref, "balanced with padding")
+
+
+# ------------------------------------------------------------------ sizes at the edges
+@pytest.mark.parametrize("H", [16, 24, 64])
+@pytest.mark.parametrize("S", [1, 2])
+def test_split_longer_than_one_resolve_chunk(H, S):
+    # a split of more than 2048 entries is resolved to rows in several chunks
+    w = workloads.make_workload("long_split", B=1, T=1, H=H, K=4500, ctx_lens=[12000], seed=H + S)
+    o, lse = run_decode(w, S)
+    o_ref, lse_ref, _ = oracle_decode(w)
+    check_o_lse(o, lse, o_ref, lse_ref, f"K=4500 H={H} S={S}")
+
+
+def test_page_table_wider_than_the_latency_kernel_holds():
+    # 9000 logical pages (576k positions) over a pool of 96 physical pages
+    # (pages aliased): one-tile splits then take the pipelined kernel
+    g = torch.Generator().manual_seed(17)
+    B, H, K, P, W = 2, 16, 2048, 96, 9000
+    q = (torch.randn(B, 1, H, 576, generator=g) * 0.5).to(torch.bfloat16)
+    cache = (torch.randn(P, 64, 576, generator=g) * 0.5).to(torch.bfloat16)
+    pt = torch.randint(0, P, (B, W), generator=g, dtype=torch.int32)
+    idx = torch.stack([torch.randperm(W * 64, generator=g)[:K] for _ in range(B)]).to(torch.int32)
+    idx = idx.view(B, 1, K)
+    w = workloads.Workload("wide_pt", q, cache, pt, idx, 576 ** -0.5, [W * 64] * B, None, ())
+    for S in (64, 16):
+        o, lse = run_decode(w, S)
+        o_ref, lse_ref, _ = oracle_decode(w)
+        check_o_lse(o, lse, o_ref, lse_ref, f"pt_stride {W} S={S}")
+
+
+@pytest.mark.parametrize("K,S", [(2048, 1024), (100, 512), (3, 1024)])
+def test_maximum_nsplit(K, S):
+    # NSPLIT at its maximum: two-entry splits, and mostly empty splits
+    w = small("max_nsplit", seed=K, B=1, T=2, H=16, K=K, ctx=5000)
+    o, lse = run_decode(w, S)
+    o_ref, lse_ref, _ = oracle_decode(w)
+    check_o_lse(o, lse, o_ref, lse_ref, f"K={K} S={S}")
