@@ -109,7 +109,7 @@ def load_peaks():
 def partial_kernel_name(H: int, K: int, nsplit: int, pt_stride: int) -> str:
     """The partial kernel the library launches for this shape (its dispatch rule)."""
     kc = -(-K // nsplit) if K > 0 else 0
-    if H <= 32 and K > 0 and kc <= 32 and pt_stride <= 8192:
+    if H <= 32 and K > 0 and kc <= 64 and pt_stride <= 8192:
         return "smla_partial_small_kernel"
     return "smla_partial_tc_kernel" if H > 32 else "smla_partial_mma_kernel"
 

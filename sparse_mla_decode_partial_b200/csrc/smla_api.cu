@@ -65,7 +65,7 @@ int current_device_sms() {
 
 // Kernel choice of launch_partial, as the schedule needs it.
 bool uses_latency_kernel(int H, int K, int kc, int pt_stride) {
-    return H <= 32 && K > 0 && kc <= 32 && pt_stride <= smla::kSmallMaxPt;
+    return H <= 32 && K > 0 && kc <= smla::kSmallMaxRows && pt_stride <= smla::kSmallMaxPt;
 }
 
 // NSPLIT model ("The Occupancy Hypothesis ...", sections "The Occupancy
@@ -163,13 +163,13 @@ smla_status launch_tc(const PartialParams &p, int grid, cudaStream_t st) {
     return e == cudaSuccess ? SMLA_OK : cuda_fail(e);
 }
 
-template <int HG, bool DIRECT>
+template <int HG, int TILES, bool DIRECT>
 smla_status launch_small(const PartialParams &p, int grid, cudaStream_t st) {
-    using C = smla::SmallCfg<HG>;
-    const void *fn = reinterpret_cast<const void *>(&smla::smla_partial_small_kernel<HG, DIRECT>);
+    using C = smla::SmallCfg<HG, TILES>;
+    const void *fn = reinterpret_cast<const void *>(&smla::smla_partial_small_kernel<HG, TILES, DIRECT>);
     cudaError_t e = ensure_smem_attr(fn, C::kMaxSmemBytes);
     if (e != cudaSuccess) return cuda_fail(e);
-    smla::smla_partial_small_kernel<HG, DIRECT>
+    smla::smla_partial_small_kernel<HG, TILES, DIRECT>
         <<<grid, C::kThreads, C::smem_bytes(p.pt_stride), st>>>(p);
     e = cudaGetLastError();
     return e == cudaSuccess ? SMLA_OK : cuda_fail(e);
@@ -179,10 +179,13 @@ template <bool DIRECT>
 smla_status launch_partial(const PartialParams &p, cudaStream_t st) {
     const long long grid = p.balanced ? (long long)p.grid : (long long)p.B * p.T * p.nsplit;
     if (grid > INT_MAX) return SMLA_ERR_INVALID_ARG;
-    // one tile per split: the latency path (see smla_partial_small_kernel)
-    if (p.H <= 32 && p.K > 0 && p.kc <= 32 && p.pt_stride <= smla::kSmallMaxPt) {
-        if (p.H <= 16) return launch_small<1, DIRECT>(p, (int)grid, st);
-        return launch_small<2, DIRECT>(p, (int)grid, st);
+    // one or two tiles per split: the latency path (see smla_partial_small_kernel)
+    if (!p.balanced && uses_latency_kernel(p.H, p.K, p.kc, p.pt_stride)) {
+        if (p.kc <= 32)
+            return p.H <= 16 ? launch_small<1, 1, DIRECT>(p, (int)grid, st)
+                             : launch_small<2, 1, DIRECT>(p, (int)grid, st);
+        return p.H <= 16 ? launch_small<1, 2, DIRECT>(p, (int)grid, st)
+                         : launch_small<2, 2, DIRECT>(p, (int)grid, st);
     }
     if (p.H > 32) return launch_tc<DIRECT>(p, (int)grid, st);
     if (p.H > 16) return launch_mma<2, 32, 4, DIRECT>(p, (int)grid, st);

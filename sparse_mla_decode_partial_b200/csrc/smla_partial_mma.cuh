@@ -515,26 +515,30 @@ __global__ void __launch_bounds__(MmaCfg<HG, NT, NSTAGE>::kThreads, MmaCfg<HG, N
 // with 16-byte cp.async copies issued by every thread (one more round trip,
 // no serial TMA queue) and runs the same consumer math on it.
 constexpr int kSmallMaxPt = 8192;  // page-table entries kept in shared memory
+constexpr int kSmallMaxRows = 64;  // rows per split the latency form takes
 
 
-template <int HG>
+template <int HG, int TILES>
 struct SmallCfg {
+    static_assert(TILES == 1 || TILES == 2, "one or two 32-row tiles per split");
     static constexpr int NT = 32;
     static constexpr int kThreads = 128 * HG;
     static constexpr int kQBytes = 16 * HG * kSmemRowBytes;
     static constexpr int kSPartBytes = HG * 2 * 4 * 16 * (NT + 8) * 4;
     static constexpr int kOffQ = 0;  // Q rows, then the S partials
     static constexpr int kOffKV = ((kQBytes > kSPartBytes ? kQBytes : kSPartBytes) + 127) / 128 * 128;
-    static constexpr int kOffRows = kOffKV + NT * kSmemRowBytes;  // int [32] rows, u32 mask
-    static constexpr int kOffPt = kOffRows + 36 * 4;             // int [pt_stride]
+    static constexpr int kOffRows = kOffKV + TILES * NT * kSmemRowBytes;  // int [32 TILES] rows, masks
+    static constexpr int kOffPt = kOffRows + (NT + 4) * TILES * 4;      // int [pt_stride]
     static constexpr int kMaxSmemBytes = kOffPt + kSmallMaxPt * 4;
     static int smem_bytes(int pt_stride) { return kOffPt + pt_stride * 4; }
 };
 
-template <int HG, bool DIRECT>
-__global__ void __launch_bounds__(SmallCfg<HG>::kThreads)
+// TILES: 32-row tiles per split (a split of up to 64 rows still takes one
+// round trip for its rows: both tiles are gathered at once).
+template <int HG, int TILES, bool DIRECT>
+__global__ void __launch_bounds__(SmallCfg<HG, TILES>::kThreads)
     smla_partial_small_kernel(const PartialParams p) {
-    using C = SmallCfg<HG>;
+    using C = SmallCfg<HG, TILES>;
     constexpr int NT = C::NT;
     extern __shared__ __align__(128) uint8_t smem[];
     const int warp = threadIdx.x >> 5;
@@ -547,7 +551,7 @@ __global__ void __launch_bounds__(SmallCfg<HG>::kThreads)
     const long long j0l = (long long)s * p.kc;
     const int j0 = (int)(j0l < p.K ? j0l : p.K);
     const int j1 = (int)((long long)j0 + p.kc < p.K ? (long long)j0 + p.kc : p.K);
-    int *rows_s = reinterpret_cast<int *>(smem + C::kOffRows);
+    int *rows_s = reinterpret_cast<int *>(smem + C::kOffRows);  // [TILES * 32] rows, then masks
     int *pt_s = reinterpret_cast<int *>(smem + C::kOffPt);
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
@@ -567,14 +571,14 @@ __global__ void __launch_bounds__(SmallCfg<HG>::kThreads)
         }
     }
     int my_idx = -1;
-    if (tid < NT && j0 + tid < j1) my_idx = __ldg(p.idx + (size_t)bt * p.K + j0 + tid);
+    if (tid < NT * TILES && j0 + tid < j1) my_idx = __ldg(p.idx + (size_t)bt * p.K + j0 + tid);
     MmaConsumer<NT, HG> cons;
     cons.init(warp, lane);
     cons.load_q(smem + C::kOffQ, p, bt);
     __syncthreads();
 
-    // 2. rows of the tile (warp 0); out-of-range entries are masked and counted
-    if (warp == 0) {
+    // 2. rows of tile w (warp w); out-of-range entries are masked and counted
+    if (warp < TILES) {
         const int i = my_idx;
         int row = -1;
         if (i != -1) {
@@ -589,17 +593,17 @@ __global__ void __launch_bounds__(SmallCfg<HG>::kThreads)
                 atomicAdd(&g_bad_index_count, 1ull);
             }
         }
-        rows_s[lane] = row;
+        rows_s[warp * NT + lane] = row;
         const uint32_t m = __ballot_sync(0xffffffffu, row >= 0);
-        if (lane == 0) rows_s[32] = (int)m;
+        if (lane == 0) rows_s[NT * TILES + warp] = (int)m;
     }
     __syncthreads();
 
-    // 3. gather: 32 rows x 72 chunks of 16 B, cp.async from every thread
+    // 3. gather: TILES x 32 rows x 72 chunks of 16 B, cp.async from every thread
     const uint8_t *cache = reinterpret_cast<const uint8_t *>(p.cache);
     const uint8_t *zero = reinterpret_cast<const uint8_t *>(g_zero_row);
     uint8_t *kv = smem + C::kOffKV;
-    for (int c = tid; c < NT * 72; c += C::kThreads) {
+    for (int c = tid; c < TILES * NT * 72; c += C::kThreads) {
         const int r = c / 72, k = c - 72 * (c / 72);
         const int row = rows_s[r];
         const uint8_t *src = (row >= 0 ? cache + (size_t)row * kRowBytes : zero) + k * 16;
@@ -609,13 +613,15 @@ __global__ void __launch_bounds__(SmallCfg<HG>::kThreads)
                      : "memory");
     }
     asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
-    const uint32_t vmask = (uint32_t)rows_s[32];
     __syncthreads();
 
-    // 4. the tile and the epilogue (the Q region now holds the S partials)
-    cons.tile(smem_addr(kv), vmask,
-              reinterpret_cast<float *>(smem + C::kOffQ) + cons.g * 2 * 4 * 16 * (NT + 8),
-              p.scale_log2);
+    // 4. the tiles and the epilogue (the Q region now holds the S partials,
+    //    double buffered by tile)
+    float *spart = reinterpret_cast<float *>(smem + C::kOffQ) + cons.g * 2 * 4 * 16 * (NT + 8);
+#pragma unroll
+    for (int t = 0; t < TILES; ++t)
+        cons.tile(smem_addr(kv + t * NT * kSmemRowBytes), (uint32_t)rows_s[NT * TILES + t],
+                  spart + (t & 1) * 4 * 16 * (NT + 8), p.scale_log2);
     cons.template epilogue<DIRECT>(p, bt, s);
 }
 

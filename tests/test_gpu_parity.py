@@ -298,7 +298,7 @@ def test_one_tile_splits_many_waves():
 def balanced_taken(B, T, H, K, S, sms):
     resident = sms * (2 if H <= 16 else 1)
     bt, units = B * T, B * T * -(-K // 32)
-    return (S >= 2 and H <= 32 and not (-(-K // S) <= 32) and bt * S > resident
+    return (S >= 2 and H <= 32 and not (-(-K // S) <= 64) and bt * S > resident
             and (S - 1) * bt >= resident and units >= 4 * resident)
 
 
@@ -306,8 +306,8 @@ def sms():
     return torch.cuda.get_device_properties(0).multi_processor_count
 
 
-@pytest.mark.parametrize("B,T,H,K,S", [(64, 1, 16, 2048, 6), (64, 1, 16, 2048, 40),
-                                       (40, 1, 24, 1000, 8), (20, 3, 16, 777, 16),
+@pytest.mark.parametrize("B,T,H,K,S", [(64, 1, 16, 2048, 6), (64, 1, 16, 2048, 24),
+                                       (40, 1, 24, 1000, 8), (20, 3, 16, 777, 8),
                                        (128, 1, 16, 2048, 4)])
 def test_balanced_schedule(B, T, H, K, S):
     w = workloads.make_workload("balanced", B=B, T=T, H=H, K=K, ctx_lens=[6000] * B, seed=B + K)
@@ -388,3 +388,15 @@ def test_maximum_nsplit(K, S):
     o, lse = run_decode(w, S)
     o_ref, lse_ref, _ = oracle_decode(w)
     check_o_lse(o, lse, o_ref, lse_ref, f"K={K} S={S}")
+
+
+@pytest.mark.parametrize("H,K,S", [(16, 2048, 32), (8, 100, 2), (24, 640, 12), (32, 130, 3),
+                                   (5, 33, 1), (16, 64, 1), (1, 1000, 16)])
+def test_two_tile_splits(H, K, S):
+    # 33..64 entries per split: the latency form gathers both tiles at once
+    assert 32 < -(-K // S) <= 64
+    w = small("two_tiles", seed=H * 7 + K, B=2, T=2, H=H, K=K, ctx=3000)
+    w.idx[1, 0, 5::9] = -1                       # interleaved padding in one token
+    o, lse = run_decode(w, S)
+    o_ref, lse_ref, _ = oracle_decode(w)
+    check_o_lse(o, lse, o_ref, lse_ref, f"two tiles H={H} K={K} S={S}")

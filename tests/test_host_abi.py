@@ -123,7 +123,7 @@ def model(B, T, H, K, sms):
     # balanced schedule: one full wave of `slots` CTAs, base + slots pieces
     s_bal = math.ceil(slots / base) + 1
     units = base * -(-K // 32)
-    latency_kernel = H <= 32 and math.ceil(K / s_bal) <= 32
+    latency_kernel = H <= 32 and math.ceil(K / s_bal) <= 64
     if H <= 32 and 2 <= s_bal <= s_max and units >= 4 * slots and not latency_kernel:
         pieces = base + slots
         t = 48.0 * pieces / slots + units * 32.0 / slots
