@@ -298,7 +298,8 @@ def test_one_tile_splits_many_waves():
 def balanced_taken(B, T, H, K, S, sms):
     resident = sms * (2 if H <= 16 else 1)
     bt, units = B * T, B * T * -(-K // 32)
-    return (S >= 2 and H <= 32 and not (-(-K // S) <= 64) and bt * S > resident
+    latency = H <= 32 and -(-K // S) <= 64
+    return (S >= 2 and H <= 32 and not latency and bt * S > resident
             and (S - 1) * bt >= resident and units >= 4 * resident)
 
 
