@@ -8,7 +8,10 @@
 //
 // One CTA = one (query token, split) and ALL of its heads, because every
 // gathered 1152-byte latent row is shared by all heads: gathering it once per
-// CTA is what keeps the pass at one HBM read per selected row.
+// CTA is what keeps the pass at one HBM read per selected row.  Under the
+// balanced schedule of the whole decode a CTA instead takes an equal run of
+// 32-row tiles that may span two tokens; it walks those pieces (work items)
+// in order, one partial slot per piece.
 //
 // Warp roles (HG = head groups of 16 rows, the mma M dimension):
 //   warp 4*HG      producer: first resolves the split's index entries to

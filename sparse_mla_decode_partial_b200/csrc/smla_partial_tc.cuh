@@ -150,7 +150,7 @@ __global__ void __launch_bounds__(TcCfg::kThreads, 1)
         constexpr int kPadRow = 0;
         int *rows_s = reinterpret_cast<int *>(smem + C::kOffRows);
         const uint8_t *cache = reinterpret_cast<const uint8_t *>(p.cache);
-        const uint32_t bar_prod = 1;  // named barrier of the 4 producer warps
+        const uint32_t bar_prod = 1;  // named barrier of the producer warps
         const int len = j1 - j0;
         int it = 0;
         for (int base = 0; base < len; base += kResolveChunk) {
