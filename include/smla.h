@@ -211,6 +211,36 @@ smla_status smla_decode_noalloc(const void *q, const void *kv_cache, int64_t num
                                 int page_size, float scale, int nsplit, void *o, float *lse,
                                 void *stream);
 
+/*
+ * Whole decode for per-step data that lives in host memory.
+ *
+ * The pages have no counterpart to this entry point; it serves decode loops
+ * whose query vectors, top-k indices and page tables are produced on the host
+ * each step and whose outputs are consumed there.  q, page_table, topk_idx, o
+ * and lse are PINNED host memory (cudaHostAlloc / cudaMallocHost /
+ * cudaHostRegister, which on a unified-addressing system the GPU can address
+ * directly); kv_cache and workspace are device memory as for smla_decode.
+ * One small copy kernel pulls q, the indices and the page table over the
+ * host link into a staging area at the end of the workspace, then the decode
+ * runs as smla_decode does and writes o and lse straight into the host
+ * buffers.  This avoids the per-transfer latency of separate copies.
+ *
+ *  - workspace_bytes must be at least smla_workspace_host_bytes(B, T, H, K,
+ *    pt_stride, nsplit) for the nsplit actually used (0 picks the heuristic's
+ *    value), else SMLA_ERR_WORKSPACE_TOO_SMALL.
+ *  - Any host pointer that is not pinned host memory visible to the current
+ *    device returns SMLA_ERR_INVALID_ARG before anything is launched.
+ *  - Asynchronous on `stream`: the host may read o and lse after
+ *    synchronising the stream, and must not rewrite q, page_table or topk_idx
+ *    before then.
+ */
+size_t smla_workspace_host_bytes(int B, int T, int H, int K, int pt_stride, int nsplit);
+smla_status smla_decode_host(const void *q_host, const void *kv_cache, int64_t num_pages,
+                             const int32_t *page_table_host, int pt_stride,
+                             const int32_t *topk_idx_host, int B, int T, int H, int K,
+                             int page_size, float scale, int nsplit, void *workspace,
+                             size_t workspace_bytes, void *o_host, float *lse_host, void *stream);
+
 /* Static text for a status code. */
 const char *smla_status_string(smla_status status);
 

@@ -37,6 +37,9 @@ SIGNATURES = {
                          _P]),
     "smla_decode_noalloc": (_I, [_P, _P, _I64, _P, _I, _P, _I, _I, _I, _I, _I, _F, _I, _P, _P,
                                  _P]),
+    "smla_workspace_host_bytes": (_SZ, [_I, _I, _I, _I, _I, _I]),
+    "smla_decode_host": (_I, [_P, _P, _I64, _P, _I, _P, _I, _I, _I, _I, _I, _F, _I, _P, _SZ, _P, _P,
+                              _P]),
     "smla_check_device": (_I, [_I, ctypes.POINTER(ctypes.c_ulonglong), _P]),
     "smla_status_string": (ctypes.c_char_p, [_I]),
     "smla_last_error": (ctypes.c_char_p, []),
@@ -209,6 +212,43 @@ def decode_noalloc(q, cache, page_table, idx, scale: float, nsplit: int = 0, *, 
                                      pt_stride, _ptr(idx), B, T, H, K, PAGE_SIZE, float(scale),
                                      int(nsplit), _ptr(o), _ptr(lse), _stream(stream)),
            "smla_decode_noalloc")
+    return o, lse
+
+
+def workspace_host_bytes(B: int, T: int, H: int, K: int, pt_stride: int, nsplit: int) -> int:
+    return int(lib().smla_workspace_host_bytes(B, T, H, K, pt_stride, nsplit))
+
+
+def decode_host(q, cache, page_table, idx, scale: float, nsplit: int = 0, *, o, lse,
+                workspace=None, stream=None):
+    """Whole decode through smla_decode_host: q, page_table, idx, o and lse are
+    pinned CPU tensors (the per-step data of a host-driven decode loop), cache
+    and workspace live on the GPU.  The inputs are pulled over the host link
+    by a copy kernel and o, lse are written straight back into host memory;
+    both are asynchronous on the stream (synchronise before reading o)."""
+    for t, n, dt in ((q, "q", torch.bfloat16), (page_table, "page_table", torch.int32),
+                     (idx, "idx", torch.int32), (o, "o", torch.bfloat16), (lse, "lse", torch.float32)):
+        if not isinstance(t, torch.Tensor) or t.dtype != dt or not t.is_contiguous():
+            raise TypeError(f"{n} must be a contiguous {dt} tensor")
+        if t.is_cuda or not t.is_pinned():
+            raise ValueError(f"{n} must be a pinned CPU tensor")
+    _need(cache, torch.bfloat16, "cache")
+    dev = cache.device
+    if q.dim() != 4 or q.shape[-1] != D:
+        raise ValueError(f"q must be [B,T,H,{D}]")
+    B, T, H, _ = q.shape
+    K, pt_stride = idx.shape[2], page_table.shape[1]
+    num_pages = cache.numel() // (PAGE_SIZE * D)
+    if nsplit == 0:
+        nsplit = choose_nsplit(B, T, H, K, 0)
+    need = workspace_host_bytes(B, T, H, K, pt_stride, nsplit)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    _need(workspace, torch.uint8, "workspace", dev)
+    _check(lib().smla_decode_host(_ptr(q), _ptr(cache), num_pages, _ptr(page_table), pt_stride,
+                                  _ptr(idx), B, T, H, K, PAGE_SIZE, float(scale), int(nsplit),
+                                  _ptr(workspace), workspace.numel(), _ptr(o), _ptr(lse),
+                                  _stream(stream)), "smla_decode_host")
     return o, lse
 
 

@@ -3,6 +3,7 @@
 // Every entry point returns a status; nothing throws across the ABI.
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <climits>
 #include <cmath>
 #include <cstdint>
@@ -461,6 +462,93 @@ smla_status smla_decode_noalloc(const void *q, const void *kv_cache, int64_t num
     return smla_decode(q, kv_cache, num_pages, page_table, pt_stride, topk_idx, B, T, H, K,
                        page_size, scale, nsplit, scratch, SMLA_NOALLOC_SCRATCH_BYTES, o, lse,
                        stream);
+}
+
+// ---------------------------------------------------------------------------
+// Decode with per-step data in pinned host memory (see include/smla.h).
+namespace {
+
+// Device alias of pinned host memory, or nullptr when `ptr` is not pinned host
+// memory that the current device can address.
+void *host_alias(const void *ptr) {
+    if (ptr == nullptr) return nullptr;
+    cudaPointerAttributes a;
+    if (cudaPointerGetAttributes(&a, ptr) != cudaSuccess) {
+        (void)cudaGetLastError();  // an unregistered pointer is not an error state
+        return nullptr;
+    }
+    if (a.type != cudaMemoryTypeHost || a.devicePointer == nullptr) return nullptr;
+    return a.devicePointer;
+}
+
+struct HostStaging {
+    size_t base, q, idx, pt, total;  // byte offsets and sizes inside the workspace
+};
+
+HostStaging host_staging(int B, int T, int H, int K, int pt_stride, int nsplit) {
+    HostStaging h{};
+    h.base = nsplit > 1 ? smla_workspace_bytes(B, T, H, nsplit) : 0;
+    const size_t q_bytes = (size_t)B * T * H * smla::kD * 2;
+    const size_t idx_bytes = (size_t)B * T * K * 4;
+    h.q = round256(h.base);
+    h.idx = h.q + round256(q_bytes);
+    h.pt = h.idx + round256(idx_bytes);
+    h.total = h.pt + round256((size_t)B * pt_stride * 4);
+    return h;
+}
+
+}  // namespace
+
+size_t smla_workspace_host_bytes(int B, int T, int H, int K, int pt_stride, int nsplit) {
+    if (B < 0 || T < 0 || H < 0 || K < 0 || pt_stride < 0 || nsplit < 1 || nsplit > SMLA_MAX_NSPLIT)
+        return 0;
+    return host_staging(B, T, H, K, pt_stride, nsplit).total;
+}
+
+smla_status smla_decode_host(const void *q_host, const void *kv_cache, int64_t num_pages,
+                             const int32_t *page_table_host, int pt_stride,
+                             const int32_t *topk_idx_host, int B, int T, int H, int K,
+                             int page_size, float scale, int nsplit, void *workspace,
+                             size_t workspace_bytes, void *o_host, float *lse_host, void *stream) {
+    if (B < 0 || T < 0 || H < 0 || K < 0 || pt_stride < 0) return SMLA_ERR_INVALID_ARG;
+    if (nsplit < 0 || nsplit > SMLA_MAX_NSPLIT) return SMLA_ERR_INVALID_ARG;
+    if (B == 0 || T == 0 || H == 0) return SMLA_OK;
+    if (nsplit == 0) nsplit = smla_choose_nsplit(B, T, H, K, 0);
+    // every host pointer must be pinned and visible to the device: checked
+    // here, before anything is launched
+    void *q_d = host_alias(q_host);
+    void *o_d = host_alias(o_host);
+    void *lse_d = host_alias(lse_host);
+    void *pt_d = K > 0 ? host_alias(page_table_host) : nullptr;
+    void *idx_d = K > 0 ? host_alias(topk_idx_host) : nullptr;
+    if (q_d == nullptr || o_d == nullptr || lse_d == nullptr || (K > 0 && (pt_d == nullptr || idx_d == nullptr))) {
+        std::snprintf(g_last_error, sizeof g_last_error,
+                      "smla_decode_host: q, page_table, topk_idx, o and lse must be pinned host memory");
+        return SMLA_ERR_INVALID_ARG;
+    }
+    if (!aligned(q_host, 16) || !aligned(o_host, 16) || !aligned(lse_host, 4) ||
+        (K > 0 && (!aligned(page_table_host, 4) || !aligned(topk_idx_host, 4))))
+        return SMLA_ERR_MISALIGNED;
+    const HostStaging hs = host_staging(B, T, H, K, pt_stride, nsplit);
+    if (workspace_bytes < hs.total) return SMLA_ERR_WORKSPACE_TOO_SMALL;
+    if (workspace == nullptr) return SMLA_ERR_INVALID_ARG;
+    if (!aligned(workspace, 16)) return SMLA_ERR_MISALIGNED;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    smla::IngestArgs a{};
+    a.r[0] = {static_cast<const uint8_t *>(q_d), ws + hs.q, (size_t)B * T * H * smla::kD * 2};
+    if (K > 0) {
+        a.r[1] = {static_cast<const uint8_t *>(idx_d), ws + hs.idx, (size_t)B * T * K * 4};
+        a.r[2] = {static_cast<const uint8_t *>(pt_d), ws + hs.pt, (size_t)B * pt_stride * 4};
+    }
+    const size_t words = (a.r[0].bytes + a.r[1].bytes + a.r[2].bytes) / 16 + 1;
+    const unsigned blocks = (unsigned)std::min<size_t>((words + 255) / 256, 148);
+    smla::smla_ingest_kernel<<<blocks, 256, 0, st>>>(a);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e);
+    return smla_decode(ws + hs.q, kv_cache, num_pages, reinterpret_cast<const int32_t *>(ws + hs.pt),
+                       pt_stride, reinterpret_cast<const int32_t *>(ws + hs.idx), B, T, H, K, page_size,
+                       scale, nsplit, workspace, hs.base, o_d, static_cast<float *>(lse_d), stream);
 }
 
 smla_status smla_check_device(int clear, unsigned long long *n_bad_index, void *stream) {

@@ -296,4 +296,32 @@ __global__ void __launch_bounds__(32 * kCombineWarpUnits)
     if (lane == 0) lse[u] = M + logf(L);
 }
 
+// Copy of the per-step inputs of smla_decode_host from pinned host memory
+// (addressed through its device alias) into the workspace's staging area:
+// up to three regions, 16-byte vectors for the body, 4-byte words for a tail.
+struct IngestRegion {
+    const uint8_t *src;
+    uint8_t *dst;
+    size_t bytes;  // multiple of 4
+};
+struct IngestArgs {
+    IngestRegion r[3];
+};
+
+__global__ void __launch_bounds__(256) smla_ingest_kernel(const IngestArgs a) {
+    const size_t tid = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const size_t nthreads = (size_t)gridDim.x * blockDim.x;
+#pragma unroll
+    for (int k = 0; k < 3; ++k) {
+        const IngestRegion r = a.r[k];
+        // destinations are 256-byte aligned; the source decides the width
+        const size_t n16 = (reinterpret_cast<uintptr_t>(r.src) & 15) ? 0 : r.bytes / 16;
+        const uint4 *s16 = reinterpret_cast<const uint4 *>(r.src);
+        uint4 *d16 = reinterpret_cast<uint4 *>(r.dst);
+        for (size_t i = tid; i < n16; i += nthreads) d16[i] = s16[i];
+        for (size_t i = n16 * 4 + tid; i < r.bytes / 4; i += nthreads)
+            reinterpret_cast<uint32_t *>(r.dst)[i] = reinterpret_cast<const uint32_t *>(r.src)[i];
+    }
+}
+
 }  // namespace smla

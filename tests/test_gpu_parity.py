@@ -401,3 +401,48 @@ def test_two_tile_splits(H, K, S):
     o, lse = run_decode(w, S)
     o_ref, lse_ref, _ = oracle_decode(w)
     check_o_lse(o, lse, o_ref, lse_ref, f"two tiles H={H} K={K} S={S}")
+
+
+# ------------------------------------------------------------------ per-step data in host memory
+@pytest.mark.parametrize("name,S", [("single_request", 0), ("spec_verify", 0), ("tiny", 1),
+                                    ("tiny", 4)])
+def test_decode_host_matches_device_decode(name, S):
+    w = workloads.WORKLOADS[name]()
+    wd = w.to(DEV)
+    o_ref, lse_ref = binding.decode(wd.q, wd.cache, wd.page_table, wd.idx, w.scale, S)
+    q_h, pt_h, idx_h = w.q.pin_memory(), w.page_table.pin_memory(), w.idx.pin_memory()
+    o_h = torch.full(o_ref.shape, 5.0, dtype=torch.bfloat16).pin_memory()
+    lse_h = torch.full(lse_ref.shape, 5.0, dtype=torch.float32).pin_memory()
+    for _ in range(2):
+        binding.decode_host(q_h, wd.cache, pt_h, idx_h, w.scale, S, o=o_h, lse=lse_h)
+        torch.cuda.synchronize()
+        # the same kernels on the same bytes: bit-identical to the device path
+        assert torch.equal(o_h, o_ref.cpu()) and torch.equal(lse_h, lse_ref.cpu())
+
+
+def test_decode_host_rejects_unpinned_memory_before_launch():
+    w = workloads.tiny()
+    wd = w.to(DEV)
+    lib = binding.lib()
+    o_h = torch.full((1, 1, 8, 512), 5.0, dtype=torch.bfloat16).pin_memory()
+    lse_h = torch.full((1, 1, 8), 5.0, dtype=torch.float32).pin_memory()
+    ws = torch.empty(binding.workspace_host_bytes(1, 1, 8, 256, w.pt_stride, 4), dtype=torch.uint8,
+                     device=DEV)
+    q_pageable = w.q.clone()                      # ordinary (pageable) host memory
+    q_h, pt_h, idx_h = w.q.pin_memory(), w.page_table.pin_memory(), w.idx.pin_memory()
+    st = lib.smla_decode_host(q_pageable.data_ptr(), wd.cache.data_ptr(), w.num_pages,
+                              pt_h.data_ptr(), w.pt_stride, idx_h.data_ptr(), 1, 1, 8, 256, 64,
+                              w.scale, 4, ws.data_ptr(), ws.numel(), o_h.data_ptr(),
+                              lse_h.data_ptr(), None)
+    assert st == 1 and "pinned" in lib.smla_last_error().decode()
+    # a device pointer where host memory is expected is refused too
+    st = lib.smla_decode_host(wd.q.data_ptr(), wd.cache.data_ptr(), w.num_pages, pt_h.data_ptr(),
+                              w.pt_stride, idx_h.data_ptr(), 1, 1, 8, 256, 64, w.scale, 4,
+                              ws.data_ptr(), ws.numel(), o_h.data_ptr(), lse_h.data_ptr(), None)
+    assert st == 1
+    st = lib.smla_decode_host(q_h.data_ptr(), wd.cache.data_ptr(), w.num_pages, pt_h.data_ptr(),
+                              w.pt_stride, idx_h.data_ptr(), 1, 1, 8, 256, 64, w.scale, 4,
+                              ws.data_ptr(), 100, o_h.data_ptr(), lse_h.data_ptr(), None)
+    assert st == 4
+    torch.cuda.synchronize()
+    assert torch.all(o_h == 5.0) and torch.all(lse_h == 5.0)   # nothing ran

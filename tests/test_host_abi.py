@@ -219,3 +219,13 @@ def test_binding_refuses_cpu_tensors():
         binding.decode(q, torch.zeros((1, 64, 576), dtype=torch.bfloat16),
                        torch.zeros((1, 1), dtype=torch.int32), torch.zeros((1, 1, 4), dtype=torch.int32),
                        0.1, 1)
+
+
+def test_workspace_host_bytes_formula(lib):
+    r = lambda x: (x + 255) // 256 * 256
+    for B, T, H, K, P, S in [(1, 1, 16, 2048, 1024, 64), (64, 1, 16, 2048, 256, 4), (2, 3, 5, 7, 9, 1)]:
+        base = binding.workspace_bytes(B, T, H, S) if S > 1 else 0
+        want = r(base) + r(B * T * H * 576 * 2) + r(B * T * K * 4) + r(B * P * 4)
+        assert binding.workspace_host_bytes(B, T, H, K, P, S) == want
+    assert binding.workspace_host_bytes(1, 1, 1, 1, 1, 0) == 0
+    assert binding.workspace_host_bytes(1, 1, 1, -1, 1, 1) == 0
