@@ -21,7 +21,10 @@
 //
 // Both are launched as programmatic dependents of the partial pass: they may
 // be scheduled while that grid still runs, and wait on griddepcontrol before
-// touching memory.
+// touching memory.  The partials are read with coherent L2 loads (__ldcg),
+// never the read-only path: that data is written by the grid that runs
+// concurrently, so no load of it may be treated as invariant and scheduled
+// ahead of the wait.
 #pragma once
 
 #include <cstdint>
@@ -60,9 +63,9 @@ __global__ void __launch_bounds__(kCombineThreads)
         for (int k = 0; k < kCombineDepth; ++k) {
             const int s = s0 + g * kCombineDepth + k;
             if (s < nsplit) {
-                mv[k] = __ldg(pm + s);
-                lv[k] = __ldg(pl + s);
-                v[k] = __ldg(po + (size_t)s * 128);
+                mv[k] = __ldcg(pm + s);
+                lv[k] = __ldcg(pl + s);
+                v[k] = __ldcg(po + (size_t)s * 128);
             } else {
                 mv[k] = -INFINITY;
                 lv[k] = -INFINITY;
@@ -162,9 +165,9 @@ __global__ void __launch_bounds__(kCombineThreads)
         for (int k = 0; k < kCombineQDepth; ++k) {
             const int sp = s0 + g + kCombineQGroups * k;
             if (sp < nsplit) {
-                mv[k] = __ldg(pm + sp);
-                lv[k] = __ldg(pl + sp);
-                v[k] = __ldg(po + (size_t)sp * 128);
+                mv[k] = __ldcg(pm + sp);
+                lv[k] = __ldcg(pl + sp);
+                v[k] = __ldcg(po + (size_t)sp * 128);
             } else {
                 mv[k] = -INFINITY;
                 lv[k] = -INFINITY;
@@ -248,10 +251,10 @@ __global__ void __launch_bounds__(32 * kCombineWarpUnits)
 #pragma unroll
     for (int s = 0; s < SMAX; ++s) {
         if (s < nsplit) {
-            mv[s] = __ldg(pm + s);
-            lv[s] = __ldg(pl + s);
+            mv[s] = __ldcg(pm + s);
+            lv[s] = __ldcg(pl + s);
 #pragma unroll
-            for (int j = 0; j < 4; ++j) v[s][j] = __ldg(po + s * 128 + j * 32);
+            for (int j = 0; j < 4; ++j) v[s][j] = __ldcg(po + s * 128 + j * 32);
         } else {
             mv[s] = -INFINITY;
             lv[s] = -INFINITY;
