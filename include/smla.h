@@ -33,11 +33,16 @@
  *
  * Split convention.  With S = nsplit, Kc = ceil(K / S): split s covers index
  * positions [s*Kc, min(K, (s+1)*Kc)).  Trailing splits may be short or empty.
+ * This is exactly what smla_decode_partial writes.  The whole-decode entry
+ * points may instead cover a token with at most S pieces of unequal length
+ * (see smla_decode); their results differ only in rounding order.
  *
  * Common rules for every entry point:
  *  - All pointers are DEVICE pointers on the current device, owned by the
- *    caller.  The library allocates no device memory; it keeps only a small
- *    host-side cache of per-device kernel attributes.
+ *    caller, except the per-step buffers of smla_decode_host (pinned host
+ *    memory).  The library allocates no device memory at run time; it keeps a
+ *    small host-side cache of per-device kernel attributes and, for
+ *    smla_decode_noalloc, one static device array per GPU.
  *  - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL is
  *    the legacy default stream).  Arguments are checked on the host before
  *    anything is launched; a failed check launches nothing.
@@ -90,8 +95,10 @@ typedef enum {
  * CTAs.  The heuristic picks the NSPLIT in [1, min(SMLA_MAX_NSPLIT, ceil(K/32))]
  * that minimises a model of wave count x rows per CTA plus per-CTA overhead
  * and the split-K scratch traffic, with two resident CTAs per SM for H <= 16
- * and one otherwise.  sm_count <= 0 queries the current
- * device.  If the environment variable SMLA_NSPLIT holds a positive integer,
+ * and one otherwise.  It also prices smla_decode's balanced schedule (one
+ * full wave of equal CTAs, ceil(SMs x resident / (B*T)) + 1 slots) and
+ * returns that slot count only when the model favours it by more than 15%.
+ * sm_count <= 0 queries the current device.  If the environment variable SMLA_NSPLIT holds a positive integer,
  * that value is returned instead (clamped to [1, SMLA_MAX_NSPLIT]).
  * Returns >= 1; returns 1 for degenerate sizes.
  */
