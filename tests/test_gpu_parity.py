@@ -446,3 +446,41 @@ def test_decode_host_rejects_unpinned_memory_before_launch():
     assert st == 4
     torch.cuda.synchronize()
     assert torch.all(o_h == 5.0) and torch.all(lse_h == 5.0)   # nothing ran
+
+
+def test_concurrent_host_threads_on_separate_streams():
+    # four host threads decode at once, each on its own stream and workspace,
+    # with shapes that take different kernels (latency form, mma, tcgen05);
+    # ctypes releases the GIL, so the library's calls really overlap
+    import threading
+    cases = [small("mt0", seed=40, B=1, T=1, H=16, K=2048, ctx=70000),
+             small("mt1", seed=41, B=3, T=2, H=16, K=700, ctx=4000),
+             small("mt2", seed=42, B=2, T=1, H=64, K=900, ctx=4000),
+             small("mt3", seed=43, B=2, T=3, H=24, K=130, ctx=4000)]
+    splits = [64, 3, 2, 5]
+    devs = [w.to(DEV) for w in cases]
+    torch.cuda.synchronize()
+    results, errors = [None] * 4, []
+
+    def run(i):
+        try:
+            s = torch.cuda.Stream()
+            wd = devs[i]
+            with torch.cuda.stream(s):
+                for _ in range(5):
+                    o, lse = binding.decode(wd.q, wd.cache, wd.page_table, wd.idx, cases[i].scale,
+                                            splits[i], stream=s)
+            s.synchronize()
+            results[i] = (o, lse)
+        except Exception as e:  # reported below, on the main thread
+            errors.append(e)
+
+    threads = [threading.Thread(target=run, args=(i,)) for i in range(4)]
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join()
+    assert not errors, errors
+    for i, w in enumerate(cases):
+        o_ref, lse_ref, _ = oracle_decode(w)
+        check_o_lse(results[i][0], results[i][1], o_ref, lse_ref, f"thread {i}")
