@@ -248,6 +248,17 @@ smla_status smla_decode_host(const void *q_host, const void *kv_cache, int64_t n
                              int page_size, float scale, int nsplit, void *workspace,
                              size_t workspace_bytes, void *o_host, float *lse_host, void *stream);
 
+/*
+ * Self-test of the bounded waits (no counterpart on the pages).  Every wait in
+ * the library's kernels gives up after a time limit, raises a sticky timeout
+ * flag and lets the kernel return, so a broken pipeline never hangs the GPU.
+ * This launches one warp that waits on a barrier nothing arrives at, through
+ * the same wait routine, with limit_ns in [1e3, 1e9]; afterwards
+ * smla_check_device() reports SMLA_ERR_TIMEOUT (and clears it when asked).
+ * SMLA_ERR_INVALID_ARG for a limit outside the range.
+ */
+smla_status smla_selftest_wait_timeout(unsigned long long limit_ns, void *stream);
+
 /* Static text for a status code. */
 const char *smla_status_string(smla_status status);
 

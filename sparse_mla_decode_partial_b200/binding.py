@@ -40,6 +40,7 @@ SIGNATURES = {
     "smla_workspace_host_bytes": (_SZ, [_I, _I, _I, _I, _I, _I]),
     "smla_decode_host": (_I, [_P, _P, _I64, _P, _I, _P, _I, _I, _I, _I, _I, _F, _I, _P, _SZ, _P, _P,
                               _P]),
+    "smla_selftest_wait_timeout": (_I, [ctypes.c_ulonglong, _P]),
     "smla_check_device": (_I, [_I, ctypes.POINTER(ctypes.c_ulonglong), _P]),
     "smla_status_string": (ctypes.c_char_p, [_I]),
     "smla_last_error": (ctypes.c_char_p, []),
@@ -257,6 +258,14 @@ def check_device(clear: bool = True, stream=None):
     n = ctypes.c_ulonglong(0)
     st = lib().smla_check_device(1 if clear else 0, ctypes.byref(n), _stream(stream))
     return int(st), int(n.value)
+
+
+def selftest_wait_timeout(limit_ns: int, stream=None) -> None:
+    """Launch the bounded-wait self-test: one warp waits on a barrier that
+    nothing arrives at and gives up after limit_ns, raising the timeout flag
+    that check_device() then reports."""
+    _check(lib().smla_selftest_wait_timeout(int(limit_ns), _stream(stream)),
+           "smla_selftest_wait_timeout")
 
 
 def status_string(status: int) -> str:

@@ -551,6 +551,13 @@ smla_status smla_decode_host(const void *q_host, const void *kv_cache, int64_t n
                        scale, nsplit, workspace, hs.base, o_d, static_cast<float *>(lse_d), stream);
 }
 
+smla_status smla_selftest_wait_timeout(unsigned long long limit_ns, void *stream) {
+    if (limit_ns < 1000ull || limit_ns > 1000000000ull) return SMLA_ERR_INVALID_ARG;
+    smla::smla_selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns);
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? SMLA_OK : cuda_fail(e);
+}
+
 smla_status smla_check_device(int clear, unsigned long long *n_bad_index, void *stream) {
     cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e);

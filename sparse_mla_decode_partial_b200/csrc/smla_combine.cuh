@@ -30,6 +30,8 @@
 #include <cstdint>
 #include <cuda_bf16.h>
 
+#include "smla_ptx.cuh"
+
 namespace smla {
 
 constexpr int kCombineThreads = 512;
@@ -297,6 +299,21 @@ __global__ void __launch_bounds__(32 * kCombineWarpUnits)
         dst[j * 32] = make_uint2(*reinterpret_cast<uint32_t *>(&lo), *reinterpret_cast<uint32_t *>(&hi));
     }
     if (lane == 0) lse[u] = M + logf(L);
+}
+
+// Self-test of the bounded waits (smla_selftest_wait_timeout): one warp waits
+// on a fresh mbarrier that nothing ever arrives at, through the same
+// mbar_wait the kernels use, with the given limit.  The wait gives up, raises
+// the timeout flag and the kernel returns.
+__global__ void __launch_bounds__(32) smla_selftest_wait_kernel(unsigned long long limit_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+    }
+    __syncwarp();
+    bool dead = false;
+    mbar_wait(&bar, 0, dead, limit_ns);
 }
 
 // Copy of the per-step inputs of smla_decode_host from pinned host memory

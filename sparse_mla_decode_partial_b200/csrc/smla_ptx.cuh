@@ -79,12 +79,13 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
 // Returns false (and raises kFlagTimeout) when the limit is reached.  Once a
 // wait of this thread has timed out (`dead`), later waits return at once, so a
 // broken pipeline costs one time limit per thread, not one per wait.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, bool &dead) {
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, bool &dead,
+                                          unsigned long long limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     if (dead) return false;
     const uint64_t t0 = global_timer_ns();
     while (!mbar_try_wait(bar, parity)) {
-        if (global_timer_ns() - t0 > kWaitLimitNs) {
+        if (global_timer_ns() - t0 > limit_ns) {
             atomicOr(&g_status_flags, kFlagTimeout);
             dead = true;
             return false;

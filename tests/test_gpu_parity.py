@@ -183,6 +183,25 @@ def test_empty_topk():
     assert torch.all(o == 0) and torch.all(torch.isneginf(lse))
 
 
+def test_bounded_wait_gives_up_and_context_survives():
+    """A wait nothing will end (a barrier no thread arrives at) gives up after
+    its limit, raises the timeout status and the kernel returns; the context
+    then decodes normally."""
+    binding.check_device(clear=True)
+    with pytest.raises(binding.SmlaError):
+        binding.selftest_wait_timeout(10)                 # below the 1 us floor: refused
+    binding.selftest_wait_timeout(5_000_000)              # 5 ms
+    st, _ = binding.check_device(clear=False)
+    assert st == 7, binding.status_string(st)
+    assert binding.check_device(clear=True)[0] == 7
+    assert binding.check_device(clear=True)[0] == 0
+    w = small(seed=11, B=1, T=1, K=200)
+    o, lse = run_decode(w, 4)
+    assert binding.check_device(clear=True)[0] == 0
+    o_ref, lse_ref, _ = oracle_decode(w)
+    check_o_lse(o, lse, o_ref, lse_ref, "after timeout self-test")
+
+
 def test_out_of_range_entries_masked_and_counted():
     w = small(H=16, K=128, B=1, T=1)
     w.idx[0, 0, 3] = -5
