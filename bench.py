@@ -59,10 +59,18 @@ def workload_bytes(w):
     partial pass, per query token: every valid selected row once (1152 B),
     its page-table entry (4 B), the K index entries (4 B each) and q
     (H * 1152 B); the combine adds o (H * 1024 B) and lse (H * 4 B).
+    Dense variant: the T query tokens of a sequence attend to nested prefixes
+    of the same rows, so each row of the longest prefix counts once (with its
+    page-table entry), plus the visible lengths (4 B per query token) and the
+    K-entry position list that the library writes and the partial pass reads
+    (8 B per entry).
     """
-    valid = w.n_valid()
     BT = w.B * w.T
-    partial = valid * (1152 + 4) + BT * w.K * 4 + BT * w.H * 1152
+    if w.dense:
+        rows = int(w.seq_lens.max(dim=1).values.to(__import__("torch").int64).sum())
+        partial = rows * (1152 + 4) + BT * (4 + w.K * 8) + BT * w.H * 1152
+    else:
+        partial = w.n_valid() * (1152 + 4) + BT * w.K * 4 + BT * w.H * 1152
     step = partial + BT * w.H * (1024 + 4)
     return partial, step
 
@@ -73,8 +81,16 @@ def workload_flops(w):
 
 
 def describe(w):
-    return (f"B{w.B} T{w.T} H{w.H} K{w.K} dc512+dr64 bf16, paged cache page64, "
+    sel = (f"dense causal prefixes of {int(w.seq_lens.min())}..{w.K} positions" if w.dense
+           else f"K{w.K}")
+    return (f"B{w.B} T{w.T} H{w.H} {sel} dc512+dr64 bf16, paged cache page64, "
             f"{w.num_pages} pages, ctx {min(w.ctx_lens)}..{max(w.ctx_lens)}")
+
+
+def data_note(w):
+    sel = ("every visible position of each draft token (dense causal verify)" if w.dense
+           else "distinct random top-k indices")
+    return f"synthetic (seeded N(0,1)*0.5 bf16 q and cache, {sel})"
 
 
 def measured_traffic(workload: str):
@@ -244,7 +260,10 @@ def cpu_baseline(w, budget_s: float):
     import oracle
     bits = lambda t: t.contiguous().view(__import__("torch").int16).numpy().view(np.uint16)
     q, cache = bits(w.q), bits(w.cache)
-    pt, idx = w.page_table.numpy(), w.idx.numpy()
+    pt = w.page_table.numpy()
+    # the dense variant's lists are every visible position (the oracle's own
+    # construction); the sparse workloads carry theirs
+    idx = oracle.dense_positions(w.seq_lens.numpy(), w.K) if w.dense else w.idx.numpy()
     threads = oracle.max_threads()
     units = w.B * w.T * w.H
     # one query token first, to size the sample
@@ -264,7 +283,7 @@ def cpu_baseline(w, budget_s: float):
     el = time.perf_counter() - t0
     tokens = reps * len(bt)
     sample = (f"{len(bt)} of {w.B * w.T} query tokens of one step (all {w.H} heads, "
-              f"K={w.K}) x {reps} repeats")
+              f"{'dense, up to ' if w.dense else ''}K={w.K}) x {reps} repeats")
     # the same oracle on one thread, over the first query token (a few repeats)
     oracle.set_threads(1)
     try:
@@ -321,14 +340,36 @@ def run_ours(args, world, rank, local):
         po = torch.empty(max(n * 512, 4), dtype=torch.float32, device=dev)
         pm = torch.empty(max(n, 1), dtype=torch.float32, device=dev)
         pl = torch.empty(max(n, 1), dtype=torch.float32, device=dev)
-        ws = torch.empty(max(16, binding.workspace_bytes(B, T, H, S)), dtype=torch.uint8, device=dev)
         o = torch.empty((B, T, H, 512), dtype=torch.bfloat16, device=dev)
         lse = torch.empty((B, T, H), dtype=torch.float32, device=dev)
+        if w.dense:
+            # smla_decode_dense writes the position lists after the split-K
+            # partials in its workspace (the layout include/smla.h states); the
+            # partial-only step reads them from there
+            ws = torch.empty(max(16, binding.dense_workspace_bytes(B, T, H, K, S)),
+                             dtype=torch.uint8, device=dev)
+            dense_args = (w.q.data_ptr(), w.cache.data_ptr(), w.num_pages, w.page_table.data_ptr(),
+                          w.pt_stride, w.seq_lens.data_ptr(), B, T, H, K, 64, w.scale)
+            st = lib.smla_decode_dense(*dense_args, S, ws.data_ptr(), ws.numel(), o.data_ptr(),
+                                       lse.data_ptr(), sptr)
+            if st != 0:
+                raise RuntimeError(binding.status_string(st))
+            base = binding.workspace_bytes(B, T, H, S) if S > 1 else 0
+            idx_ptr = ws.data_ptr() + (base + 255) // 256 * 256
+        else:
+            ws = torch.empty(max(16, binding.workspace_bytes(B, T, H, S)), dtype=torch.uint8,
+                             device=dev)
+            idx_ptr = w.idx.data_ptr()
         args_common = (w.q.data_ptr(), w.cache.data_ptr(), w.num_pages, w.page_table.data_ptr(),
-                       w.pt_stride, w.idx.data_ptr(), B, T, H, K, 64, w.scale)
+                       w.pt_stride, idx_ptr, B, T, H, K, 64, w.scale)
 
         def decode():
-            """One whole decode: smla_decode (partial pass + LSE combine)."""
+            """One whole decode: smla_decode (partial pass + LSE combine), or
+            smla_decode_dense (position lists, partial pass, combine)."""
+            if w.dense:
+                st = lib.smla_decode_dense(*dense_args, S, ws.data_ptr(), ws.numel(),
+                                           o.data_ptr(), lse.data_ptr(), sptr)
+                return st, (2 if S == 1 else 3)
             st = lib.smla_decode(*args_common, S, ws.data_ptr(), ws.numel(), o.data_ptr(),
                                  lse.data_ptr(), sptr)
             return st, (1 if S == 1 else 2)
@@ -381,7 +422,37 @@ def run_ours(args, world, rank, local):
     # page table over the host link with a copy kernel and writes o, lse
     # straight back into host memory; all of it inside the timed region.
     e2e = None
-    if True:
+    if w_host.dense:
+        # the dense entry point takes device buffers: the step's q, visible
+        # lengths and page table are copied from pinned host memory first, o
+        # and lse back after, all on the launching stream inside the interval
+        q_h, len_h = w_host.q.pin_memory(), w_host.seq_lens.pin_memory()
+        pt_h = w_host.page_table.pin_memory()
+        o_h = torch.empty((B, T, H, 512), dtype=torch.bfloat16).pin_memory()
+        lse_h = torch.empty((B, T, H), dtype=torch.float32).pin_memory()
+        q_d, len_d, pt_d = torch.empty_like(w.q), torch.empty_like(w.seq_lens), torch.empty_like(w.page_table)
+        o_d = torch.empty((B, T, H, 512), dtype=torch.bfloat16, device=dev)
+        lse_d = torch.empty((B, T, H), dtype=torch.float32, device=dev)
+        ws_e = torch.empty(max(16, binding.dense_workspace_bytes(B, T, H, K, nsplit)),
+                           dtype=torch.uint8, device=dev)
+        h2d = q_h.numel() * 2 + len_h.numel() * 4 + pt_h.numel() * 4
+        d2h = o_h.numel() * 2 + lse_h.numel() * 4
+
+        def e2e_step():
+            q_d.copy_(q_h, non_blocking=True)
+            len_d.copy_(len_h, non_blocking=True)
+            pt_d.copy_(pt_h, non_blocking=True)
+            st = lib.smla_decode_dense(q_d.data_ptr(), w.cache.data_ptr(), w.num_pages,
+                                       pt_d.data_ptr(), w.pt_stride, len_d.data_ptr(), B, T, H, K,
+                                       64, w.scale, nsplit, ws_e.data_ptr(), ws_e.numel(),
+                                       o_d.data_ptr(), lse_d.data_ptr(), sptr)
+            o_h.copy_(o_d, non_blocking=True)
+            lse_h.copy_(lse_d, non_blocking=True)
+            return st
+        e2e_note = ("smla_decode_dense every step: q, visible lengths and page table copied from "
+                    "pinned host memory, o and lse copied back, on the launching stream; the "
+                    "latent cache stays resident")
+    else:
         q_h = w_host.q.pin_memory()
         idx_h = w_host.idx.pin_memory()
         pt_h = w_host.page_table.pin_memory()
@@ -397,7 +468,10 @@ def run_ours(args, world, rank, local):
                                         pt_h.data_ptr(), w.pt_stride, idx_h.data_ptr(), B, T, H, K,
                                         64, w.scale, nsplit, ws_h.data_ptr(), ws_h.numel(),
                                         o_h.data_ptr(), lse_h.data_ptr(), sptr)
-
+        e2e_note = ("smla_decode_host every step: q, top-k indices and page table read from "
+                    "pinned host memory by the library's copy kernel, o and lse written straight "
+                    "into pinned host memory; the latent cache stays resident")
+    if True:
         for _ in range(3):
             e2e_step()
         torch.cuda.synchronize(dev)
@@ -415,10 +489,7 @@ def run_ours(args, world, rank, local):
             times.append(e0.elapsed_time(e1))
         e2e_ms = max_over_ranks(statistics.fmean(times), world)
         e2e = {"value": tokens_all / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
-               "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
-               "note": "smla_decode_host every step: q, top-k indices and page table read "
-                       "from pinned host memory by the library's copy kernel, o and lse written "
-                       "straight into pinned host memory; the latent cache stays resident"}
+               "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "note": e2e_note}
 
     # Warm-L2 reference (after the timed region, not part of value): the same
     # step back to back without the flush, so the selected rows may still sit
@@ -465,7 +536,7 @@ def run_ours(args, world, rank, local):
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step_max, 6),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic (seeded N(0,1)*0.5 bf16 q and cache, distinct random top-k indices)",
+        "data": data_note(w_host),
         "config": {"workload": args.workload, "shape": describe(w_host), "nsplit": nsplit,
                    "nsplit_policy": "explicit" if args.nsplit else "heuristic",
                    "batch": B, "q_len": T, "heads": H, "topk": K,
@@ -514,7 +585,7 @@ def run_reference(args, world, rank):
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(w.B * w.T / value * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic (seeded N(0,1)*0.5 bf16 q and cache, distinct random top-k indices)",
+        "data": data_note(w),
         "config": {"workload": args.workload, "shape": describe(w), "nsplit": nsplit,
                    "batch": w.B, "q_len": w.T, "heads": w.H, "topk": w.K},
         "impl": "reference",

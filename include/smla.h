@@ -249,6 +249,40 @@ smla_status smla_decode_host(const void *q_host, const void *kv_cache, int64_t n
                              size_t workspace_bytes, void *o_host, float *lse_host, void *stream);
 
 /*
+ * Dense-context decode: the KV-split verify variant.
+ *
+ * "The Occupancy Hypothesis: How One Kernel Parameter Unlocked 1.8x Decode
+ * Speedup on Blackwell", sections "The Road to This Experiment", "The
+ * Occupancy Insight" and "The Broader Context": the speculative-decoding
+ * verify kernel attends each of q_len query tokens to its whole visible KV
+ * sequence (46K tokens there), split into NSPLIT chunks, each a partial pass,
+ * merged by a reduce.  Here query token (b, t) attends to the positions
+ * 0 .. seq_lens[b*T + t] - 1 of sequence b, mapped through the page table
+ * like a sparse index.  For causal verify of T draft tokens appended at the
+ * end of a sequence of n tokens, seq_lens[b*T + t] = n - T + t + 1.
+ *
+ *  - seq_lens  int32 [B, T], device memory, each in [0, K].  A length outside
+ *              that range is clamped to it and raises SMLA_ERR_INDEX_RANGE in
+ *              smla_check_device (counted once per query token).
+ *  - K         the longest visible length (the width of the index lists the
+ *              call builds); the NSPLIT heuristic sees this K.
+ *  - All other arguments, layouts, the nsplit rule and the outputs are those
+ *    of smla_decode.  Positions beyond a sequence's pages are masked and
+ *    counted as smla_decode does for out-of-range indices.
+ *  - workspace_bytes must be at least smla_dense_workspace_bytes(B, T, H, K,
+ *    nsplit) for the nsplit actually used: the split-K partials followed by
+ *    the B*T*K int32 index lists, which one small kernel writes before the
+ *    sparse decode runs on them.  Else SMLA_ERR_WORKSPACE_TOO_SMALL; a
+ *    workspace not 16-byte aligned gives SMLA_ERR_MISALIGNED.
+ */
+size_t smla_dense_workspace_bytes(int B, int T, int H, int K, int nsplit);
+smla_status smla_decode_dense(const void *q, const void *kv_cache, int64_t num_pages,
+                              const int32_t *page_table, int pt_stride, const int32_t *seq_lens,
+                              int B, int T, int H, int K, int page_size, float scale, int nsplit,
+                              void *workspace, size_t workspace_bytes, void *o, float *lse,
+                              void *stream);
+
+/*
  * Self-test of the bounded waits (no counterpart on the pages).  Every wait in
  * the library's kernels gives up after a time limit, raises a sticky timeout
  * flag and lets the kernel return, so a broken pipeline never hangs the GPU.

@@ -3,7 +3,8 @@
 Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
 ``bench.py`` may import this package.  The CUDA library never uses it.
 """
-from .oracle import DC, DR, PAGE_SIZE, build, combine, decode, max_threads, partial, set_threads
+from .oracle import (DC, DR, PAGE_SIZE, build, combine, decode, decode_dense, dense_positions,
+                     max_threads, partial, set_threads)
 
-__all__ = ["DC", "DR", "PAGE_SIZE", "build", "combine", "decode", "max_threads",
-           "partial", "set_threads"]
+__all__ = ["DC", "DR", "PAGE_SIZE", "build", "combine", "decode", "decode_dense",
+           "dense_positions", "max_threads", "partial", "set_threads"]

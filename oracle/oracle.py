@@ -170,3 +170,35 @@ def combine(part_o, part_m, part_lse, *, lib=None):
                             o.ctypes.data_as(ctypes.c_void_p),
                             lse.ctypes.data_as(ctypes.c_void_p))
     return o, lse
+
+
+def dense_positions(seq_lens, K):
+    """Index lists of the dense-context (KV-split verify) variant: query token
+    (b, t) attends to every position 0 .. seq_lens[b, t] - 1 of its sequence,
+    so its list is those positions followed by -1 up to width K.
+
+    "The Occupancy Hypothesis: How One Kernel Parameter Unlocked 1.8x Decode
+    Speedup on Blackwell", sections "The Occupancy Insight" and "The Broader
+    Context": the verify kernel divides each query token's whole KV sequence
+    into NSPLIT splits (2875 tokens per split at 46K and NSPLIT 16), with a
+    partial pass and a reduce.  The visible prefix length is an input.
+    """
+    seq_lens = np.asarray(seq_lens, np.int64)
+    if seq_lens.ndim != 2:
+        raise ValueError("seq_lens must be [B, T]")
+    if seq_lens.size and (seq_lens.min() < 0 or seq_lens.max() > K):
+        raise ValueError("seq_lens must lie in [0, K]")
+    j = np.arange(K, dtype=np.int64)
+    return np.where(j[None, None, :] < seq_lens[..., None], j, -1).astype(np.int32)
+
+
+def decode_dense(q, cache, page_table, seq_lens, scale, *, K=None, dc=DC, dr=DR,
+                 page_size=PAGE_SIZE, lib=None):
+    """Dense-context decode: the sparse definition over each query token's
+    full visible prefix (``dense_positions``).  Returns (o, lse, n_bad)."""
+    seq_lens = np.asarray(seq_lens, np.int64)
+    if K is None:
+        K = int(seq_lens.max()) if seq_lens.size else 0
+    return decode(q, cache, page_table, dense_positions(seq_lens, K), scale, dc=dc, dr=dr,
+                  page_size=page_size, lib=lib)
+

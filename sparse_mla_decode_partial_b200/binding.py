@@ -40,6 +40,9 @@ SIGNATURES = {
     "smla_workspace_host_bytes": (_SZ, [_I, _I, _I, _I, _I, _I]),
     "smla_decode_host": (_I, [_P, _P, _I64, _P, _I, _P, _I, _I, _I, _I, _I, _F, _I, _P, _SZ, _P, _P,
                               _P]),
+    "smla_dense_workspace_bytes": (_SZ, [_I, _I, _I, _I, _I]),
+    "smla_decode_dense": (_I, [_P, _P, _I64, _P, _I, _P, _I, _I, _I, _I, _I, _F, _I, _P, _SZ, _P,
+                               _P, _P]),
     "smla_selftest_wait_timeout": (_I, [ctypes.c_ulonglong, _P]),
     "smla_check_device": (_I, [_I, ctypes.POINTER(ctypes.c_ulonglong), _P]),
     "smla_status_string": (ctypes.c_char_p, [_I]),
@@ -213,6 +216,53 @@ def decode_noalloc(q, cache, page_table, idx, scale: float, nsplit: int = 0, *, 
                                      pt_stride, _ptr(idx), B, T, H, K, PAGE_SIZE, float(scale),
                                      int(nsplit), _ptr(o), _ptr(lse), _stream(stream)),
            "smla_decode_noalloc")
+    return o, lse
+
+
+def dense_workspace_bytes(B: int, T: int, H: int, K: int, nsplit: int) -> int:
+    return int(lib().smla_dense_workspace_bytes(B, T, H, K, nsplit))
+
+
+def decode_dense(q, cache, page_table, seq_lens, scale: float, nsplit: int = 0, *, K=None,
+                 workspace=None, o=None, lse=None, stream=None):
+    """Dense-context decode (KV-split verify): query token (b, t) attends to
+    positions 0 .. seq_lens[b, t] - 1 of sequence b.  K defaults to the longest
+    length (read from seq_lens, which synchronises); pass it to stay
+    asynchronous.  Returns (o bf16 [B,T,H,512], lse fp32 [B,T,H])."""
+    _need(q, torch.bfloat16, "q")
+    dev = q.device
+    _need(cache, torch.bfloat16, "cache", dev)
+    _need(page_table, torch.int32, "page_table", dev)
+    _need(seq_lens, torch.int32, "seq_lens", dev)
+    if q.dim() != 4 or q.shape[-1] != D:
+        raise ValueError(f"q must be [B,T,H,{D}]")
+    B, T, H, _ = q.shape
+    if tuple(seq_lens.shape) != (B, T):
+        raise ValueError("seq_lens must be [B,T]")
+    if page_table.dim() != 2 or page_table.shape[0] != B:
+        raise ValueError("page_table must be [B, pt_stride]")
+    if cache.numel() % (PAGE_SIZE * D):
+        raise ValueError("cache must be [num_pages, 64, 576]")
+    num_pages = cache.numel() // (PAGE_SIZE * D)
+    if K is None:
+        K = int(seq_lens.max().item()) if seq_lens.numel() else 0
+    if nsplit == 0:
+        nsplit = choose_nsplit(B, T, H, K, 0)
+    need = dense_workspace_bytes(B, T, H, K, nsplit)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    _need(workspace, torch.uint8, "workspace", dev)
+    if o is None:
+        o = torch.empty((B, T, H, DC), dtype=torch.bfloat16, device=dev)
+    if lse is None:
+        lse = torch.empty((B, T, H), dtype=torch.float32, device=dev)
+    _need(o, torch.bfloat16, "o", dev)
+    _need(lse, torch.float32, "lse", dev)
+    _check(lib().smla_decode_dense(_ptr(q), _ptr(cache), num_pages, _ptr(page_table),
+                                   page_table.shape[1], _ptr(seq_lens), B, T, H, int(K),
+                                   PAGE_SIZE, float(scale), int(nsplit), _ptr(workspace),
+                                   workspace.numel(), _ptr(o), _ptr(lse), _stream(stream)),
+           "smla_decode_dense")
     return o, lse
 
 

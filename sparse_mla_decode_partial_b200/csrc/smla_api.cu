@@ -22,6 +22,7 @@
 #define SMLA_MMA_STAGES 2
 #endif
 #include "smla_combine.cuh"
+#include "smla_dense.cuh"
 #include "smla_partial_mma.cuh"
 #include "smla_partial_tc.cuh"
 
@@ -549,6 +550,49 @@ smla_status smla_decode_host(const void *q_host, const void *kv_cache, int64_t n
     return smla_decode(ws + hs.q, kv_cache, num_pages, reinterpret_cast<const int32_t *>(ws + hs.pt),
                        pt_stride, reinterpret_cast<const int32_t *>(ws + hs.idx), B, T, H, K, page_size,
                        scale, nsplit, workspace, hs.base, o_d, static_cast<float *>(lse_d), stream);
+}
+
+// ---------------------------------------------------------------------------
+// Dense-context decode (see include/smla.h): the index lists are every visible
+// position, written into the workspace by smla_dense_index_kernel, then the
+// sparse decode runs on them.
+size_t smla_dense_workspace_bytes(int B, int T, int H, int K, int nsplit) {
+    if (B < 0 || T < 0 || H < 0 || K < 0 || nsplit < 1 || nsplit > SMLA_MAX_NSPLIT) return 0;
+    const size_t base = nsplit > 1 ? smla_workspace_bytes(B, T, H, nsplit) : 0;
+    return round256(base) + round256((size_t)B * T * K * sizeof(int32_t));
+}
+
+smla_status smla_decode_dense(const void *q, const void *kv_cache, int64_t num_pages,
+                              const int32_t *page_table, int pt_stride, const int32_t *seq_lens,
+                              int B, int T, int H, int K, int page_size, float scale, int nsplit,
+                              void *workspace, size_t workspace_bytes, void *o, float *lse,
+                              void *stream) {
+    smla_status st = check_decode_args(q, kv_cache, num_pages, page_table, pt_stride, seq_lens, B,
+                                       T, H, K, page_size, scale);
+    if (st != SMLA_OK) return st;
+    if (nsplit < 0 || nsplit > SMLA_MAX_NSPLIT) return SMLA_ERR_INVALID_ARG;
+    if (B == 0 || T == 0 || H == 0) return SMLA_OK;
+    if (o == nullptr || lse == nullptr) return SMLA_ERR_INVALID_ARG;
+    if (!aligned(o, 16) || !aligned(lse, 4)) return SMLA_ERR_MISALIGNED;
+    if (nsplit == 0) nsplit = smla_choose_nsplit(B, T, H, K, 0);
+    if (K == 0)  // every list is empty: o = 0, lse = -inf
+        return smla_decode(q, kv_cache, num_pages, page_table, pt_stride, seq_lens, B, T, H, 0,
+                           page_size, scale, nsplit, workspace, workspace_bytes, o, lse, stream);
+    if (workspace_bytes < smla_dense_workspace_bytes(B, T, H, K, nsplit))
+        return SMLA_ERR_WORKSPACE_TOO_SMALL;
+    if (workspace == nullptr) return SMLA_ERR_INVALID_ARG;
+    if (!aligned(workspace, 16)) return SMLA_ERR_MISALIGNED;
+    const size_t base = nsplit > 1 ? smla_workspace_bytes(B, T, H, nsplit) : 0;
+    int32_t *idx = reinterpret_cast<int32_t *>(static_cast<uint8_t *>(workspace) + round256(base));
+    const long long n_bt = (long long)B * T;
+    const long long total = n_bt * K;
+    const unsigned blocks = (unsigned)std::min<long long>((total + 255) / 256, 148 * 8);
+    smla::smla_dense_index_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        seq_lens, n_bt, K, idx);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e);
+    return smla_decode(q, kv_cache, num_pages, page_table, pt_stride, idx, B, T, H, K, page_size,
+                       scale, nsplit, workspace, base, o, lse, stream);
 }
 
 smla_status smla_selftest_wait_timeout(unsigned long long limit_ns, void *stream) {

@@ -46,6 +46,11 @@ class Workload:
     ctx_lens: list             # tokens owned by each sequence
     nsplit: Optional[int]      # the configuration's fixed NSPLIT, None = heuristic
     nsplit_sweep: tuple        # NSPLIT values the configuration sweeps
+    seq_lens: Optional[torch.Tensor] = None  # int32 [B,T]: dense variant's visible lengths
+
+    @property
+    def dense(self) -> bool:
+        return self.seq_lens is not None
 
     @property
     def B(self):
@@ -61,6 +66,8 @@ class Workload:
 
     @property
     def K(self):
+        if self.dense:
+            return int(self.seq_lens.max()) if self.seq_lens.numel() else 0
         return self.idx.shape[2]
 
     @property
@@ -72,13 +79,17 @@ class Workload:
         return self.page_table.shape[1]
 
     def n_valid(self) -> int:
-        """Number of non-padding index entries over the whole batch."""
+        """Number of attended rows (non-padding index entries, or visible
+        positions of the dense variant) over the whole batch."""
+        if self.dense:
+            return int(self.seq_lens.to(torch.int64).sum())
         return int((self.idx >= 0).sum())
 
     def to(self, device) -> "Workload":
         return dataclasses.replace(
             self, q=self.q.to(device), cache=self.cache.to(device),
-            page_table=self.page_table.to(device), idx=self.idx.to(device))
+            page_table=self.page_table.to(device), idx=self.idx.to(device),
+            seq_lens=None if self.seq_lens is None else self.seq_lens.to(device))
 
 
 def _normal_bf16(shape, gen, chunk_rows=1 << 14) -> torch.Tensor:
@@ -147,6 +158,21 @@ def mixed_ctx_lens(B: int, seed: int, lo: int = 1024, hi: int = 131072) -> list:
     return [int(min(max(v, lo), hi)) for v in lens.tolist()]
 
 
+def make_dense_workload(name: str, *, B: int, T: int, H: int, ctx_lens: Sequence[int],
+                        seed: int, paged: bool = True, scale: Optional[float] = None,
+                        nsplit: Optional[int] = None, nsplit_sweep: Sequence[int] = ()) -> Workload:
+    """Draw a dense-context (verify) workload: the cache and query as
+    ``make_workload`` draws them, no index lists, and ``seq_lens[b, t] =
+    ctx_lens[b] - T + t + 1``: the sequence ends with its ``T`` draft tokens
+    and token ``t`` sees every position up to and including its own."""
+    w = make_workload(name, B=B, T=T, H=H, K=0, ctx_lens=ctx_lens, seed=seed, paged=paged,
+                      scale=scale, nsplit=nsplit, nsplit_sweep=nsplit_sweep)
+    lens = torch.tensor([[c - T + t + 1 for t in range(T)] for c in w.ctx_lens], dtype=torch.int32)
+    if int(lens.min()) < 0:
+        raise ValueError("every context must hold its T draft tokens")
+    return dataclasses.replace(w, seq_lens=lens)
+
+
 # name -> (description, builder)
 def tiny(seed: int = 0) -> Workload:
     """B1 T1 H8 K256, contiguous 4096-token cache, NSPLIT 4."""
@@ -179,10 +205,18 @@ def mixed(seed: int = 4, B: int = 60) -> Workload:
                          ctx_lens=mixed_ctx_lens(B, seed), seed=seed)
 
 
+def dense_verify(seed: int = 5) -> Workload:
+    """B1 T9 H8, 46080-token context + 9 draft tokens, dense causal verify
+    (every visible position), NSPLIT swept over {16, 64} as on the pages."""
+    return make_dense_workload("dense_verify", B=1, T=9, H=8, ctx_lens=[46080 + 9], seed=seed,
+                               nsplit_sweep=(16, 64))
+
+
 WORKLOADS = {
     "tiny": tiny,
     "single_request": single_request,
     "spec_verify": spec_verify,
     "batched": batched,
     "mixed": mixed,
+    "dense_verify": dense_verify,
 }

@@ -22,6 +22,8 @@ def bits(t: torch.Tensor) -> np.ndarray:
 def oracle_decode(w, sample=None):
     """Oracle o/lse for workload ``w``; ``sample`` = list of (b, t) to evaluate
     (returns arrays stacked in that order), or None for the whole batch."""
+    if w.dense:
+        return oracle_decode_dense(w, sample)
     q, cache, pt, idx = bits(w.q), bits(w.cache), w.page_table.cpu().numpy(), w.idx.cpu().numpy()
     if sample is None:
         o, lse, bad = oracle.decode(q, cache, pt, idx, w.scale)
@@ -30,6 +32,21 @@ def oracle_decode(w, sample=None):
     for b, t in sample:
         o, lse, n = oracle.decode(q[b:b + 1, t:t + 1], cache, pt[b:b + 1], idx[b:b + 1, t:t + 1],
                                   w.scale)
+        os_.append(o[0, 0])
+        ls_.append(lse[0, 0])
+        bad += n
+    return np.stack(os_), np.stack(ls_), bad
+
+
+def oracle_decode_dense(w, sample=None):
+    q, cache, pt = bits(w.q), bits(w.cache), w.page_table.cpu().numpy()
+    lens = w.seq_lens.cpu().numpy()
+    if sample is None:
+        return oracle.decode_dense(q, cache, pt, lens, w.scale)
+    os_, ls_, bad = [], [], 0
+    for b, t in sample:
+        o, lse, n = oracle.decode_dense(q[b:b + 1, t:t + 1], cache, pt[b:b + 1],
+                                        lens[b:b + 1, t:t + 1], w.scale)
         os_.append(o[0, 0])
         ls_.append(lse[0, 0])
         bad += n

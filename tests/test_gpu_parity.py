@@ -6,6 +6,8 @@ problem statement's: o max-abs <= 1e-2 and relative L2 <= 5e-3, lse <= 1e-3
 and mixed-length workloads, run in the launch configuration the benchmark
 times (heuristic NSPLIT), compare sampled query tokens.
 """
+import dataclasses
+
 import numpy as np
 import pytest
 import torch
@@ -420,6 +422,74 @@ def test_two_tile_splits(H, K, S):
     o, lse = run_decode(w, S)
     o_ref, lse_ref, _ = oracle_decode(w)
     check_o_lse(o, lse, o_ref, lse_ref, f"two tiles H={H} K={K} S={S}")
+
+
+# ------------------------------------------------------------------ dense-context variant
+# ("The Occupancy Hypothesis ...", sections "The Occupancy Insight" and "The
+# Broader Context": the verify kernel splits each query token's whole visible
+# KV sequence)
+def run_dense(w, nsplit, **kw):
+    wd = w.to(DEV)
+    o, lse = binding.decode_dense(wd.q, wd.cache, wd.page_table, wd.seq_lens, w.scale, nsplit,
+                                  K=w.K, **kw)
+    torch.cuda.synchronize()
+    return o, lse
+
+
+@pytest.mark.parametrize("H,T,ctx,S", [(8, 9, 3000, 0), (8, 9, 3000, 16), (16, 3, 777, 5),
+                                       (64, 2, 1500, 0), (64, 2, 1500, 3), (8, 4, 40, 1),
+                                       (16, 2, 100, 64), (24, 5, 2100, 0)])
+def test_dense_against_oracle(H, T, ctx, S):
+    w = workloads.make_dense_workload("dense", B=2, T=T, H=H, ctx_lens=[ctx, max(T, ctx // 2 + 7)],
+                                      seed=H + T + S)
+    o, lse = run_dense(w, S)
+    o_ref, lse_ref, _ = oracle_decode(w)
+    check_o_lse(o, lse, o_ref, lse_ref, f"dense H={H} T={T} ctx={ctx} S={S}")
+
+
+@pytest.fixture(scope="module")
+def dense_verify_ref():
+    w = workloads.dense_verify()
+    o_ref, lse_ref, bad = oracle_decode(w)
+    assert bad == 0
+    return w, o_ref, lse_ref
+
+
+@pytest.mark.parametrize("nsplit", [16, 64, 0])
+def test_dense_verify_config(dense_verify_ref, nsplit):
+    """B1 T9 H8 at 46080 + 9 tokens, every output compared."""
+    w, o_ref, lse_ref = dense_verify_ref
+    o, lse = run_dense(w, nsplit)
+    check_o_lse(o, lse, o_ref, lse_ref, f"dense_verify S={nsplit}")
+
+
+def test_dense_lengths_out_of_range_are_clamped_and_counted():
+    w = workloads.make_dense_workload("dense_bad", B=2, T=2, H=16, ctx_lens=[300, 300], seed=9)
+    K = 290
+    lens = w.seq_lens.clone()
+    lens[0, 1] = K + 7                        # clamped to K
+    lens[1, 0] = -3                           # clamped to 0: o = 0, lse = -inf
+    w = dataclasses.replace(w, seq_lens=lens)
+    binding.check_device(clear=True)
+    wd = w.to(DEV)
+    o, lse = binding.decode_dense(wd.q, wd.cache, wd.page_table, wd.seq_lens, w.scale, 4, K=K)
+    st, n = binding.check_device(clear=True)
+    assert st == 5 and n == 2, (binding.status_string(st), n)
+    ref = dataclasses.replace(w, seq_lens=lens.clamp(0, K))
+    o_ref, lse_ref, _ = oracle_decode(ref)
+    check_o_lse(o, lse, o_ref, lse_ref, "dense clamped lengths")
+
+
+def test_dense_positions_past_the_page_table_are_masked_and_counted():
+    w = workloads.make_dense_workload("dense_pt", B=1, T=2, H=16, ctx_lens=[100], seed=3)
+    lens = torch.tensor([[90, 200]], dtype=torch.int32)   # 2 pages = 128 positions mapped
+    w = dataclasses.replace(w, seq_lens=lens)
+    binding.check_device(clear=True)
+    o, lse = run_dense(w, 4)
+    st, n = binding.check_device(clear=True)
+    o_ref, lse_ref, bad = oracle_decode(w)
+    assert st == 5 and n == 200 - 128 == bad // w.H
+    check_o_lse(o, lse, o_ref, lse_ref, "dense past the page table")
 
 
 # ------------------------------------------------------------------ per-step data in host memory

@@ -97,6 +97,35 @@ def test_decode_rejects_bad_arguments(lib, kw, expect):
     assert call_decode(lib, **kw) == expect
 
 
+def call_dense(lib, q=FAKE, cache=FAKE, num_pages=10, pt=FAKE, pt_stride=4, lens=FAKE, B=1, T=9,
+               H=8, K=200, ps=64, scale=0.1, nsplit=2, ws=FAKE, ws_bytes=1 << 30, o=FAKE,
+               lse=FAKE):
+    return lib.smla_decode_dense(q, cache, num_pages, pt, pt_stride, lens, B, T, H, K, ps, scale,
+                                 nsplit, ws, ws_bytes, o, lse, None)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(ws_bytes=100), 4), (dict(ws=0), 1), (dict(ws=FAKE + 8), 3), (dict(o=FAKE + 8), 3),
+    (dict(lse=FAKE + 2), 3), (dict(o=0), 1), (dict(lens=0), 1), (dict(lens=FAKE + 2), 3),
+    (dict(nsplit=-1), 1), (dict(nsplit=1025), 1), (dict(ps=16), 2), (dict(H=65), 2),
+    (dict(K=-1), 1), (dict(scale=math.nan), 1), (dict(cache=0), 1), (dict(pt=0), 1),
+    (dict(B=0), 0), (dict(T=0), 0), (dict(H=0), 0),
+])
+def test_decode_dense_rejects_bad_arguments(lib, kw, expect):
+    assert call_dense(lib, **kw) == expect
+
+
+def test_dense_workspace_bytes_formula(lib):
+    """Split-K partials (none at nsplit 1), then the B*T*K int32 index lists."""
+    r = lambda x: (x + 255) // 256 * 256
+    for B, T, H, K, S in [(1, 9, 8, 46089, 32), (1, 9, 8, 46089, 1), (2, 3, 16, 777, 5),
+                          (1, 1, 64, 0, 4)]:
+        base = binding.workspace_bytes(B, T, H, S) if S > 1 else 0
+        assert binding.dense_workspace_bytes(B, T, H, K, S) == r(base) + r(B * T * K * 4)
+    assert binding.dense_workspace_bytes(1, 1, 1, 1, 0) == 0
+    assert binding.dense_workspace_bytes(1, 1, 1, -1, 1) == 0
+
+
 def test_combine_rejects_bad_arguments(lib):
     c = lambda **kw: lib.smla_lse_combine(kw.get("po", FAKE), kw.get("pm", FAKE),
                                           kw.get("pl", FAKE), kw.get("B", 1), 1, 16,

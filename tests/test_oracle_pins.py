@@ -349,3 +349,85 @@ def test_large_scores_no_overflow():
     oc, lc = oracle.combine(po, pm, pl)
     np.testing.assert_allclose(oc, o, rtol=1e-10, atol=1e-12)
     np.testing.assert_allclose(lc, lse, rtol=1e-13)
+
+
+# ---------------------------------------------------------------- dense-context variant
+# "The Occupancy Hypothesis: How One Kernel Parameter Unlocked 1.8x Decode
+# Speedup on Blackwell", sections "The Occupancy Insight" and "The Broader
+# Context": the verify kernel splits each query token's whole visible KV
+# sequence.  The oracle builds the positions 0 .. n-1 as an index list and
+# runs the sparse definition pinned above; these pins fix the list.
+def dense_workload(B=2, T=3, H=3, ctx=(200, 130), seed=21):
+    return workloads.make_dense_workload("pin_dense", B=B, T=T, H=H, ctx_lens=list(ctx), seed=seed)
+
+
+def dense_arrays(w):
+    return torch_bits(w.q), torch_bits(w.cache), w.page_table.numpy(), w.seq_lens.numpy()
+
+
+def test_dense_positions_hand_case():
+    got = oracle.dense_positions([[3, 0], [4, 1]], 4)
+    want = [[[0, 1, 2, -1], [-1, -1, -1, -1]], [[0, 1, 2, 3], [0, -1, -1, -1]]]
+    np.testing.assert_array_equal(got, np.asarray(want, np.int32))
+    for bad in ([[5]], [[-1]]):
+        with pytest.raises(ValueError):
+            oracle.dense_positions(bad, 4)
+
+
+def test_dense_workload_lengths_are_causal():
+    """Draft token t of a sequence of n tokens sees n - T + t + 1 positions."""
+    w = dense_workload()
+    np.testing.assert_array_equal(w.seq_lens.numpy(), [[198, 199, 200], [128, 129, 130]])
+
+
+def test_dense_single_position_returns_first_row_exactly():
+    w = dense_workload()
+    q, cache, pt, _ = dense_arrays(w)
+    o, lse, bad = oracle.decode_dense(q, cache, pt, np.ones((2, 3), np.int32), w.scale)
+    assert bad == 0
+    rows = cache.reshape(-1, 576)
+    for b in range(2):
+        want = bits_to_f64(rows[int(pt[b, 0]) * 64, :512])   # position 0 = page pt[b,0], slot 0
+        for t in range(3):
+            for h in range(3):
+                np.testing.assert_array_equal(o[b, t, h], want)
+                assert np.isfinite(lse[b, t, h])
+
+
+def test_dense_equal_scores_give_mean_of_prefix():
+    w = dense_workload()
+    q, cache, pt, lens = dense_arrays(w)
+    q = np.zeros_like(q)                      # every score is 0
+    lens = lens.copy()
+    lens[1, 0] = 0                            # an empty prefix
+    o, lse, _ = oracle.decode_dense(q, cache, pt, lens, w.scale, K=int(lens.max()) + 5)
+    rows = bits_to_f64(cache.reshape(-1, 576))
+    for b in range(2):
+        for t in range(3):
+            n = int(lens[b, t])
+            if n == 0:
+                assert np.all(o[b, t] == 0) and np.all(lse[b, t] == -np.inf)
+                continue
+            sel = [int(pt[b, i // 64]) * 64 + i % 64 for i in range(n)]
+            mean = rows[sel, :512].mean(axis=0)
+            for h in range(3):
+                np.testing.assert_allclose(o[b, t, h], mean, rtol=1e-13, atol=1e-15)
+                assert abs(lse[b, t, h] - math.log(n)) < 1e-13
+
+
+def test_dense_is_causal():
+    """Token t's output depends on the positions below its length only."""
+    w = dense_workload(B=1, T=4, H=2, ctx=(150,), seed=23)
+    q, cache, pt, lens = dense_arrays(w)              # lens 147, 148, 149, 150
+    o1, l1, _ = oracle.decode_dense(q, cache, pt, lens, w.scale)
+    cache2 = cache.copy().reshape(-1, 576)
+    rng = np.random.default_rng(4)
+    for i in (147, 148, 149):                         # the rows of the last three draft tokens
+        r = int(pt[0, i // 64]) * 64 + i % 64
+        cache2[r] = to_bits(rng.integers(-8, 8, 576) / 4.0)
+    o2, l2, _ = oracle.decode_dense(q, cache2.reshape(cache.shape), pt, lens, w.scale)
+    np.testing.assert_array_equal(o2[0, 0], o1[0, 0])
+    np.testing.assert_array_equal(l2[0, 0], l1[0, 0])
+    for t in (1, 2, 3):
+        assert np.abs(o2[0, t] - o1[0, t]).max() > 1e-6
+
