@@ -465,9 +465,9 @@ def test_dense_verify_config(dense_verify_ref, nsplit):
 
 def test_dense_lengths_out_of_range_are_clamped_and_counted():
     w = workloads.make_dense_workload("dense_bad", B=2, T=2, H=16, ctx_lens=[300, 300], seed=9)
-    K = 290
+    K = 310                                   # natural lengths 299, 300 lie inside [0, K]
     lens = w.seq_lens.clone()
-    lens[0, 1] = K + 7                        # clamped to K
+    lens[0, 1] = K + 7                        # clamped to K (positions 300.. sit on page 4)
     lens[1, 0] = -3                           # clamped to 0: o = 0, lse = -inf
     w = dataclasses.replace(w, seq_lens=lens)
     binding.check_device(clear=True)
