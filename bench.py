@@ -61,14 +61,12 @@ def workload_bytes(w):
     (H * 1152 B); the combine adds o (H * 1024 B) and lse (H * 4 B).
     Dense variant: the T query tokens of a sequence attend to nested prefixes
     of the same rows, so each row of the longest prefix counts once (with its
-    page-table entry), plus the visible lengths (4 B per query token) and the
-    K-entry position list that the library writes and the partial pass reads
-    (8 B per entry).
+    page-table entry), plus the visible lengths (4 B per query token).
     """
     BT = w.B * w.T
     if w.dense:
         rows = int(w.seq_lens.max(dim=1).values.to(__import__("torch").int64).sum())
-        partial = rows * (1152 + 4) + BT * (4 + w.K * 8) + BT * w.H * 1152
+        partial = rows * (1152 + 4) + BT * 4 + BT * w.H * 1152
     else:
         partial = w.n_valid() * (1152 + 4) + BT * w.K * 4 + BT * w.H * 1152
     step = partial + BT * w.H * (1024 + 4)
@@ -122,8 +120,11 @@ def load_peaks():
 
 
 # ----------------------------------------------------------------------------- clocks
-def partial_kernel_name(H: int, K: int, nsplit: int, pt_stride: int) -> str:
-    """The partial kernel the library launches for this shape (its dispatch rule)."""
+def partial_kernel_name(H: int, K: int, nsplit: int, pt_stride: int, dense: bool = False) -> str:
+    """The partial kernel the library launches for this shape (its dispatch rule;
+    the dense variant always runs the tcgen05 kernel)."""
+    if dense:
+        return "smla_partial_tc_kernel"
     kc = -(-K // nsplit) if K > 0 else 0
     if H <= 32 and K > 0 and kc <= 64 and pt_stride <= 8192:
         return "smla_partial_small_kernel"
@@ -318,7 +319,8 @@ def run_ours(args, world, rank, local):
     w_host = replica_workload(args.workload, rank, world)
     w = w_host.to(dev)
     B, T, H, K = w.B, w.T, w.H, w.K
-    nsplit = args.nsplit or binding.choose_nsplit(B, T, H, K, 0)
+    nsplit = args.nsplit or (binding.dense_nsplit(B, T, H, K) if w.dense
+                             else binding.choose_nsplit(B, T, H, K, 0))
     stream = torch.cuda.current_stream(dev)
     sptr = stream.cuda_stream
 
@@ -343,25 +345,16 @@ def run_ours(args, world, rank, local):
         o = torch.empty((B, T, H, 512), dtype=torch.bfloat16, device=dev)
         lse = torch.empty((B, T, H), dtype=torch.float32, device=dev)
         if w.dense:
-            # smla_decode_dense writes the position lists after the split-K
-            # partials in its workspace (the layout include/smla.h states); the
-            # partial-only step reads them from there
             ws = torch.empty(max(16, binding.dense_workspace_bytes(B, T, H, K, S)),
                              dtype=torch.uint8, device=dev)
             dense_args = (w.q.data_ptr(), w.cache.data_ptr(), w.num_pages, w.page_table.data_ptr(),
                           w.pt_stride, w.seq_lens.data_ptr(), B, T, H, K, 64, w.scale)
-            st = lib.smla_decode_dense(*dense_args, S, ws.data_ptr(), ws.numel(), o.data_ptr(),
-                                       lse.data_ptr(), sptr)
-            if st != 0:
-                raise RuntimeError(binding.status_string(st))
-            base = binding.workspace_bytes(B, T, H, S) if S > 1 else 0
-            idx_ptr = ws.data_ptr() + (base + 255) // 256 * 256
         else:
             ws = torch.empty(max(16, binding.workspace_bytes(B, T, H, S)), dtype=torch.uint8,
                              device=dev)
-            idx_ptr = w.idx.data_ptr()
-        args_common = (w.q.data_ptr(), w.cache.data_ptr(), w.num_pages, w.page_table.data_ptr(),
-                       w.pt_stride, idx_ptr, B, T, H, K, 64, w.scale)
+            args_common = (w.q.data_ptr(), w.cache.data_ptr(), w.num_pages,
+                           w.page_table.data_ptr(), w.pt_stride, w.idx.data_ptr(), B, T, H, K, 64,
+                           w.scale)
 
         def decode():
             """One whole decode: smla_decode (partial pass + LSE combine), or
@@ -369,13 +362,19 @@ def run_ours(args, world, rank, local):
             if w.dense:
                 st = lib.smla_decode_dense(*dense_args, S, ws.data_ptr(), ws.numel(),
                                            o.data_ptr(), lse.data_ptr(), sptr)
-                return st, (2 if S == 1 else 3)
+                return st, (1 if S == 1 else 2)
             st = lib.smla_decode(*args_common, S, ws.data_ptr(), ws.numel(), o.data_ptr(),
                                  lse.data_ptr(), sptr)
             return st, (1 if S == 1 else 2)
 
         def partial():
             """The partial pass alone (with S = 1 it writes o and lse directly)."""
+            if w.dense:
+                if S == 1:
+                    return lib.smla_decode_dense(*dense_args, 1, None, 0, o.data_ptr(),
+                                                 lse.data_ptr(), sptr), 1
+                return lib.smla_decode_dense_partial(*dense_args, S, po.data_ptr(), pm.data_ptr(),
+                                                     pl.data_ptr(), sptr), 1
             if S == 1:
                 return lib.smla_decode(*args_common, 1, None, 0, o.data_ptr(), lse.data_ptr(),
                                        sptr), 1
@@ -548,7 +547,7 @@ def run_ours(args, world, rank, local):
                       "note": "partial pass timed alone in a second loop of the same length; "
                               "the step runs it and the combine through one smla_decode call"},
         "roofline": {"bound": "hbm",
-                     "kernel": partial_kernel_name(H, K, nsplit, w_host.pt_stride),
+                     "kernel": partial_kernel_name(H, K, nsplit, w_host.pt_stride, w_host.dense),
                      "achieved": round(achieved, 1),
                      "peak": hbm_peak, "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),
                      "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured" else "fallback",

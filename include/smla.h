@@ -258,29 +258,44 @@ smla_status smla_decode_host(const void *q_host, const void *kv_cache, int64_t n
  * sequence (46K tokens there), split into NSPLIT chunks, each a partial pass,
  * merged by a reduce.  Here query token (b, t) attends to the positions
  * 0 .. seq_lens[b*T + t] - 1 of sequence b, mapped through the page table
- * like a sparse index.  For causal verify of T draft tokens appended at the
- * end of a sequence of n tokens, seq_lens[b*T + t] = n - T + t + 1.
+ * like a sparse index: the sparse definition with the index list of every
+ * visible position.  For causal verify of T draft tokens appended at the end
+ * of a sequence of n tokens, seq_lens[b*T + t] = n - T + t + 1.
+ *
+ * The partial kernel packs up to 64 / H query tokens of one sequence into the
+ * 64 query rows of one tcgen05 pass over the rows, each row masked at its own
+ * length, so a row read from HBM serves all of them.
  *
  *  - seq_lens  int32 [B, T], device memory, each in [0, K].  A length outside
  *              that range is clamped to it and raises SMLA_ERR_INDEX_RANGE in
  *              smla_check_device (counted once per query token).
- *  - K         the longest visible length (the width of the index lists the
- *              call builds); the NSPLIT heuristic sees this K.
- *  - All other arguments, layouts, the nsplit rule and the outputs are those
- *    of smla_decode.  Positions beyond a sequence's pages are masked and
- *    counted as smla_decode does for out-of-range indices.
+ *  - K         the longest visible length; the split boundaries are those of
+ *              an index list of width K (R7: Kc = ceil(K / nsplit) positions).
+ *  - nsplit    0 picks smla_dense_nsplit(B, T, H, K).
+ *  - Other arguments, layouts and outputs are those of smla_decode.  A
+ *    visible position that no page maps is masked and counted once per
+ *    position and packed group of query tokens.
  *  - workspace_bytes must be at least smla_dense_workspace_bytes(B, T, H, K,
- *    nsplit) for the nsplit actually used: the split-K partials followed by
- *    the B*T*K int32 index lists, which one small kernel writes before the
- *    sparse decode runs on them.  Else SMLA_ERR_WORKSPACE_TOO_SMALL; a
- *    workspace not 16-byte aligned gives SMLA_ERR_MISALIGNED.
+ *    nsplit) for the nsplit used (the split-K partials; 0 for nsplit 1), else
+ *    SMLA_ERR_WORKSPACE_TOO_SMALL; a workspace not 16-byte aligned gives
+ *    SMLA_ERR_MISALIGNED.
+ *
+ * smla_decode_dense_partial runs the partial pass alone (nsplit >= 1) and
+ * writes part_o / part_m / part_lse exactly as smla_decode_partial does for
+ * the equivalent index lists; smla_lse_combine merges them.
  */
+int smla_dense_nsplit(int B, int T, int H, int K);
 size_t smla_dense_workspace_bytes(int B, int T, int H, int K, int nsplit);
 smla_status smla_decode_dense(const void *q, const void *kv_cache, int64_t num_pages,
                               const int32_t *page_table, int pt_stride, const int32_t *seq_lens,
                               int B, int T, int H, int K, int page_size, float scale, int nsplit,
                               void *workspace, size_t workspace_bytes, void *o, float *lse,
                               void *stream);
+smla_status smla_decode_dense_partial(const void *q, const void *kv_cache, int64_t num_pages,
+                                      const int32_t *page_table, int pt_stride,
+                                      const int32_t *seq_lens, int B, int T, int H, int K,
+                                      int page_size, float scale, int nsplit, float *part_o,
+                                      float *part_m, float *part_lse, void *stream);
 
 /*
  * Self-test of the bounded waits (no counterpart on the pages).  Every wait in

@@ -40,9 +40,12 @@ SIGNATURES = {
     "smla_workspace_host_bytes": (_SZ, [_I, _I, _I, _I, _I, _I]),
     "smla_decode_host": (_I, [_P, _P, _I64, _P, _I, _P, _I, _I, _I, _I, _I, _F, _I, _P, _SZ, _P, _P,
                               _P]),
+    "smla_dense_nsplit": (_I, [_I, _I, _I, _I]),
     "smla_dense_workspace_bytes": (_SZ, [_I, _I, _I, _I, _I]),
     "smla_decode_dense": (_I, [_P, _P, _I64, _P, _I, _P, _I, _I, _I, _I, _I, _F, _I, _P, _SZ, _P,
                                _P, _P]),
+    "smla_decode_dense_partial": (_I, [_P, _P, _I64, _P, _I, _P, _I, _I, _I, _I, _I, _F, _I, _P,
+                                       _P, _P, _P]),
     "smla_selftest_wait_timeout": (_I, [ctypes.c_ulonglong, _P]),
     "smla_check_device": (_I, [_I, ctypes.POINTER(ctypes.c_ulonglong), _P]),
     "smla_status_string": (ctypes.c_char_p, [_I]),
@@ -219,16 +222,15 @@ def decode_noalloc(q, cache, page_table, idx, scale: float, nsplit: int = 0, *, 
     return o, lse
 
 
+def dense_nsplit(B: int, T: int, H: int, K: int) -> int:
+    return int(lib().smla_dense_nsplit(B, T, H, K))
+
+
 def dense_workspace_bytes(B: int, T: int, H: int, K: int, nsplit: int) -> int:
     return int(lib().smla_dense_workspace_bytes(B, T, H, K, nsplit))
 
 
-def decode_dense(q, cache, page_table, seq_lens, scale: float, nsplit: int = 0, *, K=None,
-                 workspace=None, o=None, lse=None, stream=None):
-    """Dense-context decode (KV-split verify): query token (b, t) attends to
-    positions 0 .. seq_lens[b, t] - 1 of sequence b.  K defaults to the longest
-    length (read from seq_lens, which synchronises); pass it to stay
-    asynchronous.  Returns (o bf16 [B,T,H,512], lse fp32 [B,T,H])."""
+def _dense_args(q, cache, page_table, seq_lens, K):
     _need(q, torch.bfloat16, "q")
     dev = q.device
     _need(cache, torch.bfloat16, "cache", dev)
@@ -243,11 +245,21 @@ def decode_dense(q, cache, page_table, seq_lens, scale: float, nsplit: int = 0, 
         raise ValueError("page_table must be [B, pt_stride]")
     if cache.numel() % (PAGE_SIZE * D):
         raise ValueError("cache must be [num_pages, 64, 576]")
-    num_pages = cache.numel() // (PAGE_SIZE * D)
     if K is None:
         K = int(seq_lens.max().item()) if seq_lens.numel() else 0
+    return B, T, H, int(K), page_table.shape[1], cache.numel() // (PAGE_SIZE * D)
+
+
+def decode_dense(q, cache, page_table, seq_lens, scale: float, nsplit: int = 0, *, K=None,
+                 workspace=None, o=None, lse=None, stream=None):
+    """Dense-context decode (KV-split verify): query token (b, t) attends to
+    positions 0 .. seq_lens[b, t] - 1 of sequence b.  K defaults to the longest
+    length (read from seq_lens, which synchronises); pass it to stay
+    asynchronous.  Returns (o bf16 [B,T,H,512], lse fp32 [B,T,H])."""
+    B, T, H, K, pt_stride, num_pages = _dense_args(q, cache, page_table, seq_lens, K)
+    dev = q.device
     if nsplit == 0:
-        nsplit = choose_nsplit(B, T, H, K, 0)
+        nsplit = dense_nsplit(B, T, H, K)
     need = dense_workspace_bytes(B, T, H, K, nsplit)
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
@@ -258,12 +270,33 @@ def decode_dense(q, cache, page_table, seq_lens, scale: float, nsplit: int = 0, 
         lse = torch.empty((B, T, H), dtype=torch.float32, device=dev)
     _need(o, torch.bfloat16, "o", dev)
     _need(lse, torch.float32, "lse", dev)
-    _check(lib().smla_decode_dense(_ptr(q), _ptr(cache), num_pages, _ptr(page_table),
-                                   page_table.shape[1], _ptr(seq_lens), B, T, H, int(K),
-                                   PAGE_SIZE, float(scale), int(nsplit), _ptr(workspace),
-                                   workspace.numel(), _ptr(o), _ptr(lse), _stream(stream)),
-           "smla_decode_dense")
+    _check(lib().smla_decode_dense(_ptr(q), _ptr(cache), num_pages, _ptr(page_table), pt_stride,
+                                   _ptr(seq_lens), B, T, H, K, PAGE_SIZE, float(scale),
+                                   int(nsplit), _ptr(workspace), workspace.numel(), _ptr(o),
+                                   _ptr(lse), _stream(stream)), "smla_decode_dense")
     return o, lse
+
+
+def decode_dense_partial(q, cache, page_table, seq_lens, scale: float, nsplit: int, *, K=None,
+                         part_o=None, part_m=None, part_lse=None, stream=None):
+    """Partial pass of the dense variant; returns (part_o [B,T,H,S,512],
+    part_m [B,T,H,S], part_lse [B,T,H,S])."""
+    B, T, H, K, pt_stride, num_pages = _dense_args(q, cache, page_table, seq_lens, K)
+    dev = q.device
+    if part_o is None:
+        part_o = torch.empty((B, T, H, nsplit, DC), dtype=torch.float32, device=dev)
+    if part_m is None:
+        part_m = torch.empty((B, T, H, nsplit), dtype=torch.float32, device=dev)
+    if part_lse is None:
+        part_lse = torch.empty((B, T, H, nsplit), dtype=torch.float32, device=dev)
+    for t, n in ((part_o, "part_o"), (part_m, "part_m"), (part_lse, "part_lse")):
+        _need(t, torch.float32, n, dev)
+    _check(lib().smla_decode_dense_partial(_ptr(q), _ptr(cache), num_pages, _ptr(page_table),
+                                           pt_stride, _ptr(seq_lens), B, T, H, K, PAGE_SIZE,
+                                           float(scale), int(nsplit), _ptr(part_o), _ptr(part_m),
+                                           _ptr(part_lse), _stream(stream)),
+           "smla_decode_dense_partial")
+    return part_o, part_m, part_lse
 
 
 def workspace_host_bytes(B: int, T: int, H: int, K: int, pt_stride: int, nsplit: int) -> int:

@@ -22,7 +22,6 @@
 #define SMLA_MMA_STAGES 2
 #endif
 #include "smla_combine.cuh"
-#include "smla_dense.cuh"
 #include "smla_partial_mma.cuh"
 #include "smla_partial_tc.cuh"
 
@@ -553,13 +552,84 @@ smla_status smla_decode_host(const void *q_host, const void *kv_cache, int64_t n
 }
 
 // ---------------------------------------------------------------------------
-// Dense-context decode (see include/smla.h): the index lists are every visible
-// position, written into the workspace by smla_dense_index_kernel, then the
-// sparse decode runs on them.
+// Dense-context decode (see include/smla.h).  The tcgen05 kernel reads the
+// visible lengths itself (entry j of a list is position j) and packs up to
+// 64 / H query tokens of a sequence into the M rows of one pass over the
+// rows; the combine then runs over the usual [B, T, H, S] partials.
+namespace {
+
+struct DensePlan {
+    int pack;   // query tokens per unit
+    int units;  // units per sequence
+    int nsplit;
+};
+
+DensePlan dense_plan(int B, int T, int H, int K, int nsplit) {
+    DensePlan d{};
+    const int gmax = std::max(1, std::min(T, smla::kMaxTcRows / std::max(H, 1)));
+    d.units = (T + gmax - 1) / gmax;
+    d.pack = (T + d.units - 1) / d.units;  // the same number of passes, balanced units
+    // one CTA per SM (the tcgen05 kernel): the heuristic's H > 32 model
+    d.nsplit = nsplit > 0 ? nsplit : smla_choose_nsplit(B, d.units, smla::kMaxTcRows, K, 0);
+    return d;
+}
+
+smla_status check_dense_args(const void *q, const void *kv_cache, int64_t num_pages,
+                             const int32_t *page_table, int pt_stride, const int32_t *seq_lens,
+                             int B, int T, int H, int K, int page_size, float scale, int nsplit) {
+    smla_status st = check_decode_args(q, kv_cache, num_pages, page_table, pt_stride, seq_lens, B,
+                                       T, H, K, page_size, scale);
+    if (st != SMLA_OK) return st;
+    if (nsplit < 0 || nsplit > SMLA_MAX_NSPLIT) return SMLA_ERR_INVALID_ARG;
+    if (B > 0 && T > 0 && H > 0 && seq_lens == nullptr) return SMLA_ERR_INVALID_ARG;
+    return SMLA_OK;
+}
+
+PartialParams dense_params(const void *q, const void *kv_cache, int64_t num_pages,
+                           const int32_t *page_table, int pt_stride, const int32_t *seq_lens,
+                           int B, int T, int H, int K, float scale, const DensePlan &d) {
+    PartialParams p = make_params(q, kv_cache, num_pages, page_table, pt_stride, nullptr, B,
+                                  d.units, d.pack * H, K, scale, d.nsplit);
+    p.seq_lens = seq_lens;
+    p.pack = d.pack;
+    p.dense_t = T;
+    p.dense_h = H;
+    return p;
+}
+
+}  // namespace
+
 size_t smla_dense_workspace_bytes(int B, int T, int H, int K, int nsplit) {
     if (B < 0 || T < 0 || H < 0 || K < 0 || nsplit < 1 || nsplit > SMLA_MAX_NSPLIT) return 0;
-    const size_t base = nsplit > 1 ? smla_workspace_bytes(B, T, H, nsplit) : 0;
-    return round256(base) + round256((size_t)B * T * K * sizeof(int32_t));
+    return nsplit > 1 ? smla_workspace_bytes(B, T, H, nsplit) : 0;
+}
+
+int smla_dense_nsplit(int B, int T, int H, int K) {
+    if (B <= 0 || T <= 0 || H <= 0 || H > SMLA_MAX_HEADS || K <= 0) return 1;
+    return dense_plan(B, T, H, K, 0).nsplit;
+}
+
+smla_status smla_decode_dense_partial(const void *q, const void *kv_cache, int64_t num_pages,
+                                      const int32_t *page_table, int pt_stride,
+                                      const int32_t *seq_lens, int B, int T, int H, int K,
+                                      int page_size, float scale, int nsplit, float *part_o,
+                                      float *part_m, float *part_lse, void *stream) {
+    smla_status st = check_dense_args(q, kv_cache, num_pages, page_table, pt_stride, seq_lens, B,
+                                      T, H, K, page_size, scale, nsplit);
+    if (st != SMLA_OK) return st;
+    if (nsplit < 1) return SMLA_ERR_INVALID_ARG;
+    if (B == 0 || T == 0 || H == 0) return SMLA_OK;
+    if (part_o == nullptr || part_m == nullptr || part_lse == nullptr) return SMLA_ERR_INVALID_ARG;
+    if (!aligned(part_o, 16) || !aligned(part_m, 4) || !aligned(part_lse, 4))
+        return SMLA_ERR_MISALIGNED;
+    const DensePlan d = dense_plan(B, T, H, K, nsplit);
+    if ((long long)B * d.units * d.nsplit > INT_MAX) return SMLA_ERR_INVALID_ARG;
+    PartialParams p = dense_params(q, kv_cache, num_pages, page_table, pt_stride, seq_lens, B, T,
+                                   H, K, scale, d);
+    p.part_o = part_o;
+    p.part_m = part_m;
+    p.part_lse = part_lse;
+    return launch_tc<false>(p, B * d.units * d.nsplit, static_cast<cudaStream_t>(stream));
 }
 
 smla_status smla_decode_dense(const void *q, const void *kv_cache, int64_t num_pages,
@@ -567,32 +637,36 @@ smla_status smla_decode_dense(const void *q, const void *kv_cache, int64_t num_p
                               int B, int T, int H, int K, int page_size, float scale, int nsplit,
                               void *workspace, size_t workspace_bytes, void *o, float *lse,
                               void *stream) {
-    smla_status st = check_decode_args(q, kv_cache, num_pages, page_table, pt_stride, seq_lens, B,
-                                       T, H, K, page_size, scale);
+    smla_status st = check_dense_args(q, kv_cache, num_pages, page_table, pt_stride, seq_lens, B,
+                                      T, H, K, page_size, scale, nsplit);
     if (st != SMLA_OK) return st;
-    if (nsplit < 0 || nsplit > SMLA_MAX_NSPLIT) return SMLA_ERR_INVALID_ARG;
     if (B == 0 || T == 0 || H == 0) return SMLA_OK;
     if (o == nullptr || lse == nullptr) return SMLA_ERR_INVALID_ARG;
     if (!aligned(o, 16) || !aligned(lse, 4)) return SMLA_ERR_MISALIGNED;
-    if (nsplit == 0) nsplit = smla_choose_nsplit(B, T, H, K, 0);
-    if (K == 0)  // every list is empty: o = 0, lse = -inf
-        return smla_decode(q, kv_cache, num_pages, page_table, pt_stride, seq_lens, B, T, H, 0,
-                           page_size, scale, nsplit, workspace, workspace_bytes, o, lse, stream);
-    if (workspace_bytes < smla_dense_workspace_bytes(B, T, H, K, nsplit))
-        return SMLA_ERR_WORKSPACE_TOO_SMALL;
+    const DensePlan d = dense_plan(B, T, H, K, nsplit);
+    if ((long long)B * d.units * d.nsplit > INT_MAX) return SMLA_ERR_INVALID_ARG;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    PartialParams p = dense_params(q, kv_cache, num_pages, page_table, pt_stride, seq_lens, B, T,
+                                   H, K, scale, d);
+    const int grid = B * d.units * d.nsplit;
+    if (d.nsplit == 1) {
+        p.o = static_cast<__nv_bfloat16 *>(o);
+        p.lse = lse;
+        return launch_tc<true>(p, grid, s);
+    }
+    if (workspace_bytes < smla_workspace_bytes(B, T, H, d.nsplit)) return SMLA_ERR_WORKSPACE_TOO_SMALL;
     if (workspace == nullptr) return SMLA_ERR_INVALID_ARG;
     if (!aligned(workspace, 16)) return SMLA_ERR_MISALIGNED;
-    const size_t base = nsplit > 1 ? smla_workspace_bytes(B, T, H, nsplit) : 0;
-    int32_t *idx = reinterpret_cast<int32_t *>(static_cast<uint8_t *>(workspace) + round256(base));
-    const long long n_bt = (long long)B * T;
-    const long long total = n_bt * K;
-    const unsigned blocks = (unsigned)std::min<long long>((total + 255) / 256, 148 * 8);
-    smla::smla_dense_index_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(
-        seq_lens, n_bt, K, idx);
-    const cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_fail(e);
-    return smla_decode(q, kv_cache, num_pages, page_table, pt_stride, idx, B, T, H, K, page_size,
-                       scale, nsplit, workspace, base, o, lse, stream);
+    const size_t n = (size_t)B * T * H * d.nsplit;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    const size_t off_m = round256(n * smla::kDc * sizeof(float));
+    const size_t off_l = off_m + round256(n * sizeof(float));
+    p.part_o = reinterpret_cast<float *>(ws);
+    p.part_m = reinterpret_cast<float *>(ws + off_m);
+    p.part_lse = reinterpret_cast<float *>(ws + off_l);
+    st = launch_tc<false>(p, grid, s);
+    if (st != SMLA_OK) return st;
+    return launch_combine(p.part_o, p.part_m, p.part_lse, B, T, H, d.nsplit, o, lse, s);
 }
 
 smla_status smla_selftest_wait_timeout(unsigned long long limit_ns, void *stream) {

@@ -77,6 +77,13 @@ struct PartialParams {
     int tpt;                      // 32-row tiles per query token, ceil(K / 32)
     int grid;
     long long n_units;            // U
+    // Dense-context variant (tcgen05 kernel only; idx unused): query token
+    // (b, t) attends to list entries [0, seq_lens[b * dense_t + t]), entry j
+    // being position j.  Unit bt = b * T + g packs query tokens
+    // [g * pack, min(dense_t, (g + 1) * pack)) of sequence b, dense_h heads
+    // each, into the MMA's M rows (pack * dense_h <= 64).
+    const int *seq_lens;          // [B, dense_t]; nullptr = sparse index lists
+    int pack, dense_t, dense_h;
 };
 
 // One piece of a CTA's work: rows [j0, j1) of query token bt, written as

@@ -39,6 +39,7 @@
 // pair's softmax; lane l + 16 rescales the second half of the same head's O.
 #pragma once
 
+#include <climits>
 #include <cstdint>
 #include <cuda_bf16.h>
 
@@ -46,6 +47,8 @@
 #include "smla_tc_ptx.cuh"
 
 namespace smla {
+
+constexpr int kMaxTcRows = 64;  // query rows (the MMA's M) of one CTA
 
 struct TcCfg {
 #ifndef SMLA_TC_PRODUCER_WARPS
@@ -99,6 +102,18 @@ __global__ void __launch_bounds__(TcCfg::kThreads, 1)
     const int n_tiles = (j1 - j0 + C::kTileRows - 1) / C::kTileRows;
     const int n_pairs = (n_tiles + 1) / 2;
     bool dead = false;
+    // Query rows of this unit: global row of M row 0, and how many M rows are
+    // real.  Sparse: the H heads of token bt.  Dense: the packed tokens' heads.
+    const bool dense = p.seq_lens != nullptr;
+    long long row0 = (long long)bt * p.H;
+    int nrows = p.H;
+    int tok0 = 0, ntok = 0;  // dense: first token of the unit (within sequence b), tokens in it
+    if (dense) {
+        tok0 = (bt - b * p.T) * p.pack;
+        ntok = min(p.pack, p.dense_t - tok0);
+        row0 = ((long long)b * p.dense_t + tok0) * p.dense_h;
+        nrows = ntok * p.dense_h;
+    }
 
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::kOffBar);
     uint64_t *kv_full = bars;
@@ -142,7 +157,21 @@ __global__ void __launch_bounds__(TcCfg::kThreads, 1)
         const int pw = warp - 4;
         const int ptid = threadIdx.x - 128;  // 0 .. 32 * kProducerWarps - 1
         constexpr int kPT = 32 * C::kProducerWarps;
-        const int *idx_bt = p.idx + (size_t)bt * p.K + j0;
+        const int *idx_bt = dense ? nullptr : p.idx + (size_t)bt * p.K + j0;
+        // dense: the unit's list is positions [0, n_unit), the longest visible
+        // length of its tokens (each clamped to [0, K]; split 0 counts a
+        // length outside that range once per token)
+        int n_unit = 0;
+        if (dense) {
+            for (int t = 0; t < ntok; ++t) {
+                const int raw = __ldg(p.seq_lens + (size_t)b * p.dense_t + tok0 + t);
+                n_unit = max(n_unit, min(max(raw, 0), p.K));
+                if (s == 0 && ptid == t && (raw < 0 || raw > p.K)) {
+                    atomicOr(&g_status_flags, kFlagIndexRange);
+                    atomicAdd(&g_bad_index_count, 1ull);
+                }
+            }
+        }
         const int *pt_b = p.page_table + (size_t)b * p.pt_stride;
         const long long max_pos = (long long)p.pt_stride * kPage;
         // Padding slots copy cache row 0 (always in range) and are masked to
@@ -161,7 +190,12 @@ __global__ void __launch_bounds__(TcCfg::kThreads, 1)
 #pragma unroll
                 for (int k = 0; k < 16; ++k) {
                     const int j = b0 + k * kPT + ptid;
-                    iv[k] = (j < n) ? __ldg(idx_bt + base + j) : -1;
+                    if (dense) {
+                        const int pos = j0 + base + j;
+                        iv[k] = (j < n && pos < n_unit) ? pos : -1;
+                    } else {
+                        iv[k] = (j < n) ? __ldg(idx_bt + base + j) : -1;
+                    }
                 }
                 int pg[16];
 #pragma unroll
@@ -315,14 +349,14 @@ __global__ void __launch_bounds__(TcCfg::kThreads, 1)
 
         // ---- stage Q (heads x 576, zero rows beyond H) as 9 swizzled 64-column boxes
         {
-            const uint4 *qsrc = reinterpret_cast<const uint4 *>(p.q + (size_t)bt * p.H * kD);
+            const uint4 *qsrc = reinterpret_cast<const uint4 *>(p.q + (size_t)row0 * kD);
             for (int c0 = 0; c0 < 64 * 72; c0 += 128 * 12) {
                 uint4 v[12];
 #pragma unroll
                 for (int k = 0; k < 12; ++k) {
                     const int c = c0 + k * 128 + tid;
                     const int h = c / 72;
-                    v[k] = (c < 64 * 72 && h < p.H) ? __ldg(qsrc + (size_t)h * 72 + (c % 72))
+                    v[k] = (c < 64 * 72 && h < nrows) ? __ldg(qsrc + (size_t)h * 72 + (c % 72))
                                                      : make_uint4(0u, 0u, 0u, 0u);
                 }
 #pragma unroll
@@ -341,6 +375,13 @@ __global__ void __launch_bounds__(TcCfg::kThreads, 1)
             if (lane == 0) mbar_arrive(q_ready);
         }
 
+        // dense: list entries visible to query row hrow (rows past the unit's
+        // real rows see none); sparse: no per-row limit
+        int lim = INT_MAX;
+        if (dense)
+            lim = hrow < nrows ? min(max(__ldg(p.seq_lens + (size_t)b * p.dense_t + tok0 +
+                                               hrow / p.dense_h), 0), p.K)
+                               : 0;
         float m_ref = -INFINITY;  // running reference max of head hrow (log2 units)
         float l_acc = 0.f;        // sum of P of head hrow relative to m_ref (lanes 0-15; 0 elsewhere)
         const uint32_t t_lane = tmem + ((uint32_t)(32 * q4) << 16);
@@ -357,11 +398,17 @@ __global__ void __launch_bounds__(TcCfg::kThreads, 1)
             tmem_ld32(t_lane + C::kSCol + 64 * (pr & 1) + 32, s1);
             tmem_ld_wait();
             mbar_wait(&kv_full[t0 % C::kStages], (t0 / C::kStages) & 1, dead);
-            const uint32_t vm0 = hdr[t0 % C::kStages];
+            uint32_t vm0 = hdr[t0 % C::kStages];
             uint32_t vm1 = 0;
             if (has1) {
                 mbar_wait(&kv_full[(t0 + 1) % C::kStages], ((t0 + 1) / C::kStages) & 1, dead);
                 vm1 = hdr[(t0 + 1) % C::kStages];
+            }
+            if (dense) {  // this row's causal limit, as a mask over the pair's columns
+                const int r0 = lim - (j0 + t0 * C::kTileRows);
+                const int r1 = r0 - C::kTileRows;
+                vm0 &= r0 >= 32 ? 0xffffffffu : (r0 <= 0 ? 0u : (1u << r0) - 1u);
+                vm1 &= r1 >= 32 ? 0xffffffffu : (r1 <= 0 ? 0u : (1u << r1) - 1u);
             }
             const bool owner = half == 0;  // lanes 0-15 run the softmax of head hrow
             // scores in log2 units, padding (and an absent second tile) -> -inf;
@@ -439,8 +486,8 @@ __global__ void __launch_bounds__(TcCfg::kThreads, 1)
             mbar_wait(&o_done[(n_pairs - 1) & 1], ((n_pairs - 1) >> 1) & 1, dead);
             tc_fence_after();
         }
-        const bool write = hrow < p.H;
-        const size_t row = (size_t)bt * p.H + hrow;
+        const bool write = hrow < nrows;
+        const size_t row = (size_t)row0 + hrow;
 #pragma unroll 1
         for (int c = 0; c < 256; c += 32) {
             uint32_t orr[32];

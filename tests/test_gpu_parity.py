@@ -447,6 +447,31 @@ def test_dense_against_oracle(H, T, ctx, S):
     check_o_lse(o, lse, o_ref, lse_ref, f"dense H={H} T={T} ctx={ctx} S={S}")
 
 
+@pytest.mark.parametrize("H,T,ctx,S", [(8, 9, 3000, 7), (16, 3, 777, 5), (64, 2, 1500, 3),
+                                       (24, 5, 2100, 16)])
+def test_dense_partial_pass_against_oracle_partials(H, T, ctx, S):
+    """Each split's normalised partial and lse against the oracle's partials of
+    the equivalent index lists (every visible position, width K)."""
+    w = workloads.make_dense_workload("dense_part", B=2, T=T, H=H, ctx_lens=[ctx, ctx // 2 + 40],
+                                      seed=3 * H + S)
+    wd = w.to(DEV)
+    po, pm, pl = binding.decode_dense_partial(wd.q, wd.cache, wd.page_table, wd.seq_lens, w.scale,
+                                              S, K=w.K)
+    torch.cuda.synchronize()
+    lists = oracle.dense_positions(w.seq_lens.numpy(), w.K)
+    rpo, rpm, rpl, _ = oracle.partial(bits(w.q), bits(w.cache), w.page_table.numpy(), lists,
+                                      w.scale, S)
+    got = normalised_partials(po.cpu().numpy(), pm.cpu().numpy(), pl.cpu().numpy())
+    want = normalised_partials(rpo, rpm, rpl)
+    pl_g = pl.cpu().numpy().astype(np.float64)
+    assert np.array_equal(np.isneginf(pl_g), np.isneginf(rpl)), "empty splits differ"
+    fin = ~np.isneginf(rpl)
+    assert np.abs(pl_g[fin] - rpl[fin]).max() <= 1e-3
+    err = np.abs(got - want)
+    assert err.max() <= 1e-2
+    assert np.linalg.norm(got - want) / np.linalg.norm(want) <= 5e-3
+
+
 @pytest.fixture(scope="module")
 def dense_verify_ref():
     w = workloads.dense_verify()

@@ -116,14 +116,42 @@ def test_decode_dense_rejects_bad_arguments(lib, kw, expect):
 
 
 def test_dense_workspace_bytes_formula(lib):
-    """Split-K partials (none at nsplit 1), then the B*T*K int32 index lists."""
-    r = lambda x: (x + 255) // 256 * 256
-    for B, T, H, K, S in [(1, 9, 8, 46089, 32), (1, 9, 8, 46089, 1), (2, 3, 16, 777, 5),
+    """The split-K partials of [B, T, H, S] (none at nsplit 1)."""
+    for B, T, H, K, S in [(1, 9, 8, 46089, 74), (1, 9, 8, 46089, 1), (2, 3, 16, 777, 5),
                           (1, 1, 64, 0, 4)]:
-        base = binding.workspace_bytes(B, T, H, S) if S > 1 else 0
-        assert binding.dense_workspace_bytes(B, T, H, K, S) == r(base) + r(B * T * K * 4)
+        want = binding.workspace_bytes(B, T, H, S) if S > 1 else 0
+        assert binding.dense_workspace_bytes(B, T, H, K, S) == want
     assert binding.dense_workspace_bytes(1, 1, 1, 1, 0) == 0
     assert binding.dense_workspace_bytes(1, 1, 1, -1, 1) == 0
+
+
+@pytest.mark.parametrize("shape", [(1, 9, 8, 46089), (1, 9, 8, 4105), (2, 3, 16, 777),
+                                   (2, 2, 64, 1500), (2, 4, 8, 40), (1, 1, 16, 65536),
+                                   (2, 5, 24, 2100), (3, 17, 4, 999)])
+def test_dense_nsplit_packs_tokens_into_64_rows(lib, shape, monkeypatch):
+    """Up to 64 / H query tokens share a pass, in balanced groups; the NSPLIT
+    is the heuristic's for that many units at the one-CTA-per-SM kernel."""
+    monkeypatch.delenv("SMLA_NSPLIT", raising=False)
+    B, T, H, K = shape
+    gmax = max(1, min(T, 64 // H))
+    units = -(-T // gmax)
+    assert units * gmax >= T and (units - 1) * gmax < T
+    assert binding.dense_nsplit(B, T, H, K) == binding.choose_nsplit(B, units, 64, K, 0)
+
+
+def call_dense_partial(lib, q=FAKE, cache=FAKE, num_pages=10, pt=FAKE, pt_stride=4, lens=FAKE, B=1,
+                       T=9, H=8, K=200, ps=64, scale=0.1, nsplit=2, po=FAKE, pm=FAKE, pl=FAKE):
+    return lib.smla_decode_dense_partial(q, cache, num_pages, pt, pt_stride, lens, B, T, H, K, ps,
+                                         scale, nsplit, po, pm, pl, None)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(nsplit=0), 1), (dict(nsplit=1025), 1), (dict(po=0), 1), (dict(po=FAKE + 4), 3),
+    (dict(pm=FAKE + 2), 3), (dict(lens=0), 1), (dict(H=65), 2), (dict(ps=32), 2),
+    (dict(q=FAKE + 8), 3), (dict(B=0), 0),
+])
+def test_decode_dense_partial_rejects_bad_arguments(lib, kw, expect):
+    assert call_dense_partial(lib, **kw) == expect
 
 
 def test_combine_rejects_bad_arguments(lib):
