@@ -48,7 +48,7 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-sweep", action="store_true", help="skip the NSPLIT sweep")
     ap.add_argument("--cpu-seconds", type=float, default=6.0,
-                    help="time budget of the oracle CPU baseline sample")
+                    help="seconds of oracle CPU time for the baseline sample")
     return ap.parse_args(argv)
 
 
@@ -253,10 +253,10 @@ def sum_over_ranks(x: float, world: int) -> float:
 
 
 # ----------------------------------------------------------------------------- oracle baseline
-def cpu_baseline(w, budget_s: float):
+def cpu_baseline(w, seconds: float):
     """The fp64 oracle as it stands, on this host's cores, over whole steps of
     the same workload (or the first query tokens of one step when a step alone
-    exceeds the budget)."""
+    exceeds that time)."""
     import numpy as np
     import oracle
     bits = lambda t: t.contiguous().view(__import__("torch").int16).numpy().view(np.uint16)
@@ -271,7 +271,7 @@ def cpu_baseline(w, budget_s: float):
     t0 = time.perf_counter()
     oracle.decode(q[:1, :1], cache, pt[:1], idx[:1, :1], w.scale)
     per_token = time.perf_counter() - t0
-    n_tok = max(1, min(w.B * w.T, int(budget_s / max(per_token, 1e-9))))
+    n_tok = max(1, min(w.B * w.T, int(seconds / max(per_token, 1e-9))))
     bt = [(b, t) for b in range(w.B) for t in range(w.T)][:n_tok]
     reps = 0
     t0 = time.perf_counter()
@@ -279,7 +279,7 @@ def cpu_baseline(w, budget_s: float):
         for b, t in bt:
             oracle.decode(q[b:b + 1, t:t + 1], cache, pt[b:b + 1], idx[b:b + 1, t:t + 1], w.scale)
         reps += 1
-        if time.perf_counter() - t0 >= budget_s * 0.5 or reps >= 50:
+        if time.perf_counter() - t0 >= seconds * 0.5 or reps >= 50:
             break
     el = time.perf_counter() - t0
     tokens = reps * len(bt)
@@ -289,7 +289,7 @@ def cpu_baseline(w, budget_s: float):
     oracle.set_threads(1)
     try:
         n1, t0 = 0, time.perf_counter()
-        while n1 < 5 and (n1 == 0 or time.perf_counter() - t0 < budget_s * 0.25):
+        while n1 < 5 and (n1 == 0 or time.perf_counter() - t0 < seconds * 0.25):
             b, t = bt[0]
             oracle.decode(q[b:b + 1, t:t + 1], cache, pt[b:b + 1], idx[b:b + 1, t:t + 1], w.scale)
             n1 += 1
@@ -574,9 +574,9 @@ def run_reference(args, world, rank):
         return None
     from sparse_mla_decode_partial_b200 import workloads
     w = workloads.WORKLOADS[args.workload]()
-    budget = max(2.0, args.cpu_seconds)
+    seconds = max(2.0, args.cpu_seconds)
     t_all = time.perf_counter()
-    res = cpu_baseline(w, budget)
+    res = cpu_baseline(w, seconds)
     value = res["value"]
     nsplit = args.nsplit or None
     return {
