@@ -133,3 +133,47 @@ def test_planted_mistake_is_caught(name):
         lib = build_variant(src.replace(old, new), d, name)
         failures = run_pins(lib)
     assert failures, f"no pin caught the planted mistake '{name}'"
+
+
+# ---------------------------------------------------------------- dense-context variant
+def _dense_mutant(kind):
+    """A copy of the oracle's position-list construction with one mistake."""
+    def dense_positions(seq_lens, K):
+        seq_lens = np.asarray(seq_lens, np.int64)
+        if seq_lens.size and (seq_lens.min() < 0 or seq_lens.max() > K):
+            raise ValueError("seq_lens must lie in [0, K]")
+        j = np.arange(K, dtype=np.int64)[None, None, :]
+        n = seq_lens[..., None]
+        if kind == "prefix_one_too_long":
+            return np.where(j <= n, j, -1).astype(np.int32)
+        if kind == "prefix_one_too_short":
+            return np.where(j < n - 1, j, -1).astype(np.int32)
+        if kind == "positions_from_one":
+            return np.where(j < n, j + 1, -1).astype(np.int32)
+        raise AssertionError(kind)
+    return dense_positions
+
+
+def run_dense_pins() -> list:
+    import test_oracle_pins as pins
+    failures = []
+    for name in ("test_dense_positions_hand_case", "test_dense_single_position_returns_first_row_exactly",
+                 "test_dense_equal_scores_give_mean_of_prefix", "test_dense_is_causal"):
+        try:
+            getattr(pins, name)()
+        except (AssertionError, ValueError):
+            failures.append(name)
+    return failures
+
+
+def test_unmutated_dense_oracle_passes_its_pins():
+    assert run_dense_pins() == []
+
+
+@pytest.mark.parametrize("kind", ["prefix_one_too_long", "prefix_one_too_short",
+                                  "positions_from_one"])
+def test_planted_dense_mistake_is_caught(kind, monkeypatch):
+    mutant = _dense_mutant(kind)
+    monkeypatch.setattr(oracle.oracle, "dense_positions", mutant)
+    monkeypatch.setattr(oracle, "dense_positions", mutant)
+    assert run_dense_pins(), f"no pin caught the planted dense mistake '{kind}'"
