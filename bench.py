@@ -91,22 +91,37 @@ def data_note(w):
     return f"synthetic (seeded N(0,1)*0.5 bf16 q and cache, {sel})"
 
 
+# The sources each partial kernel's code and launch shape come from: a
+# recorded ncu traffic figure stays valid while these files are unchanged.
+KERNEL_SOURCES = {
+    "smla_partial_small_kernel": ["smla_api.cu", "smla_partial_mma.cuh", "smla_ptx.cuh"],
+    "smla_partial_mma_kernel": ["smla_api.cu", "smla_partial_mma.cuh", "smla_ptx.cuh"],
+    "smla_partial_tc_kernel": ["smla_api.cu", "smla_partial_mma.cuh", "smla_partial_tc.cuh",
+                               "smla_ptx.cuh", "smla_tc_ptx.cuh"],
+}
+
+
+def kernel_sources_hash(kernel: str) -> str:
+    """sha256[:16] over the kernel's source files (KERNEL_SOURCES), in order."""
+    import hashlib
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(ROOT, "sparse_mla_decode_partial_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
 def measured_traffic(workload: str):
     """DRAM bytes (read + write) per launch of the partial kernel for this
     workload from the committed ncu capture, or None when no capture exists
-    or the kernel sources changed since it was taken."""
-    import glob
-    import hashlib
+    or that kernel's sources changed since it was taken."""
     try:
         with open(os.path.join(ROOT, "profiles", "ncu_traffic.json")) as f:
             rec = json.load(f)[workload]
+        ok = kernel_sources_hash(rec["kernel"]) == rec["sources_sha256_16"]
     except (OSError, KeyError, ValueError):
         return None
-    h = hashlib.sha256()
-    for fn in sorted(glob.glob(os.path.join(ROOT, "sparse_mla_decode_partial_b200", "csrc", "*"))):
-        with open(fn, "rb") as f:
-            h.update(f.read())
-    return rec["traffic_bytes_per_launch"] if h.hexdigest()[:16] == rec["sources_sha256_16"] else None
+    return rec["traffic_bytes_per_launch"] if ok else None
 
 
 def load_peaks():

@@ -6,20 +6,24 @@
 // the top-k candidate rows, split-K over that axis, partials merged by LSE.
 //
 // One CTA = one (query token, split), all heads (M = 64 rows of the MMA;
-// heads >= H are zero rows of Q and are never written out).  416 threads:
+// heads >= H are zero rows of Q and are never written out), or in dense mode
+// up to 64 / H query tokens of one sequence.  512 threads (16 warps x 128
+// registers: the whole register file):
 //   warps 0-3  softmax warpgroup: stages Q (128B-swizzled) once, then per
 //              PAIR of 32-row tiles reads S from TMEM (tcgen05.ld), masks,
 //              keeps a running max per head with lazy rescaling (O is only
 //              rescaled when the max grows by more than 2^8), writes P as bf16
-//              into each tile's spent k_pe box, and finally drains O.
-//   warps 4-11 producers: resolve the split's indices to rows (as the mma
+//              into each tile's spent k_pe box, and finally drains O
+//              (partials through shared memory, whole 128-B segments per
+//              store).
+//   warps 4-14 producers: resolve the split's indices to rows (as the mma
 //              kernel does), then gather each 32-row tile with 16-byte
 //              cp.async copies written straight into the 128B-swizzled
 //              K-major layout (each warp instruction moves 4 rows x 128 B,
 //              coalesced); completion reaches the tile's mbarrier through
 //              cp.async.mbarrier.arrive.  Padding slots copy row 0 and are
 //              masked.
-//   warp 12    TMEM owner + MMA issuer (one thread):
+//   warp 15    TMEM owner + MMA issuer (one thread):
 //                QK(pair): S[64 x 64] = Q[64 x 576] [K_2p K_2p+1]^T   36 x (M64 N64 K16)
 //                PV(t):    O[64 x 512] += P_t[64 x 32] C_t[32 x 512]  2 x 2 x (M64 N256 K16)
 //              A tcgen05 MMA costs at least ~46 cycles whatever its size
@@ -52,7 +56,7 @@ constexpr int kMaxTcRows = 64;  // query rows (the MMA's M) of one CTA
 
 struct TcCfg {
 #ifndef SMLA_TC_PRODUCER_WARPS
-#define SMLA_TC_PRODUCER_WARPS 8
+#define SMLA_TC_PRODUCER_WARPS 11
 #endif
     static constexpr int kProducerWarps = SMLA_TC_PRODUCER_WARPS;
     static constexpr int kMmaWarp = 4 + kProducerWarps;
@@ -227,7 +231,8 @@ __global__ void __launch_bounds__(TcCfg::kThreads, 1)
                 const int stage = it % C::kStages;
                 if (it >= C::kStages) mbar_wait(&kv_empty[stage], ((it / C::kStages) - 1) & 1, dead);
                 uint8_t *dst = smem + C::kOffKV + C::tile_off(stage);
-                // 72 warp instructions per tile, each 4 rows x 128 B; warp pw takes i = pw mod 4
+                // 72 warp instructions per tile, each 4 rows x 128 B; warp pw takes every
+                // kProducerWarps-th from i = pw
 #pragma unroll 2
                 for (int i = pw; i < 72; i += C::kProducerWarps) {
                     const int seg = 4 * i + (lane >> 3);  // 0..287: row r, column box
@@ -488,6 +493,13 @@ __global__ void __launch_bounds__(TcCfg::kThreads, 1)
         }
         const bool write = hrow < nrows;
         const size_t row = (size_t)row0 + hrow;
+        // Partials leave through shared memory so that each store instruction
+        // writes whole 128-B row segments: lane L holds 32 columns of its own
+        // row, and a direct store would touch 32 rows (32 lines) at once.
+        // Per warp, 32 lane-rows of 32 floats at a 144-B pitch (conflict-free
+        // both ways) in the Q region, which no MMA reads any more.
+        constexpr int kPitch = 36;
+        float *stage = reinterpret_cast<float *>(smem + C::kOffQ) + warp * (32 * kPitch);
 #pragma unroll 1
         for (int c = 0; c < 256; c += 32) {
             uint32_t orr[32];
@@ -498,15 +510,28 @@ __global__ void __launch_bounds__(TcCfg::kThreads, 1)
 #pragma unroll
                 for (int j = 0; j < 32; ++j) orr[j] = 0u;
             }
-            if (!write) continue;
             const int col = 256 * half + c;
             if (!DIRECT) {
-                float4 *dst = reinterpret_cast<float4 *>(p.part_o + (row * p.nsplit + s) * kDc + col);
+                float4 *mine = reinterpret_cast<float4 *>(stage + lane * kPitch);
 #pragma unroll
                 for (int j = 0; j < 8; ++j)
-                    dst[j] = make_float4(__uint_as_float(orr[4 * j]), __uint_as_float(orr[4 * j + 1]),
-                                         __uint_as_float(orr[4 * j + 2]), __uint_as_float(orr[4 * j + 3]));
-            } else {
+                    mine[j] = make_float4(__uint_as_float(orr[4 * j]), __uint_as_float(orr[4 * j + 1]),
+                                          __uint_as_float(orr[4 * j + 2]), __uint_as_float(orr[4 * j + 3]));
+                __syncwarp();
+                // eight lanes per lane-row, four lane-rows per instruction
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const int lr = 4 * k + (lane >> 3);  // lane-row: lane lr's row and half
+                    const int ch = lane & 7;             // 16-B chunk of its 128-B segment
+                    const int hr = 16 * q4 + (lr & 15);
+                    if (hr < nrows) {
+                        const float4 v = *reinterpret_cast<const float4 *>(stage + lr * kPitch + 4 * ch);
+                        *reinterpret_cast<float4 *>(p.part_o + (((size_t)row0 + hr) * p.nsplit + s) * kDc +
+                                                    256 * (lr >> 4) + c + 4 * ch) = v;
+                    }
+                }
+                __syncwarp();
+            } else if (write) {
                 const float inv = (l_tot > 0.f) ? 1.f / l_tot : 0.f;
                 uint4 *dst = reinterpret_cast<uint4 *>(p.o + row * kDc + col);
 #pragma unroll
