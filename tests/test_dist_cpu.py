@@ -88,3 +88,28 @@ def test_reference_arm_rank0_prints_one_line():
     assert d["impl"] == "reference" and d["cpu_baseline"]["kind"] == "oracle"
     assert d["unit"] == "query-tokens/s" and d["value"] > 0
     assert d["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_dense_replicas_keep_the_shape_and_change_the_data():
+    """Weak scaling for the dense verify workload: each rank's replica has the
+    same shape and visible lengths (the same work) with its own data."""
+    sys.path.insert(0, ROOT)
+    import bench
+    r0 = bench.replica_workload("dense_verify", 0, 2)
+    r1 = bench.replica_workload("dense_verify", 1, 2)
+    assert r0.dense and r1.dense
+    assert r0.q.shape == r1.q.shape and r0.cache.shape == r1.cache.shape
+    assert torch.equal(r0.seq_lens, r1.seq_lens)
+    assert not torch.equal(r0.q, r1.q)
+    assert bench.workload_bytes(r0) == bench.workload_bytes(r1)
+
+
+def test_reference_arm_dense_workload(tmp_path):
+    env = dict(os.environ, RANK="0", WORLD_SIZE="1")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--workload", "dense_verify", "--cpu-seconds", "0.5"],
+                       env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr
+    d = json.loads([l for l in r.stdout.splitlines() if l.strip()][0])
+    assert d["impl"] == "reference" and d["config"]["workload"] == "dense_verify"
+    assert "dense" in d["cpu_baseline"]["sample"] and d["value"] > 0
