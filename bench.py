@@ -372,8 +372,8 @@ def run_ours(args, world, rank, local):
                            w.scale)
 
         def decode():
-            """One whole decode: smla_decode (partial pass + LSE combine), or
-            smla_decode_dense (position lists, partial pass, combine)."""
+            """One whole decode: smla_decode, or smla_decode_dense for the dense
+            workload (partial pass + LSE combine either way)."""
             if w.dense:
                 st = lib.smla_decode_dense(*dense_args, S, ws.data_ptr(), ws.numel(),
                                            o.data_ptr(), lse.data_ptr(), sptr)
