@@ -9,13 +9,13 @@
 // heads >= H are zero rows of Q and are never written out), or in dense mode
 // up to 64 / H query tokens of one sequence.  512 threads (16 warps x 128
 // registers: the whole register file):
-//   warps 0-3  softmax warpgroup: stages Q (128B-swizzled) once, then per
-//              PAIR of 32-row tiles reads S from TMEM (tcgen05.ld), masks,
-//              keeps a running max per head with lazy rescaling (O is only
-//              rescaled when the max grows by more than 2^8), writes P as bf16
-//              into each tile's spent k_pe box, and finally drains O
-//              (partials through shared memory, whole 128-B segments per
-//              store).
+//   warps 0-3  softmax warpgroup: stages Q into TMEM once (it is the QK
+//              MMA's A operand), then per PAIR of 32-row tiles reads S from
+//              TMEM (tcgen05.ld), masks, keeps a running max per head with
+//              lazy rescaling (O is only rescaled when the max grows by more
+//              than 2^8), writes P as bf16 into each tile's spent k_pe box,
+//              and finally drains O (partials through shared memory, whole
+//              128-B segments per store).
 //   warps 4-14 producers: resolve the split's indices to rows (as the mma
 //              kernel does), then gather each 32-row tile with 16-byte
 //              cp.async copies written straight into the 128B-swizzled
@@ -24,7 +24,7 @@
 //              cp.async.mbarrier.arrive.  Padding slots copy row 0 and are
 //              masked.
 //   warp 15    TMEM owner + MMA issuer (one thread):
-//                QK(pair): S[64 x 64] = Q[64 x 576] [K_2p K_2p+1]^T   36 x (M64 N64 K16)
+//                QK(pair): S[64 x 64] = Q[64 x 576] [K_2p K_2p+1]^T   36 x (M64 N64 K16), A in TMEM
 //                PV(t):    O[64 x 512] += P_t[64 x 32] C_t[32 x 512]  2 x 2 x (M64 N256 K16)
 //              A tcgen05 MMA costs at least ~46 cycles whatever its size
 //              below M64 N64 (M64 N32 costs the same as M64 N64), so the
@@ -32,15 +32,20 @@
 //              ring keeps the pair's tiles side by side in every 64-column
 //              box.  The issuer polls: a pair's QK goes out as soon as both
 //              tiles have landed, its PV as soon as its P is ready.
-// Shared memory ring: two pair slots of 2 x 36864 B; box b (64 columns) of
-// tile h of a slot at slot + 8192 b + 4096 h, rows 128 B apart.
-// TMEM (512 columns; M = 64 accumulators occupy lanes 0-15 of each 32-lane
-// sub-partition, or 16-31 when addressed at lane offset 16):
-//   cols [0,256)   lane off 0: O[:, 0:256]     lane off 16: O[:, 256:512]
-//   cols 256+64b   lane off 0: S of pair b (b = pair parity, double buffered),
-//                  columns 0-31 its first tile, 32-63 its second
-// Softmax thread (warp q, lane l): lanes 0-15 own head 16q + l and do the
-// pair's softmax; lane l + 16 rescales the second half of the same head's O.
+// Shared memory ring: three pair slots of 2 x 36864 B (Q is not in shared
+// memory); box b (64 columns) of tile h of a slot at slot + 8192 b + 4096 h,
+// rows 128 B apart.
+// TMEM (512 columns; an M = 64 operand or accumulator occupies lanes 0-15 of
+// each 32-lane sub-partition, or 16-31 when addressed at lane offset 16; an A
+// operand in TMEM must sit at its accumulator's lanes):
+//   lanes 0-15   cols [0,288)    Q, two bf16 per column (A of QK)
+//                cols 288+64b    S of pair b (b = pair parity, double
+//                                buffered), columns 0-31 its first tile,
+//                                32-63 its second
+//   lanes 16-31  cols [0,512)    O
+// Softmax thread (warp q, lane l): head 16q + l % 16; lanes l and l + 16 take
+// the pair's first and second tile, and the first and second 32 of each 64
+// columns of O.
 #pragma once
 
 #include <climits>
@@ -62,23 +67,27 @@ struct TcCfg {
     static constexpr int kMmaWarp = 4 + kProducerWarps;
     static constexpr int kThreads = 32 * (kMmaWarp + 1);
     static constexpr int kTileRows = 32;
-    static constexpr int kStages = 4;                       // tiles in the ring (2 pair slots)
+    static constexpr int kStages = 6;                       // tiles in the ring (3 pair slots)
     static constexpr int kBoxBytes = kTileRows * 128;       // 4096: 32 rows x 64 bf16
     static constexpr int kBoxStride = 2 * kBoxBytes;        // 8192: the pair's two tiles per box
     static constexpr int kStageBytes = 9 * kBoxBytes;       // 36864 per tile
-    static constexpr int kQBoxBytes = 64 * 128;             // 8192
-    static constexpr int kOffQ = 0;                         // 9 x 8192
-    static constexpr int kOffKV = 9 * kQBoxBytes;           // 73728
+    static constexpr int kOffKV = 0;                        // Q lives in TMEM: the ring starts at 0
     static constexpr int kOffRows = kOffKV + kStages * kStageBytes;  // 221184
     static constexpr int kOffBar = kOffRows + kResolveChunk * 4;     // 229376
-    // barriers: kv_full[4], kv_empty[4], s_full[2], p_full[2], o_done[2], q_ready
-    static constexpr int kNumBars = 4 + 4 + 2 + 2 + 2 + 1;
+    // barriers: kv_full[6], kv_empty[6], s_full[2], p_full[2], o_done[2], q_ready
+    static constexpr int kNumBars = kStages + kStages + 2 + 2 + 2 + 1;
     static constexpr int kOffTmem = kOffBar + kNumBars * 8;
-    static constexpr int kOffHdr = kOffTmem + 16;           // u32 [4]
-    static constexpr int kBytes = kOffHdr + 16;
+    static constexpr int kOffHdr = kOffTmem + 16;           // u32 [kStages]
+    static constexpr int kBytes = kOffHdr + 4 * kStages;
     static constexpr int kSmemBytes = kBytes + 1024;        // + alignment slack for 1024-B atoms
     static constexpr uint32_t kTmemCols = 512;
-    static constexpr uint32_t kSCol = 256;
+    // TMEM: Q (the QK MMA's A operand, two bf16 per column) at lanes 0-15 of
+    // each sub-partition, columns [0, 288); S of a pair at the same lanes (an
+    // A operand in TMEM must share the accumulator's lanes), columns 288 +
+    // 64 * parity; O at lanes 16-31, columns [0, 512).
+    static constexpr uint32_t kQCol = 0;
+    static constexpr uint32_t kSCol = 288;
+    static constexpr uint32_t kOLane = 16;
     __host__ __device__ static constexpr int tile_off(int stage) {  // tile base inside the ring
         return (stage >> 1) * 2 * kStageBytes + (stage & 1) * kBoxBytes;
     }
@@ -121,16 +130,16 @@ __global__ void __launch_bounds__(TcCfg::kThreads, 1)
 
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::kOffBar);
     uint64_t *kv_full = bars;
-    uint64_t *kv_empty = bars + 4;
-    uint64_t *s_full = bars + 8;
-    uint64_t *p_full = bars + 10;
-    uint64_t *o_done = bars + 12;  // [pair parity]: PV of that pair complete
-    uint64_t *q_ready = bars + 14;
+    uint64_t *kv_empty = bars + C::kStages;
+    uint64_t *s_full = bars + 2 * C::kStages;
+    uint64_t *p_full = s_full + 2;
+    uint64_t *o_done = p_full + 2;  // [pair parity]: PV of that pair complete
+    uint64_t *q_ready = o_done + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::kOffTmem);
     volatile uint32_t *hdr = reinterpret_cast<volatile uint32_t *>(smem + C::kOffHdr);
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < 4; ++i) {
+        for (int i = 0; i < C::kStages; ++i) {
             // 32 cp.async arrivals per producer warp + one plain arrive that
             // publishes the tile's validity mask
             mbar_init(&kv_full[i], 32 * C::kProducerWarps + 1);
@@ -264,7 +273,6 @@ __global__ void __launch_bounds__(TcCfg::kThreads, 1)
         if (lane == 0) {
             constexpr uint32_t kIdescQK = idesc_bf16_f32(64, 64, false, false);
             constexpr uint32_t kIdescPV = idesc_bf16_f32(64, 256, false, true);
-            const uint32_t q_addr = sbase + C::kOffQ;
             mbar_wait(q_ready, 0, dead);
             tc_fence_after();
             // Issue whatever is ready: a pair's QK as soon as its tiles have
@@ -297,11 +305,10 @@ __global__ void __launch_bounds__(TcCfg::kThreads, 1)
 #pragma unroll 4
                         for (int kk = 0; kk < 36; ++kk) {
                             const uint32_t koff = (kk & 3) * 32;  // 16-element step inside the 128-B row
-                            const uint64_t a = smem_desc(q_addr + (kk >> 2) * C::kQBoxBytes + koff, 16,
-                                                         1024, kSwizzle128B);
+                            const uint32_t a = tmem + C::kQCol + 8 * kk;  // 16 bf16 = 8 columns of Q
                             const uint64_t bd = smem_desc(kv_addr + (kk >> 2) * C::kBoxStride + koff,
                                                           16, 1024, kSwizzle128B);
-                            umma_bf16(d, a, bd, kIdescQK, kk > 0 ? 1u : 0u);
+                            umma_bf16_ts(d, a, bd, kIdescQK, kk > 0 ? 1u : 0u);
                         }
                         umma_commit(&s_full[qk_next & 1]);
                         ++qk_next;
@@ -324,8 +331,8 @@ __global__ void __launch_bounds__(TcCfg::kThreads, 1)
                                                            kSwizzle128B);
                             const uint64_t bhi = smem_desc(kv_addr + 4 * C::kBoxStride + kk * 2048,
                                                            C::kBoxStride, 1024, kSwizzle128B);
-                            umma_bf16(tmem, a, blo, kIdescPV, acc);
-                            umma_bf16(tmem + (16u << 16), a, bhi, kIdescPV, acc);
+                            umma_bf16(tmem + (C::kOLane << 16), a, blo, kIdescPV, acc);
+                            umma_bf16(tmem + (C::kOLane << 16) + 256, a, bhi, kIdescPV, acc);
                         }
                         umma_commit(&kv_empty[stage]);
                     }
@@ -347,35 +354,48 @@ __global__ void __launch_bounds__(TcCfg::kThreads, 1)
         __syncwarp();
     } else {
         // ============================================================ softmax warpgroup
-        const int tid = threadIdx.x;  // 0..127
         const int q4 = warp;          // TMEM sub-partition (lanes 32*q4 .. +31)
         const int hrow = 16 * q4 + (lane & 15);
         const int half = lane >> 4;
 
-        // ---- stage Q (heads x 576, zero rows beyond H) as 9 swizzled 64-column boxes
+        const uint32_t t_lane = tmem + ((uint32_t)(32 * q4) << 16);            // lanes 0-15: Q, S
+        const uint32_t t_o = tmem + ((uint32_t)(32 * q4 + C::kOLane) << 16);  // lanes 16-31: O
+
+        // ---- stage Q (rows past the unit's real rows are zero) into TMEM, the
+        // QK MMA's A operand: row hrow at lane hrow % 16 of this sub-partition,
+        // 32-bit column j = bf16 elements 2j, 2j+1 (the row's own word order).
+        // Thread t writes columns 64 i + 32 (t / 16) + [0, 32) for i < 4, then
+        // 256 + 16 (t / 16) + [0, 16).
         {
-            const uint4 *qsrc = reinterpret_cast<const uint4 *>(p.q + (size_t)row0 * kD);
-            for (int c0 = 0; c0 < 64 * 72; c0 += 128 * 12) {
-                uint4 v[12];
+            const bool real = hrow < nrows;
+            const uint4 *qrow = reinterpret_cast<const uint4 *>(p.q + ((size_t)row0 + (real ? hrow : 0)) * kD);
+#pragma unroll 1
+            for (int i = 0; i < 4; ++i) {
+                uint32_t w[32];
 #pragma unroll
-                for (int k = 0; k < 12; ++k) {
-                    const int c = c0 + k * 128 + tid;
-                    const int h = c / 72;
-                    v[k] = (c < 64 * 72 && h < nrows) ? __ldg(qsrc + (size_t)h * 72 + (c % 72))
-                                                     : make_uint4(0u, 0u, 0u, 0u);
+                for (int k = 0; k < 8; ++k) {
+                    const uint4 v = real ? __ldg(qrow + 16 * i + 8 * half + k) : make_uint4(0u, 0u, 0u, 0u);
+                    w[4 * k] = v.x;
+                    w[4 * k + 1] = v.y;
+                    w[4 * k + 2] = v.z;
+                    w[4 * k + 3] = v.w;
                 }
-#pragma unroll
-                for (int k = 0; k < 12; ++k) {
-                    const int c = c0 + k * 128 + tid;
-                    if (c < 64 * 72) {
-                        const int h = c / 72, k16 = c % 72;
-                        const int box = k16 >> 3, ch = k16 & 7;
-                        *reinterpret_cast<uint4 *>(smem + C::kOffQ + box * C::kQBoxBytes + h * 128 +
-                                                   ((ch ^ (h & 7)) << 4)) = v[k];
-                    }
-                }
+                tmem_st16x2_32(t_lane + C::kQCol + 64 * i, w);
             }
-            fence_proxy_async_smem();
+            {
+                uint32_t w[16];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const uint4 v = real ? __ldg(qrow + 64 + 4 * half + k) : make_uint4(0u, 0u, 0u, 0u);
+                    w[4 * k] = v.x;
+                    w[4 * k + 1] = v.y;
+                    w[4 * k + 2] = v.z;
+                    w[4 * k + 3] = v.w;
+                }
+                tmem_st16x2_16(t_lane + C::kQCol + 256, w);
+            }
+            tmem_st_wait();
+            tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(q_ready);
         }
@@ -388,54 +408,49 @@ __global__ void __launch_bounds__(TcCfg::kThreads, 1)
                                                hrow / p.dense_h), 0), p.K)
                                : 0;
         float m_ref = -INFINITY;  // running reference max of head hrow (log2 units)
-        float l_acc = 0.f;        // sum of P of head hrow relative to m_ref (lanes 0-15; 0 elsewhere)
-        const uint32_t t_lane = tmem + ((uint32_t)(32 * q4) << 16);
+        float l_acc = 0.f;        // this thread's tile's share of the sum of P of head hrow
 
         for (int pr = 0; pr < n_pairs; ++pr) {
             const int t0 = 2 * pr;
             const bool has1 = t0 + 1 < n_tiles;
             mbar_wait(&s_full[pr & 1], (pr >> 1) & 1, dead);
             tc_fence_after();
-            // S of the pair: lanes 0-15 hold head hrow, columns 0-31 tile t0,
-            // 32-63 tile t0+1 (lanes 16-31 read unused TMEM lanes, ignored)
-            uint32_t s0[32], s1[32];
-            tmem_ld32(t_lane + C::kSCol + 64 * (pr & 1), s0);
-            tmem_ld32(t_lane + C::kSCol + 64 * (pr & 1) + 32, s1);
+            // S of the pair (TMEM lanes 0-15): thread t gets head hrow's scores
+            // against tile t0 + t / 16 (columns 32 (t / 16) + [0, 32)), so the
+            // two threads of a head split the pair's 64 columns
+            uint32_t sv[32];
+            tmem_ld16x2_32(t_lane + C::kSCol + 64 * (pr & 1), sv);
             tmem_ld_wait();
             mbar_wait(&kv_full[t0 % C::kStages], (t0 / C::kStages) & 1, dead);
-            uint32_t vm0 = hdr[t0 % C::kStages];
+            uint32_t vm = hdr[t0 % C::kStages];
             uint32_t vm1 = 0;
             if (has1) {
                 mbar_wait(&kv_full[(t0 + 1) % C::kStages], ((t0 + 1) / C::kStages) & 1, dead);
                 vm1 = hdr[(t0 + 1) % C::kStages];
             }
-            if (dense) {  // this row's causal limit, as a mask over the pair's columns
-                const int r0 = lim - (j0 + t0 * C::kTileRows);
-                const int r1 = r0 - C::kTileRows;
-                vm0 &= r0 >= 32 ? 0xffffffffu : (r0 <= 0 ? 0u : (1u << r0) - 1u);
-                vm1 &= r1 >= 32 ? 0xffffffffu : (r1 <= 0 ? 0u : (1u << r1) - 1u);
+            if (half) vm = vm1;  // an absent second tile: every column masked
+            if (dense) {  // this row's causal limit, as a mask over this tile's columns
+                const int r = lim - (j0 + (t0 + half) * C::kTileRows);
+                vm &= r >= 32 ? 0xffffffffu : (r <= 0 ? 0u : (1u << r) - 1u);
             }
-            const bool owner = half == 0;  // lanes 0-15 run the softmax of head hrow
-            // scores in log2 units, padding (and an absent second tile) -> -inf;
-            // selects, not branches
+            // scores in log2 units, padding -> -inf; selects, not branches
             float mt = -INFINITY;
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
-                const float x0 = ((vm0 >> j) & 1u) ? __uint_as_float(s0[j]) * p.scale_log2 : -INFINITY;
-                const float x1 = ((vm1 >> j) & 1u) ? __uint_as_float(s1[j]) * p.scale_log2 : -INFINITY;
-                s0[j] = __float_as_uint(x0);
-                s1[j] = __float_as_uint(x1);
-                mt = fmaxf(mt, fmaxf(x0, x1));
+                const float x = ((vm >> j) & 1u) ? __uint_as_float(sv[j]) * p.scale_log2 : -INFINITY;
+                sv[j] = __float_as_uint(x);
+                mt = fmaxf(mt, x);
             }
-            if (!owner) mt = -INFINITY;
+            // the pair's max of head hrow; both threads of the head then keep
+            // the same reference max (same inputs, same steps)
+            mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 16));
             float alpha = 1.f;
-            if (owner && mt > m_ref + C::kTau) {
+            if (mt > m_ref + C::kTau) {
                 alpha = (m_ref == -INFINITY) ? 0.f : fast_exp2(m_ref - mt);
                 m_ref = mt;
             }
-            alpha = __shfl_sync(0xffffffffu, alpha, lane & 15);  // lane l+16 rescales O[:, 256:512]
-            // Rescale this thread's half row of O when its head's max jumped
-            // (warp-collective TMEM access; alpha = 1 for the other threads).
+            // Rescale the head's row of O when its max jumped (warp-collective
+            // TMEM access; alpha = 1 for the other heads).
             const bool need = (pr >= 1) && (alpha != 1.f);
             if (__any_sync(0xffffffffu, need)) {
                 // O must hold PV of pair pr-1 before it is rescaled.  The tensor
@@ -444,34 +459,31 @@ __global__ void __launch_bounds__(TcCfg::kThreads, 1)
                 mbar_wait(&o_done[(pr - 1) & 1], ((pr - 1) >> 1) & 1, dead);
                 tc_fence_after();
 #pragma unroll 1
-                for (int c = 0; c < 256; c += 32) {
+                for (int c = 0; c < 512; c += 64) {  // thread t: columns c + 32 (t / 16) + [0, 32)
                     uint32_t orr[32];
-                    tmem_ld32(t_lane + c, orr);
+                    tmem_ld16x2_32(t_o + c, orr);
                     tmem_ld_wait();
 #pragma unroll
                     for (int j = 0; j < 32; ++j) orr[j] = __float_as_uint(__uint_as_float(orr[j]) * alpha);
-                    tmem_st32(t_lane + c, orr);
+                    tmem_st16x2_32(t_o + c, orr);
                 }
                 tmem_st_wait();
             }
-            if (owner) {
+            {
                 const float mu = (m_ref == -INFINITY) ? 0.f : m_ref;
                 float ps = 0.f;
+                uint32_t pk[16];
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    uint32_t pk[16];
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const uint32_t r0 = h ? s1[2 * j] : s0[2 * j], r1 = h ? s1[2 * j + 1] : s0[2 * j + 1];
-                        const float a0 = fast_exp2(__uint_as_float(r0) - mu);  // exp2(-inf) = 0
-                        const float a1 = fast_exp2(__uint_as_float(r1) - mu);
-                        ps += a0 + a1;
-                        pk[j] = pack_bf16x2(a0, a1);
-                    }
-                    if (h == 1 && !has1) continue;
-                    // P tile (64 heads x 32 rows, bf16) in the tile's spent k_pe box,
-                    // K-major 64B swizzle
-                    uint8_t *pbase = smem + C::kOffKV + C::tile_off((t0 + h) % C::kStages) + 8 * C::kBoxStride;
+                for (int j = 0; j < 16; ++j) {
+                    const float a0 = fast_exp2(__uint_as_float(sv[2 * j]) - mu);  // exp2(-inf) = 0
+                    const float a1 = fast_exp2(__uint_as_float(sv[2 * j + 1]) - mu);
+                    ps += a0 + a1;
+                    pk[j] = pack_bf16x2(a0, a1);
+                }
+                if (half == 0 || has1) {
+                    // this tile's P (64 heads x 32 rows, bf16) in its spent k_pe
+                    // box, K-major 64B swizzle
+                    uint8_t *pbase = smem + C::kOffKV + C::tile_off((t0 + half) % C::kStages) + 8 * C::kBoxStride;
 #pragma unroll
                     for (int c = 0; c < 4; ++c)
                         *reinterpret_cast<uint4 *>(pbase + hrow * 64 + ((c ^ ((hrow >> 1) & 3)) << 4)) =
@@ -493,24 +505,25 @@ __global__ void __launch_bounds__(TcCfg::kThreads, 1)
         }
         const bool write = hrow < nrows;
         const size_t row = (size_t)row0 + hrow;
-        // Partials leave through shared memory so that each store instruction
-        // writes whole 128-B row segments: lane L holds 32 columns of its own
-        // row, and a direct store would touch 32 rows (32 lines) at once.
-        // Per warp, 32 lane-rows of 32 floats at a 144-B pitch (conflict-free
-        // both ways) in the Q region, which no MMA reads any more.
+        // O of head hrow from TMEM lanes 16-31: thread t holds columns
+        // c + 32 (t / 16) + [0, 32) per step.  Partials leave through shared
+        // memory so that each store instruction writes whole 128-B row
+        // segments (a direct store would touch 16 rows at once).  Per warp, 32
+        // lane-rows of 32 floats at a 144-B pitch (conflict-free both ways),
+        // in the ring: every tile has been consumed by now.
         constexpr int kPitch = 36;
-        float *stage = reinterpret_cast<float *>(smem + C::kOffQ) + warp * (32 * kPitch);
+        float *stage = reinterpret_cast<float *>(smem + C::kOffKV) + warp * (32 * kPitch);
 #pragma unroll 1
-        for (int c = 0; c < 256; c += 32) {
+        for (int c = 0; c < 512; c += 64) {
             uint32_t orr[32];
             if (n_pairs > 0) {
-                tmem_ld32(t_lane + c, orr);
+                tmem_ld16x2_32(t_o + c, orr);
                 tmem_ld_wait();
             } else {
 #pragma unroll
                 for (int j = 0; j < 32; ++j) orr[j] = 0u;
             }
-            const int col = 256 * half + c;
+            const int col = c + 32 * half;
             if (!DIRECT) {
                 float4 *mine = reinterpret_cast<float4 *>(stage + lane * kPitch);
 #pragma unroll
@@ -521,13 +534,13 @@ __global__ void __launch_bounds__(TcCfg::kThreads, 1)
                 // eight lanes per lane-row, four lane-rows per instruction
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
-                    const int lr = 4 * k + (lane >> 3);  // lane-row: lane lr's row and half
+                    const int lr = 4 * k + (lane >> 3);  // lane-row: lane lr's head and columns
                     const int ch = lane & 7;             // 16-B chunk of its 128-B segment
                     const int hr = 16 * q4 + (lr & 15);
                     if (hr < nrows) {
                         const float4 v = *reinterpret_cast<const float4 *>(stage + lr * kPitch + 4 * ch);
                         *reinterpret_cast<float4 *>(p.part_o + (((size_t)row0 + hr) * p.nsplit + s) * kDc +
-                                                    256 * (lr >> 4) + c + 4 * ch) = v;
+                                                    c + 32 * (lr >> 4) + 4 * ch) = v;
                     }
                 }
                 __syncwarp();
