@@ -113,3 +113,23 @@ def test_reference_arm_dense_workload(tmp_path):
     d = json.loads([l for l in r.stdout.splitlines() if l.strip()][0])
     assert d["impl"] == "reference" and d["config"]["workload"] == "dense_verify"
     assert "dense" in d["cpu_baseline"]["sample"] and d["value"] > 0
+
+
+def test_traffic_record_tracks_its_kernel_sources(tmp_path, monkeypatch):
+    """roofline.traffic is reported only while the captured kernel's own source
+    files are unchanged: editing the tcgen05 kernel drops the tcgen05 figures
+    and keeps the others."""
+    import shutil
+    sys.path.insert(0, ROOT)
+    import bench
+    for sub in ("profiles", os.path.join("sparse_mla_decode_partial_b200", "csrc")):
+        shutil.copytree(os.path.join(ROOT, sub), tmp_path / sub)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    before = {wl: bench.measured_traffic(wl) for wl in ("single_request", "batched", "mixed")}
+    assert all(v is not None for v in before.values()), before
+    tc = tmp_path / "sparse_mla_decode_partial_b200" / "csrc" / "smla_partial_tc.cuh"
+    tc.write_text(tc.read_text() + "\n// edited\n")
+    assert bench.measured_traffic("mixed") is None
+    assert bench.measured_traffic("single_request") == before["single_request"]
+    assert bench.measured_traffic("batched") == before["batched"]
+    assert bench.measured_traffic("tiny") is None          # never captured
