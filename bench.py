@@ -7,9 +7,16 @@
 One step = one whole decode (partial pass + LSE combine, through the C ABI)
 over one batch of the named synthetic workload, inputs resident in HBM.  L2
 is flushed before every step; each step is timed with CUDA events on the
-launching stream.  Rank 0 prints one JSON line.  Under torchrun every rank
-runs an independent replica (its own seed), so per-GPU work is fixed
-(weak scaling) and the step time is the max over ranks.
+launching stream; `ms_per_step` is the median (the mean is reported beside
+it).  Rank 0 prints one JSON line.  Under torchrun every rank runs an
+independent replica (its own seed), so per-GPU work is fixed (weak scaling)
+and the step time is the max over ranks.
+
+On one GPU the line also carries a `workloads` record: the memory-bound
+batched and mixed-length configurations and the two verify shapes, each
+measured after the headline in the same process under the same protocol
+(decode and partial pass at the heuristic NSPLIT, medians, its own roofline
+and clock record).
 
 The metric (query tokens per second, us per call and achieved HBM GB/s,
 against NSPLIT) follows "The Occupancy Hypothesis ..." (section "The
@@ -47,6 +54,8 @@ def parse_args(argv=None):
     ap.add_argument("--nsplit", type=int, default=0, help="0 = the library's heuristic")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-sweep", action="store_true", help="skip the NSPLIT sweep")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the other configurations measured beside the headline")
     ap.add_argument("--cpu-seconds", type=float, default=6.0,
                     help="seconds of oracle CPU time for the baseline sample")
     return ap.parse_args(argv)
@@ -323,36 +332,47 @@ def cpu_baseline(w, seconds: float):
 
 
 # ----------------------------------------------------------------------------- GPU arm
-def run_ours(args, world, rank, local):
-    import torch
-    from sparse_mla_decode_partial_b200 import binding, build, workloads
+# Workloads measured beside the headline in the same invocation: the
+# memory-bound configurations the roofline target is stated on (batched,
+# mixed) and the two verify shapes.
+SIDE_WORKLOADS = ("batched", "mixed", "spec_verify", "dense_verify")
 
-    build.build()
-    lib = binding.lib()
-    dev = torch.device("cuda", local)
-    torch.cuda.set_device(dev)
-    w_host = replica_workload(args.workload, rank, world)
-    w = w_host.to(dev)
-    B, T, H, K = w.B, w.T, w.H, w.K
-    nsplit = args.nsplit or (binding.dense_nsplit(B, T, H, K) if w.dense
-                             else binding.choose_nsplit(B, T, H, K, 0))
-    stream = torch.cuda.current_stream(dev)
-    sptr = stream.cuda_stream
 
-    part_bytes, step_bytes = workload_bytes(w_host)
-    flops = workload_flops(w_host)
-    hbm_peak, tc_peak, peak_src = load_peaks()
+def bench_config(w, workload: str, nsplit_arg: int, world: int) -> dict:
+    """The `config` object of the JSON line, identical in both arms for the
+    same command line (the split count the library resolves is reported
+    beside it, as `nsplit_used`)."""
+    return {"workload": workload, "shape": describe(w),
+            "nsplit": nsplit_arg if nsplit_arg else "heuristic",
+            "batch": w.B, "q_len": w.T, "heads": w.H, "topk": w.K,
+            "l2": "flushed before every step: 256 MB write then 256 MB read",
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
 
-    flush_w = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
-    flush_r = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
-    sink = torch.empty(1, dtype=torch.float32, device=dev)
 
-    def flush():
-        flush_w.fill_(1.0)
-        torch.sum(flush_r, dim=0, out=sink[0])
+class Harness:
+    """Device-side timing through the C ABI on one stream: L2 flush before
+    every step, CUDA events on the launching stream around each step."""
 
-    def make_steps(S):
-        """(decode step, partial-only step) for NSPLIT = S, through the C ABI."""
+    def __init__(self, dev):
+        import torch
+        from sparse_mla_decode_partial_b200 import binding
+        self.torch, self.binding, self.lib = torch, binding, binding.lib()
+        self.dev = dev
+        self.stream = torch.cuda.current_stream(dev)
+        self.sptr = self.stream.cuda_stream
+        self.flush_w = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+        self.flush_r = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+        self.sink = torch.empty(1, dtype=torch.float32, device=dev)
+
+    def flush(self):
+        self.flush_w.fill_(1.0)
+        self.torch.sum(self.flush_r, dim=0, out=self.sink[0])
+
+    def steps(self, w, S):
+        """(decode step, partial-only step) for NSPLIT = S on device workload w;
+        each returns (status, kernel launches)."""
+        torch, binding, lib, sptr, dev = self.torch, self.binding, self.lib, self.sptr, self.dev
+        B, T, H, K = w.B, w.T, w.H, w.K
         n = B * T * H * S
         po = torch.empty(max(n * 512, 4), dtype=torch.float32, device=dev)
         pm = torch.empty(max(n, 1), dtype=torch.float32, device=dev)
@@ -362,74 +382,143 @@ def run_ours(args, world, rank, local):
         if w.dense:
             ws = torch.empty(max(16, binding.dense_workspace_bytes(B, T, H, K, S)),
                              dtype=torch.uint8, device=dev)
-            dense_args = (w.q.data_ptr(), w.cache.data_ptr(), w.num_pages, w.page_table.data_ptr(),
-                          w.pt_stride, w.seq_lens.data_ptr(), B, T, H, K, 64, w.scale)
+            common = (w.q.data_ptr(), w.cache.data_ptr(), w.num_pages, w.page_table.data_ptr(),
+                      w.pt_stride, w.seq_lens.data_ptr(), B, T, H, K, 64, w.scale)
+            whole, part = lib.smla_decode_dense, lib.smla_decode_dense_partial
         else:
             ws = torch.empty(max(16, binding.workspace_bytes(B, T, H, S)), dtype=torch.uint8,
                              device=dev)
-            args_common = (w.q.data_ptr(), w.cache.data_ptr(), w.num_pages,
-                           w.page_table.data_ptr(), w.pt_stride, w.idx.data_ptr(), B, T, H, K, 64,
-                           w.scale)
+            common = (w.q.data_ptr(), w.cache.data_ptr(), w.num_pages, w.page_table.data_ptr(),
+                      w.pt_stride, w.idx.data_ptr(), B, T, H, K, 64, w.scale)
+            whole, part = lib.smla_decode, lib.smla_decode_partial
 
         def decode():
-            """One whole decode: smla_decode, or smla_decode_dense for the dense
-            workload (partial pass + LSE combine either way)."""
-            if w.dense:
-                st = lib.smla_decode_dense(*dense_args, S, ws.data_ptr(), ws.numel(),
-                                           o.data_ptr(), lse.data_ptr(), sptr)
-                return st, (1 if S == 1 else 2)
-            st = lib.smla_decode(*args_common, S, ws.data_ptr(), ws.numel(), o.data_ptr(),
-                                 lse.data_ptr(), sptr)
+            """One whole decode: partial pass + LSE combine in one call."""
+            st = whole(*common, S, ws.data_ptr(), ws.numel(), o.data_ptr(), lse.data_ptr(), sptr)
             return st, (1 if S == 1 else 2)
 
         def partial():
             """The partial pass alone (with S = 1 it writes o and lse directly)."""
-            if w.dense:
-                if S == 1:
-                    return lib.smla_decode_dense(*dense_args, 1, None, 0, o.data_ptr(),
-                                                 lse.data_ptr(), sptr), 1
-                return lib.smla_decode_dense_partial(*dense_args, S, po.data_ptr(), pm.data_ptr(),
-                                                     pl.data_ptr(), sptr), 1
             if S == 1:
-                return lib.smla_decode(*args_common, 1, None, 0, o.data_ptr(), lse.data_ptr(),
-                                       sptr), 1
-            return lib.smla_decode_partial(*args_common, S, po.data_ptr(), pm.data_ptr(),
-                                           pl.data_ptr(), sptr), 1
+                return whole(*common, 1, None, 0, o.data_ptr(), lse.data_ptr(), sptr), 1
+            return part(*common, S, po.data_ptr(), pm.data_ptr(), pl.data_ptr(), sptr), 1
         return decode, partial
 
-    def timed(step, n):
+    def timed(self, step, n):
+        """n flushed steps; returns (per-step ms list, kernel launches)."""
+        torch = self.torch
         ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n)]
         launches = 0
         for i in range(n):
-            flush()
-            ev[i][0].record(stream)
+            self.flush()
+            ev[i][0].record(self.stream)
             st, nl = step()
-            ev[i][1].record(stream)
+            ev[i][1].record(self.stream)
             if st != 0:
-                raise RuntimeError(binding.status_string(st))
+                raise RuntimeError(self.binding.status_string(st))
             launches += nl
-        torch.cuda.synchronize(dev)
+        torch.cuda.synchronize(self.dev)
         return [e[0].elapsed_time(e[1]) for e in ev], launches
 
-    step, part_step = make_steps(nsplit)
-    for _ in range(max(3, args.warmup)):
-        flush()
-        step()
-        part_step()
-    torch.cuda.synchronize(dev)
+    def warm(self, fns, n):
+        for _ in range(max(3, n)):
+            for f in fns:
+                self.flush()
+                f()
+        self.torch.cuda.synchronize(self.dev)
+
+
+def roofline(w_host, nsplit, part_ms, workload, hbm_peak, tc_peak, peak_src):
+    """The partial kernel's roofline record: algorithmic bytes per launch over
+    its CUDA-event duration, against the measured HBM copy bandwidth."""
+    part_bytes, _ = workload_bytes(w_host)
+    flops = workload_flops(w_host)
+    part_us = part_ms * 1e3
+    achieved = part_bytes / (part_us * 1e-6) / 1e9
+    tc_achieved = flops / (part_us * 1e-6) / 1e12
+    return {"bound": "hbm",
+            "kernel": partial_kernel_name(w_host.H, w_host.K, nsplit, w_host.pt_stride,
+                                          w_host.dense),
+            "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
+            "frac": round(achieved / hbm_peak, 4),
+            "peak_source": (f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured"
+                            else "fallback"),
+            "traffic": measured_traffic(workload),
+            "traffic_source": "profiles/ncu_traffic.json (ncu dram__bytes_read.sum + "
+                              "dram__bytes_write.sum of one capture of this kernel)",
+            "algorithmic_bytes_per_launch": part_bytes,
+            "partial_us_median": round(part_us, 3),
+            "tensor_tflops": round(tc_achieved, 2),
+            "tensor_frac_of_bf16_peak": round(tc_achieved / tc_peak, 4)}
+
+
+def side_workload(h, name, steps, warmup, peaks):
+    """One configuration measured beside the headline: decode and partial pass
+    at the heuristic NSPLIT, the same flush protocol, its own clock record."""
+    import torch
+    from sparse_mla_decode_partial_b200 import binding, workloads
+    w_host = workloads.WORKLOADS[name]()
+    w = w_host.to(h.dev)
+    B, T, H, K = w.B, w.T, w.H, w.K
+    S = binding.dense_nsplit(B, T, H, K) if w.dense else binding.choose_nsplit(B, T, H, K, 0)
+    decode, partial = h.steps(w, S)
+    h.warm([decode, partial], warmup)
+    sampler = ClockSampler(h.dev.index)
+    with sampler:
+        tot, launches = h.timed(decode, steps)
+        part, _ = h.timed(partial, steps)
+    _, step_bytes = workload_bytes(w_host)
+    us = statistics.median(tot) * 1e3
+    rec = {"shape": describe(w_host), "nsplit": S, "steps": steps,
+           "us_per_call": round(us, 3), "us_per_call_mean": round(statistics.fmean(tot) * 1e3, 3),
+           "partial_us": round(statistics.median(part) * 1e3, 3),
+           "partial_us_mean": round(statistics.fmean(part) * 1e3, 3),
+           "q_tok_s": round(B * T / (us * 1e-6), 1),
+           "hbm_gbs_step": round(step_bytes / (us * 1e-6) / 1e9, 1),
+           "roofline": roofline(w_host, S, statistics.median(part), name, *peaks),
+           "gpu_launches": launches, "clocks": sampler.summary()}
+    del w, decode, partial
+    torch.cuda.empty_cache()
+    return rec
+
+
+def run_ours(args, world, rank, local):
+    import torch
+    from sparse_mla_decode_partial_b200 import binding, build
+
+    build.build()
+    lib = binding.lib()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    h = Harness(dev)
+    sptr = h.sptr
+    w_host = replica_workload(args.workload, rank, world)
+    w = w_host.to(dev)
+    B, T, H, K = w.B, w.T, w.H, w.K
+    nsplit = args.nsplit or (binding.dense_nsplit(B, T, H, K) if w.dense
+                             else binding.choose_nsplit(B, T, H, K, 0))
+    stream = h.stream
+
+    _, step_bytes = workload_bytes(w_host)
+    peaks = load_peaks()
+
+    step, part_step = h.steps(w, nsplit)
+    h.warm([step, part_step], args.warmup)
 
     sampler = ClockSampler(dev.index)
     barrier(world)
     torch.cuda.synchronize(dev)
     with sampler:
-        tot, launches = timed(step, args.steps)
-        part, _ = timed(part_step, args.steps)
+        tot, launches = h.timed(step, args.steps)
+        part, _ = h.timed(part_step, args.steps)
     barrier(world)
     torch.cuda.synchronize(dev)
 
-    ms_step = statistics.fmean(tot)
-    ms_part = statistics.fmean(part)
+    # median over the timed steps (the mean is reported beside it)
+    ms_step = statistics.median(tot)
+    ms_part = statistics.median(part)
     tokens_all, ms_step_max, value = aggregate(float(B * T), ms_step, world)
+    ms_mean_max = max_over_ranks(statistics.fmean(tot), world)
 
     # e2e: per-step data in pinned host memory through the C ABI's host entry
     # point (smla_decode_host): the library pulls q, the top-k indices and the
@@ -490,7 +579,7 @@ def run_ours(args, world, rank, local):
     n_e2e = max(10, min(args.steps, 200))
     times = []
     for _ in range(n_e2e):
-        flush()
+        h.flush()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         st = e2e_step()
@@ -499,9 +588,10 @@ def run_ours(args, world, rank, local):
         if st != 0:
             raise RuntimeError(binding.status_string(st))
         times.append(e0.elapsed_time(e1))
-    e2e_ms = max_over_ranks(statistics.fmean(times), world)
+    e2e_ms = max_over_ranks(statistics.median(times), world)
     e2e = {"value": tokens_all / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
-           "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "note": e2e_note}
+           "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+           "ms_per_step_mean": max_over_ranks(statistics.fmean(times), world), "note": e2e_note}
 
     # Warm-L2 reference (after the timed region, not part of value): the same
     # step back to back without the flush, so the selected rows may still sit
@@ -517,59 +607,53 @@ def run_ours(args, world, rank, local):
         e1.record(stream)
         warm.append((e0, e1))
     torch.cuda.synchronize(dev)
-    warm_us = statistics.fmean(a.elapsed_time(b) for a, b in warm) * 1e3
+    warm_us = statistics.median(a.elapsed_time(b) for a, b in warm) * 1e3
 
     # NSPLIT sweep (rank 0 only, after the timed region)
     sweep = []
     if rank == 0 and not args.no_sweep:
         cands = list(w_host.nsplit_sweep) or sorted({1, 2, 4, 8, 16, 32, 64, nsplit})
         for S in sorted(set(cands) | {nsplit}):
-            d_fn, p_fn = make_steps(S)
-            for _ in range(5):
-                flush()
-                d_fn()
-                p_fn()
+            d_fn, p_fn = h.steps(w, S)
+            h.warm([d_fn, p_fn], 5)
             nrep = max(20, min(args.steps, 200))
-            t, _ = timed(d_fn, nrep)
-            p_, _ = timed(p_fn, nrep)
-            us = statistics.fmean(t) * 1e3
+            t, _ = h.timed(d_fn, nrep)
+            p_, _ = h.timed(p_fn, nrep)
+            us = statistics.median(t) * 1e3
             sweep.append({"nsplit": S, "us_per_call": round(us, 3),
-                          "partial_us": round(statistics.fmean(p_) * 1e3, 3),
+                          "partial_us": round(statistics.median(p_) * 1e3, 3),
                           "q_tok_s": round(B * T / (us * 1e-6), 1),
                           "hbm_gbs": round(step_bytes / (us * 1e-6) / 1e9, 1)})
 
     if rank != 0:
         return None
 
-    part_us = ms_part * 1e3
-    achieved = part_bytes / (part_us * 1e-6) / 1e9
-    tc_achieved = flops / (part_us * 1e-6) / 1e12
+    # The other configurations, measured after the headline in the same
+    # process (one GPU only: under torchrun the ranks would wait on rank 0)
+    side = {}
+    if world == 1 and not args.no_workloads:
+        del w
+        torch.cuda.empty_cache()
+        for name in SIDE_WORKLOADS:
+            if name != args.workload:
+                side[name] = side_workload(h, name, min(args.steps, 200), args.warmup, peaks)
+
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step_max, 6),
+        "ms_per_step_mean": round(ms_mean_max, 6),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": data_note(w_host),
-        "config": {"workload": args.workload, "shape": describe(w_host), "nsplit": nsplit,
-                   "nsplit_policy": "explicit" if args.nsplit else "heuristic",
-                   "batch": B, "q_len": T, "heads": H, "topk": K,
-                   "l2": "flushed before every step: 256 MB write then 256 MB read",
-                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "config": bench_config(w_host, args.workload, args.nsplit, world),
+        "nsplit_used": nsplit,
         "us_per_call": round(ms_step_max * 1e3, 3),
         "hbm_gbs_step": round(step_bytes / (ms_step * 1e-3) / 1e9, 1),
-        "kernel_us": {"partial": round(part_us, 3),
-                      "note": "partial pass timed alone in a second loop of the same length; "
-                              "the step runs it and the combine through one smla_decode call"},
-        "roofline": {"bound": "hbm",
-                     "kernel": partial_kernel_name(H, K, nsplit, w_host.pt_stride, w_host.dense),
-                     "achieved": round(achieved, 1),
-                     "peak": hbm_peak, "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),
-                     "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured" else "fallback",
-                     "traffic": measured_traffic(args.workload),
-                     "traffic_source": "profiles/ncu_traffic.json (ncu dram__bytes_read.sum + "
-                                       "dram__bytes_write.sum of one capture of this kernel)",
-                     "algorithmic_bytes_per_launch": part_bytes,
-                     "tensor_tflops": round(tc_achieved, 2),
-                     "tensor_frac_of_bf16_peak": round(tc_achieved / tc_peak, 4)},
+        "kernel_us": {"partial": round(ms_part * 1e3, 3),
+                      "partial_mean": round(statistics.fmean(part) * 1e3, 3),
+                      "note": "partial pass timed alone in a second loop of the same length "
+                              "(medians); the step runs it and the combine through one "
+                              "smla_decode call"},
+        "roofline": roofline(w_host, nsplit, ms_part, args.workload, *peaks),
         "warm_l2": {"us_per_call": round(warm_us, 3),
                     "note": "same step back to back without the L2 flush (labelled reference, "
                             "not the headline: repeated inputs leave the selected rows in L2)"},
@@ -577,6 +661,7 @@ def run_ours(args, world, rank, local):
         "clocks": sampler.summary(),
         "e2e": e2e,
         "nsplit_sweep": sweep,
+        "workloads": side,
     }
     return line
 
@@ -591,15 +676,13 @@ def run_reference(args, world, rank):
     t_all = time.perf_counter()
     res = cpu_baseline(w, seconds)
     value = res["value"]
-    nsplit = args.nsplit or None
     return {
         "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(w.B * w.T / value * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": data_note(w),
-        "config": {"workload": args.workload, "shape": describe(w), "nsplit": nsplit,
-                   "batch": w.B, "q_len": w.T, "heads": w.H, "topk": w.K},
+        "config": bench_config(w, args.workload, args.nsplit, world),
         "impl": "reference",
         "cpu_baseline": res,
         "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0,

@@ -196,15 +196,26 @@ smla_status smla_check_device(int clear, unsigned long long *n_bad_index, void *
  * holds in device memory on every GPU that loads it, until the process exits.
  *
  *  - q, kv_cache, page_table, topk_idx, o, lse: as for smla_decode (device,
- *    caller-owned).  nsplit = 0 picks the heuristic's value.
+ *    caller-owned).  nsplit = 0 picks the heuristic's value, lowered to the
+ *    largest split count whose partials fit the scratch array.
  *  - If smla_workspace_bytes(B, T, H, S) for the split count actually used is
  *    larger than SMLA_NOALLOC_SCRATCH_BYTES, the call launches nothing and
  *    returns SMLA_ERR_WORKSPACE_TOO_SMALL (smla_last_error() says how many
  *    bytes were needed); pass a smaller nsplit or use smla_decode.
  *  - The first call on each device looks up that device's copy of the scratch
  *    array (cudaGetSymbolAddress, with the device current); make that first
- *    call before starting any stream capture.  It allocates nothing and calls
- *    no allocating CUDA or library routine, then or later.
+ *    call before starting any stream capture.  The call itself never calls
+ *    cudaMalloc, cudaFree or an allocating library routine.  The array is,
+ *    however, part of the library's device code image: CUDA maps that image
+ *    (code plus the 16 MiB array) into device memory when it loads the module
+ *    on a device, which under lazy module loading (the CUDA 12 default)
+ *    happens at the library's first launch or symbol lookup on that device --
+ *    possibly inside the first smla_decode_noalloc call.  A caller that may
+ *    not see device memory change at all inside its critical region should
+ *    make one call (of any library entry point that launches work) on each
+ *    device beforehand.  Later calls change no device memory reservation.
+ *  - The looked-up address is kept per device for the life of the process;
+ *    do not use this entry point across a cudaDeviceReset() of that device.
  *  - All calls on a device share the one array and it keeps whatever the last
  *    call left in it; nothing in it has to start at zero, because every split
  *    the combine reads is written first by the same call.  Calls whose work

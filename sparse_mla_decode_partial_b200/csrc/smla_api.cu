@@ -447,7 +447,13 @@ smla_status smla_decode_noalloc(const void *q, const void *kv_cache, int64_t num
     if (st != SMLA_OK) return st;
     if (nsplit < 0 || nsplit > SMLA_MAX_NSPLIT) return SMLA_ERR_INVALID_ARG;
     if (B == 0 || T == 0 || H == 0) return SMLA_OK;
-    if (nsplit == 0) nsplit = smla_choose_nsplit(B, T, H, K, 0);
+    if (nsplit == 0) {
+        // the heuristic's split count, lowered until its partials fit the
+        // scratch array (S = 1 needs none)
+        nsplit = smla_choose_nsplit(B, T, H, K, 0);
+        while (nsplit > 1 && smla_workspace_bytes(B, T, H, nsplit) > SMLA_NOALLOC_SCRATCH_BYTES)
+            --nsplit;
+    }
     const size_t need = nsplit > 1 ? smla_workspace_bytes(B, T, H, nsplit) : 0;
     if (need > SMLA_NOALLOC_SCRATCH_BYTES) {
         std::snprintf(g_last_error, sizeof g_last_error,
@@ -510,9 +516,16 @@ smla_status smla_decode_host(const void *q_host, const void *kv_cache, int64_t n
                              const int32_t *topk_idx_host, int B, int T, int H, int K,
                              int page_size, float scale, int nsplit, void *workspace,
                              size_t workspace_bytes, void *o_host, float *lse_host, void *stream) {
-    if (B < 0 || T < 0 || H < 0 || K < 0 || pt_stride < 0) return SMLA_ERR_INVALID_ARG;
+    // Every check smla_decode makes on its arguments runs here first, on the
+    // host pointers, so that a failed check launches nothing (not even the
+    // copy kernel).
+    smla_status st0 = check_decode_args(q_host, kv_cache, num_pages, page_table_host, pt_stride,
+                                        topk_idx_host, B, T, H, K, page_size, scale);
+    if (st0 != SMLA_OK) return st0;
+    if (pt_stride < 0) return SMLA_ERR_INVALID_ARG;
     if (nsplit < 0 || nsplit > SMLA_MAX_NSPLIT) return SMLA_ERR_INVALID_ARG;
     if (B == 0 || T == 0 || H == 0) return SMLA_OK;
+    if (o_host == nullptr || lse_host == nullptr) return SMLA_ERR_INVALID_ARG;
     if (nsplit == 0) nsplit = smla_choose_nsplit(B, T, H, K, 0);
     // every host pointer must be pinned and visible to the device: checked
     // here, before anything is launched
@@ -542,7 +555,7 @@ smla_status smla_decode_host(const void *q_host, const void *kv_cache, int64_t n
         a.r[2] = {static_cast<const uint8_t *>(pt_d), ws + hs.pt, (size_t)B * pt_stride * 4};
     }
     const size_t words = (a.r[0].bytes + a.r[1].bytes + a.r[2].bytes) / 16 + 1;
-    const unsigned blocks = (unsigned)std::min<size_t>((words + 255) / 256, 148);
+    const unsigned blocks = (unsigned)std::min<size_t>((words + 255) / 256, (size_t)current_device_sms());
     smla::smla_ingest_kernel<<<blocks, 256, 0, st>>>(a);
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e);

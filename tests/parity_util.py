@@ -70,6 +70,19 @@ def check_o_lse(o_gpu, lse_gpu, o_ref, lse_ref, what=""):
     assert max_abs <= O_MAX_ABS, f"{what}: o max-abs {max_abs:.3e} > {O_MAX_ABS}"
     assert rel <= O_REL_L2, f"{what}: o rel-L2 {rel:.3e} > {O_REL_L2}"
     assert lse_err <= LSE_MAX_ABS, f"{what}: lse err {lse_err:.3e} > {LSE_MAX_ABS}"
+    # The same relative-L2 bound per output row (one (b, t, h)): |o| is about
+    # |c| / sqrt(valid rows) here, so the max-abs bound alone is loose, and
+    # one wrong row among thousands could pass the whole-tensor bound.  A row
+    # whose reference is exactly zero (nothing selected) must be zero.
+    if o.size:
+        o2, r2 = o.reshape(-1, o.shape[-1]), o_ref.reshape(-1, o_ref.shape[-1])
+        num = np.linalg.norm(o2 - r2, axis=1)
+        den = np.linalg.norm(r2, axis=1)
+        zero = den == 0
+        assert np.all(num[zero] == 0), f"{what}: non-zero o where nothing is selected"
+        row_rel = num[~zero] / den[~zero]
+        worst = float(row_rel.max()) if row_rel.size else 0.0
+        assert worst <= O_REL_L2, f"{what}: o rel-L2 of one row {worst:.3e} > {O_REL_L2}"
     return max_abs, rel, lse_err
 
 

@@ -122,12 +122,19 @@ def test_traffic_record_tracks_its_kernel_sources(tmp_path, monkeypatch):
     import shutil
     sys.path.insert(0, ROOT)
     import bench
-    for sub in ("profiles", os.path.join("sparse_mla_decode_partial_b200", "csrc")):
-        shutil.copytree(os.path.join(ROOT, sub), tmp_path / sub)
+    csrc = os.path.join("sparse_mla_decode_partial_b200", "csrc")
+    shutil.copytree(os.path.join(ROOT, csrc), tmp_path / csrc)
+    (tmp_path / "profiles").mkdir()
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
-    before = {wl: bench.measured_traffic(wl) for wl in ("single_request", "batched", "mixed")}
-    assert all(v is not None for v in before.values()), before
-    tc = tmp_path / "sparse_mla_decode_partial_b200" / "csrc" / "smla_partial_tc.cuh"
+    # a record taken on the sources as they are now
+    kernels = {"single_request": "smla_partial_small_kernel", "batched": "smla_partial_mma_kernel",
+               "mixed": "smla_partial_tc_kernel"}
+    rec = {wl: {"kernel": k, "sources_sha256_16": bench.kernel_sources_hash(k),
+                "traffic_bytes_per_launch": 1000 + i} for i, (wl, k) in enumerate(kernels.items())}
+    (tmp_path / "profiles" / "ncu_traffic.json").write_text(json.dumps(rec))
+    before = {wl: bench.measured_traffic(wl) for wl in kernels}
+    assert before == {"single_request": 1000, "batched": 1001, "mixed": 1002}
+    tc = tmp_path / csrc / "smla_partial_tc.cuh"
     tc.write_text(tc.read_text() + "\n// edited\n")
     assert bench.measured_traffic("mixed") is None
     assert bench.measured_traffic("single_request") == before["single_request"]
