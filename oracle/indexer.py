@@ -45,6 +45,8 @@ def load_library(path: str):
     lib.smla_ix_oracle_scores.restype = ctypes.c_long
     lib.smla_ix_oracle_topk.argtypes = [P, P, P, P, i32, i64, P, i32, i32, i32, i32, i32, i32, P]
     lib.smla_ix_oracle_topk.restype = ctypes.c_long
+    lib.smla_ix_oracle_select.argtypes = [P, P, i32, i32, i32, P]
+    lib.smla_ix_oracle_select.restype = None
     return lib
 
 
@@ -106,3 +108,18 @@ def topk(q_bits, w, k_bits, page_table, n_vis, K, *, page_size=PAGE_SIZE, lib=No
     bad = lib.smla_ix_oracle_topk(_p(q), _p(w), _p(k), _p(pt), pt_stride, num_pages, _p(n), B, T,
                                   HI, DI, page_size, int(K), _p(out))
     return out, int(bad)
+
+
+def select(scores, n_vis, K, *, lib=None):
+    """The selection rule applied to given scores [B, T, n_max] (any float
+    dtype, widened exactly to fp64; NaN marks a position that is not a
+    candidate): [B, T, K] int32, ascending positions then -1."""
+    lib = _load(lib)
+    sc = np.ascontiguousarray(scores, np.float64)
+    n = np.ascontiguousarray(n_vis, np.int32)
+    if sc.ndim != 3 or n.shape != sc.shape[:2]:
+        raise ValueError("scores must be [B, T, n_max] and n_vis [B, T]")
+    B, T, n_max = sc.shape
+    out = np.zeros((B, T, K), np.int32)
+    lib.smla_ix_oracle_select(_p(sc), _p(n), B * T, n_max, int(K), _p(out))
+    return out

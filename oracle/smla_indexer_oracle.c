@@ -29,6 +29,11 @@
  *    lies outside [0, num_pages), or beyond pt_stride * page_size, is not a
  *    candidate and is counted (the return value).
  *
+ * smla_ix_oracle_select applies the same selection to scores given from
+ * outside (positions with a NaN score are not candidates), so that a
+ * selection made from another implementation's scores can be checked with
+ * that implementation's own rounding.
+ *
  * Inputs: qI and kI are bf16 bit patterns (uint16), widened exactly to
  * double; w is fp32, widened exactly.  Parity pins:
  * tests/test_indexer_oracle.py.  No function here is unpinned.
@@ -98,6 +103,19 @@ static int ix_by_pos(const void *a, const void *b)
     return (x > y) - (x < y);
 }
 
+/* The selection from m candidates: the first min(K, m) in selection order,
+ * written as ascending positions, then -1 up to width K. */
+static void ix_finish(ix_cand *cand, int64_t m, int K, int32_t *o)
+{
+    qsort(cand, (size_t)m, sizeof(ix_cand), ix_by_score);
+    const int64_t take = m < K ? m : K;
+    for (int64_t i = 0; i < take; ++i)
+        o[i] = (int32_t)cand[i].pos;
+    qsort(o, (size_t)take, sizeof(int32_t), ix_by_pos);
+    for (int64_t i = take; i < K; ++i)
+        o[i] = -1;
+}
+
 /*
  * Scores of every visible position of every query token.
  *   qI  bf16 bits [B, T, HI, DI]     w  fp32 [B, T, HI]
@@ -161,17 +179,33 @@ long smla_ix_oracle_topk(const uint16_t *qI, const float *w, const uint16_t *kI,
             cand[m].pos = s;
             ++m;
         }
-        /* 2. the first min(K, m) in selection order */
-        qsort(cand, (size_t)m, sizeof(ix_cand), ix_by_score);
-        const int64_t take = m < K ? m : K;
-        int32_t *o = out + (int64_t)u * K;
-        for (int64_t i = 0; i < take; ++i)
-            o[i] = (int32_t)cand[i].pos;
-        /* 3. ascending positions, then padding */
-        qsort(o, (size_t)take, sizeof(int32_t), ix_by_pos);
-        for (int64_t i = take; i < K; ++i)
-            o[i] = -1;
+        ix_finish(cand, m, K, out + (int64_t)u * K);
         free(cand);
     }
     return n_bad;
+}
+
+/*
+ * Selection from given scores [B*T, n_max] (double; NaN = not a candidate)
+ * for positions s < n_vis[u]: out [B*T, K] as smla_ix_oracle_topk writes it.
+ */
+void smla_ix_oracle_select(const double *scores, const int32_t *n_vis, int BT, int n_max, int K,
+                           int32_t *out)
+{
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int u = 0; u < BT; ++u) {
+        const int64_t n = n_vis[u] < 0 ? 0 : (n_vis[u] > n_max ? n_max : n_vis[u]);
+        ix_cand *cand = (ix_cand *)malloc(sizeof(ix_cand) * (size_t)(n > 0 ? n : 1));
+        int64_t m = 0;
+        for (int64_t s = 0; s < n; ++s) {
+            const double v = scores[(int64_t)u * n_max + s];
+            if (isnan(v))
+                continue;
+            cand[m].score = v;
+            cand[m].pos = s;
+            ++m;
+        }
+        ix_finish(cand, m, K, out + (int64_t)u * K);
+        free(cand);
+    }
 }

@@ -209,6 +209,25 @@ def test_bad_pages_are_not_candidates_and_are_counted():
     assert bad == 2 and idx[0, 0].tolist() == [0, 1, 2, 3, 4, 5, -1, -1]
 
 
+def test_select_from_scores_matches_the_whole_oracle():
+    """The selection rule on given scores (NaN = not a candidate) picks what
+    the whole oracle picks from its own scores, on general inputs and on
+    integer ones full of ties; NaN positions are skipped."""
+    for seed, integer in ((21, False), (22, True), (23, True)):
+        rng = np.random.default_rng(seed)
+        q, w, k, pt, n, ps = random_case(rng, B=3, T=2, pages=9, integer=integer)
+        sc, _ = indexer.scores(q, w, k, pt, n, page_size=ps)
+        sc = np.where(np.isneginf(sc), np.nan, sc)
+        for K in (1, 4, 17, 50):
+            want, _ = indexer.topk(q, w, k, pt, n, K, page_size=ps)
+            assert np.array_equal(indexer.select(sc, n, K), want), (seed, K)
+    # NaN skipped; fp32 scores compared as stored
+    sc = np.asarray([[[1.5, np.nan, 1.5, 0.25, np.nan, 9.0]]], np.float32)
+    assert indexer.select(sc, np.asarray([[6]], np.int32), 3).tolist() == [[[0, 2, 5]]]
+    assert indexer.select(sc, np.asarray([[6]], np.int32), 6).tolist() == [[[0, 2, 3, 5, -1, -1]]]
+    assert indexer.select(sc, np.asarray([[2]], np.int32), 2).tolist() == [[[0, -1]]]
+
+
 # ---------------------------------------------------------------- planted mistakes
 MUTATIONS = {
     "no_relu": ("double relu = logit > 0.0 ? logit : 0.0;", "double relu = logit;"),
@@ -220,7 +239,8 @@ MUTATIONS = {
     "ignore_page_table": ("return (int64_t)page * page_size + s % page_size;", "return s;"),
     "slot_from_page_number": ("return (int64_t)page * page_size + s % page_size;",
                               "return (int64_t)page * page_size + s / page_size;"),
-    "one_position_too_few": ("for (int64_t s = 0; s < n; ++s) {", "for (int64_t s = 0; s + 1 < n; ++s) {"),
+    "one_position_too_few": ("for (int64_t s = 0; s < n; ++s) {\n            int64_t r = ix_row",
+                             "for (int64_t s = 0; s + 1 < n; ++s) {\n            int64_t r = ix_row"),
     "output_in_score_order": ("qsort(o, (size_t)take, sizeof(int32_t), ix_by_pos);", "(void)ix_by_pos;"),
     "query_head_stride": ("ix_bf16(q_t[(int64_t)j * DI + d])", "ix_bf16(q_t[d])"),
 }
