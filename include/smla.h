@@ -319,6 +319,70 @@ smla_status smla_decode_dense_partial(const void *q, const void *kv_cache, int64
  */
 smla_status smla_selftest_wait_timeout(unsigned long long limit_ns, void *stream);
 
+/*
+ * Top-k indexer: the step that produces topk_idx for the decode.
+ *
+ * "The Negative Result That Refined the Hunt: Disabling the MMA FlashMLA
+ * Kernel", section "The Context: A Systematic Bisection Campaign": the
+ * deployment runs an indexer kernel and a bf16 index-key path ahead of the
+ * sparse MLA decode kernel, which attends over the top-k candidate tokens
+ * ("The Moment of Truth ...", section "The Split-K Imperative").  The pages
+ * give no formula; this library follows the published DeepSeek
+ * sparse-attention indexer.  For query token (b, t) and each visible
+ * position s in [0, n_vis[b*T + t]) of sequence b:
+ *
+ *   logit_j(s) = q_index[b,t,j,:] . k_index[row(s), :]     128 bf16 values, fp32 sum
+ *   I(s)       = sum_j w[b,t,j] * max(0, logit_j(s))        j < HI, fp32
+ *
+ * with row(s) = page_table[b*pt_stride + s/64]*64 + s%64 (the latent cache's
+ * page table; the index-key cache is paged the same way).  The selection is
+ * the min(K, number of candidates) positions with the largest I; equal scores
+ * go to the smaller position.  topk_idx[b, t, :] lists the selected positions
+ * in ascending order, then -1 up to width K -- the index-list convention of
+ * smla_decode.
+ *
+ *   q_index    bf16 [B, T, HI, 128]       device, 16-B aligned
+ *   w          fp32 [B, T, HI]            device
+ *   k_index    bf16 [num_pages, 64, 128]  device, 16-B aligned
+ *   page_table int32 [B, pt_stride]       device
+ *   n_vis      int32 [B, T]               device: visible positions per query token
+ *   HI         index heads, 1..SMLA_INDEXER_MAX_HEADS
+ *   max_n      an upper bound on n_vis (sizes the score buffer and the work);
+ *              a length outside [0, max_n] is clamped and counted
+ *   K          selection width >= 1
+ *   B * T      at most SMLA_INDEXER_MAX_TOKENS
+ * A visible position whose page entry is outside [0, num_pages), or past
+ * pt_stride*64, is not a candidate; it is counted (SMLA_ERR_INDEX_RANGE in
+ * smla_check_device).  Scores that are NaN are not candidates either.
+ *
+ * smla_indexer_topk runs both steps; its workspace must hold
+ * smla_indexer_workspace_bytes(B, T, max_n) bytes (a per-token tile plan and
+ * the fp32 scores).  The two steps are also exported:
+ *   smla_indexer_scores writes I(s) into scores [B, T, max_n] (fp32, row
+ *     stride max_n) for every visible s; a position that is not a candidate
+ *     gets NaN; entries at s >= n_vis are not written.  Its workspace needs
+ *     only the tile plan: smla_indexer_workspace_bytes(B, T, 0) bytes.
+ *   smla_indexer_select applies the selection rule to given scores of that
+ *     layout (NaN = not a candidate; -0 and +0 are equal).
+ * Asynchronous on `stream`; errors as for the decode entry points.
+ */
+#define SMLA_INDEXER_DIM 128
+#define SMLA_INDEXER_MAX_HEADS 64
+#define SMLA_INDEXER_MAX_TOKENS 1048576
+size_t smla_indexer_workspace_bytes(int B, int T, int max_n);
+smla_status smla_indexer_topk(const void *q_index, const float *w, const void *k_index,
+                              int64_t num_pages, const int32_t *page_table, int pt_stride,
+                              const int32_t *n_vis, int B, int T, int HI, int max_n, int K,
+                              int page_size, void *workspace, size_t workspace_bytes,
+                              int32_t *topk_idx, void *stream);
+smla_status smla_indexer_scores(const void *q_index, const float *w, const void *k_index,
+                                int64_t num_pages, const int32_t *page_table, int pt_stride,
+                                const int32_t *n_vis, int B, int T, int HI, int max_n,
+                                int page_size, void *workspace, size_t workspace_bytes,
+                                float *scores, void *stream);
+smla_status smla_indexer_select(const float *scores, const int32_t *n_vis, int B, int T,
+                                int max_n, int K, int32_t *topk_idx, void *stream);
+
 /* Static text for a status code. */
 const char *smla_status_string(smla_status status);
 

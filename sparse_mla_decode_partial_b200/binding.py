@@ -46,6 +46,12 @@ SIGNATURES = {
                                _P, _P]),
     "smla_decode_dense_partial": (_I, [_P, _P, _I64, _P, _I, _P, _I, _I, _I, _I, _I, _F, _I, _P,
                                        _P, _P, _P]),
+    "smla_indexer_workspace_bytes": (_SZ, [_I, _I, _I]),
+    "smla_indexer_topk": (_I, [_P, _P, _P, _I64, _P, _I, _P, _I, _I, _I, _I, _I, _I, _P, _SZ, _P,
+                               _P]),
+    "smla_indexer_scores": (_I, [_P, _P, _P, _I64, _P, _I, _P, _I, _I, _I, _I, _I, _P, _SZ, _P,
+                                 _P]),
+    "smla_indexer_select": (_I, [_P, _P, _I, _I, _I, _I, _P, _P]),
     "smla_selftest_wait_timeout": (_I, [ctypes.c_ulonglong, _P]),
     "smla_check_device": (_I, [_I, ctypes.POINTER(ctypes.c_ulonglong), _P]),
     "smla_status_string": (ctypes.c_char_p, [_I]),
@@ -334,6 +340,87 @@ def decode_host(q, cache, page_table, idx, scale: float, nsplit: int = 0, *, o, 
                                   _ptr(workspace), workspace.numel(), _ptr(o), _ptr(lse),
                                   _stream(stream)), "smla_decode_host")
     return o, lse
+
+
+INDEXER_DIM, INDEXER_MAX_HEADS = 128, 64
+
+
+def indexer_workspace_bytes(B: int, T: int, max_n: int) -> int:
+    return int(lib().smla_indexer_workspace_bytes(B, T, max_n))
+
+
+def _indexer_args(q_index, w, k_index, page_table, n_vis):
+    _need(q_index, torch.bfloat16, "q_index")
+    dev = q_index.device
+    _need(w, torch.float32, "w", dev)
+    _need(k_index, torch.bfloat16, "k_index", dev)
+    _need(page_table, torch.int32, "page_table", dev)
+    _need(n_vis, torch.int32, "n_vis", dev)
+    if q_index.dim() != 4 or q_index.shape[-1] != INDEXER_DIM:
+        raise ValueError(f"q_index must be [B,T,HI,{INDEXER_DIM}]")
+    B, T, HI, _ = q_index.shape
+    if tuple(w.shape) != (B, T, HI) or tuple(n_vis.shape) != (B, T):
+        raise ValueError("w must be [B,T,HI] and n_vis [B,T]")
+    if page_table.dim() != 2 or page_table.shape[0] != B:
+        raise ValueError("page_table must be [B, pt_stride]")
+    if k_index.numel() % (PAGE_SIZE * INDEXER_DIM):
+        raise ValueError("k_index must be [num_pages, 64, 128]")
+    return B, T, HI, page_table.shape[1], k_index.numel() // (PAGE_SIZE * INDEXER_DIM)
+
+
+def indexer_topk(q_index, w, k_index, page_table, n_vis, K: int, max_n: int, *, out=None,
+                 workspace=None, stream=None):
+    """Top-k indexer: the min(K, n) positions with the largest index score
+    per query token, ascending then -1 (int32 [B, T, K]).  max_n bounds
+    n_vis (it sizes the work and the score buffer)."""
+    B, T, HI, pt_stride, num_pages = _indexer_args(q_index, w, k_index, page_table, n_vis)
+    dev = q_index.device
+    if out is None:
+        out = torch.empty((B, T, K), dtype=torch.int32, device=dev)
+    _need(out, torch.int32, "out", dev)
+    if workspace is None:
+        workspace = torch.empty(max(16, indexer_workspace_bytes(B, T, max_n)), dtype=torch.uint8,
+                                device=dev)
+    _need(workspace, torch.uint8, "workspace", dev)
+    _check(lib().smla_indexer_topk(_ptr(q_index), _ptr(w), _ptr(k_index), num_pages,
+                                   _ptr(page_table), pt_stride, _ptr(n_vis), B, T, HI, int(max_n),
+                                   int(K), PAGE_SIZE, _ptr(workspace), workspace.numel(),
+                                   _ptr(out), _stream(stream)), "smla_indexer_topk")
+    return out
+
+
+def indexer_scores(q_index, w, k_index, page_table, n_vis, max_n: int, *, scores=None,
+                   workspace=None, stream=None):
+    """Index scores fp32 [B, T, max_n] for every visible position (NaN where
+    a position is not a candidate; entries past n_vis are not written)."""
+    B, T, HI, pt_stride, num_pages = _indexer_args(q_index, w, k_index, page_table, n_vis)
+    dev = q_index.device
+    if scores is None:
+        scores = torch.full((B, T, max(max_n, 1)), float("nan"), dtype=torch.float32, device=dev)
+    _need(scores, torch.float32, "scores", dev)
+    if workspace is None:
+        workspace = torch.empty(max(16, indexer_workspace_bytes(B, T, 0)), dtype=torch.uint8,
+                                device=dev)
+    _need(workspace, torch.uint8, "workspace", dev)
+    _check(lib().smla_indexer_scores(_ptr(q_index), _ptr(w), _ptr(k_index), num_pages,
+                                     _ptr(page_table), pt_stride, _ptr(n_vis), B, T, HI,
+                                     int(max_n), PAGE_SIZE, _ptr(workspace), workspace.numel(),
+                                     _ptr(scores), _stream(stream)), "smla_indexer_scores")
+    return scores
+
+
+def indexer_select(scores, n_vis, K: int, *, out=None, stream=None):
+    """The indexer's selection rule on given scores fp32 [B, T, max_n]."""
+    _need(scores, torch.float32, "scores")
+    dev = scores.device
+    _need(n_vis, torch.int32, "n_vis", dev)
+    B, T, max_n = scores.shape
+    if out is None:
+        out = torch.empty((B, T, K), dtype=torch.int32, device=dev)
+    _need(out, torch.int32, "out", dev)
+    _check(lib().smla_indexer_select(_ptr(scores), _ptr(n_vis), B, T, max_n, int(K), _ptr(out),
+                                     _stream(stream)), "smla_indexer_select")
+    return out
 
 
 def check_device(clear: bool = True, stream=None):

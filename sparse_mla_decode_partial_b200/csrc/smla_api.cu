@@ -2,6 +2,7 @@
 // checks, the NSPLIT heuristic, workspace carving and kernel launches.
 // Every entry point returns a status; nothing throws across the ABI.
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 
 #include <algorithm>
 #include <climits>
@@ -24,6 +25,7 @@
 #include "smla_combine.cuh"
 #include "smla_partial_mma.cuh"
 #include "smla_partial_tc.cuh"
+#include "smla_indexer.cuh"
 
 namespace {
 
@@ -707,6 +709,207 @@ smla_status smla_check_device(int clear, unsigned long long *n_bad_index, void *
     if (flags & smla::kFlagTimeout) return SMLA_ERR_TIMEOUT;
     if (flags & smla::kFlagIndexRange) return SMLA_ERR_INDEX_RANGE;
     return SMLA_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Top-k indexer (see include/smla.h and smla_indexer.cuh).
+}  // extern "C"
+
+namespace {
+
+// cuTensorMapEncodeTiled, reached through the runtime (no link against the
+// driver library).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+        (void)cudaGetLastError();
+    });
+    return fn;
+}
+
+// 2-D bf16 tensor of `rows` rows of 128 values (256-byte rows), read in boxes
+// of 64 values x box_rows rows with the 128-byte swizzle.
+smla_status encode_rows128(CUtensorMap *map, const void *base, uint64_t rows, uint32_t box_rows) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (enc == nullptr) {
+        std::snprintf(g_last_error, sizeof g_last_error, "cuTensorMapEncodeTiled unavailable");
+        return SMLA_ERR_CUDA;
+    }
+    const cuuint64_t dims[2] = {(cuuint64_t)smla::kIxDim, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)smla::kIxDim * 2};
+    const cuuint32_t box[2] = {64u, box_rows};
+    const cuuint32_t estr[2] = {1u, 1u};
+    const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims,
+                           strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        std::snprintf(g_last_error, sizeof g_last_error, "cuTensorMapEncodeTiled failed: %d", (int)r);
+        return SMLA_ERR_CUDA;
+    }
+    return SMLA_OK;
+}
+
+smla_status check_indexer_args(const void *q_index, const float *w, const void *k_index,
+                               int64_t num_pages, const int32_t *page_table, int pt_stride,
+                               const int32_t *n_vis, int B, int T, int HI, int max_n,
+                               int page_size) {
+    if (B < 0 || T < 0 || HI < 1 || max_n < 0) return SMLA_ERR_INVALID_ARG;
+    if (page_size != SMLA_PAGE_SIZE) return SMLA_ERR_UNSUPPORTED;
+    if (HI > SMLA_INDEXER_MAX_HEADS) return SMLA_ERR_UNSUPPORTED;
+    if (B == 0 || T == 0) return SMLA_OK;
+    if ((long long)B * T > SMLA_INDEXER_MAX_TOKENS) return SMLA_ERR_UNSUPPORTED;
+    if ((long long)B * T * HI > INT_MAX) return SMLA_ERR_INVALID_ARG;
+    if (!q_index || !w || !n_vis) return SMLA_ERR_INVALID_ARG;
+    if (!aligned(q_index, 16) || !aligned(w, 4) || !aligned(n_vis, 4)) return SMLA_ERR_MISALIGNED;
+    if (max_n > 0) {
+        if (!k_index || !page_table || num_pages < 1 || pt_stride < 1) return SMLA_ERR_INVALID_ARG;
+        if (num_pages > SMLA_MAX_PAGES) return SMLA_ERR_UNSUPPORTED;
+        if (!aligned(k_index, 16) || !aligned(page_table, 4)) return SMLA_ERR_MISALIGNED;
+    }
+    return SMLA_OK;
+}
+
+size_t ix_plan_bytes(int B, int T) { return round256(((size_t)B * T + 1) * sizeof(int)); }
+
+// Plan + scores into `scores` (row stride `stride` floats).
+smla_status launch_ix_scores(const void *q_index, const float *w, const void *k_index,
+                             int64_t num_pages, const int32_t *page_table, int pt_stride,
+                             const int32_t *n_vis, int B, int T, int HI, int max_n, int *plan,
+                             float *scores, long long stride, cudaStream_t st) {
+    smla::IndexerParams p{};
+    p.page_table = page_table;
+    p.pt_stride = pt_stride;
+    p.num_pages = num_pages;
+    p.n_vis = n_vis;
+    p.w = w;
+    p.BT = B * T;
+    p.T = T;
+    p.HI = HI;
+    p.max_n = max_n;
+    p.tile_start = plan;
+    p.scores = scores;
+    p.score_stride = stride;
+    smla::smla_ix_plan_kernel<<<1, 1024, 0, st>>>(p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (max_n == 0) return SMLA_OK;
+    const int npad = HI <= 16 ? 16 : (HI <= 32 ? 32 : 64);
+    CUtensorMap map_k, map_q;
+    smla_status s = encode_rows128(&map_k, k_index, (uint64_t)num_pages * SMLA_PAGE_SIZE, 64u);
+    if (s != SMLA_OK) return s;
+    s = encode_rows128(&map_q, q_index, (uint64_t)B * T * HI, (uint32_t)npad);
+    if (s != SMLA_OK) return s;
+    const int grid = current_device_sms();
+    const void *fn;
+    int smem;
+    if (npad == 16) {
+        fn = reinterpret_cast<const void *>(&smla::smla_ix_score_kernel<16>);
+        smem = smla::IxCfg<16>::kSmemBytes;
+    } else if (npad == 32) {
+        fn = reinterpret_cast<const void *>(&smla::smla_ix_score_kernel<32>);
+        smem = smla::IxCfg<32>::kSmemBytes;
+    } else {
+        fn = reinterpret_cast<const void *>(&smla::smla_ix_score_kernel<64>);
+        smem = smla::IxCfg<64>::kSmemBytes;
+    }
+    e = ensure_smem_attr(fn, smem);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (npad == 16)
+        smla::smla_ix_score_kernel<16><<<grid, smla::IxCfg<16>::kThreads, smem, st>>>(map_k, map_q, p);
+    else if (npad == 32)
+        smla::smla_ix_score_kernel<32><<<grid, smla::IxCfg<32>::kThreads, smem, st>>>(map_k, map_q, p);
+    else
+        smla::smla_ix_score_kernel<64><<<grid, smla::IxCfg<64>::kThreads, smem, st>>>(map_k, map_q, p);
+    e = cudaGetLastError();
+    return e == cudaSuccess ? SMLA_OK : cuda_fail(e);
+}
+
+smla_status launch_ix_select(const float *scores, long long stride, const int32_t *n_vis, int B,
+                             int T, int max_n, int K, int32_t *out, cudaStream_t st) {
+    smla::IndexerParams p{};
+    p.n_vis = n_vis;
+    p.BT = B * T;
+    p.T = T;
+    p.max_n = max_n;
+    p.K = K;
+    p.scores = const_cast<float *>(scores);
+    p.score_stride = stride;
+    p.out = out;
+    smla::smla_ix_select_kernel<<<B * T, smla::kIxSelectThreads, 0, st>>>(p);
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? SMLA_OK : cuda_fail(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t smla_indexer_workspace_bytes(int B, int T, int max_n) {
+    if (B < 0 || T < 0 || max_n < 0) return 0;
+    return ix_plan_bytes(B, T) + round256((size_t)B * T * max_n * sizeof(float));
+}
+
+smla_status smla_indexer_scores(const void *q_index, const float *w, const void *k_index,
+                                int64_t num_pages, const int32_t *page_table, int pt_stride,
+                                const int32_t *n_vis, int B, int T, int HI, int max_n,
+                                int page_size, void *workspace, size_t workspace_bytes,
+                                float *scores, void *stream) {
+    smla_status st = check_indexer_args(q_index, w, k_index, num_pages, page_table, pt_stride,
+                                        n_vis, B, T, HI, max_n, page_size);
+    if (st != SMLA_OK) return st;
+    if (B == 0 || T == 0 || max_n == 0) return SMLA_OK;
+    if (scores == nullptr) return SMLA_ERR_INVALID_ARG;
+    if (!aligned(scores, 4)) return SMLA_ERR_MISALIGNED;
+    if (workspace_bytes < ix_plan_bytes(B, T)) return SMLA_ERR_WORKSPACE_TOO_SMALL;
+    if (workspace == nullptr) return SMLA_ERR_INVALID_ARG;
+    if (!aligned(workspace, 16)) return SMLA_ERR_MISALIGNED;
+    return launch_ix_scores(q_index, w, k_index, num_pages, page_table, pt_stride, n_vis, B, T, HI,
+                            max_n, static_cast<int *>(workspace), scores, max_n,
+                            static_cast<cudaStream_t>(stream));
+}
+
+smla_status smla_indexer_select(const float *scores, const int32_t *n_vis, int B, int T, int max_n,
+                                int K, int32_t *topk_idx, void *stream) {
+    if (B < 0 || T < 0 || max_n < 0 || K < 1) return SMLA_ERR_INVALID_ARG;
+    if (B == 0 || T == 0) return SMLA_OK;
+    if ((long long)B * T > SMLA_INDEXER_MAX_TOKENS) return SMLA_ERR_UNSUPPORTED;
+    if (!n_vis || !topk_idx || (max_n > 0 && !scores)) return SMLA_ERR_INVALID_ARG;
+    if (!aligned(n_vis, 4) || !aligned(topk_idx, 4) || !aligned(scores, 4)) return SMLA_ERR_MISALIGNED;
+    return launch_ix_select(scores, max_n, n_vis, B, T, max_n, K, topk_idx,
+                            static_cast<cudaStream_t>(stream));
+}
+
+smla_status smla_indexer_topk(const void *q_index, const float *w, const void *k_index,
+                              int64_t num_pages, const int32_t *page_table, int pt_stride,
+                              const int32_t *n_vis, int B, int T, int HI, int max_n, int K,
+                              int page_size, void *workspace, size_t workspace_bytes,
+                              int32_t *topk_idx, void *stream) {
+    smla_status st = check_indexer_args(q_index, w, k_index, num_pages, page_table, pt_stride,
+                                        n_vis, B, T, HI, max_n, page_size);
+    if (st != SMLA_OK) return st;
+    if (K < 1) return SMLA_ERR_INVALID_ARG;
+    if (B == 0 || T == 0) return SMLA_OK;
+    if (topk_idx == nullptr) return SMLA_ERR_INVALID_ARG;
+    if (!aligned(topk_idx, 4)) return SMLA_ERR_MISALIGNED;
+    if (workspace_bytes < smla_indexer_workspace_bytes(B, T, max_n)) return SMLA_ERR_WORKSPACE_TOO_SMALL;
+    if (workspace == nullptr) return SMLA_ERR_INVALID_ARG;
+    if (!aligned(workspace, 16)) return SMLA_ERR_MISALIGNED;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    int *plan = reinterpret_cast<int *>(ws);
+    float *scores = reinterpret_cast<float *>(ws + ix_plan_bytes(B, T));
+    st = launch_ix_scores(q_index, w, k_index, num_pages, page_table, pt_stride, n_vis, B, T, HI,
+                          max_n, plan, scores, max_n, s);
+    if (st != SMLA_OK) return st;
+    return launch_ix_select(scores, max_n, n_vis, B, T, max_n, K, topk_idx, s);
 }
 
 }  // extern "C"

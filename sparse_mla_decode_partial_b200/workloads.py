@@ -212,6 +212,98 @@ def dense_verify(seed: int = 5) -> Workload:
                                nsplit_sweep=(16, 64))
 
 
+# ---------------------------------------------------------------- top-k indexer inputs
+INDEX_DIM = 128
+
+
+@dataclasses.dataclass
+class IndexerWorkload:
+    """Inputs of the top-k indexer: per-token index queries and head weights,
+    a paged index-key cache (the latent cache's page numbering), and the
+    visible length of every query token."""
+    name: str
+    q_index: torch.Tensor      # bf16 [B, T, HI, 128]
+    w: torch.Tensor            # fp32 [B, T, HI]
+    k_index: torch.Tensor      # bf16 [P, PAGE_SIZE, 128]
+    page_table: torch.Tensor   # int32 [B, pt_stride]
+    n_vis: torch.Tensor        # int32 [B, T]
+    K: int
+    ctx_lens: list
+
+    @property
+    def B(self):
+        return self.q_index.shape[0]
+
+    @property
+    def T(self):
+        return self.q_index.shape[1]
+
+    @property
+    def HI(self):
+        return self.q_index.shape[2]
+
+    @property
+    def num_pages(self):
+        return self.k_index.shape[0]
+
+    @property
+    def pt_stride(self):
+        return self.page_table.shape[1]
+
+    @property
+    def max_n(self):
+        return int(self.n_vis.max()) if self.n_vis.numel() else 0
+
+    def to(self, device) -> "IndexerWorkload":
+        return dataclasses.replace(self, q_index=self.q_index.to(device), w=self.w.to(device),
+                                   k_index=self.k_index.to(device),
+                                   page_table=self.page_table.to(device),
+                                   n_vis=self.n_vis.to(device))
+
+
+def make_indexer_workload(name: str, *, B: int, T: int, HI: int, K: int, ctx_lens: Sequence[int],
+                          seed: int, causal: bool = False, integer: bool = False,
+                          shuffle_pages: bool = True) -> IndexerWorkload:
+    """Draw indexer inputs.  Values are N(0,1)*0.5 rounded to bf16 (query and
+    keys) and N(0,1)*0.5 fp32 weights; with ``integer`` they are small
+    integers instead (queries and keys in [-2, 2], weights in [-2, 2]), so
+    that every score is an exact integer in fp32 whatever the summation
+    order.  n_vis[b, t] = ctx_lens[b], or with ``causal`` ctx_lens[b] - T + t
+    + 1 (draft token t sees the context and the drafts up to itself)."""
+    gen = torch.Generator().manual_seed(seed)
+    ctx_lens = [int(c) for c in ctx_lens]
+    assert len(ctx_lens) == B
+    pages_per_seq = [max(1, (c + PAGE_SIZE - 1) // PAGE_SIZE) for c in ctx_lens]
+    total_pages = sum(pages_per_seq)
+    pt_stride = max(pages_per_seq)
+    if integer:
+        q = torch.randint(-2, 3, (B, T, HI, INDEX_DIM), generator=gen).to(torch.bfloat16)
+        k = torch.randint(-2, 3, (total_pages, PAGE_SIZE, INDEX_DIM), generator=gen).to(torch.bfloat16)
+        w = torch.randint(-2, 3, (B, T, HI), generator=gen).to(torch.float32)
+    else:
+        q = _normal_bf16((B, T, HI, INDEX_DIM), gen)
+        k = _normal_bf16((total_pages, PAGE_SIZE, INDEX_DIM), gen)
+        w = torch.randn((B, T, HI), generator=gen) * 0.5
+    perm = (torch.randperm(total_pages, generator=gen) if shuffle_pages
+            else torch.arange(total_pages)).to(torch.int32)
+    page_table = torch.full((B, pt_stride), -1, dtype=torch.int32)
+    off = 0
+    for b, n in enumerate(pages_per_seq):
+        page_table[b, :n] = perm[off:off + n]
+        off += n
+    n_vis = torch.tensor([[(c - T + t + 1) if causal else c for t in range(T)] for c in ctx_lens],
+                         dtype=torch.int32)
+    return IndexerWorkload(name=name, q_index=q, w=w.to(torch.float32), k_index=k,
+                           page_table=page_table, n_vis=n_vis, K=K, ctx_lens=ctx_lens)
+
+
+def indexer_mixed(seed: int = 6, B: int = 60) -> IndexerWorkload:
+    """The indexer ahead of the mixed-length decode: B60 T1, contexts
+    log-uniform in [1024, 131072], 64 index heads of 128 values, top-2048."""
+    return make_indexer_workload("indexer_mixed", B=B, T=1, HI=64, K=2048,
+                                 ctx_lens=mixed_ctx_lens(B, seed), seed=seed)
+
+
 WORKLOADS = {
     "tiny": tiny,
     "single_request": single_request,
