@@ -16,7 +16,7 @@ On one GPU the line also carries a `workloads` record: the memory-bound
 batched and mixed-length configurations and the two verify shapes, each
 measured after the headline in the same process under the same protocol
 (decode and partial pass at the heuristic NSPLIT, medians, its own roofline
-and clock record).
+and clock record), plus the top-k indexer ahead of the mixed-length decode.
 
 The metric (query tokens per second, us per call and achieved HBM GB/s,
 against NSPLIT) follows "The Occupancy Hypothesis ..." (section "The
@@ -482,6 +482,80 @@ def side_workload(h, name, steps, warmup, peaks):
     return rec
 
 
+def indexer_bytes(w):
+    """Algorithmic bytes of one indexer call: every visible index key once
+    (256 B), its page-table entry once per 64 positions, the index queries
+    (HI x 256 B) and weights (HI x 4 B) of every query token, its visible
+    length, and the K output entries (4 B)."""
+    n = w.n_vis.to(__import__("torch").int64).clamp(min=0)
+    keys = int(n.sum())
+    pages = int(((n + 63) // 64).sum())
+    BT = w.B * w.T
+    return keys * 256 + pages * 4 + BT * w.HI * (256 + 4) + BT * 4 + BT * w.K * 4
+
+
+def side_indexer(h, steps, warmup, peaks):
+    """The top-k indexer ahead of the mixed-length decode (B60 T1, contexts
+    1K..128K, 64 index heads, top-2048), timed through smla_indexer_topk,
+    with its scoring and selection steps also timed alone."""
+    import torch
+    from sparse_mla_decode_partial_b200 import binding, workloads
+    w_host = workloads.indexer_mixed()
+    w = w_host.to(h.dev)
+    B, T, HI, K, max_n = w.B, w.T, w.HI, w.K, w_host.max_n
+    lib, sptr = h.lib, h.sptr
+    ws = torch.empty(binding.indexer_workspace_bytes(B, T, max_n), dtype=torch.uint8, device=h.dev)
+    out = torch.empty((B, T, K), dtype=torch.int32, device=h.dev)
+    sc = torch.empty((B, T, max_n), dtype=torch.float32, device=h.dev)
+    common = (w.q_index.data_ptr(), w.w.data_ptr(), w.k_index.data_ptr(), w.num_pages,
+              w.page_table.data_ptr(), w.pt_stride, w.n_vis.data_ptr(), B, T, HI, max_n)
+
+    def topk():
+        return lib.smla_indexer_topk(*common, K, 64, ws.data_ptr(), ws.numel(), out.data_ptr(),
+                                     sptr), 3
+
+    def scores():
+        return lib.smla_indexer_scores(*common, 64, ws.data_ptr(), ws.numel(), sc.data_ptr(),
+                                       sptr), 2
+
+    def select():
+        return lib.smla_indexer_select(sc.data_ptr(), w.n_vis.data_ptr(), B, T, max_n, K,
+                                       out.data_ptr(), sptr), 1
+    h.warm([topk, scores, select], warmup)
+    sampler = ClockSampler(h.dev.index)
+    with sampler:
+        t_all, launches = h.timed(topk, steps)
+        t_sc, _ = h.timed(scores, steps)
+        t_sel, _ = h.timed(select, steps)
+    us, us_sc, us_sel = (statistics.median(t) * 1e3 for t in (t_all, t_sc, t_sel))
+    nbytes = indexer_bytes(w_host)
+    hbm_peak, tc_peak, peak_src = peaks
+    key_bytes = nbytes - B * T * K * 4
+    flops = 2 * int(w_host.n_vis.clamp(min=0).sum()) * HI * 128
+    rec = {"shape": f"B{B} T{T} HI{HI} x128 bf16 index keys, top-{K}, ctx "
+                    f"{min(w_host.ctx_lens)}..{max(w_host.ctx_lens)}",
+           "steps": steps, "us_per_call": round(us, 3),
+           "us_per_call_mean": round(statistics.fmean(t_all) * 1e3, 3),
+           "q_tok_s": round(B * T / (us * 1e-6), 1),
+           "scores_us": round(us_sc, 3), "select_us": round(us_sel, 3),
+           "roofline": {"bound": "hbm", "kernel": "smla_ix_score_kernel",
+                        "achieved": round(key_bytes / (us_sc * 1e-6) / 1e9, 1),
+                        "peak": hbm_peak, "unit": "GB/s",
+                        "frac": round(key_bytes / (us_sc * 1e-6) / 1e9 / hbm_peak, 4),
+                        "peak_source": peak_src,
+                        "traffic": measured_traffic("indexer_mixed"),
+                        "algorithmic_bytes_per_launch": key_bytes,
+                        "tensor_tflops": round(flops / (us_sc * 1e-6) / 1e12, 2),
+                        "tensor_frac_of_bf16_peak": round(flops / (us_sc * 1e-6) / 1e12 / tc_peak, 4),
+                        "note": "scoring kernel (plan + scores) timed alone; bytes: keys, page "
+                                "entries, queries, weights and lengths, read once"},
+           "whole_call_frac_of_hbm": round(nbytes / (us * 1e-6) / 1e9 / hbm_peak, 4),
+           "gpu_launches": launches, "clocks": sampler.summary()}
+    del w, ws, sc
+    torch.cuda.empty_cache()
+    return rec
+
+
 def run_ours(args, world, rank, local):
     import torch
     from sparse_mla_decode_partial_b200 import binding, build
@@ -637,6 +711,7 @@ def run_ours(args, world, rank, local):
         for name in SIDE_WORKLOADS:
             if name != args.workload:
                 side[name] = side_workload(h, name, min(args.steps, 200), args.warmup, peaks)
+        side["indexer_mixed"] = side_indexer(h, min(args.steps, 100), args.warmup, peaks)
 
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
