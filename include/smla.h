@@ -97,7 +97,8 @@ typedef enum {
  * and the split-K scratch traffic, with two resident CTAs per SM for H <= 16
  * and one otherwise.  It also prices smla_decode's balanced schedule (one
  * full wave of equal CTAs, ceil(SMs x resident / (B*T)) + 1 slots) and
- * returns that slot count only when the model favours it by more than 15%.
+ * returns that slot count when the model favours it (by more than 15% for
+ * H <= 32, whose kernels stall at a token boundary; at all for H > 32).
  * sm_count <= 0 queries the current device.  If the environment variable SMLA_NSPLIT holds a positive integer,
  * that value is returned instead (clamped to [1, SMLA_MAX_NSPLIT]).
  * Returns >= 1; returns 1 for degenerate sizes.
@@ -347,8 +348,9 @@ smla_status smla_selftest_wait_timeout(unsigned long long limit_ns, void *stream
  *   page_table int32 [B, pt_stride]       device
  *   n_vis      int32 [B, T]               device: visible positions per query token
  *   HI         index heads, 1..SMLA_INDEXER_MAX_HEADS
- *   max_n      an upper bound on n_vis (sizes the score buffer and the work);
- *              a length outside [0, max_n] is clamped and counted
+ *   max_n      an upper bound on n_vis (sizes the score buffer and the work),
+ *              at most SMLA_INDEXER_MAX_N; a length outside [0, max_n] is
+ *              clamped and counted
  *   K          selection width >= 1
  *   B * T      at most SMLA_INDEXER_MAX_TOKENS
  * A visible position whose page entry is outside [0, num_pages), or past
@@ -369,6 +371,7 @@ smla_status smla_selftest_wait_timeout(unsigned long long limit_ns, void *stream
 #define SMLA_INDEXER_DIM 128
 #define SMLA_INDEXER_MAX_HEADS 64
 #define SMLA_INDEXER_MAX_TOKENS 1048576
+#define SMLA_INDEXER_MAX_N 524288   /* visible positions per query token */
 size_t smla_indexer_workspace_bytes(int B, int T, int max_n);
 smla_status smla_indexer_topk(const void *q_index, const float *w, const void *k_index,
                               int64_t num_pages, const int32_t *page_table, int pt_stride,

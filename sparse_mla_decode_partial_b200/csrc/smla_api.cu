@@ -114,12 +114,15 @@ int nsplit_model(int B, int T, int H, int K, int sm_count) {
     // of the pass), so the balanced choice must win by kBalancedMargin.
     const long long s_bal = (long long)std::ceil((double)slots / (double)base) + 1;
     const double units = (double)base * ((K + 31) / 32);
-    if (H <= 32 && s_bal >= 2 && s_bal <= s_max && units >= 4.0 * slots &&
+    if (s_bal >= 2 && s_bal <= s_max && units >= 4.0 * slots &&
         !uses_latency_kernel(H, K, (K + (int)s_bal - 1) / (int)s_bal, 0)) {
         const double pieces = (double)base + slots;
         double t = kFixedRows * pieces / slots + units * 32.0 / slots;
         t += kScratchWeight * pieces * H * kPartialBytesPerHead * 2.0 / smla::kRowBytes / slots;
-        if (t < best * (1.0 - kBalancedMargin)) best_s = (int)s_bal;
+        // the tcgen05 kernel overlaps an item boundary with the next item's
+        // work (Q staged early, O drained through a spent ring slot)
+        const double margin = H > 32 ? 0.0 : kBalancedMargin;
+        if (t < best * (1.0 - margin)) best_s = (int)s_bal;
     }
     return best_s;
 }
@@ -230,9 +233,9 @@ int resident_per_sm(int H) {
 // flattened (token, 32-row tile) space; a token then spans at most
 // ceil(R / (B*T)) + 1 CTAs, each writing one of its S slots.  Used when it
 // fits in S slots and each CTA gets at least 4 tiles.  The tcgen05 kernel
-// (H > 32) keeps equal splits.
+// (H > 32) walks its items the same way, one CTA per SM.
 bool use_balanced(int B, int T, int H, int K, int nsplit, int pt_stride, int sms, int *grid) {
-    if (nsplit < 2 || K <= 0 || H > 32) return false;
+    if (nsplit < 2 || K <= 0) return false;
     const int kc = (K + nsplit - 1) / nsplit;
     if (uses_latency_kernel(H, K, kc, pt_stride)) return false;
     const long long bt = (long long)B * T;
@@ -715,6 +718,8 @@ smla_status smla_check_device(int clear, unsigned long long *n_bad_index, void *
 // Top-k indexer (see include/smla.h and smla_indexer.cuh).
 }  // extern "C"
 
+static_assert(SMLA_INDEXER_MAX_N <= smla::kIxSelectMaxN, "selection bitmaps must fit shared memory");
+
 namespace {
 
 // cuTensorMapEncodeTiled, reached through the runtime (no link against the
@@ -763,7 +768,7 @@ smla_status check_indexer_args(const void *q_index, const float *w, const void *
                                int page_size) {
     if (B < 0 || T < 0 || HI < 1 || max_n < 0) return SMLA_ERR_INVALID_ARG;
     if (page_size != SMLA_PAGE_SIZE) return SMLA_ERR_UNSUPPORTED;
-    if (HI > SMLA_INDEXER_MAX_HEADS) return SMLA_ERR_UNSUPPORTED;
+    if (HI > SMLA_INDEXER_MAX_HEADS || max_n > SMLA_INDEXER_MAX_N) return SMLA_ERR_UNSUPPORTED;
     if (B == 0 || T == 0) return SMLA_OK;
     if ((long long)B * T > SMLA_INDEXER_MAX_TOKENS) return SMLA_ERR_UNSUPPORTED;
     if ((long long)B * T * HI > INT_MAX) return SMLA_ERR_INVALID_ARG;
@@ -843,8 +848,11 @@ smla_status launch_ix_select(const float *scores, long long stride, const int32_
     p.scores = const_cast<float *>(scores);
     p.score_stride = stride;
     p.out = out;
-    smla::smla_ix_select_kernel<<<B * T, smla::kIxSelectThreads, 0, st>>>(p);
-    const cudaError_t e = cudaGetLastError();
+    const void *fn = reinterpret_cast<const void *>(&smla::smla_ix_select_kernel);
+    cudaError_t e = ensure_smem_attr(fn, smla::ix_select_smem_bytes(smla::kIxSelectMaxN));
+    if (e != cudaSuccess) return cuda_fail(e);
+    smla::smla_ix_select_kernel<<<B * T, smla::kIxSelectThreads, smla::ix_select_smem_bytes(max_n), st>>>(p);
+    e = cudaGetLastError();
     return e == cudaSuccess ? SMLA_OK : cuda_fail(e);
 }
 
@@ -879,6 +887,7 @@ smla_status smla_indexer_scores(const void *q_index, const float *w, const void 
 smla_status smla_indexer_select(const float *scores, const int32_t *n_vis, int B, int T, int max_n,
                                 int K, int32_t *topk_idx, void *stream) {
     if (B < 0 || T < 0 || max_n < 0 || K < 1) return SMLA_ERR_INVALID_ARG;
+    if (max_n > SMLA_INDEXER_MAX_N) return SMLA_ERR_UNSUPPORTED;
     if (B == 0 || T == 0) return SMLA_OK;
     if ((long long)B * T > SMLA_INDEXER_MAX_TOKENS) return SMLA_ERR_UNSUPPORTED;
     if (!n_vis || !topk_idx || (max_n > 0 && !scores)) return SMLA_ERR_INVALID_ARG;

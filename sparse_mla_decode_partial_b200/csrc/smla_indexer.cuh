@@ -124,6 +124,46 @@ __device__ __forceinline__ int ix_token_of(const IndexerParams &p, long long uni
     return lo;
 }
 
+// What a role needs to know about one unit, computed by one lane for a batch
+// of 32 consecutive units (the dependent loads of 32 units then overlap).
+// pg[h]: physical page of the tile's h-th page; -1 when none of its
+// positions is visible, -2 when visible positions sit on a page no entry
+// maps (not candidates; counted by the producer).
+struct IxUnit {
+    int tok, tile, n, pg0, pg1;
+};
+
+__device__ __forceinline__ IxUnit ix_unit(const IndexerParams &p, long long unit) {
+    IxUnit m;
+    m.tok = ix_token_of(p, unit);
+    m.tile = (int)(unit - __ldg(p.tile_start + m.tok));
+    m.n = ix_visible(p, m.tok);
+    const int *pt_b = p.page_table + (size_t)(m.tok / p.T) * p.pt_stride;
+    int pg[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int lp = 2 * m.tile + h;
+        pg[h] = -1;
+        if (lp * 64 < m.n) {
+            const int v = lp < p.pt_stride ? __ldg(pt_b + lp) : -1;
+            pg[h] = (v >= 0 && (long long)v < p.num_pages) ? v : -2;
+        }
+    }
+    m.pg0 = pg[0];
+    m.pg1 = pg[1];
+    return m;
+}
+
+__device__ __forceinline__ IxUnit ix_unit_from(const IxUnit &m, int k) {
+    IxUnit r;
+    r.tok = __shfl_sync(0xffffffffu, m.tok, k);
+    r.tile = __shfl_sync(0xffffffffu, m.tile, k);
+    r.n = __shfl_sync(0xffffffffu, m.n, k);
+    r.pg0 = __shfl_sync(0xffffffffu, m.pg0, k);
+    r.pg1 = __shfl_sync(0xffffffffu, m.pg1, k);
+    return r;
+}
+
 // ---------------------------------------------------------------- TMA (tiled, no multicast)
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y,
                                             uint64_t *bar, uint64_t policy) {
@@ -183,13 +223,14 @@ struct IxCfg {
     static constexpr int kOffStages = 0;
     static constexpr int kOffQ = kIxStages * kStageBytes;   // two query slots
     static constexpr int kOffBar = kOffQ + 2 * kQBytes;
-    // full[S], empty[S], q_full[2], q_empty[2], acc_full[2], acc_empty[2]
-    static constexpr int kNumBars = 2 * kIxStages + 8;
+    // full[S], empty[S], q_full[2], q_empty[2], acc_full[A], acc_empty[A]
+    static constexpr int kAcc = 4;                           // accumulators of 64 TMEM columns
+    static constexpr int kNumBars = 2 * kIxStages + 4 + 2 * kAcc;
     static constexpr int kOffTmem = kOffBar + kNumBars * 8;
     static constexpr int kOffW = kOffTmem + 16;              // fp32 [64] weights of the token
     static constexpr int kBytes = kOffW + kIxMaxHeads * 4;
     static constexpr int kSmemBytes = kBytes + 1024;         // alignment slack (1024-B atoms)
-    static constexpr uint32_t kTmemCols = 128;               // two accumulators of 64 columns
+    static constexpr uint32_t kTmemCols = 64 * kAcc;
 };
 
 template <int NPAD>
@@ -203,7 +244,7 @@ __global__ void __launch_bounds__(IxCfg<NPAD>::kThreads, 1)
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::kOffBar);
     uint64_t *full = bars, *empty = bars + kIxStages;
     uint64_t *q_full = bars + 2 * kIxStages, *q_empty = q_full + 2;
-    uint64_t *acc_full = q_empty + 2, *acc_empty = acc_full + 2;
+    uint64_t *acc_full = q_empty + 2, *acc_empty = acc_full + C::kAcc;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::kOffTmem);
     float *w_s = reinterpret_cast<float *>(smem + C::kOffW);
 
@@ -215,6 +256,8 @@ __global__ void __launch_bounds__(IxCfg<NPAD>::kThreads, 1)
         for (int i = 0; i < 2; ++i) {
             mbar_init(&q_full[i], 1);
             mbar_init(&q_empty[i], 1);
+        }
+        for (int i = 0; i < C::kAcc; ++i) {
             mbar_init(&acc_full[i], 1);
             mbar_init(&acc_empty[i], 128);
         }
@@ -238,54 +281,51 @@ __global__ void __launch_bounds__(IxCfg<NPAD>::kThreads, 1)
 
     if (warp == 0) {
         // ============================================================ TMA producer
-        if (lane == 0 && u_begin < u_end) {
+        if (u_begin < u_end) {
             const uint64_t keep = l2_policy_evict_last();   // a query is read again per tile
             const uint64_t once = l2_policy_evict_first();  // keys are read once
-            int tok = ix_token_of(p, u_begin), changes = -1;
-            for (long long unit = u_begin, i = 0; unit < u_end; ++unit, ++i) {
-                bool fresh = unit == u_begin;
-                while (__ldg(p.tile_start + tok + 1) <= unit) {
-                    ++tok;
-                    fresh = true;
-                }
-                if (fresh) {  // the token's query heads into the next slot
-                    ++changes;
-                    const int sl = changes & 1, use = changes >> 1;
-                    if (use >= 1) mbar_wait(&q_empty[sl], (use - 1) & 1, dead);
-                    mbar_arrive_expect_tx(&q_full[sl], (uint32_t)C::kQBytes);
-                    const uint32_t qd = sbase + C::kOffQ + sl * C::kQBytes;
-                    tma_load_2d(qd, &map_q, 0, tok * p.HI, &q_full[sl], keep);
-                    tma_load_2d(qd + C::kQBoxBytes, &map_q, 64, tok * p.HI, &q_full[sl], keep);
-                }
-                const int st = (int)(i % kIxStages);
-                if (i >= kIxStages) mbar_wait(&empty[st], (int)((i / kIxStages) - 1) & 1, dead);
-                const int tile = (int)(unit - __ldg(p.tile_start + tok));
-                const int n = ix_visible(p, tok);
-                const int *pt_b = p.page_table + (size_t)(tok / p.T) * p.pt_stride;
-                int pages[2];
-                uint32_t bytes = 0;
+            int prev_tok = -1, changes = -1;
+            long long i = 0;
+            for (long long ub = u_begin; ub < u_end; ub += 32) {
+                const int cnt = (int)min(32ll, u_end - ub);
+                const IxUnit mine = ix_unit(p, min(ub + lane, u_end - 1));
+                for (int k = 0; k < cnt; ++k, ++i) {
+                    const IxUnit m = ix_unit_from(mine, k);
+                    if (lane == 0) {
+                        if (m.tok != prev_tok) {  // the token's query heads into the next slot
+                            prev_tok = m.tok;
+                            ++changes;
+                            const int sl = changes & 1, use = changes >> 1;
+                            if (use >= 1) mbar_wait(&q_empty[sl], (use - 1) & 1, dead);
+                            mbar_arrive_expect_tx(&q_full[sl], (uint32_t)C::kQBytes);
+                            const uint32_t qd = sbase + C::kOffQ + sl * C::kQBytes;
+                            tma_load_2d(qd, &map_q, 0, m.tok * p.HI, &q_full[sl], keep);
+                            tma_load_2d(qd + C::kQBoxBytes, &map_q, 64, m.tok * p.HI, &q_full[sl], keep);
+                        }
+                        const int st = (int)(i % kIxStages);
+                        if (i >= kIxStages) mbar_wait(&empty[st], (int)((i / kIxStages) - 1) & 1, dead);
+                        const int pgs[2] = {m.pg0, m.pg1};
+                        uint32_t bytes = 0;
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int lp = 2 * tile + h;  // logical page
-                    pages[h] = -1;
-                    const int first = lp * 64;
-                    if (first >= n) continue;     // no visible position on it
-                    const int pg = lp < p.pt_stride ? __ldg(pt_b + lp) : -1;
-                    if (pg >= 0 && (long long)pg < p.num_pages) {
-                        pages[h] = pg;
-                        bytes += 2 * 64 * 128;
-                    } else {  // visible positions on a page no entry maps: not candidates
-                        atomicOr(&g_status_flags, kFlagIndexRange);
-                        atomicAdd(&g_bad_index_count, (unsigned long long)(min(n, first + 64) - first));
+                        for (int h = 0; h < 2; ++h) {
+                            if (pgs[h] >= 0) {
+                                bytes += 2 * 64 * 128;
+                            } else if (pgs[h] == -2) {  // visible positions no page entry maps
+                                const int first = (2 * m.tile + h) * 64;
+                                atomicOr(&g_status_flags, kFlagIndexRange);
+                                atomicAdd(&g_bad_index_count, (unsigned long long)(min(m.n, first + 64) - first));
+                            }
+                        }
+                        mbar_arrive_expect_tx(&full[st], bytes);
+                        const uint32_t dst = sbase + C::kOffStages + st * C::kStageBytes;
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            if (pgs[h] < 0) continue;
+                            tma_load_2d(dst + h * 8192, &map_k, 0, pgs[h] * 64, &full[st], once);
+                            tma_load_2d(dst + C::kBoxBytes + h * 8192, &map_k, 64, pgs[h] * 64, &full[st], once);
+                        }
                     }
-                }
-                mbar_arrive_expect_tx(&full[st], bytes);
-                const uint32_t dst = sbase + C::kOffStages + st * C::kStageBytes;
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    if (pages[h] < 0) continue;
-                    tma_load_2d(dst + h * 8192, &map_k, 0, pages[h] * 64, &full[st], once);
-                    tma_load_2d(dst + C::kBoxBytes + h * 8192, &map_k, 64, pages[h] * 64, &full[st], once);
+                    __syncwarp();
                 }
             }
         }
@@ -304,9 +344,9 @@ __global__ void __launch_bounds__(IxCfg<NPAD>::kThreads, 1)
                     ++changes;
                     mbar_wait(&q_full[changes & 1], (changes >> 1) & 1, dead);
                 }
-                const int st = (int)(i % kIxStages), a = (int)(i & 1);
+                const int st = (int)(i % kIxStages), a = (int)(i % C::kAcc);
                 mbar_wait(&full[st], (int)(i / kIxStages) & 1, dead);
-                if (i >= 2) mbar_wait(&acc_empty[a], (int)((i >> 1) - 1) & 1, dead);
+                if (i >= C::kAcc) mbar_wait(&acc_empty[a], (int)((i / C::kAcc) - 1) & 1, dead);
                 tc_fence_after();
                 const uint32_t ka = sbase + C::kOffStages + st * C::kStageBytes;
                 const uint32_t qa = sbase + C::kOffQ + (changes & 1) * C::kQBytes;
@@ -330,38 +370,39 @@ __global__ void __launch_bounds__(IxCfg<NPAD>::kThreads, 1)
         const int q4 = warp & 3;                 // TMEM lanes 32 q4 .. + 31
         const int row = 32 * q4 + lane;          // key of the tile
         const int et = threadIdx.x - 128;        // 0 .. 127
-        int tok = u_begin < u_end ? ix_token_of(p, u_begin) : 0, w_tok = -1;
-        for (long long unit = u_begin, i = 0; unit < u_end; ++unit, ++i) {
-            while (__ldg(p.tile_start + tok + 1) <= unit) ++tok;
-            if (tok != w_tok) {  // the token's head weights (0 past HI)
-                named_bar_sync(1, 128);
-                if (et < kIxMaxHeads) w_s[et] = et < p.HI ? __ldg(p.w + (size_t)tok * p.HI + et) : 0.f;
-                named_bar_sync(1, 128);
-                w_tok = tok;
-            }
-            const int a = (int)(i & 1);
-            mbar_wait(&acc_full[a], (int)(i >> 1) & 1, dead);
-            tc_fence_after();
-            uint32_t x[NPAD];
-            tmem_ld_cols<NPAD>(tmem + ((uint32_t)(32 * q4) << 16) + a * 64, x);
-            tmem_ld_wait();
-            tc_fence_before();
-            mbar_arrive(&acc_empty[a]);
-            const int tile = (int)(unit - __ldg(p.tile_start + tok));
-            const int s = tile * kIxTile + row;
-            const int n = ix_visible(p, tok);
-            if (s < n) {
-                const int lp = s >> 6;
-                const int pg = lp < p.pt_stride ? __ldg(p.page_table + (size_t)(tok / p.T) * p.pt_stride + lp) : -1;
-                float score = __uint_as_float(0x7fffffffu);  // NaN: not a candidate
-                if (pg >= 0 && (long long)pg < p.num_pages) {
-                    float acc = 0.f;
-#pragma unroll
-                    for (int j = 0; j < NPAD; ++j)
-                        acc = (j < p.HI) ? fmaf(w_s[j], fmaxf(__uint_as_float(x[j]), 0.f), acc) : acc;
-                    score = acc;
+        int w_tok = -1;
+        long long i = 0;
+        for (long long ub = u_begin; ub < u_end; ub += 32) {
+            const int cnt = (int)min(32ll, u_end - ub);
+            const IxUnit mine = ix_unit(p, min(ub + lane, u_end - 1));
+            for (int k = 0; k < cnt; ++k, ++i) {
+                const IxUnit m = ix_unit_from(mine, k);
+                if (m.tok != w_tok) {  // the token's head weights (0 past HI)
+                    named_bar_sync(1, 128);
+                    if (et < kIxMaxHeads) w_s[et] = et < p.HI ? __ldg(p.w + (size_t)m.tok * p.HI + et) : 0.f;
+                    named_bar_sync(1, 128);
+                    w_tok = m.tok;
                 }
-                p.scores[(size_t)tok * p.score_stride + s] = score;
+                const int a = (int)(i % C::kAcc);
+                mbar_wait(&acc_full[a], (int)(i / C::kAcc) & 1, dead);
+                tc_fence_after();
+                uint32_t x[NPAD];
+                tmem_ld_cols<NPAD>(tmem + ((uint32_t)(32 * q4) << 16) + a * 64, x);
+                tmem_ld_wait();
+                tc_fence_before();
+                mbar_arrive(&acc_empty[a]);
+                const int s = m.tile * kIxTile + row;
+                if (s < m.n) {
+                    float score = __uint_as_float(0x7fffffffu);  // NaN: not a candidate
+                    if ((row < 64 ? m.pg0 : m.pg1) >= 0) {
+                        float acc = 0.f;
+#pragma unroll
+                        for (int j = 0; j < NPAD; ++j)
+                            acc = (j < p.HI) ? fmaf(w_s[j], fmaxf(__uint_as_float(x[j]), 0.f), acc) : acc;
+                        score = acc;
+                    }
+                    p.scores[(size_t)m.tok * p.score_stride + s] = score;
+                }
             }
         }
     }
@@ -383,85 +424,211 @@ __device__ __forceinline__ uint32_t ix_key(float f) {
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// Shared memory of the selection kernel: the digit histogram, the crossing
+// bucket's candidates and two bitmaps over the visible positions (selected,
+// equal to the threshold).
+constexpr int kIxCandCap = 8192;   // candidates of the crossing bucket kept in shared memory
+__host__ __device__ constexpr int ix_select_smem_bytes(int max_n) {
+    return 2048 * 4 + kIxCandCap * 8 + 2 * 4 * ((max_n + 31) / 32);
+}
+constexpr int kIxSelectMaxN = (232448 - 2048 * 4 - kIxCandCap * 8 - 1024) / 8 * 32;
+
+// Histogram of digit (key >> shift) & (nb - 1) over the keys whose bits above
+// the digit equal `prefix`; keys from global scores (8 loads in flight per
+// thread) or from the candidate list.
+__device__ __forceinline__ void ix_hist_add(unsigned *hist, uint32_t key, bool match, uint32_t d) {
+    const uint32_t peers = __match_any_sync(__activemask(), match ? d : 0xffffffffu);
+    if (match && (__ffs(peers) - 1) == (int)(threadIdx.x & 31)) atomicAdd(&hist[d], (unsigned)__popc(peers));
+}
+
+// Bucket of the histogram (nb bins) holding the need-th largest key counted
+// from the top: writes (bucket, keys above it) to found[]; returns the total.
+__device__ __forceinline__ int ix_find_bucket(const unsigned *hist, int nb, int need, int *scratch,
+                                              int *found) {
+    int v = 0, b_hi = -1, b_lo = -1;
+    if (2 * (int)threadIdx.x < nb) {
+        b_hi = nb - 1 - 2 * threadIdx.x;
+        b_lo = b_hi - 1;
+        v = (int)hist[b_hi] + (b_lo >= 0 ? (int)hist[b_lo] : 0);
+    }
+    int total;
+    const int incl = ix_block_scan(v, scratch, &total);
+    const int excl = incl - v;
+    if (b_hi >= 0 && excl < need && need <= incl) {
+        const int h = (int)hist[b_hi];
+        if (excl + h >= need) {
+            found[0] = b_hi;
+            found[1] = excl;
+        } else {
+            found[0] = b_lo;
+            found[1] = excl + h;
+        }
+    }
+    __syncthreads();
+    return total;
+}
+
+// Ordered scan of a bitmap of `words` words: calls emit(rank, position) for
+// every set bit in ascending position order (rank = its index among set bits).
+template <typename F>
+__device__ __forceinline__ int ix_bitmap_scan(const uint32_t *bits, int words, int *scratch, F emit) {
+    const int per = (words + blockDim.x - 1) / blockDim.x;
+    const int w0 = min(words, (int)threadIdx.x * per), w1 = min(words, w0 + per);
+    int cnt = 0;
+    for (int i = w0; i < w1; ++i) cnt += __popc(bits[i]);
+    int total;
+    int rank = ix_block_scan(cnt, scratch, &total) - cnt;
+    for (int i = w0; i < w1; ++i) {
+        uint32_t m = bits[i];
+        while (m) {
+            const int b = __ffs(m) - 1;
+            m &= m - 1;
+            emit(rank++, 32 * i + b);
+        }
+    }
+    return total;
+}
+
+// One CTA per query token.  Pass A (global): histogram of the top 11 bits of
+// the key -> the crossing bucket d0.  Pass B (global): positions with a digit
+// above d0 are selected (bitmap); those in d0 become candidates in shared
+// memory.  Two radix passes over the candidates give the exact threshold key
+// and how many keys equal to it are taken; the first of those by position are
+// found by an ordered scan of an "equal" bitmap, and an ordered scan of the
+// selection bitmap writes the output.  If d0 holds more than kIxCandCap
+// keys, the two finer passes and the marking read the global scores instead.
 __global__ void __launch_bounds__(kIxSelectThreads) smla_ix_select_kernel(const IndexerParams p) {
-    __shared__ unsigned hist[2048];
+    extern __shared__ __align__(16) uint8_t ix_smem[];
+    unsigned *hist = reinterpret_cast<unsigned *>(ix_smem);
+    uint32_t *cand_key = reinterpret_cast<uint32_t *>(ix_smem + 2048 * 4);
+    int *cand_pos = reinterpret_cast<int *>(ix_smem + 2048 * 4 + kIxCandCap * 4);
+    uint32_t *sel_bits = reinterpret_cast<uint32_t *>(ix_smem + 2048 * 4 + kIxCandCap * 8);
     __shared__ int scratch[33];
     __shared__ int found[2];
-    const int u = blockIdx.x, tid = threadIdx.x;
+    __shared__ int n_cand;
+    const int u = blockIdx.x, tid = threadIdx.x, nt = blockDim.x;
     const int n = ix_visible(p, u), K = p.K;
+    const int words = (n + 31) / 32;
+    uint32_t *eq_bits = sel_bits + words;
     const float *sc = p.scores + (size_t)u * p.score_stride;
     int *out = p.out + (size_t)u * K;
+    constexpr int kIlp = 8;
 
-    // Three radix passes find the K-th largest key (thresh) and how many keys
-    // equal to it are taken (need); with K or fewer candidates, all are.
-    uint32_t prefix = 0, thresh = 0;
-    int need = K, valid = 0;
-    const int shifts[3] = {21, 10, 0}, widths[3] = {11, 11, 10};
-    for (int pass = 0; pass < 3; ++pass) {
-        const int shift = shifts[pass], nb = 1 << widths[pass];
-        for (int i = tid; i < 2048; i += blockDim.x) hist[i] = 0;
-        __syncthreads();
-        const int hi_shift = shift + widths[pass];  // bits above this digit must match prefix
-        for (int s = tid; s < n; s += blockDim.x) {
-            const uint32_t key = ix_key(__ldg(sc + s));
-            const bool match = key != 0u && (hi_shift >= 32 || (key >> hi_shift) == prefix);
-            const uint32_t d = (key >> shift) & (uint32_t)(nb - 1);
-            // aggregate equal digits within the warp (scores cluster in few buckets)
-            const uint32_t peers = __match_any_sync(__activemask(), match ? d : 0xffffffffu);
-            if (match && (__ffs(peers) - 1) == (tid & 31)) atomicAdd(&hist[d], (unsigned)__popc(peers));
+    for (int i = tid; i < 2048; i += nt) hist[i] = 0;
+    for (int i = tid; i < 2 * words; i += nt) sel_bits[i] = 0;
+    if (tid == 0) n_cand = 0;
+    __syncthreads();
+
+    // ---- pass A: top 11 bits
+    for (int base = 0; base < n; base += nt * kIlp) {
+        uint32_t key[kIlp];
+#pragma unroll
+        for (int j = 0; j < kIlp; ++j) {
+            const int s = base + j * nt + tid;
+            key[j] = s < n ? ix_key(__ldg(sc + s)) : 0u;
         }
-        __syncthreads();
-        // bins from the top: thread i sums bins nb-1-2i and nb-2-2i
-        int v = 0, b_hi = -1, b_lo = -1;
-        if (2 * tid < nb) {
-            b_hi = nb - 1 - 2 * tid;
-            b_lo = b_hi - 1;
-            v = (int)hist[b_hi] + (b_lo >= 0 ? (int)hist[b_lo] : 0);
+#pragma unroll
+        for (int j = 0; j < kIlp; ++j) ix_hist_add(hist, key[j], key[j] != 0u, key[j] >> 21);
+    }
+    __syncthreads();
+    int need = K;
+    const int valid = ix_find_bucket(hist, 2048, need, scratch, found);
+    const bool take_all = valid <= K;
+    const uint32_t d0 = take_all ? 0u : (uint32_t)found[0];
+    if (!take_all) need -= found[1];
+
+    // ---- pass B: digits above d0 are in; d0's keys become candidates
+    for (int base = 0; base < n; base += nt * kIlp) {
+        uint32_t key[kIlp];
+#pragma unroll
+        for (int j = 0; j < kIlp; ++j) {
+            const int s = base + j * nt + tid;
+            key[j] = s < n ? ix_key(__ldg(sc + s)) : 0u;
         }
-        int total;
-        const int incl = ix_block_scan(v, scratch, &total);
-        if (pass == 0) {
-            valid = total;
-            if (valid <= K) {  // every candidate is taken
-                thresh = 0u;
-                need = 0;
-                break;
+#pragma unroll
+        for (int j = 0; j < kIlp; ++j) {
+            const int s = base + j * nt + tid;
+            if (key[j] == 0u) continue;
+            const uint32_t d = key[j] >> 21;
+            if (take_all || d > d0) {
+                atomicOr(&sel_bits[s >> 5], 1u << (s & 31));
+            } else if (d == d0) {
+                const int c = atomicAdd(&n_cand, 1);
+                if (c < kIxCandCap) {
+                    cand_key[c] = key[j];
+                    cand_pos[c] = s;
+                }
             }
         }
-        const int excl = incl - v;
-        if (b_hi >= 0 && excl < need && need <= incl) {
-            const int h = (int)hist[b_hi];
-            if (excl + h >= need) {
-                found[0] = b_hi;
-                found[1] = excl;
+    }
+    __syncthreads();
+
+    if (!take_all) {
+        // ---- the two finer digits, over the candidates (or the global scores)
+        const int m = n_cand;
+        const bool in_smem = m <= kIxCandCap;
+        uint32_t prefix = d0;
+#pragma unroll
+        for (int pass = 0; pass < 2; ++pass) {
+            const int shift = pass == 0 ? 10 : 0, width = pass == 0 ? 11 : 10, nb = 1 << width;
+            const int hi_shift = shift + width;
+            for (int i = tid; i < 2048; i += nt) hist[i] = 0;
+            __syncthreads();
+            if (in_smem) {
+                for (int c = tid; c < ((m + 31) & ~31); c += nt) {
+                    const uint32_t key = c < m ? cand_key[c] : 0u;
+                    ix_hist_add(hist, key, c < m && (key >> hi_shift) == prefix, (key >> shift) & (nb - 1));
+                }
             } else {
-                found[0] = b_lo;
-                found[1] = excl + h;
+                for (int base = 0; base < n; base += nt * kIlp) {
+                    uint32_t key[kIlp];
+#pragma unroll
+                    for (int j = 0; j < kIlp; ++j) {
+                        const int s = base + j * nt + tid;
+                        key[j] = s < n ? ix_key(__ldg(sc + s)) : 0u;
+                    }
+#pragma unroll
+                    for (int j = 0; j < kIlp; ++j)
+                        ix_hist_add(hist, key[j], key[j] != 0u && (key[j] >> hi_shift) == prefix,
+                                    (key[j] >> shift) & (nb - 1));
+                }
+            }
+            __syncthreads();
+            ix_find_bucket(hist, nb, need, scratch, found);
+            prefix = (prefix << width) | (uint32_t)found[0];
+            need -= found[1];
+            __syncthreads();
+        }
+        const uint32_t thresh = prefix;
+        // ---- mark: above the threshold -> selected; equal -> the "equal" bitmap
+        if (in_smem) {
+            for (int c = tid; c < m; c += nt) {
+                const uint32_t key = cand_key[c];
+                const int s = cand_pos[c];
+                if (key > thresh) atomicOr(&sel_bits[s >> 5], 1u << (s & 31));
+                else if (key == thresh) atomicOr(&eq_bits[s >> 5], 1u << (s & 31));
+            }
+        } else {
+            for (int s = tid; s < n; s += nt) {
+                const uint32_t key = ix_key(__ldg(sc + s));
+                if ((key >> 21) != d0) continue;  // the bits above d0 are set already
+                if (key > thresh) atomicOr(&sel_bits[s >> 5], 1u << (s & 31));
+                else if (key == thresh) atomicOr(&eq_bits[s >> 5], 1u << (s & 31));
             }
         }
         __syncthreads();
-        prefix = (prefix << widths[pass]) | (uint32_t)found[0];
-        need -= found[1];
+        // ---- the first `need` equal keys by position
+        ix_bitmap_scan(eq_bits, words, scratch, [&](int rank, int s) {
+            if (rank < need) atomicOr(&sel_bits[s >> 5], 1u << (s & 31));
+        });
         __syncthreads();
-        if (pass == 2) thresh = prefix;
     }
 
-    // Ascending scan: keys above thresh, and the first `need` equal to it.
-    int eq_carry = 0, sel_carry = 0, total;
-    for (int base = 0; base < n; base += blockDim.x) {
-        const int s = base + tid;
-        const uint32_t key = s < n ? ix_key(__ldg(sc + s)) : 0u;
-        const int eq = (need > 0 && key == thresh) ? 1 : 0;
-        const int eq_incl = ix_block_scan(eq, scratch, &total);
-        const int eq_rank = eq_carry + eq_incl - eq;
-        eq_carry += total;
-        const int sel = (key > thresh || (eq && eq_rank < need)) ? 1 : 0;
-        const int sel_incl = ix_block_scan(sel, scratch, &total);
-        const int at = sel_carry + sel_incl - sel;
-        if (sel && at < K) out[at] = s;
-        sel_carry += total;
-    }
-    for (int i = min(sel_carry, K) + tid; i < K; i += blockDim.x) out[i] = -1;
+    // ---- output: selected positions in ascending order, then -1
+    const int taken = ix_bitmap_scan(sel_bits, words, scratch, [&](int rank, int s) {
+        if (rank < K) out[rank] = s;
+    });
+    for (int i = min(taken, K) + tid; i < K; i += nt) out[i] = -1;
 }
 
 }  // namespace smla

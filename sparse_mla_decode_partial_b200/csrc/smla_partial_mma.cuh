@@ -147,6 +147,49 @@ __device__ __forceinline__ void mark_unused_slots(const PartialParams &p, const 
     }
 }
 
+// Index entries [j0 + base, j0 + base + n) of query token bt -> physical rows
+// in rows_s[0, n) (-1 = masked), resolved by threads tid, tid + nthreads, ...
+// of the caller with every load of a batch in flight at once.  Entries other
+// than -1 that are out of range are counted.
+template <int BATCH>
+__device__ __forceinline__ void resolve_rows(const PartialParams &p, int bt, int j0, int base, int n,
+                                             int *rows_s, int tid, int nthreads) {
+    const int *idx_bt = p.idx + (size_t)bt * p.K + j0 + base;
+    const int *pt_b = p.page_table + (size_t)(bt / p.T) * p.pt_stride;
+    const long long max_pos = (long long)p.pt_stride * kPage;
+    for (int b0 = 0; b0 < n; b0 += nthreads * BATCH) {
+        int iv[BATCH];
+#pragma unroll
+        for (int k = 0; k < BATCH; ++k) {
+            const int j = b0 + k * nthreads + tid;
+            iv[k] = (j < n) ? __ldg(idx_bt + j) : -1;
+        }
+        int pg[BATCH];
+#pragma unroll
+        for (int k = 0; k < BATCH; ++k) {
+            const int i = iv[k];
+            pg[k] = (i >= 0 && (long long)i < max_pos) ? __ldg(pt_b + (i >> 6)) : -1;
+        }
+#pragma unroll
+        for (int k = 0; k < BATCH; ++k) {
+            const int j = b0 + k * nthreads + tid;
+            const int i = iv[k];
+            int row = -1;
+            if (i != -1) {
+                const bool ok = (i >= 0) && ((long long)i < max_pos) && (pg[k] >= 0) &&
+                                ((long long)pg[k] < p.num_pages);
+                if (ok) {
+                    row = pg[k] * kPage + (i & (kPage - 1));
+                } else if (j < n) {
+                    atomicOr(&g_status_flags, kFlagIndexRange);
+                    atomicAdd(&g_bad_index_count, 1ull);
+                }
+            }
+            if (j < n) rows_s[j] = row;
+        }
+    }
+}
+
 template <int HG, int NT, int NSTAGE>
 struct MmaCfg {
     static_assert(NT == 16 || NT == 32 || NT == 64, "tile rows");
@@ -394,57 +437,37 @@ __global__ void __launch_bounds__(MmaCfg<HG, NT, NSTAGE>::kThreads, MmaCfg<HG, N
     // The combine kernel is launched as a programmatic dependent: let it be
     // scheduled now; it waits for this grid's completion before reading.
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    // Every thread helps resolve the first chunk of the first item, so that
+    // the first copies start after two memory round trips (one warp alone
+    // took several microseconds for a 512-entry split).
+    int *rows_s0 = reinterpret_cast<int *>(smem + C::kOffRows);
+    {
+        long long u0 = item_begin(p, cta);
+        WorkItem w0;
+        if (next_item(p, cta, u0, w0))
+            resolve_rows<4>(p, w0.bt, w0.j0, 0, min(kResolveChunk, w0.j1 - w0.j0), rows_s0,
+                            threadIdx.x, C::kThreads);
+    }
     __syncthreads();
 
     if (warp == C::kComputeWarps) {
         // ============================================================ producer
-        const long long max_pos = (long long)p.pt_stride * kPage;
         const uint64_t policy = l2_policy_evict_first();
         int *rows_s = reinterpret_cast<int *>(smem + C::kOffRows);
         constexpr int kResolveBatch = HG <= 2 ? 32 : 16;  // loads in flight per lane
         int it = 0;  // tile counter over all of this CTA's items (ring position)
         long long u = item_begin(p, cta);
         WorkItem w;
+        bool first_chunk = true;  // resolved by the whole CTA above
         while (next_item(p, cta, u, w)) {
-            const int *idx_bt = p.idx + (size_t)w.bt * p.K + w.j0;
-            const int *pt_b = p.page_table + (size_t)(w.bt / p.T) * p.pt_stride;
             const int len = w.j1 - w.j0;
             for (int base = 0; base < len; base += kResolveChunk) {
                 const int n = min(kResolveChunk, len - base);
                 __syncwarp();  // rows_s is rewritten below
-                // Resolve the whole chunk before the first copy: index loads, then
-                // page-table loads, each batch of 32 per lane in flight at once.
-                for (int b0 = 0; b0 < n; b0 += 32 * kResolveBatch) {
-                    int iv[kResolveBatch];
-#pragma unroll
-                    for (int k = 0; k < kResolveBatch; ++k) {
-                        const int j = b0 + k * 32 + lane;
-                        iv[k] = (j < n) ? __ldg(idx_bt + base + j) : -1;
-                    }
-                    int pg[kResolveBatch];
-#pragma unroll
-                    for (int k = 0; k < kResolveBatch; ++k) {
-                        const int i = iv[k];
-                        pg[k] = (i >= 0 && (long long)i < max_pos) ? __ldg(pt_b + (i >> 6)) : -1;
-                    }
-#pragma unroll
-                    for (int k = 0; k < kResolveBatch; ++k) {
-                        const int j = b0 + k * 32 + lane;
-                        const int i = iv[k];
-                        int row = -1;
-                        if (i != -1) {
-                            const bool ok = (i >= 0) && ((long long)i < max_pos) && (pg[k] >= 0) &&
-                                            ((long long)pg[k] < p.num_pages);
-                            if (ok) {
-                                row = pg[k] * kPage + (i & (kPage - 1));
-                            } else if (j < n) {
-                                atomicOr(&g_status_flags, kFlagIndexRange);
-                                atomicAdd(&g_bad_index_count, 1ull);
-                            }
-                        }
-                        if (j < n) rows_s[j] = row;
-                    }
-                }
+                // Resolve the whole chunk before its first copy: index loads,
+                // then page-table loads, a batch per lane in flight at once.
+                if (!first_chunk) resolve_rows<kResolveBatch>(p, w.bt, w.j0, base, n, rows_s, lane, 32);
+                first_chunk = false;
                 __syncwarp();
                 // Issue one bulk copy per row (or per padding slot, from the zero row).
                 const int chunk_tiles = (n + NT - 1) / NT;
