@@ -96,9 +96,8 @@ typedef enum {
  * that minimises a model of wave count x rows per CTA plus per-CTA overhead
  * and the split-K scratch traffic, with two resident CTAs per SM for H <= 16
  * and one otherwise.  It also prices smla_decode's balanced schedule (one
- * full wave of equal CTAs, ceil(SMs x resident / (B*T)) + 1 slots) and
- * returns that slot count when the model favours it (by more than 15% for
- * H <= 32, whose kernels stall at a token boundary; at all for H > 32).
+ * full wave of equal CTAs, ceil(SMs x resident / (B*T)) + 1 slots, H <= 32)
+ * and returns that slot count only when the model favours it by more than 15%.
  * sm_count <= 0 queries the current device.  If the environment variable SMLA_NSPLIT holds a positive integer,
  * that value is returned instead (clamped to [1, SMLA_MAX_NSPLIT]).
  * Returns >= 1; returns 1 for degenerate sizes.
@@ -172,6 +171,24 @@ smla_status smla_decode(const void *q, const void *kv_cache, int64_t num_pages,
                         int B, int T, int H, int K, int page_size, float scale, int nsplit,
                         void *workspace, size_t workspace_bytes, void *o, float *lse,
                         void *stream);
+
+/*
+ * The partial pass of smla_decode alone (nsplit >= 2): the same kernel,
+ * schedule and workspace layout smla_decode uses -- equal splits, or the
+ * balanced schedule's pieces in nsplit slots per token -- with the partials
+ * left in the workspace.  The workspace holds, at offsets 0, round256(n * 512
+ * * 4) and that plus round256(n * 4) with n = B*T*H*nsplit, part_o
+ * [B,T,H,nsplit,512], part_m and part_lse [B,T,H,nsplit]; smla_lse_combine on
+ * them completes the decode (it ignores a slot with part_m = -inf).  Splitting
+ * the decode this way lets a caller schedule other work between the two
+ * launches or time the partial pass alone.  Arguments and errors as for
+ * smla_decode.
+ */
+smla_status smla_decode_partial_ws(const void *q, const void *kv_cache, int64_t num_pages,
+                                   const int32_t *page_table, int pt_stride,
+                                   const int32_t *topk_idx, int B, int T, int H, int K,
+                                   int page_size, float scale, int nsplit, void *workspace,
+                                   size_t workspace_bytes, void *stream);
 
 /*
  * Checked mode: synchronises `stream`, then reads the current device's
@@ -281,8 +298,13 @@ smla_status smla_decode_host(const void *q_host, const void *kv_cache, int64_t n
  *  - seq_lens  int32 [B, T], device memory, each in [0, K].  A length outside
  *              that range is clamped to it and raises SMLA_ERR_INDEX_RANGE in
  *              smla_check_device (counted once per query token).
- *  - K         the longest visible length; the split boundaries are those of
- *              an index list of width K (R7: Kc = ceil(K / nsplit) positions).
+ *  - K         the longest visible length.  smla_decode_dense rounds the
+ *              split length ceil(K / nsplit) up to whole pages (64 positions)
+ *              and uses the ceil(K / that) <= nsplit splits it needs, so that
+ *              every 32-row tile is half a page of consecutive cache rows;
+ *              smla_decode_dense_partial keeps split s at positions
+ *              [s Kc, (s+1) Kc), Kc = ceil(K / nsplit), as for an index list
+ *              of width K.
  *  - nsplit    0 picks smla_dense_nsplit(B, T, H, K).
  *  - Other arguments, layouts and outputs are those of smla_decode.  A
  *    visible position that no page maps is masked and counted once per

@@ -35,6 +35,8 @@ SIGNATURES = {
     "smla_lse_combine": (_I, [_P, _P, _P, _I, _I, _I, _I, _P, _P, _P]),
     "smla_decode": (_I, [_P, _P, _I64, _P, _I, _P, _I, _I, _I, _I, _I, _F, _I, _P, _SZ, _P, _P,
                          _P]),
+    "smla_decode_partial_ws": (_I, [_P, _P, _I64, _P, _I, _P, _I, _I, _I, _I, _I, _F, _I, _P, _SZ,
+                                    _P]),
     "smla_decode_noalloc": (_I, [_P, _P, _I64, _P, _I, _P, _I, _I, _I, _I, _I, _F, _I, _P, _P,
                                  _P]),
     "smla_workspace_host_bytes": (_SZ, [_I, _I, _I, _I, _I, _I]),

@@ -114,15 +114,12 @@ int nsplit_model(int B, int T, int H, int K, int sm_count) {
     // of the pass), so the balanced choice must win by kBalancedMargin.
     const long long s_bal = (long long)std::ceil((double)slots / (double)base) + 1;
     const double units = (double)base * ((K + 31) / 32);
-    if (s_bal >= 2 && s_bal <= s_max && units >= 4.0 * slots &&
+    if (H <= 32 && s_bal >= 2 && s_bal <= s_max && units >= 4.0 * slots &&
         !uses_latency_kernel(H, K, (K + (int)s_bal - 1) / (int)s_bal, 0)) {
         const double pieces = (double)base + slots;
         double t = kFixedRows * pieces / slots + units * 32.0 / slots;
         t += kScratchWeight * pieces * H * kPartialBytesPerHead * 2.0 / smla::kRowBytes / slots;
-        // the tcgen05 kernel overlaps an item boundary with the next item's
-        // work (Q staged early, O drained through a spent ring slot)
-        const double margin = H > 32 ? 0.0 : kBalancedMargin;
-        if (t < best * (1.0 - margin)) best_s = (int)s_bal;
+        if (t < best * (1.0 - kBalancedMargin)) best_s = (int)s_bal;
     }
     return best_s;
 }
@@ -159,12 +156,23 @@ smla_status launch_mma(const PartialParams &p, int grid, cudaStream_t st) {
     return e == cudaSuccess ? SMLA_OK : cuda_fail(e);
 }
 
+}  // namespace
+smla_status encode_cache_tiles(CUtensorMap *map, const void *cache, int64_t num_pages);
+namespace {
+
 template <bool DIRECT>
 smla_status launch_tc(const PartialParams &p, int grid, cudaStream_t st) {
     const void *fn = reinterpret_cast<const void *>(&smla::smla_partial_tc_kernel<DIRECT>);
     cudaError_t e = ensure_smem_attr(fn, smla::TcCfg::kSmemBytes);
     if (e != cudaSuccess) return cuda_fail(e);
-    smla::smla_partial_tc_kernel<DIRECT><<<grid, smla::TcCfg::kThreads, smla::TcCfg::kSmemBytes, st>>>(p);
+    // dense lists load whole half-pages by TMA; sparse lists never use the map
+    CUtensorMap map;
+    std::memset(&map, 0, sizeof map);
+    if (p.seq_lens != nullptr && p.K > 0) {
+        const smla_status s = encode_cache_tiles(&map, p.cache, p.num_pages);
+        if (s != SMLA_OK) return s;
+    }
+    smla::smla_partial_tc_kernel<DIRECT><<<grid, smla::TcCfg::kThreads, smla::TcCfg::kSmemBytes, st>>>(p, map);
     e = cudaGetLastError();
     return e == cudaSuccess ? SMLA_OK : cuda_fail(e);
 }
@@ -233,9 +241,11 @@ int resident_per_sm(int H) {
 // flattened (token, 32-row tile) space; a token then spans at most
 // ceil(R / (B*T)) + 1 CTAs, each writing one of its S slots.  Used when it
 // fits in S slots and each CTA gets at least 4 tiles.  The tcgen05 kernel
-// (H > 32) walks its items the same way, one CTA per SM.
+// (H > 32) keeps equal splits: its gather is bound by the device-wide 16-byte
+// cp.async rate, not by the SMs it occupies (a balanced form measured no
+// faster).
 bool use_balanced(int B, int T, int H, int K, int nsplit, int pt_stride, int sms, int *grid) {
-    if (nsplit < 2 || K <= 0) return false;
+    if (nsplit < 2 || K <= 0 || H > 32) return false;
     const int kc = (K + nsplit - 1) / nsplit;
     if (uses_latency_kernel(H, K, kc, pt_stride)) return false;
     const long long bt = (long long)B * T;
@@ -368,30 +378,19 @@ smla_status smla_lse_combine(const float *part_o, const float *part_m, const flo
                           static_cast<cudaStream_t>(stream));
 }
 
-smla_status smla_decode(const void *q, const void *kv_cache, int64_t num_pages,
-                        const int32_t *page_table, int pt_stride, const int32_t *topk_idx, int B,
-                        int T, int H, int K, int page_size, float scale, int nsplit,
-                        void *workspace, size_t workspace_bytes, void *o, float *lse,
-                        void *stream) {
-    smla_status st = check_decode_args(q, kv_cache, num_pages, page_table, pt_stride, topk_idx, B,
-                                       T, H, K, page_size, scale);
-    if (st != SMLA_OK) return st;
-    if (nsplit < 0 || nsplit > SMLA_MAX_NSPLIT) return SMLA_ERR_INVALID_ARG;
-    if (B == 0 || T == 0 || H == 0) return SMLA_OK;
-    if (o == nullptr || lse == nullptr) return SMLA_ERR_INVALID_ARG;
-    if (!aligned(o, 16) || !aligned(lse, 4)) return SMLA_ERR_MISALIGNED;
-    if (nsplit == 0) nsplit = smla_choose_nsplit(B, T, H, K, 0);
-    const cudaStream_t s = static_cast<cudaStream_t>(stream);
-    PartialParams p = make_params(q, kv_cache, num_pages, page_table, pt_stride, topk_idx, B, T, H,
-                                  K, scale, nsplit);
-    if (nsplit == 1) {
-        p.o = static_cast<__nv_bfloat16 *>(o);
-        p.lse = lse;
-        return launch_partial<true>(p, s);
-    }
+namespace {
+
+// The partial pass of the whole decode into the workspace (nsplit >= 2):
+// equal splits, or the balanced schedule when it applies.
+smla_status decode_partial_pass(const void *q, const void *kv_cache, int64_t num_pages,
+                                const int32_t *page_table, int pt_stride, const int32_t *topk_idx,
+                                int B, int T, int H, int K, float scale, int nsplit, void *workspace,
+                                size_t workspace_bytes, cudaStream_t s, PartialParams *out) {
     if (workspace_bytes < smla_workspace_bytes(B, T, H, nsplit)) return SMLA_ERR_WORKSPACE_TOO_SMALL;
     if (workspace == nullptr) return SMLA_ERR_INVALID_ARG;
     if (!aligned(workspace, 16)) return SMLA_ERR_MISALIGNED;
+    PartialParams p = make_params(q, kv_cache, num_pages, page_table, pt_stride, topk_idx, B, T, H,
+                                  K, scale, nsplit);
     const size_t n = (size_t)B * T * H * nsplit;
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     const size_t off_m = round256(n * smla::kDc * sizeof(float));
@@ -406,9 +405,54 @@ smla_status smla_decode(const void *q, const void *kv_cache, int64_t num_pages,
         p.tpt = (K + 31) / 32;
         p.n_units = (long long)B * T * p.tpt;
     }
-    st = launch_partial<false>(p, s);
+    *out = p;
+    return launch_partial<false>(p, s);
+}
+
+}  // namespace
+
+smla_status smla_decode(const void *q, const void *kv_cache, int64_t num_pages,
+                        const int32_t *page_table, int pt_stride, const int32_t *topk_idx, int B,
+                        int T, int H, int K, int page_size, float scale, int nsplit,
+                        void *workspace, size_t workspace_bytes, void *o, float *lse,
+                        void *stream) {
+    smla_status st = check_decode_args(q, kv_cache, num_pages, page_table, pt_stride, topk_idx, B,
+                                       T, H, K, page_size, scale);
+    if (st != SMLA_OK) return st;
+    if (nsplit < 0 || nsplit > SMLA_MAX_NSPLIT) return SMLA_ERR_INVALID_ARG;
+    if (B == 0 || T == 0 || H == 0) return SMLA_OK;
+    if (o == nullptr || lse == nullptr) return SMLA_ERR_INVALID_ARG;
+    if (!aligned(o, 16) || !aligned(lse, 4)) return SMLA_ERR_MISALIGNED;
+    if (nsplit == 0) nsplit = smla_choose_nsplit(B, T, H, K, 0);
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (nsplit == 1) {
+        PartialParams p = make_params(q, kv_cache, num_pages, page_table, pt_stride, topk_idx, B, T,
+                                      H, K, scale, nsplit);
+        p.o = static_cast<__nv_bfloat16 *>(o);
+        p.lse = lse;
+        return launch_partial<true>(p, s);
+    }
+    PartialParams p{};
+    st = decode_partial_pass(q, kv_cache, num_pages, page_table, pt_stride, topk_idx, B, T, H, K,
+                             scale, nsplit, workspace, workspace_bytes, s, &p);
     if (st != SMLA_OK) return st;
     return launch_combine(p.part_o, p.part_m, p.part_lse, B, T, H, nsplit, o, lse, s);
+}
+
+smla_status smla_decode_partial_ws(const void *q, const void *kv_cache, int64_t num_pages,
+                                   const int32_t *page_table, int pt_stride,
+                                   const int32_t *topk_idx, int B, int T, int H, int K,
+                                   int page_size, float scale, int nsplit, void *workspace,
+                                   size_t workspace_bytes, void *stream) {
+    smla_status st = check_decode_args(q, kv_cache, num_pages, page_table, pt_stride, topk_idx, B,
+                                       T, H, K, page_size, scale);
+    if (st != SMLA_OK) return st;
+    if (nsplit < 2 || nsplit > SMLA_MAX_NSPLIT) return SMLA_ERR_INVALID_ARG;
+    if (B == 0 || T == 0 || H == 0) return SMLA_OK;
+    PartialParams p{};
+    return decode_partial_pass(q, kv_cache, num_pages, page_table, pt_stride, topk_idx, B, T, H, K,
+                               scale, nsplit, workspace, workspace_bytes,
+                               static_cast<cudaStream_t>(stream), &p);
 }
 
 // ---------------------------------------------------------------------------
@@ -661,11 +705,17 @@ smla_status smla_decode_dense(const void *q, const void *kv_cache, int64_t num_p
     if (B == 0 || T == 0 || H == 0) return SMLA_OK;
     if (o == nullptr || lse == nullptr) return SMLA_ERR_INVALID_ARG;
     if (!aligned(o, 16) || !aligned(lse, 4)) return SMLA_ERR_MISALIGNED;
-    const DensePlan d = dense_plan(B, T, H, K, nsplit);
+    DensePlan d = dense_plan(B, T, H, K, nsplit);
+    // Split boundaries on whole pages: every 32-row tile is then half a page
+    // of consecutive cache rows, which the kernel moves by TMA.  Kc rounds up
+    // to 64 positions, and ceil(K / Kc) <= nsplit splits remain.
+    const int kc64 = K > 0 ? ((K + d.nsplit - 1) / d.nsplit + 63) / 64 * 64 : 0;
+    if (K > 0) d.nsplit = (K + kc64 - 1) / kc64;
     if ((long long)B * d.units * d.nsplit > INT_MAX) return SMLA_ERR_INVALID_ARG;
     const cudaStream_t s = static_cast<cudaStream_t>(stream);
     PartialParams p = dense_params(q, kv_cache, num_pages, page_table, pt_stride, seq_lens, B, T,
                                    H, K, scale, d);
+    if (K > 0) p.kc = kc64;
     const int grid = B * d.units * d.nsplit;
     if (d.nsplit == 1) {
         p.o = static_cast<__nv_bfloat16 *>(o);
@@ -761,6 +811,33 @@ smla_status encode_rows128(CUtensorMap *map, const void *base, uint64_t rows, ui
     }
     return SMLA_OK;
 }
+
+}  // namespace
+
+// The latent cache as a 2-D bf16 tensor [num_pages * 64 rows, 576], read in
+// boxes of 32 rows x 64 values with the 128-byte swizzle.
+smla_status encode_cache_tiles(CUtensorMap *map, const void *cache, int64_t num_pages) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (enc == nullptr) {
+        std::snprintf(g_last_error, sizeof g_last_error, "cuTensorMapEncodeTiled unavailable");
+        return SMLA_ERR_CUDA;
+    }
+    const cuuint64_t dims[2] = {(cuuint64_t)smla::kD, (cuuint64_t)num_pages * smla::kPage};
+    const cuuint64_t strides[1] = {(cuuint64_t)smla::kRowBytes};
+    const cuuint32_t box[2] = {64u, (cuuint32_t)smla::TcCfg::kTileRows};
+    const cuuint32_t estr[2] = {1u, 1u};
+    const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(cache), dims,
+                           strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        std::snprintf(g_last_error, sizeof g_last_error, "cuTensorMapEncodeTiled failed: %d", (int)r);
+        return SMLA_ERR_CUDA;
+    }
+    return SMLA_OK;
+}
+
+namespace {
 
 smla_status check_indexer_args(const void *q_index, const float *w, const void *k_index,
                                int64_t num_pages, const int32_t *page_table, int pt_stride,

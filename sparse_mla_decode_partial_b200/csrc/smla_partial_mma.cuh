@@ -14,11 +14,13 @@
 // in order, one partial slot per piece.
 //
 // Warp roles (HG = head groups of 16 rows, the mma M dimension):
-//   warp 4*HG      producer: first resolves the split's index entries to
-//                  physical rows (index loads, then page-table loads, 32 per
-//                  lane in flight) into shared memory, then issues one 1-D
-//                  bulk async copy (TMA engine, 1152 B) per row into a ring of
-//                  NSTAGE tiles of NT rows, each completing on an mbarrier.
+//   warps 4*HG,    producers: every thread of the CTA first resolves the
+//   4*HG+1         split's index entries to physical rows (index loads, then
+//                  page-table loads, a batch in flight at once) into shared
+//                  memory; then the two producer warps take alternate tiles
+//                  and issue one 1-D bulk async copy (TMA engine, 1152 B) per
+//                  row into a ring of NSTAGE tiles of NT rows, each completing
+//                  on an mbarrier.
 //   warps 0..4HG-1 consumers, 4 per head group.  Each warp keeps the Q
 //                  fragments of one quarter of the 576 dims in registers and
 //                  computes that quarter's partial S = Q K^T for all NT rows
@@ -195,7 +197,11 @@ struct MmaCfg {
     static_assert(NT == 16 || NT == 32 || NT == 64, "tile rows");
     static constexpr int kHeads = 16 * HG;
     static constexpr int kComputeWarps = 4 * HG;
-    static constexpr int kThreads = (kComputeWarps + 1) * 32;
+    // Two producer warps take alternate tiles: one warp issues about 22 GB/s
+    // of 1-D bulk copies, and two per CTA (four per SM) keep the TMA engine
+    // near the HBM rate.
+    static constexpr int kProducerWarps = 2;
+    static constexpr int kThreads = (kComputeWarps + kProducerWarps) * 32;
     static constexpr int kSRow = NT + 8;  // floats per S-partial row (32-byte pad: conflict-free float2)
     static constexpr int kStageBytes = NT * kSmemRowBytes;
     static constexpr int kQBytes = kHeads * kSmemRowBytes;
@@ -416,6 +422,7 @@ __global__ void __launch_bounds__(MmaCfg<HG, NT, NSTAGE>::kThreads, MmaCfg<HG, N
     smla_partial_mma_kernel(const PartialParams p) {
     using C = MmaCfg<HG, NT, NSTAGE>;
     static_assert(NT == 32, "the balanced schedule counts 32-row tiles");
+    static_assert(NSTAGE % 2 == 0, "the two producer warps own alternate stages");
     extern __shared__ __align__(128) uint8_t smem[];
 
     const int warp = threadIdx.x >> 5;
@@ -450,11 +457,13 @@ __global__ void __launch_bounds__(MmaCfg<HG, NT, NSTAGE>::kThreads, MmaCfg<HG, N
     }
     __syncthreads();
 
-    if (warp == C::kComputeWarps) {
-        // ============================================================ producer
+    if (warp >= C::kComputeWarps) {
+        // ============================================================ producers
+        const int pw = warp - C::kComputeWarps;  // takes the tiles it with it % 2 == pw
+        const uint32_t bar_prod = 2 + HG;        // named barrier of the producer warps
         const uint64_t policy = l2_policy_evict_first();
         int *rows_s = reinterpret_cast<int *>(smem + C::kOffRows);
-        constexpr int kResolveBatch = HG <= 2 ? 32 : 16;  // loads in flight per lane
+        constexpr int kResolveBatch = HG <= 2 ? 16 : 8;  // loads in flight per lane
         int it = 0;  // tile counter over all of this CTA's items (ring position)
         long long u = item_begin(p, cta);
         WorkItem w;
@@ -463,15 +472,19 @@ __global__ void __launch_bounds__(MmaCfg<HG, NT, NSTAGE>::kThreads, MmaCfg<HG, N
             const int len = w.j1 - w.j0;
             for (int base = 0; base < len; base += kResolveChunk) {
                 const int n = min(kResolveChunk, len - base);
-                __syncwarp();  // rows_s is rewritten below
                 // Resolve the whole chunk before its first copy: index loads,
                 // then page-table loads, a batch per lane in flight at once.
-                if (!first_chunk) resolve_rows<kResolveBatch>(p, w.bt, w.j0, base, n, rows_s, lane, 32);
+                if (!first_chunk) {
+                    named_bar_sync(bar_prod, 32 * C::kProducerWarps);  // rows_s free for rewriting
+                    resolve_rows<kResolveBatch>(p, w.bt, w.j0, base, n, rows_s, 32 * pw + lane,
+                                                32 * C::kProducerWarps);
+                    named_bar_sync(bar_prod, 32 * C::kProducerWarps);  // rows_s complete
+                }
                 first_chunk = false;
-                __syncwarp();
                 // Issue one bulk copy per row (or per padding slot, from the zero row).
                 const int chunk_tiles = (n + NT - 1) / NT;
                 for (int t = 0; t < chunk_tiles; ++t, ++it) {
+                    if ((it & 1) != pw) continue;
                     const int stage = it % NSTAGE;
                     if (it >= NSTAGE) mbar_wait(&empty[stage], ((it / NSTAGE) - 1) & 1, dead);
                     if (lane == 0) mbar_expect_tx(&full[stage], (uint32_t)(NT * kRowBytes));
@@ -503,7 +516,7 @@ __global__ void __launch_bounds__(MmaCfg<HG, NT, NSTAGE>::kThreads, MmaCfg<HG, N
         }
         // Copies still in flight must land before the CTA may exit.
         for (int k = (it > NSTAGE ? it - NSTAGE : 0); k < it; ++k)
-            mbar_wait(&full[k % NSTAGE], (k / NSTAGE) & 1, dead);
+            if ((k & 1) == pw) mbar_wait(&full[k % NSTAGE], (k / NSTAGE) & 1, dead);
         return;
     }
 

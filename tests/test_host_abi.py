@@ -181,12 +181,11 @@ def model(B, T, H, K, sms):
     s_bal = math.ceil(slots / base) + 1
     units = base * -(-K // 32)
     latency_kernel = H <= 32 and math.ceil(K / s_bal) <= 64
-    if 2 <= s_bal <= s_max and units >= 4 * slots and not latency_kernel:
+    if H <= 32 and 2 <= s_bal <= s_max and units >= 4 * slots and not latency_kernel:
         pieces = base + slots
         t = 48.0 * pieces / slots + units * 32.0 / slots
         t += 0.5 * pieces * H * (514 * 4.0) * 2.0 / 1152 / slots
-        margin = 0.0 if H > 32 else 0.15   # the tcgen05 kernel overlaps item boundaries
-        if t < best * (1 - margin):
+        if t < best * (1 - 0.15):
             best_s = s_bal
     return best_s
 
