@@ -559,10 +559,39 @@ def side_indexer(h, steps, warmup, peaks):
     return rec
 
 
+def run_indexer_headline(args, world, rank, local):
+    """`--workload indexer_mixed`: the top-k indexer as the timed step (the
+    profiling recipe's launch list and captures of the indexer kernels use
+    it); the line carries the indexer record's figures."""
+    import torch
+    from sparse_mla_decode_partial_b200 import build
+    build.build()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    h = Harness(dev)
+    rec = side_indexer(h, args.steps, args.warmup, load_peaks())
+    if rank != 0:
+        return None
+    from sparse_mla_decode_partial_b200 import workloads
+    w = workloads.indexer_mixed()
+    us = rec["us_per_call"]
+    return {"metric": "top-k indexer query-tokens/s", "value": rec["q_tok_s"],
+            "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(us * 1e-3, 6), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded index queries, keys "
+            "and weights)", "config": {"workload": "indexer_mixed", "shape": rec["shape"],
+                                       "l2": "flushed before every step: 256 MB write then 256 MB read",
+                                       "parallelism": "single GPU"},
+            "roofline": rec["roofline"], "clocks": rec["clocks"], "gpu_launches": rec["gpu_launches"],
+            "indexer": rec}
+
+
 def run_ours(args, world, rank, local):
     import torch
     from sparse_mla_decode_partial_b200 import binding, build
 
+    if args.workload == "indexer_mixed":
+        return run_indexer_headline(args, world, rank, local)
     build.build()
     lib = binding.lib()
     dev = torch.device("cuda", local)
@@ -745,11 +774,45 @@ def run_ours(args, world, rank, local):
     return line
 
 
+def indexer_cpu_baseline(seconds: float):
+    """The fp64 indexer oracle on this host's cores over the first query
+    tokens of the indexer workload (one token at a time until the time is
+    spent)."""
+    import numpy as np
+    import torch
+    from oracle import indexer as ix_oracle
+    from sparse_mla_decode_partial_b200 import workloads
+    w = workloads.indexer_mixed()
+    bits = lambda t: t.contiguous().view(torch.int16).numpy().view(np.uint16)
+    q, k = bits(w.q_index), bits(w.k_index)
+    wt, pt, nv = w.w.numpy(), w.page_table.numpy(), w.n_vis.numpy()
+    done, keys = 0, 0
+    t0 = time.perf_counter()
+    while done < w.B and time.perf_counter() - t0 < seconds:
+        b = done
+        ix_oracle.topk(q[b:b + 1], wt[b:b + 1], k, pt[b:b + 1], nv[b:b + 1], w.K)
+        keys += int(nv[b, 0])
+        done += 1
+    el = time.perf_counter() - t0
+    return {"value": done / el, "unit": UNIT, "cores": __import__("os").cpu_count(),
+            "kind": "oracle", "sample": f"the first {done} of {w.B} query tokens ({keys} keys)",
+            "us_per_token": el / done * 1e6}
+
+
 def run_reference(args, world, rank):
     """The oracle (CPU, fp64) as the reference arm, on this host's cores."""
     if rank != 0:
         return None
     from sparse_mla_decode_partial_b200 import workloads
+    if args.workload == "indexer_mixed":
+        res = indexer_cpu_baseline(max(2.0, args.cpu_seconds))
+        return {"metric": "top-k indexer query-tokens/s", "value": round(res["value"], 3),
+                "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": round(1e3 / res["value"], 3), "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "config": {"workload": "indexer_mixed"}, "impl": "reference", "cpu_baseline": res,
+                "e2e": {"value": round(res["value"], 3), "unit": UNIT, "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
     w = workloads.WORKLOADS[args.workload]()
     seconds = max(2.0, args.cpu_seconds)
     t_all = time.perf_counter()
@@ -783,7 +846,7 @@ def main(argv=None):
         return 0
     world, rank, local = dist_init()
     line = run_ours(args, world, rank, local)
-    if rank == 0 and line is not None:
+    if rank == 0 and line is not None and args.workload != "indexer_mixed":
         from sparse_mla_decode_partial_b200 import workloads
         line["cpu_baseline"] = cpu_baseline(workloads.WORKLOADS[args.workload](),
                                             args.cpu_seconds)

@@ -22,10 +22,12 @@
 // epilogue thread that owns a key reduces over its heads without talking to
 // any other thread.  Warp roles: warp 0 TMA producer, warp 1 TMEM owner and
 // MMA issuer, warps 4-7 epilogue (TMEM lanes 0-127).
-// Selection (smla_ix_select_kernel): one CTA per query token; three radix
-// passes (11, 11, 10 bits) over an order-preserving key of the fp32 score
-// find the K-th largest score, then one ascending scan writes the positions
-// above it and the first ones (by position) equal to it.
+// Selection (smla_ix_select_kernel): one CTA per query token; radix passes
+// (8, 12, 12 bits) over an order-preserving key of the fp32 score find the
+// K-th largest score -- the first over all scores, the others over the
+// crossing bucket's candidates in shared memory -- then ordered scans of two
+// position bitmaps write the positions above it and the first ones (by
+// position) equal to it.
 #pragma once
 
 #include <cuda.h>
@@ -402,44 +404,44 @@ __device__ __forceinline__ uint32_t ix_key(float f) {
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// Shared memory of the selection kernel: the digit histogram, the crossing
-// bucket's candidates and two bitmaps over the visible positions (selected,
-// equal to the threshold).
-constexpr int kIxCandCap = 8192;   // candidates of the crossing bucket kept in shared memory
+// Shared memory of the selection kernel: the histograms (per-warp private
+// ones for the first digit), the crossing bucket's candidates and two bitmaps
+// over the visible positions (selected, equal to the threshold).
+constexpr int kIxCandCap = 8192;    // candidates of the crossing bucket kept in shared memory
+constexpr int kIxHistBytes = 32 * 256 * 4;  // 32 warps x 256 bins, or one 4096-bin histogram
 __host__ __device__ constexpr int ix_select_smem_bytes(int max_n) {
-    return 2048 * 4 + kIxCandCap * 8 + 2 * 4 * ((max_n + 31) / 32);
+    return kIxHistBytes + kIxCandCap * 8 + 2 * 4 * ((max_n + 31) / 32);
 }
-constexpr int kIxSelectMaxN = (232448 - 2048 * 4 - kIxCandCap * 8 - 1024) / 8 * 32;
+constexpr int kIxSelectMaxN = (232448 - kIxHistBytes - kIxCandCap * 8 - 1024) / 8 * 32;
 
-// Histogram of digit (key >> shift) & (nb - 1) over the keys whose bits above
-// the digit equal `prefix`; keys from global scores (8 loads in flight per
-// thread) or from the candidate list.
-__device__ __forceinline__ void ix_hist_add(unsigned *hist, uint32_t key, bool match, uint32_t d) {
+// Warp-aggregated increment of hist[d] (lanes with the same digit add once).
+__device__ __forceinline__ void ix_hist_add(unsigned *hist, bool match, uint32_t d) {
     const uint32_t peers = __match_any_sync(__activemask(), match ? d : 0xffffffffu);
     if (match && (__ffs(peers) - 1) == (int)(threadIdx.x & 31)) atomicAdd(&hist[d], (unsigned)__popc(peers));
 }
 
 // Bucket of the histogram (nb bins) holding the need-th largest key counted
 // from the top: writes (bucket, keys above it) to found[]; returns the total.
+// Thread i sums bins nb-1-i*per .. nb-per-i*per (per = nb / blockDim.x).
 __device__ __forceinline__ int ix_find_bucket(const unsigned *hist, int nb, int need, int *scratch,
                                               int *found) {
-    int v = 0, b_hi = -1, b_lo = -1;
-    if (2 * (int)threadIdx.x < nb) {
-        b_hi = nb - 1 - 2 * threadIdx.x;
-        b_lo = b_hi - 1;
-        v = (int)hist[b_hi] + (b_lo >= 0 ? (int)hist[b_lo] : 0);
-    }
+    const int per = (nb + blockDim.x - 1) / blockDim.x;
+    const int top = nb - 1 - (int)threadIdx.x * per;
+    int v = 0;
+    for (int k = 0; k < per; ++k)
+        if (top - k >= 0) v += (int)hist[top - k];
     int total;
     const int incl = ix_block_scan(v, scratch, &total);
-    const int excl = incl - v;
-    if (b_hi >= 0 && excl < need && need <= incl) {
-        const int h = (int)hist[b_hi];
-        if (excl + h >= need) {
-            found[0] = b_hi;
-            found[1] = excl;
-        } else {
-            found[0] = b_lo;
-            found[1] = excl + h;
+    int excl = incl - v;
+    if (excl < need && need <= incl) {
+        for (int k = 0; k < per && top - k >= 0; ++k) {
+            const int h = (int)hist[top - k];
+            if (excl + h >= need) {
+                found[0] = top - k;
+                found[1] = excl;
+                break;
+            }
+            excl += h;
         }
     }
     __syncthreads();
@@ -467,24 +469,27 @@ __device__ __forceinline__ int ix_bitmap_scan(const uint32_t *bits, int words, i
     return total;
 }
 
-// One CTA per query token.  Pass A (global): histogram of the top 11 bits of
-// the key -> the crossing bucket d0.  Pass B (global): positions with a digit
-// above d0 are selected (bitmap); those in d0 become candidates in shared
-// memory.  Two radix passes over the candidates give the exact threshold key
-// and how many keys equal to it are taken; the first of those by position are
-// found by an ordered scan of an "equal" bitmap, and an ordered scan of the
-// selection bitmap writes the output.  If d0 holds more than kIxCandCap
-// keys, the two finer passes and the marking read the global scores instead.
+// One CTA per query token.  Pass A (global): histogram of the top 8 bits of
+// the key, one private histogram per warp (scores crowd into few buckets;
+// shared bins would serialise the warps) -> the crossing bucket d0.  Pass B
+// (global): positions with a digit above d0 are selected (bitmap); those in
+// d0 become candidates in shared memory.  Two 12-bit radix passes over the
+// candidates give the exact threshold key and how many keys equal to it are
+// taken; the first of those by position are found by an ordered scan of an
+// "equal" bitmap, and an ordered scan of the selection bitmap writes the
+// output.  If d0 holds more than kIxCandCap keys, the finer passes and the
+// marking read the global scores instead.
 __global__ void __launch_bounds__(kIxSelectThreads) smla_ix_select_kernel(const IndexerParams p) {
     extern __shared__ __align__(16) uint8_t ix_smem[];
     unsigned *hist = reinterpret_cast<unsigned *>(ix_smem);
-    uint32_t *cand_key = reinterpret_cast<uint32_t *>(ix_smem + 2048 * 4);
-    int *cand_pos = reinterpret_cast<int *>(ix_smem + 2048 * 4 + kIxCandCap * 4);
-    uint32_t *sel_bits = reinterpret_cast<uint32_t *>(ix_smem + 2048 * 4 + kIxCandCap * 8);
+    uint32_t *cand_key = reinterpret_cast<uint32_t *>(ix_smem + kIxHistBytes);
+    int *cand_pos = reinterpret_cast<int *>(ix_smem + kIxHistBytes + kIxCandCap * 4);
+    uint32_t *sel_bits = reinterpret_cast<uint32_t *>(ix_smem + kIxHistBytes + kIxCandCap * 8);
     __shared__ int scratch[33];
     __shared__ int found[2];
     __shared__ int n_cand;
     const int u = blockIdx.x, tid = threadIdx.x, nt = blockDim.x;
+    const int warp = tid >> 5, lane = tid & 31;
     const int n = ix_visible(p, u), K = p.K;
     const int words = (n + 31) / 32;
     uint32_t *eq_bits = sel_bits + words;
@@ -492,12 +497,13 @@ __global__ void __launch_bounds__(kIxSelectThreads) smla_ix_select_kernel(const 
     int *out = p.out + (size_t)u * K;
     constexpr int kIlp = 8;
 
-    for (int i = tid; i < 2048; i += nt) hist[i] = 0;
+    for (int i = tid; i < kIxHistBytes / 4; i += nt) hist[i] = 0;
     for (int i = tid; i < 2 * words; i += nt) sel_bits[i] = 0;
     if (tid == 0) n_cand = 0;
     __syncthreads();
 
-    // ---- pass A: top 11 bits
+    // ---- pass A: top 8 bits into this warp's own 256 bins
+    unsigned *my_hist = hist + warp * 256;
     for (int base = 0; base < n; base += nt * kIlp) {
         uint32_t key[kIlp];
 #pragma unroll
@@ -506,11 +512,18 @@ __global__ void __launch_bounds__(kIxSelectThreads) smla_ix_select_kernel(const 
             key[j] = s < n ? ix_key(__ldg(sc + s)) : 0u;
         }
 #pragma unroll
-        for (int j = 0; j < kIlp; ++j) ix_hist_add(hist, key[j], key[j] != 0u, key[j] >> 21);
+        for (int j = 0; j < kIlp; ++j) ix_hist_add(my_hist, key[j] != 0u, key[j] >> 24);
+    }
+    __syncthreads();
+    // fold the 32 private histograms into bins 0..255 of warp 0's
+    if (tid < 256) {
+        unsigned sum = 0;
+        for (int w = 0; w < 32; ++w) sum += hist[w * 256 + tid];
+        hist[tid] = sum;
     }
     __syncthreads();
     int need = K;
-    const int valid = ix_find_bucket(hist, 2048, need, scratch, found);
+    const int valid = ix_find_bucket(hist, 256, need, scratch, found);
     const bool take_all = valid <= K;
     const uint32_t d0 = take_all ? 0u : (uint32_t)found[0];
     if (!take_all) need -= found[1];
@@ -526,12 +539,17 @@ __global__ void __launch_bounds__(kIxSelectThreads) smla_ix_select_kernel(const 
 #pragma unroll
         for (int j = 0; j < kIlp; ++j) {
             const int s = base + j * nt + tid;
-            if (key[j] == 0u) continue;
-            const uint32_t d = key[j] >> 21;
-            if (take_all || d > d0) {
-                atomicOr(&sel_bits[s >> 5], 1u << (s & 31));
-            } else if (d == d0) {
-                const int c = atomicAdd(&n_cand, 1);
+            const uint32_t d = key[j] >> 24;
+            const bool above = key[j] != 0u && (take_all || d > d0);
+            const bool cand = key[j] != 0u && !take_all && d == d0;
+            if (above) atomicOr(&sel_bits[s >> 5], 1u << (s & 31));
+            // warp-aggregated append of the candidates
+            const uint32_t cm = __ballot_sync(0xffffffffu, cand);
+            int slot0 = 0;
+            if (lane == 0 && cm) slot0 = atomicAdd(&n_cand, __popc(cm));
+            slot0 = __shfl_sync(0xffffffffu, slot0, 0);
+            if (cand) {
+                const int c = slot0 + __popc(cm & ((1u << lane) - 1u));
                 if (c < kIxCandCap) {
                     cand_key[c] = key[j];
                     cand_pos[c] = s;
@@ -542,20 +560,19 @@ __global__ void __launch_bounds__(kIxSelectThreads) smla_ix_select_kernel(const 
     __syncthreads();
 
     if (!take_all) {
-        // ---- the two finer digits, over the candidates (or the global scores)
+        // ---- the two finer 12-bit digits, over the candidates (or the global scores)
         const int m = n_cand;
         const bool in_smem = m <= kIxCandCap;
         uint32_t prefix = d0;
 #pragma unroll
         for (int pass = 0; pass < 2; ++pass) {
-            const int shift = pass == 0 ? 10 : 0, width = pass == 0 ? 11 : 10, nb = 1 << width;
-            const int hi_shift = shift + width;
-            for (int i = tid; i < 2048; i += nt) hist[i] = 0;
+            const int shift = pass == 0 ? 12 : 0, hi_shift = shift + 12;
+            for (int i = tid; i < 4096; i += nt) hist[i] = 0;
             __syncthreads();
             if (in_smem) {
                 for (int c = tid; c < ((m + 31) & ~31); c += nt) {
                     const uint32_t key = c < m ? cand_key[c] : 0u;
-                    ix_hist_add(hist, key, c < m && (key >> hi_shift) == prefix, (key >> shift) & (nb - 1));
+                    ix_hist_add(hist, c < m && (key >> hi_shift) == prefix, (key >> shift) & 4095u);
                 }
             } else {
                 for (int base = 0; base < n; base += nt * kIlp) {
@@ -567,13 +584,13 @@ __global__ void __launch_bounds__(kIxSelectThreads) smla_ix_select_kernel(const 
                     }
 #pragma unroll
                     for (int j = 0; j < kIlp; ++j)
-                        ix_hist_add(hist, key[j], key[j] != 0u && (key[j] >> hi_shift) == prefix,
-                                    (key[j] >> shift) & (nb - 1));
+                        ix_hist_add(hist, key[j] != 0u && (key[j] >> hi_shift) == prefix,
+                                    (key[j] >> shift) & 4095u);
                 }
             }
             __syncthreads();
-            ix_find_bucket(hist, nb, need, scratch, found);
-            prefix = (prefix << width) | (uint32_t)found[0];
+            ix_find_bucket(hist, 4096, need, scratch, found);
+            prefix = (prefix << 12) | (uint32_t)found[0];
             need -= found[1];
             __syncthreads();
         }
@@ -589,7 +606,7 @@ __global__ void __launch_bounds__(kIxSelectThreads) smla_ix_select_kernel(const 
         } else {
             for (int s = tid; s < n; s += nt) {
                 const uint32_t key = ix_key(__ldg(sc + s));
-                if ((key >> 21) != d0) continue;  // the bits above d0 are set already
+                if (key == 0u || (key >> 24) != d0) continue;  // the bits above d0 are set already
                 if (key > thresh) atomicOr(&sel_bits[s >> 5], 1u << (s & 31));
                 else if (key == thresh) atomicOr(&eq_bits[s >> 5], 1u << (s & 31));
             }
