@@ -41,7 +41,7 @@ namespace smla {
 constexpr int kIxDim = 128;        // index-key width (bf16 values)
 constexpr int kIxTile = 128;       // keys per unit: the MMA's M
 constexpr int kIxMaxHeads = 64;    // index heads: the MMA's N (padded to 16, 32, 64)
-constexpr int kIxStages = 4;       // key tiles in flight per CTA
+constexpr int kIxStages = 5;       // key tiles in flight per CTA
 constexpr int kIxSelectThreads = 1024;
 
 struct IndexerParams {
@@ -135,9 +135,13 @@ struct IxUnit {
     int tok, tile, n, pg0, pg1;
 };
 
-__device__ __forceinline__ IxUnit ix_unit(const IndexerParams &p, long long unit) {
+// `hint`: a token at or before the unit's (units are walked in order, and
+// consecutive units rarely change token, so the advance is a step or two of
+// cached loads).
+__device__ __forceinline__ IxUnit ix_unit(const IndexerParams &p, long long unit, int hint) {
     IxUnit m;
-    m.tok = ix_token_of(p, unit);
+    m.tok = hint;
+    while (__ldg(p.tile_start + m.tok + 1) <= unit) ++m.tok;
     m.tile = (int)(unit - __ldg(p.tile_start + m.tok));
     m.n = ix_visible(p, m.tok);
     const int *pt_b = p.page_table + (size_t)(m.tok / p.T) * p.pt_stride;
@@ -265,10 +269,12 @@ __global__ void __launch_bounds__(IxCfg<NPAD>::kThreads, 1)
             const uint64_t keep = l2_policy_evict_last();   // a query is read again per tile
             const uint64_t once = l2_policy_evict_first();  // keys are read once
             int prev_tok = -1, changes = -1;
+            int hint = ix_token_of(p, u_begin);
             long long i = 0;
             for (long long ub = u_begin; ub < u_end; ub += 32) {
                 const int cnt = (int)min(32ll, u_end - ub);
-                const IxUnit mine = ix_unit(p, min(ub + lane, u_end - 1));
+                const IxUnit mine = ix_unit(p, min(ub + lane, u_end - 1), hint);
+                hint = __shfl_sync(0xffffffffu, mine.tok, cnt - 1);
                 for (int k = 0; k < cnt; ++k, ++i) {
                     const IxUnit m = ix_unit_from(mine, k);
                     if (lane == 0) {
@@ -351,10 +357,12 @@ __global__ void __launch_bounds__(IxCfg<NPAD>::kThreads, 1)
         const int row = 32 * q4 + lane;          // key of the tile
         const int et = threadIdx.x - 128;        // 0 .. 127
         int w_tok = -1;
+        int hint = u_begin < u_end ? ix_token_of(p, u_begin) : 0;
         long long i = 0;
         for (long long ub = u_begin; ub < u_end; ub += 32) {
             const int cnt = (int)min(32ll, u_end - ub);
-            const IxUnit mine = ix_unit(p, min(ub + lane, u_end - 1));
+            const IxUnit mine = ix_unit(p, min(ub + lane, u_end - 1), hint);
+            hint = __shfl_sync(0xffffffffu, mine.tok, cnt - 1);
             for (int k = 0; k < cnt; ++k, ++i) {
                 const IxUnit m = ix_unit_from(mine, k);
                 if (m.tok != w_tok) {  // the token's head weights (0 past HI)
