@@ -510,12 +510,14 @@ def side_indexer(h, steps, warmup, peaks):
     ws = torch.empty(binding.indexer_workspace_bytes(B, T, max_n), dtype=torch.uint8, device=h.dev)
     out = torch.empty((B, T, K), dtype=torch.int32, device=h.dev)
     sc = torch.empty((B, T, max_n), dtype=torch.float32, device=h.dev)
+    sel_ws = torch.empty(binding.indexer_select_workspace_bytes(B, T, max_n), dtype=torch.uint8,
+                         device=h.dev)
     common = (w.q_index.data_ptr(), w.w.data_ptr(), w.k_index.data_ptr(), w.num_pages,
               w.page_table.data_ptr(), w.pt_stride, w.n_vis.data_ptr(), B, T, HI, max_n)
 
     def topk():
         return lib.smla_indexer_topk(*common, K, 64, ws.data_ptr(), ws.numel(), out.data_ptr(),
-                                     sptr), 3
+                                     sptr), 5
 
     def scores():
         return lib.smla_indexer_scores(*common, 64, ws.data_ptr(), ws.numel(), sc.data_ptr(),
@@ -523,7 +525,7 @@ def side_indexer(h, steps, warmup, peaks):
 
     def select():
         return lib.smla_indexer_select(sc.data_ptr(), w.n_vis.data_ptr(), B, T, max_n, K,
-                                       out.data_ptr(), sptr), 1
+                                       sel_ws.data_ptr(), sel_ws.numel(), out.data_ptr(), sptr), 3
     h.warm([topk, scores, select], warmup)
     sampler = ClockSampler(h.dev.index)
     with sampler:
@@ -554,7 +556,7 @@ def side_indexer(h, steps, warmup, peaks):
                                 "entries, queries, weights and lengths, read once"},
            "whole_call_frac_of_hbm": round(nbytes / (us * 1e-6) / 1e9 / hbm_peak, 4),
            "gpu_launches": launches, "clocks": sampler.summary()}
-    del w, ws, sc
+    del w, ws, sc, sel_ws
     torch.cuda.empty_cache()
     return rec
 

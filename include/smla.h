@@ -380,14 +380,21 @@ smla_status smla_selftest_wait_timeout(unsigned long long limit_ns, void *stream
  * smla_check_device).  Scores that are NaN are not candidates either.
  *
  * smla_indexer_topk runs both steps; its workspace must hold
- * smla_indexer_workspace_bytes(B, T, max_n) bytes (a per-token tile plan and
- * the fp32 scores).  The two steps are also exported:
+ * smla_indexer_workspace_bytes(B, T, max_n) bytes (a per-token tile plan,
+ * the fp32 scores and the selection scratch).  The two steps are also
+ * exported:
  *   smla_indexer_scores writes I(s) into scores [B, T, max_n] (fp32, row
  *     stride max_n) for every visible s; a position that is not a candidate
  *     gets NaN; entries at s >= n_vis are not written.  Its workspace needs
- *     only the tile plan: smla_indexer_workspace_bytes(B, T, 0) bytes.
+ *     only the tile plan, which smla_indexer_workspace_bytes(B, T, 0) bytes
+ *     cover.
  *   smla_indexer_select applies the selection rule to given scores of that
- *     layout (NaN = not a candidate; -0 and +0 are equal).
+ *     layout (NaN = not a candidate; -0 and +0 are equal).  Its workspace
+ *     must hold smla_indexer_select_workspace_bytes(B, T, max_n) bytes: per
+ *     token a 16 KiB digit histogram, a position bitmap and a candidate list
+ *     of max_n positions.  Scratch only: nothing carries over between calls.
+ * Workspaces are device memory, 16-B aligned, owned by the caller and in use
+ * until the call's work on `stream` completes.
  * Asynchronous on `stream`; errors as for the decode entry points.
  */
 #define SMLA_INDEXER_DIM 128
@@ -395,6 +402,7 @@ smla_status smla_selftest_wait_timeout(unsigned long long limit_ns, void *stream
 #define SMLA_INDEXER_MAX_TOKENS 1048576
 #define SMLA_INDEXER_MAX_N 524288   /* visible positions per query token */
 size_t smla_indexer_workspace_bytes(int B, int T, int max_n);
+size_t smla_indexer_select_workspace_bytes(int B, int T, int max_n);
 smla_status smla_indexer_topk(const void *q_index, const float *w, const void *k_index,
                               int64_t num_pages, const int32_t *page_table, int pt_stride,
                               const int32_t *n_vis, int B, int T, int HI, int max_n, int K,
@@ -406,7 +414,8 @@ smla_status smla_indexer_scores(const void *q_index, const float *w, const void 
                                 int page_size, void *workspace, size_t workspace_bytes,
                                 float *scores, void *stream);
 smla_status smla_indexer_select(const float *scores, const int32_t *n_vis, int B, int T,
-                                int max_n, int K, int32_t *topk_idx, void *stream);
+                                int max_n, int K, void *workspace, size_t workspace_bytes,
+                                int32_t *topk_idx, void *stream);
 
 /* Static text for a status code. */
 const char *smla_status_string(smla_status status);

@@ -53,7 +53,8 @@ SIGNATURES = {
                                _P]),
     "smla_indexer_scores": (_I, [_P, _P, _P, _I64, _P, _I, _P, _I, _I, _I, _I, _I, _P, _SZ, _P,
                                  _P]),
-    "smla_indexer_select": (_I, [_P, _P, _I, _I, _I, _I, _P, _P]),
+    "smla_indexer_select": (_I, [_P, _P, _I, _I, _I, _I, _P, _SZ, _P, _P]),
+    "smla_indexer_select_workspace_bytes": (_SZ, [_I, _I, _I]),
     "smla_selftest_wait_timeout": (_I, [ctypes.c_ulonglong, _P]),
     "smla_check_device": (_I, [_I, ctypes.POINTER(ctypes.c_ulonglong), _P]),
     "smla_status_string": (ctypes.c_char_p, [_I]),
@@ -351,6 +352,10 @@ def indexer_workspace_bytes(B: int, T: int, max_n: int) -> int:
     return int(lib().smla_indexer_workspace_bytes(B, T, max_n))
 
 
+def indexer_select_workspace_bytes(B: int, T: int, max_n: int) -> int:
+    return int(lib().smla_indexer_select_workspace_bytes(B, T, max_n))
+
+
 def _indexer_args(q_index, w, k_index, page_table, n_vis):
     _need(q_index, torch.bfloat16, "q_index")
     dev = q_index.device
@@ -411,7 +416,7 @@ def indexer_scores(q_index, w, k_index, page_table, n_vis, max_n: int, *, scores
     return scores
 
 
-def indexer_select(scores, n_vis, K: int, *, out=None, stream=None):
+def indexer_select(scores, n_vis, K: int, *, out=None, workspace=None, stream=None):
     """The indexer's selection rule on given scores fp32 [B, T, max_n]."""
     _need(scores, torch.float32, "scores")
     dev = scores.device
@@ -420,7 +425,12 @@ def indexer_select(scores, n_vis, K: int, *, out=None, stream=None):
     if out is None:
         out = torch.empty((B, T, K), dtype=torch.int32, device=dev)
     _need(out, torch.int32, "out", dev)
-    _check(lib().smla_indexer_select(_ptr(scores), _ptr(n_vis), B, T, max_n, int(K), _ptr(out),
+    if workspace is None:
+        workspace = torch.empty(max(16, indexer_select_workspace_bytes(B, T, max_n)),
+                                dtype=torch.uint8, device=dev)
+    _need(workspace, torch.uint8, "workspace", dev)
+    _check(lib().smla_indexer_select(_ptr(scores), _ptr(n_vis), B, T, max_n, int(K),
+                                     _ptr(workspace), workspace.numel(), _ptr(out),
                                      _stream(stream)), "smla_indexer_select")
     return out
 

@@ -768,7 +768,7 @@ smla_status smla_check_device(int clear, unsigned long long *n_bad_index, void *
 // Top-k indexer (see include/smla.h and smla_indexer.cuh).
 }  // extern "C"
 
-static_assert(SMLA_INDEXER_MAX_N <= smla::kIxSelectMaxN, "selection bitmaps must fit shared memory");
+static_assert(smla::ix_finish_smem_bytes(SMLA_INDEXER_MAX_N) <= 232448, "selection bitmaps must fit shared memory");
 
 namespace {
 
@@ -914,8 +914,19 @@ smla_status launch_ix_scores(const void *q_index, const float *w, const void *k_
     return e == cudaSuccess ? SMLA_OK : cuda_fail(e);
 }
 
+// Selection scratch: [hist | meta] (cleared per call), the position bitmap
+// and the candidate list.
+size_t ix_select_zeroed_bytes(int B, int T) {
+    return (size_t)B * T * (smla::kIxSelBins * sizeof(unsigned) + sizeof(smla::IxSelMeta));
+}
+size_t ix_select_bytes(int B, int T, int max_n) {
+    const size_t bt = (size_t)B * T, words = ((size_t)max_n + 31) / 32;
+    return round256(ix_select_zeroed_bytes(B, T)) + round256(bt * words * sizeof(uint32_t)) +
+           round256(bt * max_n * sizeof(uint2));
+}
+
 smla_status launch_ix_select(const float *scores, long long stride, const int32_t *n_vis, int B,
-                             int T, int max_n, int K, int32_t *out, cudaStream_t st) {
+                             int T, int max_n, int K, void *workspace, int32_t *out, cudaStream_t st) {
     smla::IndexerParams p{};
     p.n_vis = n_vis;
     p.BT = B * T;
@@ -925,11 +936,52 @@ smla_status launch_ix_select(const float *scores, long long stride, const int32_
     p.scores = const_cast<float *>(scores);
     p.score_stride = stride;
     p.out = out;
-    const void *fn = reinterpret_cast<const void *>(&smla::smla_ix_select_kernel);
-    cudaError_t e = ensure_smem_attr(fn, smla::ix_select_smem_bytes(smla::kIxSelectMaxN));
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    const size_t bt = (size_t)B * T;
+    p.sel_hist = reinterpret_cast<unsigned *>(ws);
+    p.sel_meta = reinterpret_cast<smla::IxSelMeta *>(ws + bt * smla::kIxSelBins * sizeof(unsigned));
+    p.sel_words = (max_n + 31) / 32;
+    const size_t off_bits = round256(ix_select_zeroed_bytes(B, T));
+    p.sel_bits = reinterpret_cast<uint32_t *>(ws + off_bits);
+    p.sel_cand = reinterpret_cast<uint2 *>(ws + off_bits + round256(bt * p.sel_words * sizeof(uint32_t)));
+    p.sel_chunks = (max_n + smla::kIxSelChunk - 1) / smla::kIxSelChunk;
+    // The chain: clear (stream-ordered after whatever wrote the scores), then
+    // hist, mark and finish, each allowed to start early and waiting on its
+    // predecessor in-kernel.
+    cudaLaunchConfig_t cfg = {};
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e;
+    if (max_n > 0) {
+        const long long n16 = (long long)(ix_select_zeroed_bytes(B, T) / 16);
+        const long long blocks = std::min<long long>((n16 + 255) / 256, 4ll * current_device_sms());
+        smla::smla_ix_clear_kernel<<<(unsigned)blocks, 256, 0, st>>>(reinterpret_cast<uint4 *>(ws), n16);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(e);
+        cfg.gridDim = dim3((unsigned)((long long)p.BT * p.sel_chunks));
+        cfg.blockDim = dim3(smla::kIxSelThreads);
+        cfg.dynamicSmemBytes = 0;
+        e = cudaLaunchKernelEx(&cfg, smla::smla_ix_hist_kernel, p);
+        if (e != cudaSuccess) return cuda_fail(e);
+        e = ensure_smem_attr(reinterpret_cast<const void *>(&smla::smla_ix_mark_kernel),
+                             smla::kIxMarkSmemBytes);
+        if (e != cudaSuccess) return cuda_fail(e);
+        cfg.dynamicSmemBytes = smla::kIxMarkSmemBytes;
+        e = cudaLaunchKernelEx(&cfg, smla::smla_ix_mark_kernel, p);
+        if (e != cudaSuccess) return cuda_fail(e);
+    }
+    e = ensure_smem_attr(reinterpret_cast<const void *>(&smla::smla_ix_finish_kernel),
+                         smla::ix_finish_smem_bytes(SMLA_INDEXER_MAX_N));
     if (e != cudaSuccess) return cuda_fail(e);
-    smla::smla_ix_select_kernel<<<B * T, smla::kIxSelectThreads, smla::ix_select_smem_bytes(max_n), st>>>(p);
-    e = cudaGetLastError();
+    cfg.gridDim = dim3((unsigned)p.BT);
+    cfg.blockDim = dim3(smla::kIxFinishThreads);
+    cfg.dynamicSmemBytes = smla::ix_finish_smem_bytes(max_n);
+    e = cudaLaunchKernelEx(&cfg, smla::smla_ix_finish_kernel, p);
+    if (e == cudaSuccess) e = cudaGetLastError();
     return e == cudaSuccess ? SMLA_OK : cuda_fail(e);
 }
 
@@ -939,7 +991,13 @@ extern "C" {
 
 size_t smla_indexer_workspace_bytes(int B, int T, int max_n) {
     if (B < 0 || T < 0 || max_n < 0) return 0;
-    return ix_plan_bytes(B, T) + round256((size_t)B * T * max_n * sizeof(float));
+    return ix_plan_bytes(B, T) + round256((size_t)B * T * max_n * sizeof(float)) +
+           ix_select_bytes(B, T, max_n);
+}
+
+size_t smla_indexer_select_workspace_bytes(int B, int T, int max_n) {
+    if (B < 0 || T < 0 || max_n < 0) return 0;
+    return ix_select_bytes(B, T, max_n);
 }
 
 smla_status smla_indexer_scores(const void *q_index, const float *w, const void *k_index,
@@ -962,14 +1020,18 @@ smla_status smla_indexer_scores(const void *q_index, const float *w, const void 
 }
 
 smla_status smla_indexer_select(const float *scores, const int32_t *n_vis, int B, int T, int max_n,
-                                int K, int32_t *topk_idx, void *stream) {
+                                int K, void *workspace, size_t workspace_bytes, int32_t *topk_idx,
+                                void *stream) {
     if (B < 0 || T < 0 || max_n < 0 || K < 1) return SMLA_ERR_INVALID_ARG;
     if (max_n > SMLA_INDEXER_MAX_N) return SMLA_ERR_UNSUPPORTED;
     if (B == 0 || T == 0) return SMLA_OK;
     if ((long long)B * T > SMLA_INDEXER_MAX_TOKENS) return SMLA_ERR_UNSUPPORTED;
     if (!n_vis || !topk_idx || (max_n > 0 && !scores)) return SMLA_ERR_INVALID_ARG;
     if (!aligned(n_vis, 4) || !aligned(topk_idx, 4) || !aligned(scores, 4)) return SMLA_ERR_MISALIGNED;
-    return launch_ix_select(scores, max_n, n_vis, B, T, max_n, K, topk_idx,
+    if (workspace_bytes < ix_select_bytes(B, T, max_n)) return SMLA_ERR_WORKSPACE_TOO_SMALL;
+    if (workspace == nullptr) return SMLA_ERR_INVALID_ARG;
+    if (!aligned(workspace, 16)) return SMLA_ERR_MISALIGNED;
+    return launch_ix_select(scores, max_n, n_vis, B, T, max_n, K, workspace, topk_idx,
                             static_cast<cudaStream_t>(stream));
 }
 
@@ -992,10 +1054,11 @@ smla_status smla_indexer_topk(const void *q_index, const float *w, const void *k
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     int *plan = reinterpret_cast<int *>(ws);
     float *scores = reinterpret_cast<float *>(ws + ix_plan_bytes(B, T));
+    void *sel_ws = ws + ix_plan_bytes(B, T) + round256((size_t)B * T * max_n * sizeof(float));
     st = launch_ix_scores(q_index, w, k_index, num_pages, page_table, pt_stride, n_vis, B, T, HI,
                           max_n, plan, scores, max_n, s);
     if (st != SMLA_OK) return st;
-    return launch_ix_select(scores, max_n, n_vis, B, T, max_n, K, topk_idx, s);
+    return launch_ix_select(scores, max_n, n_vis, B, T, max_n, K, sel_ws, topk_idx, s);
 }
 
 }  // extern "C"

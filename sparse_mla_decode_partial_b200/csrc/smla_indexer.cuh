@@ -22,12 +22,15 @@
 // epilogue thread that owns a key reduces over its heads without talking to
 // any other thread.  Warp roles: warp 0 TMA producer, warp 1 TMEM owner and
 // MMA issuer, warps 4-7 epilogue (TMEM lanes 0-127).
-// Selection (smla_ix_select_kernel): one CTA per query token; radix passes
-// (8, 12, 12 bits) over an order-preserving key of the fp32 score find the
-// K-th largest score -- the first over all scores, the others over the
-// crossing bucket's candidates in shared memory -- then ordered scans of two
-// position bitmaps write the positions above it and the first ones (by
-// position) equal to it.
+// Selection: a radix select on an order-preserving key of the fp32 score.
+// The first digit (12 bits) is counted and its crossing bucket found over
+// every position, split into chunks so that one long context keeps the whole
+// device busy (smla_ix_hist_kernel); a second chunked pass selects the
+// positions above that bucket (a position bitmap) and gathers those in it as
+// candidates (smla_ix_mark_kernel); per token, two 10-bit digits over the
+// candidates give the exact K-th largest key, and ordered scans of position
+// bitmaps write the positions above it and the first ones (by position)
+// equal to it (smla_ix_finish_kernel).
 #pragma once
 
 #include <cuda.h>
@@ -42,7 +45,8 @@ constexpr int kIxDim = 128;        // index-key width (bf16 values)
 constexpr int kIxTile = 128;       // keys per unit: the MMA's M
 constexpr int kIxMaxHeads = 64;    // index heads: the MMA's N (padded to 16, 32, 64)
 constexpr int kIxStages = 5;       // key tiles in flight per CTA
-constexpr int kIxSelectThreads = 1024;
+
+struct IxSelMeta;
 
 struct IndexerParams {
     const int *page_table;   // [B, pt_stride]
@@ -55,6 +59,13 @@ struct IndexerParams {
     float *scores;           // [B * T, score_stride]; NaN = not a candidate
     long long score_stride;
     int *out;                // [B * T, K]
+    // selection scratch (see smla_ix_hist_kernel)
+    unsigned *sel_hist;      // [B * T, 4096]
+    IxSelMeta *sel_meta;     // [B * T]
+    uint32_t *sel_bits;      // [B * T, sel_words]
+    uint2 *sel_cand;         // [B * T, max_n]: (key, position)
+    int sel_words;
+    int sel_chunks;          // chunks of kIxSelChunk positions per token
 };
 
 // Visible positions of token u, clamped to [0, max_n].
@@ -403,6 +414,41 @@ __global__ void __launch_bounds__(IxCfg<NPAD>::kThreads, 1)
 }
 
 // ---------------------------------------------------------------- selection
+// Four kernels over a per-call scratch (workspace), chained by programmatic
+// dependent launch (each calls griddepcontrol.wait before it touches what
+// its predecessor writes):
+//   hist   [BT][4096] u32    counts of the first digit (key >> 20)
+//   meta   [BT]              crossing bucket, keys still needed, candidate count
+//   bits   [BT][sel_words]   positions selected by the first digit
+//   cand   [BT][max_n] uint2 (key, position) of those in the crossing bucket
+// smla_ix_clear_kernel zeroes hist and meta.  smla_ix_hist_kernel and
+// smla_ix_mark_kernel split every token into chunks of kIxSelChunk positions,
+// one CTA per (token, chunk), so a long context is spread over the whole
+// device; smla_ix_finish_kernel (one CTA per token) resolves the remaining
+// 20 bits over the candidates and writes the output.
+constexpr int kIxSelBins = 4096;
+constexpr int kIxSelThreads = 512;     // chunked passes
+constexpr int kIxSelIlp = 16;          // positions per thread: one load round trip
+constexpr int kIxSelChunk = kIxSelThreads * kIxSelIlp;
+constexpr int kIxMarkSmemBytes = kIxSelChunk * 8;   // staged candidates
+constexpr int kIxFinishThreads = 512;
+constexpr int kIxCandCap = 8192;       // candidates the finish kernel holds in shared memory
+constexpr int kIxFineBins = 1024;      // the two finer digits: 10 bits each
+
+struct IxSelMeta {
+    int d0;        // crossing bucket of the first digit
+    int need;      // keys still to take from it
+    int take_all;  // every candidate is selected (at most K of them)
+    int count;     // entries appended to cand
+    int done;      // chunks of the histogram pass finished
+    int pad[3];
+};
+static_assert(sizeof(IxSelMeta) == 32, "meta is 32 bytes");
+
+__host__ __device__ constexpr int ix_finish_smem_bytes(int max_n) {
+    return kIxCandCap * 8 + kIxFineBins * 4 + 2 * 4 * ((max_n + 31) / 32);
+}
+
 // Order-preserving key of a score: larger score -> larger key; -0 and +0
 // share one key; NaN (not a candidate) -> 0, below every real score.
 __device__ __forceinline__ uint32_t ix_key(float f) {
@@ -412,20 +458,9 @@ __device__ __forceinline__ uint32_t ix_key(float f) {
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// Shared memory of the selection kernel: the histograms (per-warp private
-// ones for the first digit), the crossing bucket's candidates and two bitmaps
-// over the visible positions (selected, equal to the threshold).
-constexpr int kIxCandCap = 8192;    // candidates of the crossing bucket kept in shared memory
-constexpr int kIxHistBytes = 32 * 256 * 4;  // 32 warps x 256 bins, or one 4096-bin histogram
-__host__ __device__ constexpr int ix_select_smem_bytes(int max_n) {
-    return kIxHistBytes + kIxCandCap * 8 + 2 * 4 * ((max_n + 31) / 32);
-}
-constexpr int kIxSelectMaxN = (232448 - kIxHistBytes - kIxCandCap * 8 - 1024) / 8 * 32;
-
-// Warp-aggregated increment of hist[d] (lanes with the same digit add once).
-__device__ __forceinline__ void ix_hist_add(unsigned *hist, bool match, uint32_t d) {
-    const uint32_t peers = __match_any_sync(__activemask(), match ? d : 0xffffffffu);
-    if (match && (__ffs(peers) - 1) == (int)(threadIdx.x & 31)) atomicAdd(&hist[d], (unsigned)__popc(peers));
+__device__ __forceinline__ void ix_pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void ix_pdl_trigger() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 // Bucket of the histogram (nb bins) holding the need-th largest key counted
@@ -457,17 +492,33 @@ __device__ __forceinline__ int ix_find_bucket(const unsigned *hist, int nb, int 
 }
 
 // Ordered scan of a bitmap of `words` words: calls emit(rank, position) for
-// every set bit in ascending position order (rank = its index among set bits).
+// every set bit in ascending position order (rank = its index among set
+// bits).  Each warp owns a contiguous run of words and reads it 32 words at
+// a time (lane i the i-th word), so the reads are conflict-free.
 template <typename F>
 __device__ __forceinline__ int ix_bitmap_scan(const uint32_t *bits, int words, int *scratch, F emit) {
-    const int per = (words + blockDim.x - 1) / blockDim.x;
-    const int w0 = min(words, (int)threadIdx.x * per), w1 = min(words, w0 + per);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    const int per = ((words + nw - 1) / nw + 31) & ~31;
+    const int w0 = min(words, warp * per), w1 = min(words, w0 + per);
     int cnt = 0;
-    for (int i = w0; i < w1; ++i) cnt += __popc(bits[i]);
+    for (int i = w0 + lane; i < w1; i += 32) cnt += __popc(bits[i]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
     int total;
-    int rank = ix_block_scan(cnt, scratch, &total) - cnt;
-    for (int i = w0; i < w1; ++i) {
-        uint32_t m = bits[i];
+    const int incl = ix_block_scan(lane == 0 ? cnt : 0, scratch, &total);
+    int base = __shfl_sync(0xffffffffu, incl, 0) - cnt;
+    for (int i0 = w0; i0 < w1; i0 += 32) {
+        const int i = i0 + lane;
+        uint32_t m = i < w1 ? bits[i] : 0u;
+        const int c = __popc(m);
+        int x = c;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+        }
+        int rank = base + x - c;
+        base += __shfl_sync(0xffffffffu, x, 31);
         while (m) {
             const int b = __ffs(m) - 1;
             m &= m - 1;
@@ -477,158 +528,241 @@ __device__ __forceinline__ int ix_bitmap_scan(const uint32_t *bits, int words, i
     return total;
 }
 
-// One CTA per query token.  Pass A (global): histogram of the top 8 bits of
-// the key, one private histogram per warp (scores crowd into few buckets;
-// shared bins would serialise the warps) -> the crossing bucket d0.  Pass B
-// (global): positions with a digit above d0 are selected (bitmap); those in
-// d0 become candidates in shared memory.  Two 12-bit radix passes over the
-// candidates give the exact threshold key and how many keys equal to it are
-// taken; the first of those by position are found by an ordered scan of an
-// "equal" bitmap, and an ordered scan of the selection bitmap writes the
-// output.  If d0 holds more than kIxCandCap keys, the finer passes and the
-// marking read the global scores instead.
-__global__ void __launch_bounds__(kIxSelectThreads) smla_ix_select_kernel(const IndexerParams p) {
+// Zeroes the per-token histograms and meta (n16 16-byte words).
+__global__ void __launch_bounds__(256) smla_ix_clear_kernel(uint4 *buf, long long n16) {
+    ix_pdl_trigger();
+    for (long long i = blockIdx.x * 256ll + threadIdx.x; i < n16; i += (long long)gridDim.x * 256)
+        buf[i] = make_uint4(0u, 0u, 0u, 0u);
+}
+
+// The (token, chunk) pair of a CTA of the chunked passes: a 1-D grid over
+// B*T x sel_chunks, token-major, so that the CTAs with work (chunks below a
+// token's length) are spread along the launch order.
+struct IxChunk {
+    int u, s0, s1;
+};
+__device__ __forceinline__ IxChunk ix_chunk(const IndexerParams &p) {
+    const int u = blockIdx.x / p.sel_chunks;
+    const int s0 = (blockIdx.x - u * p.sel_chunks) * kIxSelChunk;
+    return {u, s0, min(ix_visible(p, u), s0 + kIxSelChunk)};
+}
+
+// The chunk's keys, one load round trip (lane-consecutive positions).
+__device__ __forceinline__ void ix_load_chunk(const float *sc, const IxChunk &ck,
+                                              uint32_t (&key)[kIxSelIlp]) {
+#pragma unroll
+    for (int j = 0; j < kIxSelIlp; ++j) {
+        const int s = ck.s0 + j * kIxSelThreads + (int)threadIdx.x;
+        key[j] = s < ck.s1 ? ix_key(__ldg(sc + s)) : 0u;
+    }
+}
+
+// Pass 1, one CTA per (token, chunk): histogram of the first digit in shared
+// memory, added into the token's global histogram.  The CTA that finishes
+// the token's last chunk finds the crossing bucket and writes meta.  The
+// scores are complete before the chain starts (stream order), so they are
+// read before the wait; the global histogram only after it.
+__global__ void __launch_bounds__(kIxSelThreads) smla_ix_hist_kernel(const IndexerParams p) {
+    __shared__ unsigned hist[kIxSelBins];
+    __shared__ int scratch[33];
+    __shared__ int last;
+    ix_pdl_trigger();
+    const int tid = threadIdx.x, nt = blockDim.x;
+    const IxChunk ck = ix_chunk(p);
+    if (ck.s0 >= ck.s1) return;
+    const int u = ck.u;
+    unsigned *gh = p.sel_hist + (size_t)u * kIxSelBins;
+    uint32_t key[kIxSelIlp];
+    ix_load_chunk(p.scores + (size_t)u * p.score_stride, ck, key);
+    for (int i = tid; i < kIxSelBins; i += nt) hist[i] = 0;
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < kIxSelIlp; ++j)
+        if (key[j] != 0u) atomicAdd(&hist[key[j] >> 20], 1u);
+    __syncthreads();
+    ix_pdl_wait();
+    for (int i = tid; i < kIxSelBins; i += nt) {
+        const unsigned v = hist[i];
+        if (v) atomicAdd(gh + i, v);
+    }
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) {
+        const int chunks = (ix_visible(p, u) + kIxSelChunk - 1) / kIxSelChunk;
+        last = atomicAdd(&p.sel_meta[u].done, 1) == chunks - 1;
+    }
+    __syncthreads();
+    if (!last) return;
+    __threadfence();
+    // The crossing bucket: thread i holds bins [4096 - per*(i+1), 4096 - per*i)
+    // in registers, counted from the top.
+    constexpr int kPer = kIxSelBins / kIxSelThreads;
+    static_assert(kPer % 4 == 0, "bins per thread load as uint4");
+    uint32_t b[kPer];
+    const int lo = kIxSelBins - kPer * (tid + 1);
+#pragma unroll
+    for (int q = 0; q < kPer / 4; ++q) {
+        const uint4 v = __ldcg(reinterpret_cast<const uint4 *>(gh + lo) + q);
+        b[4 * q] = v.x;
+        b[4 * q + 1] = v.y;
+        b[4 * q + 2] = v.z;
+        b[4 * q + 3] = v.w;
+    }
+    int v = 0;
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) v += (int)b[k];
+    int total;
+    const int incl = ix_block_scan(v, scratch, &total);
+    IxSelMeta *m = p.sel_meta + u;
+    if (total <= p.K) {
+        if (tid == 0) {
+            m->take_all = 1;
+            m->d0 = 0;
+            m->need = 0;
+        }
+        return;
+    }
+    int excl = incl - v;
+    if (excl < p.K && p.K <= incl) {
+#pragma unroll
+        for (int k = kPer - 1; k >= 0; --k) {    // from the highest bin down
+            if (excl >= 0 && excl + (int)b[k] >= p.K) {
+                m->take_all = 0;
+                m->d0 = lo + k;
+                m->need = p.K - excl;
+                excl = -1;
+            } else if (excl >= 0) {
+                excl += (int)b[k];
+            }
+        }
+    }
+}
+
+// Pass 2, one CTA per (token, chunk): positions whose first digit is above
+// the crossing bucket are selected (one bitmap word per warp step, written
+// whole, so the bitmap needs no clearing); those in it are staged in shared
+// memory and appended to the token's candidates with one reservation.
+__global__ void __launch_bounds__(kIxSelThreads) smla_ix_mark_kernel(const IndexerParams p) {
     extern __shared__ __align__(16) uint8_t ix_smem[];
-    unsigned *hist = reinterpret_cast<unsigned *>(ix_smem);
-    uint32_t *cand_key = reinterpret_cast<uint32_t *>(ix_smem + kIxHistBytes);
-    int *cand_pos = reinterpret_cast<int *>(ix_smem + kIxHistBytes + kIxCandCap * 4);
-    uint32_t *sel_bits = reinterpret_cast<uint32_t *>(ix_smem + kIxHistBytes + kIxCandCap * 8);
+    uint2 *stage = reinterpret_cast<uint2 *>(ix_smem);
+    __shared__ int ccount, cbase;
+    ix_pdl_trigger();
+    const int tid = threadIdx.x, lane = tid & 31;
+    const IxChunk ck = ix_chunk(p);
+    if (ck.s0 >= ck.s1) return;
+    const int u = ck.u;
+    if (tid == 0) ccount = 0;
+    uint32_t key[kIxSelIlp];
+    ix_load_chunk(p.scores + (size_t)u * p.score_stride, ck, key);
+    ix_pdl_wait();
+    IxSelMeta *meta = p.sel_meta + u;
+    const bool take_all = meta->take_all != 0;
+    const uint32_t d0 = (uint32_t)meta->d0;
+    uint32_t *bits = p.sel_bits + (size_t)u * p.sel_words;
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < kIxSelIlp; ++j) {
+        const int s = ck.s0 + j * kIxSelThreads + tid;   // a warp covers 32 consecutive positions
+        const uint32_t d = key[j] >> 20;
+        const bool above = key[j] != 0u && (take_all || d > d0);
+        const bool is_cand = key[j] != 0u && !take_all && d == d0;
+        const uint32_t word = __ballot_sync(0xffffffffu, above);
+        if (lane == 0 && s < ck.s1) bits[s >> 5] = word;
+        const uint32_t cm = __ballot_sync(0xffffffffu, is_cand);
+        if (cm) {
+            int slot0 = 0;
+            if (lane == 0) slot0 = atomicAdd(&ccount, __popc(cm));
+            slot0 = __shfl_sync(0xffffffffu, slot0, 0);
+            if (is_cand) stage[slot0 + __popc(cm & ((1u << lane) - 1u))] = make_uint2(key[j], (uint32_t)s);
+        }
+    }
+    __syncthreads();
+    const int m = ccount;
+    if (m == 0) return;
+    if (tid == 0) cbase = atomicAdd(&meta->count, m);
+    __syncthreads();
+    uint2 *cand = p.sel_cand + (size_t)u * p.max_n + cbase;
+    for (int i = tid; i < m; i += kIxSelThreads) cand[i] = stage[i];
+}
+
+// Pass 3, one CTA per token: two 10-bit digits over the candidates (held in
+// shared memory when they fit, else re-read) give the exact threshold key and
+// how many keys equal to it are taken; the first of those by position come
+// from an ordered scan of an "equal" bitmap; an ordered scan of the selection
+// bitmap writes the output.
+__global__ void __launch_bounds__(kIxFinishThreads) smla_ix_finish_kernel(const IndexerParams p) {
+    extern __shared__ __align__(16) uint8_t ix_smem[];
+    uint32_t *cand_key = reinterpret_cast<uint32_t *>(ix_smem);
+    int *cand_pos = reinterpret_cast<int *>(ix_smem + kIxCandCap * 4);
+    unsigned *hist = reinterpret_cast<unsigned *>(ix_smem + kIxCandCap * 8);
+    uint32_t *sel = reinterpret_cast<uint32_t *>(ix_smem + kIxCandCap * 8 + kIxFineBins * 4);
     __shared__ int scratch[33];
     __shared__ int found[2];
-    __shared__ int n_cand;
     const int u = blockIdx.x, tid = threadIdx.x, nt = blockDim.x;
-    const int warp = tid >> 5, lane = tid & 31;
     const int n = ix_visible(p, u), K = p.K;
-    const int words = (n + 31) / 32;
-    uint32_t *eq_bits = sel_bits + words;
-    const float *sc = p.scores + (size_t)u * p.score_stride;
     int *out = p.out + (size_t)u * K;
-    constexpr int kIlp = 8;
-
-    for (int i = tid; i < kIxHistBytes / 4; i += nt) hist[i] = 0;
-    for (int i = tid; i < 2 * words; i += nt) sel_bits[i] = 0;
-    if (tid == 0) n_cand = 0;
-    __syncthreads();
-
-    // ---- pass A: top 8 bits into this warp's own 256 bins
-    unsigned *my_hist = hist + warp * 256;
-    for (int base = 0; base < n; base += nt * kIlp) {
-        uint32_t key[kIlp];
-#pragma unroll
-        for (int j = 0; j < kIlp; ++j) {
-            const int s = base + j * nt + tid;
-            key[j] = s < n ? ix_key(__ldg(sc + s)) : 0u;
-        }
-#pragma unroll
-        for (int j = 0; j < kIlp; ++j) ix_hist_add(my_hist, key[j] != 0u, key[j] >> 24);
+    ix_pdl_wait();
+    if (n == 0) {
+        for (int i = tid; i < K; i += nt) out[i] = -1;
+        return;
     }
-    __syncthreads();
-    // fold the 32 private histograms into bins 0..255 of warp 0's
-    if (tid < 256) {
-        unsigned sum = 0;
-        for (int w = 0; w < 32; ++w) sum += hist[w * 256 + tid];
-        hist[tid] = sum;
-    }
-    __syncthreads();
-    int need = K;
-    const int valid = ix_find_bucket(hist, 256, need, scratch, found);
-    const bool take_all = valid <= K;
-    const uint32_t d0 = take_all ? 0u : (uint32_t)found[0];
-    if (!take_all) need -= found[1];
-
-    // ---- pass B: digits above d0 are in; d0's keys become candidates
-    for (int base = 0; base < n; base += nt * kIlp) {
-        uint32_t key[kIlp];
-#pragma unroll
-        for (int j = 0; j < kIlp; ++j) {
-            const int s = base + j * nt + tid;
-            key[j] = s < n ? ix_key(__ldg(sc + s)) : 0u;
-        }
-#pragma unroll
-        for (int j = 0; j < kIlp; ++j) {
-            const int s = base + j * nt + tid;
-            const uint32_t d = key[j] >> 24;
-            const bool above = key[j] != 0u && (take_all || d > d0);
-            const bool cand = key[j] != 0u && !take_all && d == d0;
-            if (above) atomicOr(&sel_bits[s >> 5], 1u << (s & 31));
-            // warp-aggregated append of the candidates
-            const uint32_t cm = __ballot_sync(0xffffffffu, cand);
-            int slot0 = 0;
-            if (lane == 0 && cm) slot0 = atomicAdd(&n_cand, __popc(cm));
-            slot0 = __shfl_sync(0xffffffffu, slot0, 0);
-            if (cand) {
-                const int c = slot0 + __popc(cm & ((1u << lane) - 1u));
-                if (c < kIxCandCap) {
-                    cand_key[c] = key[j];
-                    cand_pos[c] = s;
-                }
-            }
+    const int words = (n + 31) / 32;
+    uint32_t *eq = sel + words;
+    const IxSelMeta meta = p.sel_meta[u];
+    const uint32_t *gbits = p.sel_bits + (size_t)u * p.sel_words;
+    const uint2 *gcand = p.sel_cand + (size_t)u * p.max_n;
+    const int m = meta.take_all ? 0 : meta.count;
+    const bool in_smem = m <= kIxCandCap;
+    if (in_smem) {
+        for (int c = tid; c < m; c += nt) {
+            const uint2 e = gcand[c];
+            cand_key[c] = e.x;
+            cand_pos[c] = (int)e.y;
         }
     }
-    __syncthreads();
-
-    if (!take_all) {
-        // ---- the two finer 12-bit digits, over the candidates (or the global scores)
-        const int m = n_cand;
-        const bool in_smem = m <= kIxCandCap;
-        uint32_t prefix = d0;
+    for (int i = tid; i < words; i += nt) {
+        sel[i] = gbits[i];
+        eq[i] = 0u;
+    }
+    if (!meta.take_all) {
+        int need = meta.need;
+        uint32_t prefix = (uint32_t)meta.d0;
 #pragma unroll
         for (int pass = 0; pass < 2; ++pass) {
-            const int shift = pass == 0 ? 12 : 0, hi_shift = shift + 12;
-            for (int i = tid; i < 4096; i += nt) hist[i] = 0;
+            const int shift = pass == 0 ? 10 : 0, hi_shift = shift + 10;
+            for (int i = tid; i < kIxFineBins; i += nt) hist[i] = 0;
             __syncthreads();
-            if (in_smem) {
-                for (int c = tid; c < ((m + 31) & ~31); c += nt) {
-                    const uint32_t key = c < m ? cand_key[c] : 0u;
-                    ix_hist_add(hist, c < m && (key >> hi_shift) == prefix, (key >> shift) & 4095u);
-                }
-            } else {
-                for (int base = 0; base < n; base += nt * kIlp) {
-                    uint32_t key[kIlp];
-#pragma unroll
-                    for (int j = 0; j < kIlp; ++j) {
-                        const int s = base + j * nt + tid;
-                        key[j] = s < n ? ix_key(__ldg(sc + s)) : 0u;
-                    }
-#pragma unroll
-                    for (int j = 0; j < kIlp; ++j)
-                        ix_hist_add(hist, key[j] != 0u && (key[j] >> hi_shift) == prefix,
-                                    (key[j] >> shift) & 4095u);
-                }
+            for (int c = tid; c < m; c += nt) {
+                const uint32_t key = in_smem ? cand_key[c] : gcand[c].x;
+                if ((key >> hi_shift) == prefix) atomicAdd(&hist[(key >> shift) & 1023u], 1u);
             }
             __syncthreads();
-            ix_find_bucket(hist, 4096, need, scratch, found);
-            prefix = (prefix << 12) | (uint32_t)found[0];
+            ix_find_bucket(hist, kIxFineBins, need, scratch, found);
+            prefix = (prefix << 10) | (uint32_t)found[0];
             need -= found[1];
-            __syncthreads();
         }
         const uint32_t thresh = prefix;
-        // ---- mark: above the threshold -> selected; equal -> the "equal" bitmap
-        if (in_smem) {
-            for (int c = tid; c < m; c += nt) {
-                const uint32_t key = cand_key[c];
-                const int s = cand_pos[c];
-                if (key > thresh) atomicOr(&sel_bits[s >> 5], 1u << (s & 31));
-                else if (key == thresh) atomicOr(&eq_bits[s >> 5], 1u << (s & 31));
+        for (int c = tid; c < m; c += nt) {
+            uint32_t key;
+            int s;
+            if (in_smem) {
+                key = cand_key[c];
+                s = cand_pos[c];
+            } else {
+                const uint2 e = gcand[c];
+                key = e.x;
+                s = (int)e.y;
             }
-        } else {
-            for (int s = tid; s < n; s += nt) {
-                const uint32_t key = ix_key(__ldg(sc + s));
-                if (key == 0u || (key >> 24) != d0) continue;  // the bits above d0 are set already
-                if (key > thresh) atomicOr(&sel_bits[s >> 5], 1u << (s & 31));
-                else if (key == thresh) atomicOr(&eq_bits[s >> 5], 1u << (s & 31));
-            }
+            if (key > thresh) atomicOr(&sel[s >> 5], 1u << (s & 31));
+            else if (key == thresh) atomicOr(&eq[s >> 5], 1u << (s & 31));
         }
         __syncthreads();
-        // ---- the first `need` equal keys by position
-        ix_bitmap_scan(eq_bits, words, scratch, [&](int rank, int s) {
-            if (rank < need) atomicOr(&sel_bits[s >> 5], 1u << (s & 31));
+        ix_bitmap_scan(eq, words, scratch, [&](int rank, int s) {
+            if (rank < need) atomicOr(&sel[s >> 5], 1u << (s & 31));
         });
-        __syncthreads();
     }
-
-    // ---- output: selected positions in ascending order, then -1
-    const int taken = ix_bitmap_scan(sel_bits, words, scratch, [&](int rank, int s) {
+    __syncthreads();
+    const int taken = ix_bitmap_scan(sel, words, scratch, [&](int rank, int s) {
         if (rank < K) out[rank] = s;
     });
     for (int i = min(taken, K) + tid; i < K; i += nt) out[i] = -1;

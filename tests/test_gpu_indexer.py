@@ -152,6 +152,65 @@ def test_selection_bit_exact_on_the_kernels_own_scores(seed):
     assert np.array_equal(gpu_topk(w), want)
 
 
+def crafted_scores(rng, B, T, max_n, kind):
+    """Score rows that stress the selection: special values, heavy ties that
+    straddle chunk boundaries, one value everywhere."""
+    sc = np.full((B, T, max_n), np.nan, np.float32)
+    for b in range(B):
+        for t in range(T):
+            if kind == "special":
+                row = rng.choice(np.array([np.nan, np.inf, -np.inf, 0.0, -0.0, 1.0, -1.0, 3.0e38,
+                                           -3.0e38, 1e-45, -1e-45, 2.0, 2.0], np.float32), max_n)
+            elif kind == "ties":
+                row = rng.integers(-3, 4, max_n).astype(np.float32)
+            elif kind == "constant":
+                row = np.full(max_n, 0.25, np.float32)
+            else:
+                row = rng.standard_normal(max_n).astype(np.float32)
+            sc[b, t] = row
+    return sc
+
+
+SELECT_CASES = [
+    # kind, n_vis rows, K
+    ("special", [[20000], [8192], [8193], [1]], 700),
+    ("ties", [[30000, 7], [16384, 100]], 2048),
+    ("constant", [[40000], [9000]], 300),      # crossing bucket holds every position
+    ("normal", [[65536], [12345], [0]], 2048),
+    ("normal", [[5000], [4999]], 5000),        # K >= n: everything, in order
+]
+
+
+@pytest.mark.parametrize("kind,nv,K", SELECT_CASES,
+                         ids=[f"{c[0]}-{len(c[1])}x{len(c[1][0])}-K{c[2]}" for c in SELECT_CASES])
+def test_selection_on_crafted_scores_bit_exact(kind, nv, K):
+    rng = np.random.default_rng(len(kind) * 1000 + K)
+    n_vis = np.array(nv, np.int32)
+    B, T = n_vis.shape
+    max_n = int(n_vis.max()) or 1
+    sc = crafted_scores(rng, B, T, max_n, kind)
+    got = binding.indexer_select(torch.from_numpy(sc).to(DEV), torch.from_numpy(n_vis).to(DEV), K)
+    torch.cuda.synchronize()
+    want = ix_oracle.select(sc, n_vis, K)
+    assert np.array_equal(got.cpu().numpy(), want)
+
+
+def test_select_workspace_is_scratch_only():
+    """A workspace left dirty by an earlier call (or filled with garbage)
+    gives the same selection."""
+    rng = np.random.default_rng(77)
+    n_vis = np.array([[30000], [9000], [500]], np.int32)
+    sc = crafted_scores(rng, 3, 1, 30000, "ties")
+    scd, nvd = torch.from_numpy(sc).to(DEV), torch.from_numpy(n_vis).to(DEV)
+    ws = torch.full((binding.indexer_select_workspace_bytes(3, 1, 30000),), 0xA5, dtype=torch.uint8,
+                    device=DEV)
+    want = ix_oracle.select(sc, n_vis, 1000)
+    for _ in range(2):
+        got = binding.indexer_select(scd, nvd, 1000, workspace=ws)
+        torch.cuda.synchronize()
+        assert np.array_equal(got.cpu().numpy(), want)
+
+
 def valid_topk(sel, exact, n, K, eps):
     """sel is a valid top-K of the exact scores up to eps: ascending, unique,
     exactly min(K, candidates) entries, and nothing is misplaced by more than
