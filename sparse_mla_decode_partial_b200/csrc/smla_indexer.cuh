@@ -222,8 +222,7 @@ struct IxCfg {
     static constexpr int kAcc = 4;                           // accumulators of 64 TMEM columns
     static constexpr int kNumBars = 2 * kIxStages + 4 + 2 * kAcc;
     static constexpr int kOffTmem = kOffBar + kNumBars * 8;
-    static constexpr int kOffW = kOffTmem + 16;              // fp32 [64] weights of the token
-    static constexpr int kBytes = kOffW + kIxMaxHeads * 4;
+    static constexpr int kBytes = kOffTmem + 16;
     static constexpr int kSmemBytes = kBytes + 1024;         // alignment slack (1024-B atoms)
     static constexpr uint32_t kTmemCols = 64 * kAcc;
 };
@@ -241,7 +240,6 @@ __global__ void __launch_bounds__(IxCfg<NPAD>::kThreads, 1)
     uint64_t *q_full = bars + 2 * kIxStages, *q_empty = q_full + 2;
     uint64_t *acc_full = q_empty + 2, *acc_empty = acc_full + C::kAcc;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::kOffTmem);
-    float *w_s = reinterpret_cast<float *>(smem + C::kOffW);
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kIxStages; ++i) {
@@ -368,6 +366,7 @@ __global__ void __launch_bounds__(IxCfg<NPAD>::kThreads, 1)
         const int row = 32 * q4 + lane;          // key of the tile
         const int et = threadIdx.x - 128;        // 0 .. 127
         int w_tok = -1;
+        float wr[NPAD];                          // the token's head weights (0 past HI)
         int hint = u_begin < u_end ? ix_token_of(p, u_begin) : 0;
         long long i = 0;
         for (long long ub = u_begin; ub < u_end; ub += 32) {
@@ -376,10 +375,10 @@ __global__ void __launch_bounds__(IxCfg<NPAD>::kThreads, 1)
             hint = __shfl_sync(0xffffffffu, mine.tok, cnt - 1);
             for (int k = 0; k < cnt; ++k, ++i) {
                 const IxUnit m = ix_unit_from(mine, k);
-                if (m.tok != w_tok) {  // the token's head weights (0 past HI)
-                    named_bar_sync(1, 128);
-                    if (et < kIxMaxHeads) w_s[et] = et < p.HI ? __ldg(p.w + (size_t)m.tok * p.HI + et) : 0.f;
-                    named_bar_sync(1, 128);
+                if (m.tok != w_tok) {
+#pragma unroll
+                    for (int j = 0; j < NPAD; ++j)
+                        wr[j] = j < p.HI ? __ldg(p.w + (size_t)m.tok * p.HI + j) : 0.f;
                     w_tok = m.tok;
                 }
                 const int a = (int)(i % C::kAcc);
@@ -394,11 +393,12 @@ __global__ void __launch_bounds__(IxCfg<NPAD>::kThreads, 1)
                 if (s < m.n) {
                     float score = __uint_as_float(0x7fffffffu);  // NaN: not a candidate
                     if ((row < 64 ? m.pg0 : m.pg1) >= 0) {
-                        float acc = 0.f;
+                        // four interleaved partial sums (heads j = r mod 4), added pairwise
+                        float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                         for (int j = 0; j < NPAD; ++j)
-                            acc = (j < p.HI) ? fmaf(w_s[j], fmaxf(__uint_as_float(x[j]), 0.f), acc) : acc;
-                        score = acc;
+                            if (j < p.HI) acc[j & 3] = fmaf(wr[j], fmaxf(__uint_as_float(x[j]), 0.f), acc[j & 3]);
+                        score = (acc[0] + acc[1]) + (acc[2] + acc[3]);
                     }
                     p.scores[(size_t)m.tok * p.score_stride + s] = score;
                 }
