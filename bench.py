@@ -517,7 +517,7 @@ def side_indexer(h, steps, warmup, peaks):
 
     def topk():
         return lib.smla_indexer_topk(*common, K, 64, ws.data_ptr(), ws.numel(), out.data_ptr(),
-                                     sptr), 5
+                                     sptr), 4
 
     def scores():
         return lib.smla_indexer_scores(*common, 64, ws.data_ptr(), ws.numel(), sc.data_ptr(),
@@ -525,7 +525,7 @@ def side_indexer(h, steps, warmup, peaks):
 
     def select():
         return lib.smla_indexer_select(sc.data_ptr(), w.n_vis.data_ptr(), B, T, max_n, K,
-                                       sel_ws.data_ptr(), sel_ws.numel(), out.data_ptr(), sptr), 3
+                                       sel_ws.data_ptr(), sel_ws.numel(), out.data_ptr(), sptr), 4
     h.warm([topk, scores, select], warmup)
     sampler = ClockSampler(h.dev.index)
     with sampler:

@@ -861,11 +861,34 @@ smla_status check_indexer_args(const void *q_index, const float *w, const void *
 
 size_t ix_plan_bytes(int B, int T) { return round256(((size_t)B * T + 1) * sizeof(int)); }
 
-// Plan + scores into `scores` (row stride `stride` floats).
+// Selection scratch: [hist | meta] (cleared per call), the position bitmap
+// and the candidate list.
+size_t ix_select_zeroed_bytes(int B, int T) {
+    return (size_t)B * T * (smla::kIxSelBins * sizeof(unsigned) + sizeof(smla::IxSelMeta));
+}
+size_t ix_select_bytes(int B, int T, int max_n) {
+    const size_t bt = (size_t)B * T, words = ((size_t)max_n + 31) / 32;
+    return round256(ix_select_zeroed_bytes(B, T)) + round256(bt * words * sizeof(uint32_t)) +
+           round256(bt * max_n * sizeof(uint2));
+}
+
+cudaLaunchConfig_t pdl_config(cudaStream_t st, cudaLaunchAttribute *attr) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.stream = st;
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cfg;
+}
+
+// Plan + scores into `scores` (row stride `stride` floats).  With sel_ws
+// (the selection scratch), the plan kernel also clears its histograms and
+// the score kernel fills them.
 smla_status launch_ix_scores(const void *q_index, const float *w, const void *k_index,
                              int64_t num_pages, const int32_t *page_table, int pt_stride,
                              const int32_t *n_vis, int B, int T, int HI, int max_n, int *plan,
-                             float *scores, long long stride, cudaStream_t st) {
+                             float *scores, long long stride, void *sel_ws, cudaStream_t st) {
     smla::IndexerParams p{};
     p.page_table = page_table;
     p.pt_stride = pt_stride;
@@ -879,7 +902,15 @@ smla_status launch_ix_scores(const void *q_index, const float *w, const void *k_
     p.tile_start = plan;
     p.scores = scores;
     p.score_stride = stride;
-    smla::smla_ix_plan_kernel<<<1, 1024, 0, st>>>(p);
+    int plan_grid = 1;
+    if (sel_ws != nullptr && max_n > 0) {
+        p.sel_hist = static_cast<unsigned *>(sel_ws);
+        p.zero = static_cast<uint4 *>(sel_ws);
+        p.n_zero = (long long)(ix_select_zeroed_bytes(B, T) / 16);
+        plan_grid = (int)std::min<long long>(std::max<long long>(1, (p.n_zero + 1023) / 1024),
+                                             current_device_sms());
+    }
+    smla::smla_ix_plan_kernel<<<plan_grid, 1024, 0, st>>>(p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e);
     if (max_n == 0) return SMLA_OK;
@@ -889,7 +920,6 @@ smla_status launch_ix_scores(const void *q_index, const float *w, const void *k_
     if (s != SMLA_OK) return s;
     s = encode_rows128(&map_q, q_index, (uint64_t)B * T * HI, (uint32_t)npad);
     if (s != SMLA_OK) return s;
-    const int grid = current_device_sms();
     const void *fn;
     int smem;
     if (npad == 16) {
@@ -904,29 +934,29 @@ smla_status launch_ix_scores(const void *q_index, const float *w, const void *k_
     }
     e = ensure_smem_attr(fn, smem);
     if (e != cudaSuccess) return cuda_fail(e);
+    // the score kernel may start while the plan runs; it waits for it in-kernel
+    cudaLaunchAttribute attr[1];
+    cudaLaunchConfig_t cfg = pdl_config(st, attr);
+    cfg.gridDim = dim3((unsigned)current_device_sms());
+    cfg.blockDim = dim3(smla::IxCfg<16>::kThreads);
+    cfg.dynamicSmemBytes = (size_t)smem;
     if (npad == 16)
-        smla::smla_ix_score_kernel<16><<<grid, smla::IxCfg<16>::kThreads, smem, st>>>(map_k, map_q, p);
+        e = cudaLaunchKernelEx(&cfg, smla::smla_ix_score_kernel<16>, map_k, map_q, p);
     else if (npad == 32)
-        smla::smla_ix_score_kernel<32><<<grid, smla::IxCfg<32>::kThreads, smem, st>>>(map_k, map_q, p);
+        e = cudaLaunchKernelEx(&cfg, smla::smla_ix_score_kernel<32>, map_k, map_q, p);
     else
-        smla::smla_ix_score_kernel<64><<<grid, smla::IxCfg<64>::kThreads, smem, st>>>(map_k, map_q, p);
-    e = cudaGetLastError();
+        e = cudaLaunchKernelEx(&cfg, smla::smla_ix_score_kernel<64>, map_k, map_q, p);
+    if (e == cudaSuccess) e = cudaGetLastError();
     return e == cudaSuccess ? SMLA_OK : cuda_fail(e);
 }
 
-// Selection scratch: [hist | meta] (cleared per call), the position bitmap
-// and the candidate list.
-size_t ix_select_zeroed_bytes(int B, int T) {
-    return (size_t)B * T * (smla::kIxSelBins * sizeof(unsigned) + sizeof(smla::IxSelMeta));
-}
-size_t ix_select_bytes(int B, int T, int max_n) {
-    const size_t bt = (size_t)B * T, words = ((size_t)max_n + 31) / 32;
-    return round256(ix_select_zeroed_bytes(B, T)) + round256(bt * words * sizeof(uint32_t)) +
-           round256(bt * max_n * sizeof(uint2));
-}
-
+// The selection chain over scores (row stride `stride`).  hist_filled: the
+// score kernel filled the histograms just before (smla_indexer_topk), so
+// the clear and histogram kernels are skipped and the scores are read only
+// after the wait.
 smla_status launch_ix_select(const float *scores, long long stride, const int32_t *n_vis, int B,
-                             int T, int max_n, int K, void *workspace, int32_t *out, cudaStream_t st) {
+                             int T, int max_n, int K, void *workspace, int32_t *out, bool hist_filled,
+                             cudaStream_t st) {
     smla::IndexerParams p{};
     p.n_vis = n_vis;
     p.BT = B * T;
@@ -945,28 +975,25 @@ smla_status launch_ix_select(const float *scores, long long stride, const int32_
     p.sel_bits = reinterpret_cast<uint32_t *>(ws + off_bits);
     p.sel_cand = reinterpret_cast<uint2 *>(ws + off_bits + round256(bt * p.sel_words * sizeof(uint32_t)));
     p.sel_chunks = (max_n + smla::kIxSelChunk - 1) / smla::kIxSelChunk;
-    // The chain: clear (stream-ordered after whatever wrote the scores), then
-    // hist, mark and finish, each allowed to start early and waiting on its
-    // predecessor in-kernel.
-    cudaLaunchConfig_t cfg = {};
-    cfg.stream = st;
+    // The chain: [clear, hist,] mark, finish; every kernel after the first
+    // may start early and waits on its predecessor in-kernel.
     cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cudaLaunchConfig_t cfg = pdl_config(st, attr);
     cudaError_t e;
     if (max_n > 0) {
-        const long long n16 = (long long)(ix_select_zeroed_bytes(B, T) / 16);
-        const long long blocks = std::min<long long>((n16 + 255) / 256, 4ll * current_device_sms());
-        smla::smla_ix_clear_kernel<<<(unsigned)blocks, 256, 0, st>>>(reinterpret_cast<uint4 *>(ws), n16);
-        e = cudaGetLastError();
-        if (e != cudaSuccess) return cuda_fail(e);
         cfg.gridDim = dim3((unsigned)((long long)p.BT * p.sel_chunks));
         cfg.blockDim = dim3(smla::kIxSelThreads);
-        cfg.dynamicSmemBytes = 0;
-        e = cudaLaunchKernelEx(&cfg, smla::smla_ix_hist_kernel, p);
-        if (e != cudaSuccess) return cuda_fail(e);
+        if (!hist_filled) {
+            const long long n16 = (long long)(ix_select_zeroed_bytes(B, T) / 16);
+            const long long blocks = std::min<long long>((n16 + 255) / 256, 4ll * current_device_sms());
+            smla::smla_ix_clear_kernel<<<(unsigned)blocks, 256, 0, st>>>(reinterpret_cast<uint4 *>(ws), n16);
+            e = cudaGetLastError();
+            if (e != cudaSuccess) return cuda_fail(e);
+            cfg.dynamicSmemBytes = 0;
+            e = cudaLaunchKernelEx(&cfg, smla::smla_ix_hist_kernel, p);
+            if (e != cudaSuccess) return cuda_fail(e);
+            p.sel_prefetch = 1;
+        }
         e = ensure_smem_attr(reinterpret_cast<const void *>(&smla::smla_ix_mark_kernel),
                              smla::kIxMarkSmemBytes);
         if (e != cudaSuccess) return cuda_fail(e);
@@ -1015,7 +1042,7 @@ smla_status smla_indexer_scores(const void *q_index, const float *w, const void 
     if (workspace == nullptr) return SMLA_ERR_INVALID_ARG;
     if (!aligned(workspace, 16)) return SMLA_ERR_MISALIGNED;
     return launch_ix_scores(q_index, w, k_index, num_pages, page_table, pt_stride, n_vis, B, T, HI,
-                            max_n, static_cast<int *>(workspace), scores, max_n,
+                            max_n, static_cast<int *>(workspace), scores, max_n, nullptr,
                             static_cast<cudaStream_t>(stream));
 }
 
@@ -1031,7 +1058,7 @@ smla_status smla_indexer_select(const float *scores, const int32_t *n_vis, int B
     if (workspace_bytes < ix_select_bytes(B, T, max_n)) return SMLA_ERR_WORKSPACE_TOO_SMALL;
     if (workspace == nullptr) return SMLA_ERR_INVALID_ARG;
     if (!aligned(workspace, 16)) return SMLA_ERR_MISALIGNED;
-    return launch_ix_select(scores, max_n, n_vis, B, T, max_n, K, workspace, topk_idx,
+    return launch_ix_select(scores, max_n, n_vis, B, T, max_n, K, workspace, topk_idx, false,
                             static_cast<cudaStream_t>(stream));
 }
 
@@ -1056,9 +1083,9 @@ smla_status smla_indexer_topk(const void *q_index, const float *w, const void *k
     float *scores = reinterpret_cast<float *>(ws + ix_plan_bytes(B, T));
     void *sel_ws = ws + ix_plan_bytes(B, T) + round256((size_t)B * T * max_n * sizeof(float));
     st = launch_ix_scores(q_index, w, k_index, num_pages, page_table, pt_stride, n_vis, B, T, HI,
-                          max_n, plan, scores, max_n, s);
+                          max_n, plan, scores, max_n, sel_ws, s);
     if (st != SMLA_OK) return st;
-    return launch_ix_select(scores, max_n, n_vis, B, T, max_n, K, sel_ws, topk_idx, s);
+    return launch_ix_select(scores, max_n, n_vis, B, T, max_n, K, sel_ws, topk_idx, true, s);
 }
 
 }  // extern "C"

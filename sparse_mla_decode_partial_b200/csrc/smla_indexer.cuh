@@ -45,8 +45,17 @@ constexpr int kIxDim = 128;        // index-key width (bf16 values)
 constexpr int kIxTile = 128;       // keys per unit: the MMA's M
 constexpr int kIxMaxHeads = 64;    // index heads: the MMA's N (padded to 16, 32, 64)
 constexpr int kIxStages = 5;       // key tiles in flight per CTA
+constexpr int kIxSelBins = 4096;   // selection: bins of the first digit (key >> 20)
 
-struct IxSelMeta;
+// Selection state of one query token (in the selection scratch).
+struct IxSelMeta {
+    int d0;        // crossing bucket of the first digit
+    int need;      // keys still to take from it
+    int take_all;  // every candidate is selected (at most K of them)
+    int count;     // entries appended to cand
+    int pad[4];
+};
+static_assert(sizeof(IxSelMeta) == 32, "meta is 32 bytes");
 
 struct IndexerParams {
     const int *page_table;   // [B, pt_stride]
@@ -59,13 +68,16 @@ struct IndexerParams {
     float *scores;           // [B * T, score_stride]; NaN = not a candidate
     long long score_stride;
     int *out;                // [B * T, K]
-    // selection scratch (see smla_ix_hist_kernel)
-    unsigned *sel_hist;      // [B * T, 4096]
+    // selection scratch (see the selection section below)
+    unsigned *sel_hist;      // [B * T, 4096]; the score kernel adds to it when non-null
     IxSelMeta *sel_meta;     // [B * T]
     uint32_t *sel_bits;      // [B * T, sel_words]
     uint2 *sel_cand;         // [B * T, max_n]: (key, position)
     int sel_words;
     int sel_chunks;          // chunks of kIxSelChunk positions per token
+    int sel_prefetch;        // the scores are complete before the selection chain starts
+    uint4 *zero;             // plan kernel: n_zero 16-byte words to clear (or null)
+    long long n_zero;
 };
 
 // Visible positions of token u, clamped to [0, max_n].
@@ -102,11 +114,104 @@ __device__ __forceinline__ int ix_block_scan(int v, int *scratch, int *total) {
     return v;
 }
 
+// Inclusive sum over a group of NT threads (t = 0 .. NT-1, whole warps) that
+// synchronise with sync(); *total receives the group's sum.  scratch holds
+// NT / 32 ints.
+template <int NT, typename Sync>
+__device__ __forceinline__ int ix_group_scan(int v, int t, int *scratch, int *total, Sync sync) {
+    const int lane = t & 31, warp = t >> 5;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int x = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += x;
+    }
+    if (lane == 31) scratch[warp] = v;
+    sync();
+    int base = 0, tot = 0;
+#pragma unroll
+    for (int k = 0; k < NT / 32; ++k) {
+        const int x = scratch[k];
+        base += k < warp ? x : 0;
+        tot += x;
+    }
+    *total = tot;
+    sync();  // scratch may be reused at once
+    return v + base;
+}
+
+// The crossing bucket of token u's first digit from its complete histogram
+// (4096 bins, counted from the top): group thread t holds bins
+// [4096 - per*(t+1), 4096 - per*t) in registers.  Writes (take_all, d0,
+// need) to dec[] (shared); dec is complete after the group's next sync.
+template <int NT, typename Sync>
+__device__ __forceinline__ void ix_decide(const unsigned *gh, int K, int t, int *scratch, int *dec,
+                                          Sync sync) {
+    constexpr int kPer = 4096 / NT;
+    static_assert(kPer % 4 == 0, "bins per thread load as uint4");
+    uint32_t b[kPer];
+    const int lo = 4096 - kPer * (t + 1);
+#pragma unroll
+    for (int q = 0; q < kPer / 4; ++q) {
+        const uint4 v = __ldcg(reinterpret_cast<const uint4 *>(gh + lo) + q);
+        b[4 * q] = v.x;
+        b[4 * q + 1] = v.y;
+        b[4 * q + 2] = v.z;
+        b[4 * q + 3] = v.w;
+    }
+    int v = 0;
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) v += (int)b[k];
+    int total;
+    const int incl = ix_group_scan<NT>(v, t, scratch, &total, sync);
+    if (total <= K) {
+        if (t == 0) {
+            dec[0] = 1;
+            dec[1] = 0;
+            dec[2] = 0;
+        }
+        return;
+    }
+    int excl = incl - v;
+    if (excl < K && K <= incl) {
+#pragma unroll
+        for (int k = kPer - 1; k >= 0; --k) {    // from the highest bin down
+            if (excl >= 0 && excl + (int)b[k] >= K) {
+                dec[0] = 0;
+                dec[1] = lo + k;
+                dec[2] = K - excl;
+                excl = -1;
+            } else if (excl >= 0) {
+                excl += (int)b[k];
+            }
+        }
+    }
+}
+
+// Order-preserving key of a score: larger score -> larger key; -0 and +0
+// share one key; NaN (not a candidate) -> 0, below every real score.
+__device__ __forceinline__ uint32_t ix_key(float f) {
+    if (f != f) return 0u;
+    if (f == 0.f) f = 0.f;
+    const uint32_t u = __float_as_uint(f);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ void ix_pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void ix_pdl_trigger() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- plan
 // Units of work: token u has ceil(n_u / 128) key tiles; tile_start is their
-// exclusive prefix sum.  A length outside [0, max_n] is clamped and counted.
+// exclusive prefix sum (CTA 0).  A length outside [0, max_n] is clamped and
+// counted.  Every CTA also clears its share of p.zero (the selection's
+// histograms when the score kernel fills them).
 __global__ void __launch_bounds__(1024) smla_ix_plan_kernel(const IndexerParams p) {
     __shared__ int scratch[33];
+    ix_pdl_trigger();
+    for (long long i = blockIdx.x * 1024ll + threadIdx.x; i < p.n_zero; i += (long long)gridDim.x * 1024)
+        p.zero[i] = make_uint4(0u, 0u, 0u, 0u);
+    if (blockIdx.x != 0) return;
     int carry = 0;
     for (int base = 0; base < p.BT; base += blockDim.x) {
         const int u = base + threadIdx.x;
@@ -222,9 +327,11 @@ struct IxCfg {
     static constexpr int kAcc = 4;                           // accumulators of 64 TMEM columns
     static constexpr int kNumBars = 2 * kIxStages + 4 + 2 * kAcc;
     static constexpr int kOffTmem = kOffBar + kNumBars * 8;
-    static constexpr int kBytes = kOffTmem + 16;
+    static constexpr int kOffHist = kOffTmem + 16;            // u32 [4096]: selection digits of a token
+    static constexpr int kBytes = kOffHist + kIxSelBins * 4;
     static constexpr int kSmemBytes = kBytes + 1024;         // alignment slack (1024-B atoms)
     static constexpr uint32_t kTmemCols = 64 * kAcc;
+    static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 };
 
 template <int NPAD>
@@ -233,6 +340,7 @@ __global__ void __launch_bounds__(IxCfg<NPAD>::kThreads, 1)
                          const __grid_constant__ CUtensorMap map_q, const IndexerParams p) {
     using C = IxCfg<NPAD>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
+    ix_pdl_trigger();
     uint8_t *smem = smem_raw + ((1024 - (smem_addr(smem_raw) & 1023)) & 1023);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::kOffBar);
@@ -260,6 +368,7 @@ __global__ void __launch_bounds__(IxCfg<NPAD>::kThreads, 1)
         tmem_alloc(tmem_slot, C::kTmemCols);
         tmem_relinquish();
     }
+    ix_pdl_wait();   // the plan (and the cleared histograms) are complete
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -365,6 +474,28 @@ __global__ void __launch_bounds__(IxCfg<NPAD>::kThreads, 1)
         const int q4 = warp & 3;                 // TMEM lanes 32 q4 .. + 31
         const int row = 32 * q4 + lane;          // key of the tile
         const int et = threadIdx.x - 128;        // 0 .. 127
+        // The selection's first-digit counts of the current token gather in
+        // shared memory and go to the token's global histogram when the token
+        // changes (global atomics per key would pile onto a few hot bins).
+        unsigned *hist_s = reinterpret_cast<unsigned *>(smem + C::kOffHist);
+        const bool count = p.sel_hist != nullptr;
+        int h_tok = -1;
+        auto flush = [&]() {
+            named_bar_sync(1, 128);
+            unsigned *gh = p.sel_hist + (size_t)h_tok * kIxSelBins;
+            for (int b = et; b < kIxSelBins; b += 128) {
+                const unsigned v = hist_s[b];
+                if (v) {
+                    atomicAdd(gh + b, v);
+                    hist_s[b] = 0u;
+                }
+            }
+            named_bar_sync(1, 128);
+        };
+        if (count) {
+            for (int b = et; b < kIxSelBins; b += 128) hist_s[b] = 0u;
+            named_bar_sync(1, 128);
+        }
         int w_tok = -1;
         float wr[NPAD];                          // the token's head weights (0 past HI)
         int hint = u_begin < u_end ? ix_token_of(p, u_begin) : 0;
@@ -380,6 +511,10 @@ __global__ void __launch_bounds__(IxCfg<NPAD>::kThreads, 1)
                     for (int j = 0; j < NPAD; ++j)
                         wr[j] = j < p.HI ? __ldg(p.w + (size_t)m.tok * p.HI + j) : 0.f;
                     w_tok = m.tok;
+                    if (count) {
+                        if (h_tok >= 0) flush();
+                        h_tok = m.tok;
+                    }
                 }
                 const int a = (int)(i % C::kAcc);
                 mbar_wait(&acc_full[a], (int)(i / C::kAcc) & 1, dead);
@@ -401,9 +536,14 @@ __global__ void __launch_bounds__(IxCfg<NPAD>::kThreads, 1)
                         score = (acc[0] + acc[1]) + (acc[2] + acc[3]);
                     }
                     p.scores[(size_t)m.tok * p.score_stride + s] = score;
+                    if (count) {  // the selection's first digit, counted here
+                        const uint32_t key = ix_key(score);
+                        if (key != 0u) atomicAdd(&hist_s[key >> 20], 1u);
+                    }
                 }
             }
         }
+        if (count && h_tok >= 0) flush();
     }
     tc_fence_before();
     __syncthreads();
@@ -414,19 +554,20 @@ __global__ void __launch_bounds__(IxCfg<NPAD>::kThreads, 1)
 }
 
 // ---------------------------------------------------------------- selection
-// Four kernels over a per-call scratch (workspace), chained by programmatic
-// dependent launch (each calls griddepcontrol.wait before it touches what
-// its predecessor writes):
+// A per-call scratch (workspace):
 //   hist   [BT][4096] u32    counts of the first digit (key >> 20)
 //   meta   [BT]              crossing bucket, keys still needed, candidate count
 //   bits   [BT][sel_words]   positions selected by the first digit
 //   cand   [BT][max_n] uint2 (key, position) of those in the crossing bucket
-// smla_ix_clear_kernel zeroes hist and meta.  smla_ix_hist_kernel and
-// smla_ix_mark_kernel split every token into chunks of kIxSelChunk positions,
-// one CTA per (token, chunk), so a long context is spread over the whole
-// device; smla_ix_finish_kernel (one CTA per token) resolves the remaining
-// 20 bits over the candidates and writes the output.
-constexpr int kIxSelBins = 4096;
+// The histogram is filled by the score kernel's epilogue when the scores are
+// computed here (smla_indexer_topk), else by smla_ix_hist_kernel over given
+// scores (after smla_ix_clear_kernel).  smla_ix_mark_kernel then finds the
+// crossing bucket and marks; hist and mark split every token into chunks of
+// kIxSelChunk positions, one CTA per (token, chunk), so a long context is
+// spread over the whole device.  smla_ix_finish_kernel (one CTA per token)
+// resolves the remaining 20 bits over the candidates and writes the output.
+// The kernels are chained by programmatic dependent launch: each calls
+// griddepcontrol.wait before it touches what its predecessor writes.
 constexpr int kIxSelThreads = 512;     // chunked passes
 constexpr int kIxSelIlp = 16;          // positions per thread: one load round trip
 constexpr int kIxSelChunk = kIxSelThreads * kIxSelIlp;
@@ -435,33 +576,11 @@ constexpr int kIxFinishThreads = 512;
 constexpr int kIxCandCap = 8192;       // candidates the finish kernel holds in shared memory
 constexpr int kIxFineBins = 1024;      // the two finer digits: 10 bits each
 
-struct IxSelMeta {
-    int d0;        // crossing bucket of the first digit
-    int need;      // keys still to take from it
-    int take_all;  // every candidate is selected (at most K of them)
-    int count;     // entries appended to cand
-    int done;      // chunks of the histogram pass finished
-    int pad[3];
-};
-static_assert(sizeof(IxSelMeta) == 32, "meta is 32 bytes");
 
 __host__ __device__ constexpr int ix_finish_smem_bytes(int max_n) {
     return kIxCandCap * 8 + kIxFineBins * 4 + 2 * 4 * ((max_n + 31) / 32);
 }
 
-// Order-preserving key of a score: larger score -> larger key; -0 and +0
-// share one key; NaN (not a candidate) -> 0, below every real score.
-__device__ __forceinline__ uint32_t ix_key(float f) {
-    if (f != f) return 0u;
-    if (f == 0.f) f = 0.f;
-    const uint32_t u = __float_as_uint(f);
-    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-
-__device__ __forceinline__ void ix_pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-__device__ __forceinline__ void ix_pdl_trigger() {
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
 
 // Bucket of the histogram (nb bins) holding the need-th largest key counted
 // from the top: writes (bucket, keys above it) to found[]; returns the total.
@@ -557,23 +676,19 @@ __device__ __forceinline__ void ix_load_chunk(const float *sc, const IxChunk &ck
     }
 }
 
-// Pass 1, one CTA per (token, chunk): histogram of the first digit in shared
-// memory, added into the token's global histogram.  The CTA that finishes
-// the token's last chunk finds the crossing bucket and writes meta.  The
-// scores are complete before the chain starts (stream order), so they are
-// read before the wait; the global histogram only after it.
+// Pass 1 over given scores, one CTA per (token, chunk): histogram of the
+// first digit in shared memory, added into the token's global histogram.
+// The scores are complete before the chain starts (stream order), so they
+// are read before the wait; the global histogram (cleared by the
+// predecessor) only after it.
 __global__ void __launch_bounds__(kIxSelThreads) smla_ix_hist_kernel(const IndexerParams p) {
     __shared__ unsigned hist[kIxSelBins];
-    __shared__ int scratch[33];
-    __shared__ int last;
     ix_pdl_trigger();
     const int tid = threadIdx.x, nt = blockDim.x;
     const IxChunk ck = ix_chunk(p);
     if (ck.s0 >= ck.s1) return;
-    const int u = ck.u;
-    unsigned *gh = p.sel_hist + (size_t)u * kIxSelBins;
     uint32_t key[kIxSelIlp];
-    ix_load_chunk(p.scores + (size_t)u * p.score_stride, ck, key);
+    ix_load_chunk(p.scores + (size_t)ck.u * p.score_stride, ck, key);
     for (int i = tid; i < kIxSelBins; i += nt) hist[i] = 0;
     __syncthreads();
 #pragma unroll
@@ -581,70 +696,25 @@ __global__ void __launch_bounds__(kIxSelThreads) smla_ix_hist_kernel(const Index
         if (key[j] != 0u) atomicAdd(&hist[key[j] >> 20], 1u);
     __syncthreads();
     ix_pdl_wait();
+    unsigned *gh = p.sel_hist + (size_t)ck.u * kIxSelBins;
     for (int i = tid; i < kIxSelBins; i += nt) {
         const unsigned v = hist[i];
         if (v) atomicAdd(gh + i, v);
     }
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) {
-        const int chunks = (ix_visible(p, u) + kIxSelChunk - 1) / kIxSelChunk;
-        last = atomicAdd(&p.sel_meta[u].done, 1) == chunks - 1;
-    }
-    __syncthreads();
-    if (!last) return;
-    __threadfence();
-    // The crossing bucket: thread i holds bins [4096 - per*(i+1), 4096 - per*i)
-    // in registers, counted from the top.
-    constexpr int kPer = kIxSelBins / kIxSelThreads;
-    static_assert(kPer % 4 == 0, "bins per thread load as uint4");
-    uint32_t b[kPer];
-    const int lo = kIxSelBins - kPer * (tid + 1);
-#pragma unroll
-    for (int q = 0; q < kPer / 4; ++q) {
-        const uint4 v = __ldcg(reinterpret_cast<const uint4 *>(gh + lo) + q);
-        b[4 * q] = v.x;
-        b[4 * q + 1] = v.y;
-        b[4 * q + 2] = v.z;
-        b[4 * q + 3] = v.w;
-    }
-    int v = 0;
-#pragma unroll
-    for (int k = 0; k < kPer; ++k) v += (int)b[k];
-    int total;
-    const int incl = ix_block_scan(v, scratch, &total);
-    IxSelMeta *m = p.sel_meta + u;
-    if (total <= p.K) {
-        if (tid == 0) {
-            m->take_all = 1;
-            m->d0 = 0;
-            m->need = 0;
-        }
-        return;
-    }
-    int excl = incl - v;
-    if (excl < p.K && p.K <= incl) {
-#pragma unroll
-        for (int k = kPer - 1; k >= 0; --k) {    // from the highest bin down
-            if (excl >= 0 && excl + (int)b[k] >= p.K) {
-                m->take_all = 0;
-                m->d0 = lo + k;
-                m->need = p.K - excl;
-                excl = -1;
-            } else if (excl >= 0) {
-                excl += (int)b[k];
-            }
-        }
-    }
 }
 
-// Pass 2, one CTA per (token, chunk): positions whose first digit is above
-// the crossing bucket are selected (one bitmap word per warp step, written
-// whole, so the bitmap needs no clearing); those in it are staged in shared
-// memory and appended to the token's candidates with one reservation.
+// Pass 2, one CTA per (token, chunk): the crossing bucket from the token's
+// histogram (every CTA of the token finds the same one; chunk 0 records it
+// in meta); positions whose first digit is above it are selected (one bitmap
+// word per warp step, written whole, so the bitmap needs no clearing); those
+// in it are staged in shared memory and appended to the token's candidates
+// with one reservation.  Scores are read before the wait only when they were
+// complete before the chain started.
 __global__ void __launch_bounds__(kIxSelThreads) smla_ix_mark_kernel(const IndexerParams p) {
     extern __shared__ __align__(16) uint8_t ix_smem[];
     uint2 *stage = reinterpret_cast<uint2 *>(ix_smem);
+    __shared__ int scratch[kIxSelThreads / 32];
+    __shared__ int dec[3];
     __shared__ int ccount, cbase;
     ix_pdl_trigger();
     const int tid = threadIdx.x, lane = tid & 31;
@@ -652,14 +722,23 @@ __global__ void __launch_bounds__(kIxSelThreads) smla_ix_mark_kernel(const Index
     if (ck.s0 >= ck.s1) return;
     const int u = ck.u;
     if (tid == 0) ccount = 0;
+    const float *sc = p.scores + (size_t)u * p.score_stride;
     uint32_t key[kIxSelIlp];
-    ix_load_chunk(p.scores + (size_t)u * p.score_stride, ck, key);
+    if (p.sel_prefetch) ix_load_chunk(sc, ck, key);
     ix_pdl_wait();
+    if (!p.sel_prefetch) ix_load_chunk(sc, ck, key);
     IxSelMeta *meta = p.sel_meta + u;
-    const bool take_all = meta->take_all != 0;
-    const uint32_t d0 = (uint32_t)meta->d0;
+    ix_decide<kIxSelThreads>(p.sel_hist + (size_t)u * kIxSelBins, p.K, tid, scratch, dec,
+                             [] { __syncthreads(); });
+    __syncthreads();   // dec[] complete (written by one thread)
+    if (ck.s0 == 0 && tid == 0) {
+        meta->take_all = dec[0];
+        meta->d0 = dec[1];
+        meta->need = dec[2];
+    }
+    const bool take_all = dec[0] != 0;
+    const uint32_t d0 = (uint32_t)dec[1];
     uint32_t *bits = p.sel_bits + (size_t)u * p.sel_words;
-    __syncthreads();
 #pragma unroll
     for (int j = 0; j < kIxSelIlp; ++j) {
         const int s = ck.s0 + j * kIxSelThreads + tid;   // a warp covers 32 consecutive positions
@@ -725,7 +804,7 @@ __global__ void __launch_bounds__(kIxFinishThreads) smla_ix_finish_kernel(const 
         eq[i] = 0u;
     }
     if (!meta.take_all) {
-        int need = meta.need;
+        int need = meta.need, n_eq = 0;
         uint32_t prefix = (uint32_t)meta.d0;
 #pragma unroll
         for (int pass = 0; pass < 2; ++pass) {
@@ -740,8 +819,10 @@ __global__ void __launch_bounds__(kIxFinishThreads) smla_ix_finish_kernel(const 
             ix_find_bucket(hist, kIxFineBins, need, scratch, found);
             prefix = (prefix << 10) | (uint32_t)found[0];
             need -= found[1];
+            if (pass == 1) n_eq = (int)hist[found[0] & (kIxFineBins - 1)];   // keys equal to the threshold
         }
         const uint32_t thresh = prefix;
+        const bool all_eq = n_eq == need;   // no tie to break by position
         for (int c = tid; c < m; c += nt) {
             uint32_t key;
             int s;
@@ -753,13 +834,14 @@ __global__ void __launch_bounds__(kIxFinishThreads) smla_ix_finish_kernel(const 
                 key = e.x;
                 s = (int)e.y;
             }
-            if (key > thresh) atomicOr(&sel[s >> 5], 1u << (s & 31));
+            if (key > thresh || (all_eq && key == thresh)) atomicOr(&sel[s >> 5], 1u << (s & 31));
             else if (key == thresh) atomicOr(&eq[s >> 5], 1u << (s & 31));
         }
         __syncthreads();
-        ix_bitmap_scan(eq, words, scratch, [&](int rank, int s) {
-            if (rank < need) atomicOr(&sel[s >> 5], 1u << (s & 31));
-        });
+        if (!all_eq)
+            ix_bitmap_scan(eq, words, scratch, [&](int rank, int s) {
+                if (rank < need) atomicOr(&sel[s >> 5], 1u << (s & 31));
+            });
     }
     __syncthreads();
     const int taken = ix_bitmap_scan(sel, words, scratch, [&](int rank, int s) {
