@@ -197,9 +197,10 @@ struct MmaCfg {
     static_assert(NT == 16 || NT == 32 || NT == 64, "tile rows");
     static constexpr int kHeads = 16 * HG;
     static constexpr int kComputeWarps = 4 * HG;
-    // Two producer warps take alternate tiles: one warp issues about 22 GB/s
-    // of 1-D bulk copies, and two per CTA (four per SM) keep the TMA engine
-    // near the HBM rate.
+    // Two producer warps share every tile's rows (slot s by warp s % 2): one
+    // warp issues only about 22 GB/s of 1-D bulk copies, so a tile issued by
+    // both lands in about half the time, and two per CTA (four per SM) keep
+    // the TMA engine near the HBM rate.
     static constexpr int kProducerWarps = 2;
     static constexpr int kThreads = (kComputeWarps + kProducerWarps) * 32;
     static constexpr int kSRow = NT + 8;  // floats per S-partial row (32-byte pad: conflict-free float2)
@@ -436,7 +437,7 @@ __global__ void __launch_bounds__(MmaCfg<HG, NT, NSTAGE>::kThreads, MmaCfg<HG, N
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < NSTAGE; ++i) {
-            mbar_init(&full[i], 1);
+            mbar_init(&full[i], C::kProducerWarps);  // one arrival (+ its bytes) per producer warp
             mbar_init(&empty[i], C::kComputeWarps);
         }
         fence_mbar_init();
@@ -459,7 +460,7 @@ __global__ void __launch_bounds__(MmaCfg<HG, NT, NSTAGE>::kThreads, MmaCfg<HG, N
 
     if (warp >= C::kComputeWarps) {
         // ============================================================ producers
-        const int pw = warp - C::kComputeWarps;  // takes the tiles it with it % 2 == pw
+        const int pw = warp - C::kComputeWarps;  // issues the rows of slots s with s % 2 == pw
         const uint32_t bar_prod = 2 + HG;        // named barrier of the producer warps
         const uint64_t policy = l2_policy_evict_first();
         int *rows_s = reinterpret_cast<int *>(smem + C::kOffRows);
@@ -484,10 +485,10 @@ __global__ void __launch_bounds__(MmaCfg<HG, NT, NSTAGE>::kThreads, MmaCfg<HG, N
                 // Issue one bulk copy per row (or per padding slot, from the zero row).
                 const int chunk_tiles = (n + NT - 1) / NT;
                 for (int t = 0; t < chunk_tiles; ++t, ++it) {
-                    if ((it & 1) != pw) continue;
                     const int stage = it % NSTAGE;
                     if (it >= NSTAGE) mbar_wait(&empty[stage], ((it / NSTAGE) - 1) & 1, dead);
-                    if (lane == 0) mbar_expect_tx(&full[stage], (uint32_t)(NT * kRowBytes));
+                    constexpr int kMine = (NT - 1) / C::kProducerWarps + 1;  // slots per warp (NT even)
+                    if (lane == 0) mbar_expect_tx(&full[stage], (uint32_t)(kMine * kRowBytes));
                     __syncwarp();
                     uint8_t *dst = smem + C::kOffKV + stage * C::kStageBytes;
                     uint64_t mask = 0;
@@ -497,7 +498,7 @@ __global__ void __launch_bounds__(MmaCfg<HG, NT, NSTAGE>::kThreads, MmaCfg<HG, N
                         const int r = t * NT + slot;
                         const int row = (slot < NT && r < n) ? rows_s[r] : -1;
                         uint8_t *d = dst + slot * kSmemRowBytes;
-                        if (slot < NT) {
+                        if (slot < NT && slot % C::kProducerWarps == pw) {
                             if (row >= 0)
                                 bulk_g2s_hint(d, reinterpret_cast<const uint8_t *>(p.cache) +
                                                      (size_t)row * kRowBytes,
@@ -508,7 +509,7 @@ __global__ void __launch_bounds__(MmaCfg<HG, NT, NSTAGE>::kThreads, MmaCfg<HG, N
                         mask |= (uint64_t)__ballot_sync(0xffffffffu, row >= 0) << (32 * k);
                     }
                     if (lane == 0) {
-                        hdr[stage] = mask;
+                        if (pw == 0) hdr[stage] = mask;
                         mbar_arrive(&full[stage]);  // release: hdr is visible to the waiters
                     }
                 }
@@ -516,7 +517,7 @@ __global__ void __launch_bounds__(MmaCfg<HG, NT, NSTAGE>::kThreads, MmaCfg<HG, N
         }
         // Copies still in flight must land before the CTA may exit.
         for (int k = (it > NSTAGE ? it - NSTAGE : 0); k < it; ++k)
-            if ((k & 1) == pw) mbar_wait(&full[k % NSTAGE], (k / NSTAGE) & 1, dead);
+            mbar_wait(&full[k % NSTAGE], (k / NSTAGE) & 1, dead);
         return;
     }
 
