@@ -107,6 +107,7 @@ KERNEL_SOURCES = {
     "smla_partial_mma_kernel": ["smla_api.cu", "smla_partial_mma.cuh", "smla_ptx.cuh"],
     "smla_partial_tc_kernel": ["smla_api.cu", "smla_partial_mma.cuh", "smla_partial_tc.cuh",
                                "smla_ptx.cuh", "smla_tc_ptx.cuh"],
+    "smla_ix_score_kernel": ["smla_api.cu", "smla_indexer.cuh", "smla_ptx.cuh", "smla_tc_ptx.cuh"],
 }
 
 
