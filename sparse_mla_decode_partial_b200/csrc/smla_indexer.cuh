@@ -454,11 +454,15 @@ __global__ void __launch_bounds__(IxCfg<NPAD>::kThreads, 1)
                 tc_fence_after();
                 const uint32_t ka = sbase + C::kOffStages + st * C::kStageBytes;
                 const uint32_t qa = sbase + C::kOffQ + (changes & 1) * C::kQBytes;
+                // descriptors built once; a k-step adds a constant to the
+                // address field (16-byte units, no carry below 2^18)
+                const uint64_t ad0 = smem_desc(ka, 16, 1024, kSwizzle128B);
+                const uint64_t bd0 = smem_desc(qa, 16, 1024, kSwizzle128B);
 #pragma unroll
                 for (int kk = 0; kk < kIxDim / 16; ++kk) {
                     const uint32_t koff = (kk & 3) * 32;
-                    const uint64_t ad = smem_desc(ka + (kk >> 2) * C::kBoxBytes + koff, 16, 1024, kSwizzle128B);
-                    const uint64_t bd = smem_desc(qa + (kk >> 2) * C::kQBoxBytes + koff, 16, 1024, kSwizzle128B);
+                    const uint64_t ad = ad0 + (uint64_t)(((kk >> 2) * C::kBoxBytes + koff) >> 4);
+                    const uint64_t bd = bd0 + (uint64_t)(((kk >> 2) * C::kQBoxBytes + koff) >> 4);
                     umma_bf16(tmem + a * 64, ad, bd, kIdesc, kk > 0 ? 1u : 0u);
                 }
                 umma_commit(&empty[st]);
