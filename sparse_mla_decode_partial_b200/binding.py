@@ -345,7 +345,7 @@ def decode_host(q, cache, page_table, idx, scale: float, nsplit: int = 0, *, o, 
     return o, lse
 
 
-INDEXER_DIM, INDEXER_MAX_HEADS = 128, 64
+INDEXER_DIM, INDEXER_MAX_HEADS, INDEXER_MAX_N = 128, 64, 524288
 
 
 def indexer_workspace_bytes(B: int, T: int, max_n: int) -> int:

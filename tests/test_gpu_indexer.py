@@ -195,6 +195,34 @@ def test_selection_on_crafted_scores_bit_exact(kind, nv, K):
     assert np.array_equal(got.cpu().numpy(), want)
 
 
+def test_selection_at_the_maximum_length():
+    """max_n = SMLA_INDEXER_MAX_N: the finishing kernel's largest shared-memory
+    configuration (position bitmaps of 524288 positions), the chunked passes'
+    longest grid row, and a K that takes every candidate of a shorter row."""
+    rng = np.random.default_rng(2024)
+    max_n = binding.INDEXER_MAX_N
+    n_vis = np.array([[max_n], [max_n - 37], [1000]], np.int32)
+    sc = rng.standard_normal((3, 1, max_n)).astype(np.float32)
+    sc[1, 0, ::7] = np.nan                        # non-candidates spread over the row
+    scd, nvd = torch.from_numpy(sc).to(DEV), torch.from_numpy(n_vis).to(DEV)
+    for K in (2048, 4096):
+        got = binding.indexer_select(scd, nvd, K)
+        torch.cuda.synchronize()
+        assert np.array_equal(got.cpu().numpy(), ix_oracle.select(sc, n_vis, K)), K
+
+
+def test_selection_many_short_tokens():
+    """Thousands of query tokens with short rows (most chunk CTAs of the 1-D
+    grid have no positions; many tokens take everything)."""
+    rng = np.random.default_rng(99)
+    B, T, max_n = 512, 8, 700
+    n_vis = rng.integers(0, max_n + 1, (B, T)).astype(np.int32)
+    sc = rng.integers(-4, 5, (B, T, max_n)).astype(np.float32)   # many ties
+    got = binding.indexer_select(torch.from_numpy(sc).to(DEV), torch.from_numpy(n_vis).to(DEV), 300)
+    torch.cuda.synchronize()
+    assert np.array_equal(got.cpu().numpy(), ix_oracle.select(sc, n_vis, 300))
+
+
 def test_select_workspace_is_scratch_only():
     """A workspace left dirty by an earlier call (or filled with garbage)
     gives the same selection."""

@@ -45,6 +45,18 @@ def test_status_strings(lib):
     assert lib.smla_version() >= 100
 
 
+def test_binding_constants_match_the_header():
+    """The binding's shape constants are the header's #defines."""
+    import re
+    text = open(os.path.join(ROOT, "include", "smla.h")).read()
+    want = {name: int(v) for name, v in re.findall(r"#define (SMLA_\w+) \(?(\d+)", text)}
+    assert want["SMLA_PAGE_SIZE"] == binding.PAGE_SIZE
+    assert want["SMLA_MAX_NSPLIT"] == binding.MAX_NSPLIT
+    assert want["SMLA_INDEXER_DIM"] == binding.INDEXER_DIM
+    assert want["SMLA_INDEXER_MAX_HEADS"] == binding.INDEXER_MAX_HEADS
+    assert want["SMLA_INDEXER_MAX_N"] == binding.INDEXER_MAX_N
+
+
 def test_workspace_bytes_formula(lib):
     r = lambda x: (x + 255) // 256 * 256
     for B, T, H, S in [(1, 1, 16, 64), (64, 1, 16, 8), (60, 1, 64, 3), (1, 9, 8, 16), (2, 3, 5, 7)]:
