@@ -139,16 +139,15 @@ __device__ __forceinline__ int ix_group_scan(int v, int t, int *scratch, int *to
     return v + base;
 }
 
-// The crossing bucket of token u's first digit from its complete histogram
+// The crossing bucket of a token's first digit from its complete histogram
 // (4096 bins, counted from the top): group thread t holds bins
-// [4096 - per*(t+1), 4096 - per*t) in registers.  Writes (take_all, d0,
-// need) to dec[] (shared); dec is complete after the group's next sync.
-template <int NT, typename Sync>
-__device__ __forceinline__ void ix_decide(const unsigned *gh, int K, int t, int *scratch, int *dec,
-                                          Sync sync) {
+// [4096 - per*(t+1), 4096 - per*t) in registers (ix_decide_load), then one
+// group scan finds the bucket (ix_decide).  Writes (take_all, d0, need) to
+// dec[] (shared); dec is complete after the group's next sync.
+template <int NT>
+__device__ __forceinline__ void ix_decide_load(const unsigned *gh, int t, uint32_t (&b)[4096 / NT]) {
     constexpr int kPer = 4096 / NT;
     static_assert(kPer % 4 == 0, "bins per thread load as uint4");
-    uint32_t b[kPer];
     const int lo = 4096 - kPer * (t + 1);
 #pragma unroll
     for (int q = 0; q < kPer / 4; ++q) {
@@ -158,6 +157,14 @@ __device__ __forceinline__ void ix_decide(const unsigned *gh, int K, int t, int 
         b[4 * q + 2] = v.z;
         b[4 * q + 3] = v.w;
     }
+}
+
+// The scan half of the above over bins already loaded by ix_decide_load.
+template <int NT, typename Sync>
+__device__ __forceinline__ void ix_decide(const uint32_t (&b)[4096 / NT], int K, int t, int *scratch,
+                                          int *dec, Sync sync) {
+    constexpr int kPer = 4096 / NT;
+    const int lo = 4096 - kPer * (t + 1);
     int v = 0;
 #pragma unroll
     for (int k = 0; k < kPer; ++k) v += (int)b[k];
@@ -730,10 +737,12 @@ __global__ void __launch_bounds__(kIxSelThreads) smla_ix_mark_kernel(const Index
     uint32_t key[kIxSelIlp];
     if (p.sel_prefetch) ix_load_chunk(sc, ck, key);
     ix_pdl_wait();
+    // the histogram's loads go out first: the scan needs them before the keys
+    uint32_t bins[kIxSelBins / kIxSelThreads];
+    ix_decide_load<kIxSelThreads>(p.sel_hist + (size_t)u * kIxSelBins, tid, bins);
     if (!p.sel_prefetch) ix_load_chunk(sc, ck, key);
     IxSelMeta *meta = p.sel_meta + u;
-    ix_decide<kIxSelThreads>(p.sel_hist + (size_t)u * kIxSelBins, p.K, tid, scratch, dec,
-                             [] { __syncthreads(); });
+    ix_decide<kIxSelThreads>(bins, p.K, tid, scratch, dec, [] { __syncthreads(); });
     __syncthreads();   // dec[] complete (written by one thread)
     if (ck.s0 == 0 && tid == 0) {
         meta->take_all = dec[0];
@@ -794,6 +803,10 @@ __global__ void __launch_bounds__(kIxFinishThreads) smla_ix_finish_kernel(const 
     const IxSelMeta meta = p.sel_meta[u];
     const uint32_t *gbits = p.sel_bits + (size_t)u * p.sel_words;
     const uint2 *gcand = p.sel_cand + (size_t)u * p.max_n;
+    for (int i = tid; i < words; i += nt) {  // independent of meta: first
+        sel[i] = gbits[i];
+        eq[i] = 0u;
+    }
     const int m = meta.take_all ? 0 : meta.count;
     const bool in_smem = m <= kIxCandCap;
     if (in_smem) {
@@ -802,10 +815,6 @@ __global__ void __launch_bounds__(kIxFinishThreads) smla_ix_finish_kernel(const 
             cand_key[c] = e.x;
             cand_pos[c] = (int)e.y;
         }
-    }
-    for (int i = tid; i < words; i += nt) {
-        sel[i] = gbits[i];
-        eq[i] = 0u;
     }
     if (!meta.take_all) {
         int need = meta.need, n_eq = 0;
