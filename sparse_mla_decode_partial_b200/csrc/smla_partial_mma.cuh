@@ -17,10 +17,11 @@
 //   warps 4*HG,    producers: every thread of the CTA first resolves the
 //   4*HG+1         split's index entries to physical rows (index loads, then
 //                  page-table loads, a batch in flight at once) into shared
-//                  memory; then the two producer warps take alternate tiles
-//                  and issue one 1-D bulk async copy (TMA engine, 1152 B) per
-//                  row into a ring of NSTAGE tiles of NT rows, each completing
-//                  on an mbarrier.
+//                  memory; then both producer warps issue every tile (one
+//                  the rows of even slots, the other the odd ones), one 1-D
+//                  bulk async copy (TMA engine, 1152 B) per row into a ring of
+//                  NSTAGE tiles of NT rows, each tile completing on an
+//                  mbarrier that counts both warps and their bytes.
 //   warps 0..4HG-1 consumers, 4 per head group.  Each warp keeps the Q
 //                  fragments of one quarter of the 576 dims in registers and
 //                  computes that quarter's partial S = Q K^T for all NT rows

@@ -22,7 +22,9 @@
 //              K-major layout (each warp instruction moves 4 rows x 128 B,
 //              coalesced); completion reaches the tile's mbarrier through
 //              cp.async.mbarrier.arrive.  Padding slots copy row 0 and are
-//              masked.
+//              masked.  In dense mode a tile of 32 consecutive cache rows
+//              moves instead with nine TMA tile loads (32 rows x 64 values,
+//              128B swizzle) on the same barrier.
 //   warp 15    TMEM owner + MMA issuer (one thread):
 //                QK(pair): S[64 x 64] = Q[64 x 576] [K_2p K_2p+1]^T   36 x (M64 N64 K16), A in TMEM
 //                PV(t):    O[64 x 512] += P_t[64 x 32] C_t[32 x 512]  2 x 2 x (M64 N256 K16)
@@ -30,7 +32,10 @@
 //              below M64 N64 (M64 N32 costs the same as M64 N64), so the
 //              two tiles of a pair share one N = 64 score MMA per k-step: the
 //              ring keeps the pair's tiles side by side in every 64-column
-//              box.  The issuer polls: a pair's QK goes out as soon as both
+//              box.  The 36 score MMAs of a pair go out as one burst from
+//              descriptors built once per pair (rebuilding them per MMA, or
+//              splitting the burst, left the tensor pipe waiting).  The
+//              issuer polls: a pair's QK goes out as soon as both
 //              tiles have landed, its PV as soon as its P is ready.
 // Shared memory ring: three pair slots of 2 x 36864 B (Q is not in shared
 // memory); box b (64 columns) of tile h of a slot at slot + 8192 b + 4096 h,
