@@ -112,12 +112,18 @@ KERNEL_SOURCES = {
 
 
 def kernel_sources_hash(kernel: str) -> str:
-    """sha256[:16] over the kernel's source files (KERNEL_SOURCES), in order."""
+    """sha256[:16] over the kernel's source files (KERNEL_SOURCES), in order,
+    with comments and whitespace removed (a comment edit does not change the
+    kernel)."""
     import hashlib
+    import re
     h = hashlib.sha256()
     for name in KERNEL_SOURCES[kernel]:
-        with open(os.path.join(ROOT, "sparse_mla_decode_partial_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "sparse_mla_decode_partial_b200", "csrc", name)) as f:
+            text = f.read()
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)   # block comments
+        text = re.sub(r"//[^\n]*", " ", text)                 # line comments
+        h.update(re.sub(r"\s+", "", text).encode())
     return h.hexdigest()[:16]
 
 
