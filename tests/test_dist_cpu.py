@@ -117,8 +117,8 @@ def test_reference_arm_dense_workload(tmp_path):
 
 def test_traffic_record_tracks_its_kernel_sources(tmp_path, monkeypatch):
     """roofline.traffic is reported only while the captured kernel's own source
-    files are unchanged: editing the tcgen05 kernel drops the tcgen05 figures
-    and keeps the others."""
+    files are unchanged (comments aside): editing the tcgen05 kernel's code
+    drops the tcgen05 figures and keeps the others."""
     import shutil
     sys.path.insert(0, ROOT)
     import bench
@@ -135,7 +135,9 @@ def test_traffic_record_tracks_its_kernel_sources(tmp_path, monkeypatch):
     before = {wl: bench.measured_traffic(wl) for wl in kernels}
     assert before == {"single_request": 1000, "batched": 1001, "mixed": 1002}
     tc = tmp_path / csrc / "smla_partial_tc.cuh"
-    tc.write_text(tc.read_text() + "\n// edited\n")
+    tc.write_text(tc.read_text() + "\n// a comment edit does not change the kernel\n")
+    assert bench.measured_traffic("mixed") == before["mixed"]
+    tc.write_text(tc.read_text() + "\nstatic_assert(true, \"a code edit\");\n")
     assert bench.measured_traffic("mixed") is None
     assert bench.measured_traffic("single_request") == before["single_request"]
     assert bench.measured_traffic("batched") == before["batched"]
