@@ -123,9 +123,12 @@ size_t smla_workspace_bytes(int B, int T, int H, int nsplit);
  *   nsplit     S in [1, SMLA_MAX_NSPLIT]
  * Outputs (fp32, device, caller-owned):
  *   part_o   [B, T, H, S, 512]  sum_j exp(s_j - part_m) c_j   (unnormalised)
- *   part_m   [B, T, H, S]       the reference point part_o is scaled by: the
- *                               split's maximum score (-inf for a split with
- *                               no valid entry)
+ *   part_m   [B, T, H, S]       the reference point part_o is scaled by: at
+ *                               most 8 ln 2 below the split's maximum score
+ *                               and never above it (the tcgen05 kernel moves
+ *                               it only when a score exceeds it by more than
+ *                               that; the others keep the exact maximum);
+ *                               -inf for a split with no valid entry
  *   part_lse [B, T, H, S]       ln sum_j exp(s_j) over the split (-inf if empty)
  * so part_o * exp(part_m - part_lse) is the split's normalised output.
  * An empty split writes part_o = 0, part_m = part_lse = -inf.
