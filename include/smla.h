@@ -46,6 +46,11 @@
  *  - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL is
  *    the legacy default stream).  Arguments are checked on the host before
  *    anything is launched; a failed check launches nothing.
+ *  - The first kernel of a decode is launched as a programmatic dependent
+ *    of the stream's previous work: its grid may be scheduled early, but it
+ *    waits for that work to complete before it touches global memory.  This
+ *    keeps stream order for every predecessor that is itself ordered (any
+ *    kernel launched without the programmatic attribute, a copy, an event).
  *  - q, kv_cache, part_o, o and workspace must be 16-byte aligned; int32 and
  *    fp32 arrays 4-byte aligned.  Otherwise SMLA_ERR_MISALIGNED.
  *  - Dimensions are fixed at 512 + 64 and page_size must be 64; heads per

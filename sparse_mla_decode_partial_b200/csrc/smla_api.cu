@@ -12,6 +12,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
+#include <utility>
 #include <set>
 #include <utility>
 
@@ -145,14 +146,36 @@ smla_status check_decode_args(const void *q, const void *kv_cache, int64_t num_p
     return SMLA_OK;
 }
 
+// Launch of a partial-pass kernel as a programmatic dependent of whatever
+// precedes it on the stream (the host entry point's copy kernel, a previous
+// decode, a user's kernel): its grid may be scheduled as soon as the
+// predecessor lets it, and every partial kernel executes griddepcontrol.wait
+// before its first global memory access and before it takes tensor memory.
+// With no programmatic predecessor the wait returns at once.
+template <typename... Params, typename... Args>
+cudaError_t launch_dependent(void (*kernel)(Params...), int grid, int threads, size_t smem,
+                             cudaStream_t st, Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3((unsigned)threads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 template <int HG, int NT, int NS, bool DIRECT>
 smla_status launch_mma(const PartialParams &p, int grid, cudaStream_t st) {
     using C = smla::MmaCfg<HG, NT, NS>;
     const void *fn = reinterpret_cast<const void *>(&smla::smla_partial_mma_kernel<HG, NT, NS, DIRECT>);
     cudaError_t e = ensure_smem_attr(fn, C::kSmemBytes);
     if (e != cudaSuccess) return cuda_fail(e);
-    smla::smla_partial_mma_kernel<HG, NT, NS, DIRECT><<<grid, C::kThreads, C::kSmemBytes, st>>>(p);
-    e = cudaGetLastError();
+    e = launch_dependent(smla::smla_partial_mma_kernel<HG, NT, NS, DIRECT>, grid, C::kThreads,
+                         C::kSmemBytes, st, p);
     return e == cudaSuccess ? SMLA_OK : cuda_fail(e);
 }
 
@@ -172,8 +195,8 @@ smla_status launch_tc(const PartialParams &p, int grid, cudaStream_t st) {
         const smla_status s = encode_cache_tiles(&map, p.cache, p.num_pages);
         if (s != SMLA_OK) return s;
     }
-    smla::smla_partial_tc_kernel<DIRECT><<<grid, smla::TcCfg::kThreads, smla::TcCfg::kSmemBytes, st>>>(p, map);
-    e = cudaGetLastError();
+    e = launch_dependent(smla::smla_partial_tc_kernel<DIRECT>, grid, smla::TcCfg::kThreads,
+                         smla::TcCfg::kSmemBytes, st, p, map);
     return e == cudaSuccess ? SMLA_OK : cuda_fail(e);
 }
 
@@ -183,9 +206,8 @@ smla_status launch_small(const PartialParams &p, int grid, cudaStream_t st) {
     const void *fn = reinterpret_cast<const void *>(&smla::smla_partial_small_kernel<HG, TILES, DIRECT>);
     cudaError_t e = ensure_smem_attr(fn, C::kMaxSmemBytes);
     if (e != cudaSuccess) return cuda_fail(e);
-    smla::smla_partial_small_kernel<HG, TILES, DIRECT>
-        <<<grid, C::kThreads, C::smem_bytes(p.pt_stride), st>>>(p);
-    e = cudaGetLastError();
+    e = launch_dependent(smla::smla_partial_small_kernel<HG, TILES, DIRECT>, grid, C::kThreads,
+                         C::smem_bytes(p.pt_stride), st, p);
     return e == cudaSuccess ? SMLA_OK : cuda_fail(e);
 }
 
@@ -603,9 +625,16 @@ smla_status smla_decode_host(const void *q_host, const void *kv_cache, int64_t n
         a.r[1] = {static_cast<const uint8_t *>(idx_d), ws + hs.idx, (size_t)B * T * K * 4};
         a.r[2] = {static_cast<const uint8_t *>(pt_d), ws + hs.pt, (size_t)B * pt_stride * 4};
     }
-    const size_t words = (a.r[0].bytes + a.r[1].bytes + a.r[2].bytes) / 16 + 1;
-    const unsigned blocks = (unsigned)std::min<size_t>((words + 255) / 256, (size_t)current_device_sms());
-    smla::smla_ingest_kernel<<<blocks, 256, 0, st>>>(a);
+    // one item per thread while the step is small (a single round trip over
+    // the host link), at most one CTA per SM beyond that
+    size_t items = 0;  // the kernel's item count (ingest_counts)
+    for (const smla::IngestRegion &r : a.r) {
+        const size_t n16 = aligned(r.src, 16) ? r.bytes / 16 : 0;
+        items += n16 + (r.bytes - n16 * 16) / 4;
+    }
+    const unsigned blocks = (unsigned)std::min<size_t>(
+        (items + smla::kIngestThreads - 1) / smla::kIngestThreads, (size_t)current_device_sms());
+    smla::smla_ingest_kernel<<<blocks, smla::kIngestThreads, 0, st>>>(a);
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e);
     return smla_decode(ws + hs.q, kv_cache, num_pages, reinterpret_cast<const int32_t *>(ws + hs.pt),

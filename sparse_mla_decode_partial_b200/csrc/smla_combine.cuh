@@ -317,8 +317,13 @@ __global__ void __launch_bounds__(32) smla_selftest_wait_kernel(unsigned long lo
 }
 
 // Copy of the per-step inputs of smla_decode_host from pinned host memory
-// (addressed through its device alias) into the workspace's staging area:
-// up to three regions, 16-byte vectors for the body, 4-byte words for a tail.
+// (addressed through its device alias) into the workspace's staging area.
+// Every read crosses the host link, so its latency (about a microsecond)
+// dominates a small step: the three regions are flattened into one item
+// space (16-byte vectors where the source allows them, then 4-byte words for
+// a tail) and each thread issues the loads of all its items, up to
+// kIngestDepth of them, before it stores any.  A step whose items fit the
+// grid's threads then costs one round trip, not one per region.
 struct IngestRegion {
     const uint8_t *src;
     uint8_t *dst;
@@ -327,20 +332,63 @@ struct IngestRegion {
 struct IngestArgs {
     IngestRegion r[3];
 };
+constexpr int kIngestThreads = 256;
+constexpr int kIngestDepth = 4;  // items in flight per thread
 
-__global__ void __launch_bounds__(256) smla_ingest_kernel(const IngestArgs a) {
-    const size_t tid = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
-    const size_t nthreads = (size_t)gridDim.x * blockDim.x;
+// Item counts of one region: n16 vectors (none when the source is not
+// 16-byte aligned) followed by the remaining 4-byte words.
+__device__ __forceinline__ void ingest_counts(const IngestRegion &r, size_t &n16, size_t &n) {
+    n16 = (reinterpret_cast<uintptr_t>(r.src) & 15) ? 0 : r.bytes / 16;
+    n = n16 + (r.bytes - n16 * 16) / 4;
+}
+
+__global__ void __launch_bounds__(kIngestThreads) smla_ingest_kernel(const IngestArgs a) {
+    // the partial pass is launched as a programmatic dependent: let it be
+    // scheduled now (it waits for this grid's completion before reading)
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    size_t n16[3], end[3];
+    size_t total = 0;
 #pragma unroll
     for (int k = 0; k < 3; ++k) {
-        const IngestRegion r = a.r[k];
-        // destinations are 256-byte aligned; the source decides the width
-        const size_t n16 = (reinterpret_cast<uintptr_t>(r.src) & 15) ? 0 : r.bytes / 16;
-        const uint4 *s16 = reinterpret_cast<const uint4 *>(r.src);
-        uint4 *d16 = reinterpret_cast<uint4 *>(r.dst);
-        for (size_t i = tid; i < n16; i += nthreads) d16[i] = s16[i];
-        for (size_t i = n16 * 4 + tid; i < r.bytes / 4; i += nthreads)
-            reinterpret_cast<uint32_t *>(r.dst)[i] = reinterpret_cast<const uint32_t *>(r.src)[i];
+        size_t n;
+        ingest_counts(a.r[k], n16[k], n);
+        total += n;
+        end[k] = total;
+    }
+    const size_t nthreads = (size_t)gridDim.x * blockDim.x;
+    for (size_t i0 = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i0 < total;
+         i0 += nthreads * kIngestDepth) {
+        uint4 v[kIngestDepth];
+        uint8_t *dst[kIngestDepth];
+        bool wide[kIngestDepth];
+#pragma unroll
+        for (int j = 0; j < kIngestDepth; ++j) {
+            const size_t i = i0 + (size_t)j * nthreads;
+            dst[j] = nullptr;
+            wide[j] = false;
+            if (i < total) {
+                const int k = i < end[0] ? 0 : (i < end[1] ? 1 : 2);
+                const size_t local = i - (k == 0 ? 0 : end[k - 1]);
+                const IngestRegion &r = a.r[k];
+                if (local < n16[k]) {
+                    v[j] = reinterpret_cast<const uint4 *>(r.src)[local];
+                    dst[j] = r.dst + local * 16;
+                    wide[j] = true;
+                } else {
+                    const size_t off = n16[k] * 16 + (local - n16[k]) * 4;
+                    v[j].x = *reinterpret_cast<const uint32_t *>(r.src + off);
+                    dst[j] = r.dst + off;
+                }
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < kIngestDepth; ++j) {
+            if (dst[j] == nullptr) continue;
+            if (wide[j])
+                *reinterpret_cast<uint4 *>(dst[j]) = v[j];
+            else
+                *reinterpret_cast<uint32_t *>(dst[j]) = v[j].x;
+        }
     }
 }
 

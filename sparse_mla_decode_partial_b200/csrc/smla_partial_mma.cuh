@@ -446,6 +446,9 @@ __global__ void __launch_bounds__(MmaCfg<HG, NT, NSTAGE>::kThreads, MmaCfg<HG, N
     // The combine kernel is launched as a programmatic dependent: let it be
     // scheduled now; it waits for this grid's completion before reading.
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    // This grid is itself a programmatic dependent of what precedes it on the
+    // stream: wait for that to complete before the first global access.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     // Every thread helps resolve the first chunk of the first item, so that
     // the first copies start after two memory round trips (one warp alone
     // took several microseconds for a 512-entry split).
@@ -602,6 +605,9 @@ __global__ void __launch_bounds__(SmallCfg<HG, TILES>::kThreads)
     int *rows_s = reinterpret_cast<int *>(smem + C::kOffRows);  // [TILES * 32] rows, then masks
     int *pt_s = reinterpret_cast<int *>(smem + C::kOffPt);
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    // launched as a programmatic dependent: the predecessor on the stream
+    // completes before the first global access
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 
     // 1. page-table row, this split's indices and Q: all loads in flight at once
     const int *pt_b = p.page_table + (size_t)b * p.pt_stride;

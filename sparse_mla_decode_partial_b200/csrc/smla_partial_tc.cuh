@@ -159,6 +159,11 @@ __global__ void __launch_bounds__(TcCfg::kThreads, 1)
         mbar_init(q_ready, 4);
         fence_mbar_init();
     }
+    // Launched as a programmatic dependent of whatever precedes it on the
+    // stream: everything above touches only shared memory; from here on the
+    // kernel reads global memory and takes tensor memory, so it first waits
+    // for its predecessor to complete.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     if (warp == C::kMmaWarp) {
         tmem_alloc(tmem_slot, C::kTmemCols);
         tmem_relinquish();
