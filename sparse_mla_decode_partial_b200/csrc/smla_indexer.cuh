@@ -239,12 +239,17 @@ __global__ void __launch_bounds__(1024) smla_ix_plan_kernel(const IndexerParams 
     if (threadIdx.x == 0) p.tile_start[p.BT] = carry;
 }
 
+// tile_start is written by the plan kernel, whose programmatic dependent (the
+// score kernel) is resident while it runs: it is read with weak global loads
+// (ld_input), never through the read-only path.  The caller's inputs (n_vis, w, the page
+// table, the keys) are complete before the plan kernel starts.
+//
 // Token holding unit `unit` (tile_start ascending; tokens with no tile skipped).
 __device__ __forceinline__ int ix_token_of(const IndexerParams &p, long long unit) {
     int lo = 0, hi = p.BT - 1;  // the last token with tile_start <= unit
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
-        if (__ldg(p.tile_start + mid) <= unit) lo = mid; else hi = mid - 1;
+        if (ld_input(p.tile_start + mid) <= unit) lo = mid; else hi = mid - 1;
     }
     return lo;
 }
@@ -264,8 +269,8 @@ struct IxUnit {
 __device__ __forceinline__ IxUnit ix_unit(const IndexerParams &p, long long unit, int hint) {
     IxUnit m;
     m.tok = hint;
-    while (__ldg(p.tile_start + m.tok + 1) <= unit) ++m.tok;
-    m.tile = (int)(unit - __ldg(p.tile_start + m.tok));
+    while (ld_input(p.tile_start + m.tok + 1) <= unit) ++m.tok;
+    m.tile = (int)(unit - ld_input(p.tile_start + m.tok));
     m.n = ix_visible(p, m.tok);
     const int *pt_b = p.page_table + (size_t)(m.tok / p.T) * p.pt_stride;
     int pg[2];
@@ -384,7 +389,7 @@ __global__ void __launch_bounds__(IxCfg<NPAD>::kThreads, 1)
     bool dead = false;
 
     // this CTA's units: an equal share of all (token, tile) units
-    const long long n_units = __ldg(p.tile_start + p.BT);
+    const long long n_units = ld_input(p.tile_start + p.BT);
     const long long u_begin = n_units * blockIdx.x / gridDim.x;
     const long long u_end = n_units * (blockIdx.x + 1) / gridDim.x;
 
@@ -447,7 +452,7 @@ __global__ void __launch_bounds__(IxCfg<NPAD>::kThreads, 1)
             int tok = ix_token_of(p, u_begin), changes = -1;
             for (long long unit = u_begin, i = 0; unit < u_end; ++unit, ++i) {
                 bool fresh = unit == u_begin;
-                while (__ldg(p.tile_start + tok + 1) <= unit) {
+                while (ld_input(p.tile_start + tok + 1) <= unit) {
                     ++tok;
                     fresh = true;
                 }
@@ -475,7 +480,7 @@ __global__ void __launch_bounds__(IxCfg<NPAD>::kThreads, 1)
                 umma_commit(&empty[st]);
                 umma_commit(&acc_full[a]);
                 // the token's last unit here: its query slot may be refilled
-                if (unit + 1 == u_end || __ldg(p.tile_start + tok + 1) <= unit + 1)
+                if (unit + 1 == u_end || ld_input(p.tile_start + tok + 1) <= unit + 1)
                     umma_commit(&q_empty[changes & 1]);
             }
         }
@@ -677,13 +682,15 @@ __device__ __forceinline__ IxChunk ix_chunk(const IndexerParams &p) {
     return {u, s0, min(ix_visible(p, u), s0 + kIxSelChunk)};
 }
 
-// The chunk's keys, one load round trip (lane-consecutive positions).
+// The chunk's keys, one load round trip (lane-consecutive positions); coherent
+// loads, since the score kernel may have written them while this grid was
+// already resident.
 __device__ __forceinline__ void ix_load_chunk(const float *sc, const IxChunk &ck,
                                               uint32_t (&key)[kIxSelIlp]) {
 #pragma unroll
     for (int j = 0; j < kIxSelIlp; ++j) {
         const int s = ck.s0 + j * kIxSelThreads + (int)threadIdx.x;
-        key[j] = s < ck.s1 ? ix_key(__ldg(sc + s)) : 0u;
+        key[j] = s < ck.s1 ? ix_key(__ldcg(sc + s)) : 0u;
     }
 }
 

@@ -34,6 +34,15 @@
 //                  128 of the 512 output columns in fp32 registers.
 // Shared-memory rows are 1168 B apart (1152 + 16) so that the 8 row addresses
 // of every ldmatrix phase fall in distinct 16-byte bank groups.
+//
+// Every partial kernel is launched as a programmatic dependent of what
+// precedes it on the stream and waits (griddepcontrol.wait) before its first
+// global access.  Its inputs (q, the indices, the page table) may therefore
+// be written by the predecessor while this grid is already resident, so they
+// are read with weak global loads (ld_input), which the wait makes see the
+// predecessor's writes, never through the read-only path, whose contract is
+// that the data stays unchanged for the kernel's lifetime.
+// The cache rows arrive by cp.async.cg, bulk or tensor copies (all through L2).
 #pragma once
 
 #include <cstdint>
@@ -165,13 +174,13 @@ __device__ __forceinline__ void resolve_rows(const PartialParams &p, int bt, int
 #pragma unroll
         for (int k = 0; k < BATCH; ++k) {
             const int j = b0 + k * nthreads + tid;
-            iv[k] = (j < n) ? __ldg(idx_bt + j) : -1;
+            iv[k] = (j < n) ? ld_input(idx_bt + j) : -1;
         }
         int pg[BATCH];
 #pragma unroll
         for (int k = 0; k < BATCH; ++k) {
             const int i = iv[k];
-            pg[k] = (i >= 0 && (long long)i < max_pos) ? __ldg(pt_b + (i >> 6)) : -1;
+            pg[k] = (i >= 0 && (long long)i < max_pos) ? ld_input(pt_b + (i >> 6)) : -1;
         }
 #pragma unroll
         for (int k = 0; k < BATCH; ++k) {
@@ -260,7 +269,7 @@ struct MmaConsumer {
         for (int i = 0; i < 9; ++i) {
             const int c = lane + 32 * i;  // 16 rows x 18 chunks of 8 dims
             const int h = 16 * g + c / 18;
-            qv[i] = (h < p.H) ? __ldg(qsrc + (size_t)h * (kD / 8) + KQ * 2 * qw + c % 18)
+            qv[i] = (h < p.H) ? ld_input(qsrc + (size_t)h * (kD / 8) + KQ * 2 * qw + c % 18)
                               : make_uint4(0u, 0u, 0u, 0u);
         }
 #pragma unroll
@@ -616,7 +625,7 @@ __global__ void __launch_bounds__(SmallCfg<HG, TILES>::kThreads)
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
             const int i = i0 + k * C::kThreads + tid;
-            v[k] = (i < p.pt_stride) ? __ldg(pt_b + i) : -1;
+            v[k] = (i < p.pt_stride) ? ld_input(pt_b + i) : -1;
         }
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
@@ -625,7 +634,7 @@ __global__ void __launch_bounds__(SmallCfg<HG, TILES>::kThreads)
         }
     }
     int my_idx = -1;
-    if (tid < NT * TILES && j0 + tid < j1) my_idx = __ldg(p.idx + (size_t)bt * p.K + j0 + tid);
+    if (tid < NT * TILES && j0 + tid < j1) my_idx = ld_input(p.idx + (size_t)bt * p.K + j0 + tid);
     MmaConsumer<NT, HG> cons;
     cons.init(warp, lane);
     cons.load_q(smem + C::kOffQ, p, bt);

@@ -37,6 +37,10 @@
 //              splitting the burst, left the tensor pipe waiting).  The
 //              issuer polls: a pair's QK goes out as soon as both
 //              tiles have landed, its PV as soon as its P is ready.
+// Like the other partial kernels it is a programmatic dependent of what
+// precedes it on the stream: it waits before touching global memory or tensor
+// memory, and reads q, the indices, the lengths and the page table with weak
+// global loads (ld_input), never through the read-only path.
 // Shared memory ring: three pair slots of 2 x 36864 B (Q is not in shared
 // memory); box b (64 columns) of tile h of a slot at slot + 8192 b + 4096 h,
 // rows 128 B apart.
@@ -187,7 +191,7 @@ __global__ void __launch_bounds__(TcCfg::kThreads, 1)
         int n_unit = 0;
         if (dense) {
             for (int t = 0; t < ntok; ++t) {
-                const int raw = __ldg(p.seq_lens + (size_t)b * p.dense_t + tok0 + t);
+                const int raw = ld_input(p.seq_lens + (size_t)b * p.dense_t + tok0 + t);
                 n_unit = max(n_unit, min(max(raw, 0), p.K));
                 if (s == 0 && ptid == t && (raw < 0 || raw > p.K)) {
                     atomicOr(&g_status_flags, kFlagIndexRange);
@@ -219,14 +223,14 @@ __global__ void __launch_bounds__(TcCfg::kThreads, 1)
                         const int pos = j0 + base + j;
                         iv[k] = (j < n && pos < n_unit) ? pos : -1;
                     } else {
-                        iv[k] = (j < n) ? __ldg(idx_bt + base + j) : -1;
+                        iv[k] = (j < n) ? ld_input(idx_bt + base + j) : -1;
                     }
                 }
                 int pg[16];
 #pragma unroll
                 for (int k = 0; k < 16; ++k) {
                     const int i = iv[k];
-                    pg[k] = (i >= 0 && (long long)i < max_pos) ? __ldg(pt_b + (i >> 6)) : -1;
+                    pg[k] = (i >= 0 && (long long)i < max_pos) ? ld_input(pt_b + (i >> 6)) : -1;
                 }
 #pragma unroll
                 for (int k = 0; k < 16; ++k) {
@@ -406,7 +410,7 @@ __global__ void __launch_bounds__(TcCfg::kThreads, 1)
                 uint32_t w[32];
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
-                    const uint4 v = real ? __ldg(qrow + 16 * i + 8 * half + k) : make_uint4(0u, 0u, 0u, 0u);
+                    const uint4 v = real ? ld_input(qrow + 16 * i + 8 * half + k) : make_uint4(0u, 0u, 0u, 0u);
                     w[4 * k] = v.x;
                     w[4 * k + 1] = v.y;
                     w[4 * k + 2] = v.z;
@@ -418,7 +422,7 @@ __global__ void __launch_bounds__(TcCfg::kThreads, 1)
                 uint32_t w[16];
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
-                    const uint4 v = real ? __ldg(qrow + 64 + 4 * half + k) : make_uint4(0u, 0u, 0u, 0u);
+                    const uint4 v = real ? ld_input(qrow + 64 + 4 * half + k) : make_uint4(0u, 0u, 0u, 0u);
                     w[4 * k] = v.x;
                     w[4 * k + 1] = v.y;
                     w[4 * k + 2] = v.z;
@@ -436,7 +440,7 @@ __global__ void __launch_bounds__(TcCfg::kThreads, 1)
         // real rows see none); sparse: no per-row limit
         int lim = INT_MAX;
         if (dense)
-            lim = hrow < nrows ? min(max(__ldg(p.seq_lens + (size_t)b * p.dense_t + tok0 +
+            lim = hrow < nrows ? min(max(ld_input(p.seq_lens + (size_t)b * p.dense_t + tok0 +
                                                hrow / p.dense_h), 0), p.K)
                                : 0;
         float m_ref = -INFINITY;  // running reference max of head hrow (log2 units)

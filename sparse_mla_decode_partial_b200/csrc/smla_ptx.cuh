@@ -29,6 +29,25 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
 }
 
 // ---------------------------------------------------------------- mbarrier
+// Weak global loads (the default cache policy, L1 included) for data that a
+// programmatic predecessor may write while this grid is resident: once
+// griddepcontrol.wait has returned, the predecessor's writes are visible to
+// them.  The read-only path (ld.global.nc, __ldg) is not used for such data:
+// it requires the data to stay unchanged for the kernel's whole lifetime.
+// Volatile asm keeps each load after the wait in program order.
+__device__ __forceinline__ int ld_input(const int *p) {
+    int v;
+    asm volatile("ld.global.s32 %0, [%1];" : "=r"(v) : "l"(p));
+    return v;
+}
+__device__ __forceinline__ uint4 ld_input(const uint4 *p) {
+    uint4 v;
+    asm volatile("ld.global.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
 __device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count)
                  : "memory");

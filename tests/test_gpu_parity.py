@@ -663,3 +663,78 @@ def test_concurrent_host_threads_on_separate_streams():
     for i, w in enumerate(cases):
         o_ref, lse_ref, _ = oracle_decode(w)
         check_o_lse(results[i][0], results[i][1], o_ref, lse_ref, f"thread {i}")
+
+
+# ------------------------------------------------------------------ inputs rewritten between calls
+def _second_inputs(w, seed):
+    """Same shapes and cache, another q and another selection (every valid
+    position moved to the next one of its sequence, padding kept), so that a
+    stale read of either input from the previous call shows in the output."""
+    g = torch.Generator().manual_seed(seed)
+    q2 = (torch.randn(w.q.shape, generator=g) * 0.5).to(torch.bfloat16)
+    ctx = torch.tensor(w.ctx_lens, dtype=torch.int32).view(-1, 1, 1)
+    idx2 = torch.where(w.idx >= 0, (w.idx + 1) % ctx, w.idx).to(torch.int32).contiguous()
+    return q2, idx2
+
+
+@pytest.mark.parametrize("name", ["single_request", "spec_verify", "tiny", "batched", "mixed"])
+def test_decode_host_inputs_change_every_call(name):
+    """The partial pass is a programmatic dependent of the copy kernel that
+    fills the workspace's staging area, so every call overwrites inputs that
+    the previous call read.  Alternate two input sets on one workspace: each
+    call must match the device decode of its own inputs bit for bit."""
+    w = workloads.WORKLOADS[name]()
+    wd = w.to(DEV)
+    q2, idx2 = _second_inputs(w, 11)
+    sets = [(w.q, w.idx), (q2, idx2)]
+    refs = [binding.decode(q.to(DEV), wd.cache, wd.page_table, i.to(DEV), w.scale, 0) for q, i in sets]
+    torch.cuda.synchronize()
+    q_h, idx_h, pt_h = w.q.pin_memory(), w.idx.pin_memory(), w.page_table.pin_memory()
+    o_h = torch.empty(refs[0][0].shape, dtype=torch.bfloat16).pin_memory()
+    lse_h = torch.empty(refs[0][1].shape, dtype=torch.float32).pin_memory()
+    B, T, H, K = w.B, w.T, w.H, w.K
+    S = binding.choose_nsplit(B, T, H, K, 0)
+    ws = torch.empty(binding.workspace_host_bytes(B, T, H, K, w.pt_stride, S), dtype=torch.uint8,
+                     device=DEV)
+    calls = 12 if name in ("batched", "mixed") else 24
+    for c in range(calls):
+        q, i = sets[c % 2]
+        q_h.copy_(q)
+        idx_h.copy_(i)
+        binding.decode_host(q_h, wd.cache, pt_h, idx_h, w.scale, S, o=o_h, lse=lse_h, workspace=ws)
+        torch.cuda.synchronize()
+        o_ref, lse_ref = refs[c % 2]
+        assert torch.equal(o_h, o_ref.cpu()) and torch.equal(lse_h, lse_ref.cpu()), f"call {c}"
+
+
+@pytest.mark.parametrize("name", ["single_request", "spec_verify", "batched", "mixed", "dense_verify"])
+def test_decode_right_after_a_kernel_that_rewrites_its_inputs(name):
+    """Device path: a copy kernel rewrites q and the selection (or the visible
+    lengths) on the stream just before each decode, alternating two sets; the
+    decode's first kernel may be scheduled while that copy still runs and
+    must still read the new inputs."""
+    w = workloads.WORKLOADS[name]()
+    wd = w.to(DEV)
+    if w.dense:
+        g = torch.Generator().manual_seed(12)
+        q2 = (torch.randn(w.q.shape, generator=g) * 0.5).to(torch.bfloat16)
+        lens2 = (w.seq_lens - 37).clamp(min=0)
+        sets = [(w.q.to(DEV), w.seq_lens.to(DEV)), (q2.to(DEV), lens2.to(DEV))]
+        refs = [binding.decode_dense(q, wd.cache, wd.page_table, l, w.scale, 0, K=w.K) for q, l in sets]
+    else:
+        q2, idx2 = _second_inputs(w, 12)
+        sets = [(w.q.to(DEV), w.idx.to(DEV)), (q2.to(DEV), idx2.to(DEV))]
+        refs = [binding.decode(q, wd.cache, wd.page_table, i, w.scale, 0) for q, i in sets]
+    torch.cuda.synchronize()
+    q_d, sel_d = sets[0][0].clone(), sets[0][1].clone()
+    for c in range(16):
+        q, sel = sets[c % 2]
+        q_d.copy_(q)
+        sel_d.copy_(sel)
+        if w.dense:
+            o, lse = binding.decode_dense(q_d, wd.cache, wd.page_table, sel_d, w.scale, 0, K=w.K)
+        else:
+            o, lse = binding.decode(q_d, wd.cache, wd.page_table, sel_d, w.scale, 0)
+        torch.cuda.synchronize()
+        o_ref, lse_ref = refs[c % 2]
+        assert torch.equal(o, o_ref) and torch.equal(lse, lse_ref), f"call {c}"
