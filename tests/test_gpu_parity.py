@@ -427,6 +427,30 @@ def test_page_table_wider_than_the_latency_kernel_holds():
         check_o_lse(o, lse, o_ref, lse_ref, f"pt_stride {W} S={S}")
 
 
+@pytest.mark.parametrize("H,W", [(16, 20000), (64, 9000), (64, 60000)])
+def test_wide_page_tables_on_the_pipelined_kernels(H, W):
+    # Page-table rows of 9000 to 60000 logical pages (up to 3.8M positions)
+    # over a pool of 96 physical pages, one logical page mapped past the pool:
+    # the mma kernel (H = 16) and the tcgen05 kernel (H = 64) must give the
+    # oracle's answer with that page's positions masked and counted.
+    g = torch.Generator().manual_seed(W + H)
+    B, K, P = 2, 2048, 96
+    q = (torch.randn(B, 1, H, 576, generator=g) * 0.5).to(torch.bfloat16)
+    cache = (torch.randn(P, 64, 576, generator=g) * 0.5).to(torch.bfloat16)
+    pt = torch.randint(0, P, (B, W), generator=g, dtype=torch.int32)
+    pt[:, 5] = P + 3  # a page past the pool: its positions are masked and counted
+    idx = torch.stack([torch.randperm(W * 64, generator=g)[:K] for _ in range(B)]).to(torch.int32)
+    idx[:, 0, ] = 5 * 64 + 7
+    idx = idx.view(B, 1, K)
+    w = workloads.Workload("pt_row", q, cache, pt, idx, 576 ** -0.5, [W * 64] * B, None, ())
+    binding.check_device(clear=True)
+    o, lse = run_decode(w, 4)
+    st, n = binding.check_device(clear=True)
+    o_ref, lse_ref, bad = oracle_decode(w)
+    assert st == 5 and n == bad // H and n >= B
+    check_o_lse(o, lse, o_ref, lse_ref, f"H={H} pt_stride {W}")
+
+
 @pytest.mark.parametrize("K,S", [(2048, 1024), (100, 512), (3, 1024)])
 def test_maximum_nsplit(K, S):
     # NSPLIT at its maximum: two-entry splits, and mostly empty splits
