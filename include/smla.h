@@ -240,8 +240,10 @@ smla_status smla_check_device(int clear, unsigned long long *n_bad_index, void *
  *    not see device memory change at all inside its critical region should
  *    make one call (of any library entry point that launches work) on each
  *    device beforehand.  Later calls change no device memory reservation.
- *  - The looked-up address is kept per device for the life of the process;
- *    do not use this entry point across a cudaDeviceReset() of that device.
+ *  - The looked-up address is kept per device together with the context it
+ *    belongs to, and looked up again when the device's current context has
+ *    changed (after a cudaDeviceReset(), the next call runs in the new
+ *    primary context and finds its array there).
  *  - All calls on a device share the one array and it keeps whatever the last
  *    call left in it; nothing in it has to start at zero, because every split
  *    the combine reads is written first by the same call.  Calls whose work

@@ -481,28 +481,59 @@ smla_status smla_decode_partial_ws(const void *q, const void *kv_cache, int64_t 
 // Allocation-free decode.  The split-K partials go to a scratch array that the
 // library owns in device memory (one copy per device that loads this module).
 // In host code `g_noalloc_scratch` names a host-side stand-in, not a device
-// address, so each device's real address is looked up once with
+// address, so each device's real address is looked up with
 // cudaGetSymbolAddress while that device is current, and only that address is
-// handed to the kernels.
+// handed to the kernels.  The address belongs to the device's current context:
+// it is cached together with that context and looked up again when the
+// context changes (a cudaDeviceReset() creates a new primary context).
 static __device__ __align__(256) uint8_t g_noalloc_scratch[SMLA_NOALLOC_SCRATCH_BYTES];
 
 namespace {
 constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mu;
 void *g_noalloc_ptr[kMaxDevices] = {};
+CUcontext g_noalloc_ctx[kMaxDevices] = {};
 
-// Device address of this device's scratch array (set up on first use).
+// cuCtxGetCurrent, reached through the runtime (no link against the driver
+// library); null if the driver does not provide it.
+PFN_cuCtxGetCurrent_v4000 ctx_getter() {
+    static PFN_cuCtxGetCurrent_v4000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(ptr);
+        (void)cudaGetLastError();
+    });
+    return fn;
+}
+
+// Device address of this device's scratch array in its current context
+// (looked up on first use and again whenever the context has changed).
 smla_status noalloc_scratch(void **out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return cuda_fail(e);
     if (dev < 0 || dev >= kMaxDevices) return SMLA_ERR_UNSUPPORTED;
+    // The thread's current context: null until the runtime has made the
+    // device's primary context current in this thread (then the address is
+    // simply looked up again, which also makes it current).
+    PFN_cuCtxGetCurrent_v4000 get_ctx = ctx_getter();
+    auto current_ctx = [get_ctx]() {
+        CUcontext c = nullptr;
+        if (get_ctx == nullptr || get_ctx(&c) != CUDA_SUCCESS) c = nullptr;
+        return c;
+    };
+    const CUcontext ctx = current_ctx();
     std::lock_guard<std::mutex> lock(g_noalloc_mu);
-    if (g_noalloc_ptr[dev] == nullptr) {
+    if (g_noalloc_ptr[dev] == nullptr || ctx == nullptr || g_noalloc_ctx[dev] != ctx) {
         void *ptr = nullptr;
         e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
         if (e != cudaSuccess) return cuda_fail(e);
         g_noalloc_ptr[dev] = ptr;
+        g_noalloc_ctx[dev] = current_ctx();
     }
     *out = g_noalloc_ptr[dev];
     return SMLA_OK;
