@@ -314,3 +314,41 @@ def test_indexer_feeds_the_decode():
                                         dw.scale)
     assert bad == 0
     check_o_lse(o, lse, o_ref, lse_ref, "indexer -> decode")
+
+
+@pytest.mark.parametrize("H", [16, 64])
+def test_selection_feeds_the_decode_on_one_stream(H):
+    """The production chain: the top-k indexer writes the selection and the
+    decode consumes it on the same stream with no synchronisation in between
+    (the indexer's last kernel lets its dependents launch early; the decode's
+    first kernel waits before it reads).  Two query sets alternate, so a
+    decode that read the previous call's selection would differ; each decode
+    must equal, bit for bit, a decode of the same selection taken after a
+    synchronisation."""
+    B, HI, K = 3, 32, 512
+    wi = workloads.make_indexer_workload("chain", B=B, T=1, HI=HI, K=K,
+                                         ctx_lens=[3000, 9000, 20000], seed=21)
+    g = torch.Generator().manual_seed(22)
+    qi2 = (torch.randn(wi.q_index.shape, generator=g) * 0.5).to(torch.bfloat16)
+    cache = (torch.randn(wi.num_pages, 64, 576, generator=g) * 0.5).to(torch.bfloat16).to(DEV)
+    q = (torch.randn(B, 1, H, 576, generator=g) * 0.5).to(torch.bfloat16).to(DEV)
+    wd = wi.to(DEV)
+    qsets = [wd.q_index, qi2.to(DEV)]
+    idx = torch.empty((B, 1, K), dtype=torch.int32, device=DEV)
+    scale = 576 ** -0.5
+    binding.indexer_topk(qsets[0], wd.w, wd.k_index, wd.page_table, wd.n_vis, K, wi.max_n, out=idx)
+    binding.decode(q, cache, wd.page_table, idx, scale, 0)  # allocator warm-up
+    torch.cuda.synchronize()
+    picks = []
+    for c in range(8):
+        binding.indexer_topk(qsets[c % 2], wd.w, wd.k_index, wd.page_table, wd.n_vis, K, wi.max_n,
+                             out=idx)
+        o, lse = binding.decode(q, cache, wd.page_table, idx, scale, 0)
+        torch.cuda.synchronize()
+        sel = idx.clone()
+        o_ref, lse_ref = binding.decode(q, cache, wd.page_table, sel, scale, 0)
+        torch.cuda.synchronize()
+        assert torch.equal(o, o_ref) and torch.equal(lse, lse_ref), f"call {c}"
+        picks.append(sel.cpu())
+    assert not torch.equal(picks[0], picks[1])  # the two query sets select differently
+    assert all(torch.equal(picks[c], picks[c % 2]) for c in range(8))
