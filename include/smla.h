@@ -269,7 +269,10 @@ smla_status smla_decode_noalloc(const void *q, const void *kv_cache, int64_t num
  * One small copy kernel pulls q, the indices and the page table over the
  * host link into a staging area at the end of the workspace, then the decode
  * runs as smla_decode does and writes o and lse straight into the host
- * buffers.  This avoids the per-transfer latency of separate copies.
+ * buffers.  This avoids the per-transfer latency of separate copies.  The
+ * copy kernel issues all of a thread's loads before its stores (one round trip
+ * over the host link for a small step), and the decode's first kernel is its
+ * programmatic dependent, so that kernel's launch overlaps the copy.
  *
  *  - workspace_bytes must be at least smla_workspace_host_bytes(B, T, H, K,
  *    pt_stride, nsplit) for the nsplit actually used (0 picks the heuristic's
