@@ -689,6 +689,29 @@ def test_concurrent_host_threads_on_separate_streams():
         check_o_lse(results[i][0], results[i][1], o_ref, lse_ref, f"thread {i}")
 
 
+@pytest.mark.parametrize("name", ["tiny", "spec_verify"])
+def test_decode_host_word_aligned_index_and_page_table(name):
+    """Index and page-table buffers that are 4-byte but not 16-byte aligned
+    (views one int32 into pinned buffers): the copy kernel moves them as
+    4-byte words; the result must equal the device decode bit for bit."""
+    w = workloads.WORKLOADS[name]()
+    wd = w.to(DEV)
+    o_ref, lse_ref = binding.decode(wd.q, wd.cache, wd.page_table, wd.idx, w.scale, 0)
+    idx_buf = torch.empty(w.idx.numel() + 1, dtype=torch.int32).pin_memory()
+    pt_buf = torch.empty(w.page_table.numel() + 3, dtype=torch.int32).pin_memory()
+    idx_h = idx_buf[1:].view(w.idx.shape)
+    pt_h = pt_buf[3:].view(w.page_table.shape)
+    idx_h.copy_(w.idx)
+    pt_h.copy_(w.page_table)
+    assert idx_h.data_ptr() % 16 != 0 and pt_h.data_ptr() % 16 != 0
+    q_h = w.q.pin_memory()
+    o_h = torch.empty(o_ref.shape, dtype=torch.bfloat16).pin_memory()
+    lse_h = torch.empty(lse_ref.shape, dtype=torch.float32).pin_memory()
+    binding.decode_host(q_h, wd.cache, pt_h, idx_h, w.scale, 0, o=o_h, lse=lse_h)
+    torch.cuda.synchronize()
+    assert torch.equal(o_h, o_ref.cpu()) and torch.equal(lse_h, lse_ref.cpu())
+
+
 # ------------------------------------------------------------------ inputs rewritten between calls
 def _second_inputs(w, seed):
     """Same shapes and cache, another q and another selection (every valid
