@@ -685,12 +685,21 @@ __device__ __forceinline__ IxChunk ix_chunk(const IndexerParams &p) {
 // The chunk's keys, one load round trip (lane-consecutive positions); coherent
 // loads, since the score kernel may have written them while this grid was
 // already resident.
+// Every load is issued before any key is formed: the loads are volatile, so a
+// branch on one loaded value between two loads would hold the next load back
+// for a full round trip.
 __device__ __forceinline__ void ix_load_chunk(const float *sc, const IxChunk &ck,
                                               uint32_t (&key)[kIxSelIlp]) {
+    float v[kIxSelIlp];
 #pragma unroll
     for (int j = 0; j < kIxSelIlp; ++j) {
         const int s = ck.s0 + j * kIxSelThreads + (int)threadIdx.x;
-        key[j] = s < ck.s1 ? ix_key(__ldcg(sc + s)) : 0u;
+        v[j] = __ldcg(sc + min(s, ck.s1 - 1));   // ck.s1 > ck.s0: in range
+    }
+#pragma unroll
+    for (int j = 0; j < kIxSelIlp; ++j) {
+        const int s = ck.s0 + j * kIxSelThreads + (int)threadIdx.x;
+        key[j] = s < ck.s1 ? ix_key(v[j]) : 0u;
     }
 }
 
