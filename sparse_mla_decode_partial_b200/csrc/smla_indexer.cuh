@@ -340,7 +340,10 @@ struct IxCfg {
     static constexpr int kNumBars = 2 * kIxStages + 4 + 2 * kAcc;
     static constexpr int kOffTmem = kOffBar + kNumBars * 8;
     static constexpr int kOffHist = kOffTmem + 16;            // u32 [4096]: selection digits of a token
-    static constexpr int kBytes = kOffHist + kIxSelBins * 4;
+    // head weights of the CTA's tokens (when they span at most kWTokens)
+    static constexpr int kWTokens = 64;
+    static constexpr int kOffW = kOffHist + kIxSelBins * 4;   // f32 [kWTokens][NPAD]
+    static constexpr int kBytes = kOffW + kWTokens * NPAD * 4;
     static constexpr int kSmemBytes = kBytes + 1024;         // alignment slack (1024-B atoms)
     static constexpr uint32_t kTmemCols = 64 * kAcc;
     static_assert(kSmemBytes <= 232448, "shared memory per CTA");
@@ -515,6 +518,28 @@ __global__ void __launch_bounds__(IxCfg<NPAD>::kThreads, 1)
         int w_tok = -1;
         float wr[NPAD];                          // the token's head weights (0 past HI)
         int hint = u_begin < u_end ? ix_token_of(p, u_begin) : 0;
+        // The weights of every token this CTA touches (a contiguous span) wait
+        // in shared memory, loaded once, so that a token change reads them
+        // there instead of paying a memory round trip.
+        float *w_s = reinterpret_cast<float *>(smem + C::kOffW);
+        const int w_first = hint;
+        const int w_last = u_begin < u_end ? ix_token_of(p, u_end - 1) : hint - 1;
+        const bool w_staged = w_last - w_first < C::kWTokens;
+        if (w_staged) {
+            const int n = (w_last - w_first + 1) * NPAD;
+            for (int i0 = 0; i0 < n; i0 += 128 * 8) {
+                float v[8];
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const int e = i0 + k * 128 + et, j = e % NPAD;
+                    v[k] = (e < n && j < p.HI) ? __ldg(p.w + (size_t)(w_first + e / NPAD) * p.HI + j) : 0.f;
+                }
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    if (i0 + k * 128 + et < n) w_s[i0 + k * 128 + et] = v[k];
+            }
+            named_bar_sync(1, 128);
+        }
         long long i = 0;
         for (long long ub = u_begin; ub < u_end; ub += 32) {
             const int cnt = (int)min(32ll, u_end - ub);
@@ -523,9 +548,21 @@ __global__ void __launch_bounds__(IxCfg<NPAD>::kThreads, 1)
             for (int k = 0; k < cnt; ++k, ++i) {
                 const IxUnit m = ix_unit_from(mine, k);
                 if (m.tok != w_tok) {
+                    if (w_staged) {
+                        const float4 *src = reinterpret_cast<const float4 *>(w_s + (m.tok - w_first) * NPAD);
 #pragma unroll
-                    for (int j = 0; j < NPAD; ++j)
-                        wr[j] = j < p.HI ? __ldg(p.w + (size_t)m.tok * p.HI + j) : 0.f;
+                        for (int j = 0; j < NPAD / 4; ++j) {
+                            const float4 x = src[j];
+                            wr[4 * j] = x.x;
+                            wr[4 * j + 1] = x.y;
+                            wr[4 * j + 2] = x.z;
+                            wr[4 * j + 3] = x.w;
+                        }
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < NPAD; ++j)
+                            wr[j] = j < p.HI ? __ldg(p.w + (size_t)m.tok * p.HI + j) : 0.f;
+                    }
                     w_tok = m.tok;
                     if (count) {
                         if (h_tok >= 0) flush();
