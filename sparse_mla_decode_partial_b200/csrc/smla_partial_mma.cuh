@@ -62,9 +62,13 @@ constexpr float kLog2e = 1.4426950408889634f;     // log2(e)
 constexpr float kLn2 = 0.69314718055994531f;      // ln(2)
 constexpr int kResolveChunk = 2048;  // index entries resolved to rows ahead of the copies
 
-// Source of the bulk copy for a padding slot: a row of zeros, so that masked
+// Sources of the bulk copies for padding slots: rows of zeros, so that masked
 // slots hold finite values (their probability is 0, and 0 * finite = 0).
-__device__ __align__(128) uint16_t g_zero_row[kD];
+// Slot s of a tile copies zero row s: thousands of CTAs copying one shared row
+// at once serialised on its few L2 lines.  (The cp.async gathers zero-fill
+// padding slots without reading memory at all.)
+constexpr int kZeroRows = 32;
+__device__ __align__(128) uint16_t g_zero_rows[kZeroRows][kD];
 
 struct PartialParams {
     const __nv_bfloat16 *q;       // [B, T, H, 576]
@@ -517,7 +521,7 @@ __global__ void __launch_bounds__(MmaCfg<HG, NT, NSTAGE>::kThreads, MmaCfg<HG, N
                                                      (size_t)row * kRowBytes,
                                               kRowBytes, &full[stage], policy);
                             else
-                                bulk_g2s(d, g_zero_row, kRowBytes, &full[stage]);
+                                bulk_g2s(d, g_zero_rows[slot % kZeroRows], kRowBytes, &full[stage]);
                         }
                         mask |= (uint64_t)__ballot_sync(0xffffffffu, row >= 0) << (32 * k);
                     }
@@ -663,16 +667,18 @@ __global__ void __launch_bounds__(SmallCfg<HG, TILES>::kThreads)
     __syncthreads();
 
     // 3. gather: TILES x 32 rows x 72 chunks of 16 B, cp.async from every thread
+    // Padding slots (no row) are zero-filled by the copy itself (source size
+    // 0: nothing is read), so that they hold finite values.
     const uint8_t *cache = reinterpret_cast<const uint8_t *>(p.cache);
-    const uint8_t *zero = reinterpret_cast<const uint8_t *>(g_zero_row);
     uint8_t *kv = smem + C::kOffKV;
     for (int c = tid; c < TILES * NT * 72; c += C::kThreads) {
         const int r = c / 72, k = c - 72 * (c / 72);
         const int row = rows_s[r];
-        const uint8_t *src = (row >= 0 ? cache + (size_t)row * kRowBytes : zero) + k * 16;
-        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+        const uint8_t *src = cache + (size_t)(row >= 0 ? row : 0) * kRowBytes + k * 16;
+        const uint32_t nbytes = row >= 0 ? 16u : 0u;
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(
                          smem_addr(kv + r * kSmemRowBytes + k * 16)),
-                     "l"(src)
+                     "l"(src), "r"(nbytes)
                      : "memory");
     }
     asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");

@@ -201,8 +201,9 @@ __global__ void __launch_bounds__(TcCfg::kThreads, 1)
         }
         const int *pt_b = p.page_table + (size_t)b * p.pt_stride;
         const long long max_pos = (long long)p.pt_stride * kPage;
-        // Padding slots copy cache row 0 (always in range) and are masked to
-        // probability 0 by the softmax, so they add 0 * row 0 to O.
+        // Padding slots are zero-filled by the copy itself (source size 0:
+        // nothing is read; the address stays that of row 0, always in range)
+        // and are masked to probability 0 by the softmax.
         constexpr int kPadRow = 0;
         int *rows_s = reinterpret_cast<int *>(smem + C::kOffRows);
         const uint8_t *cache = reinterpret_cast<const uint8_t *>(p.cache);
@@ -283,7 +284,9 @@ __global__ void __launch_bounds__(TcCfg::kThreads, 1)
                     const uint8_t *src = cache + (size_t)(row >= 0 ? row : kPadRow) * kRowBytes +
                                          box * 128 + ch * 16;
                     const uint32_t d = smem_addr(dst + box * C::kBoxStride + r * 128 + ((ch ^ (r & 7)) << 4));
-                    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(src) : "memory");
+                    const uint32_t nbytes = row >= 0 ? 16u : 0u;
+                    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(src), "r"(nbytes)
+                                 : "memory");
                 }
                 asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(
                                  smem_addr(&kv_full[stage]))
