@@ -499,7 +499,7 @@ __global__ void __launch_bounds__(MmaCfg<HG, NT, NSTAGE>::kThreads, MmaCfg<HG, N
                     named_bar_sync(bar_prod, 32 * C::kProducerWarps);  // rows_s complete
                 }
                 first_chunk = false;
-                // Issue one bulk copy per row (or per padding slot, from the zero row).
+                // Issue one bulk copy per row (or per padding slot, from its zero row).
                 const int chunk_tiles = (n + NT - 1) / NT;
                 for (int t = 0; t < chunk_tiles; ++t, ++it) {
                     const int stage = it % NSTAGE;

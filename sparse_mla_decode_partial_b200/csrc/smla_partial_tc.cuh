@@ -21,7 +21,7 @@
 //              cp.async copies written straight into the 128B-swizzled
 //              K-major layout (each warp instruction moves 4 rows x 128 B,
 //              coalesced); completion reaches the tile's mbarrier through
-//              cp.async.mbarrier.arrive.  Padding slots copy row 0 and are
+//              cp.async.mbarrier.arrive.  Padding slots are zero-filled (nothing read) and are
 //              masked.  In dense mode a tile of 32 consecutive cache rows
 //              moves instead with nine TMA tile loads (32 rows x 64 values,
 //              128B swizzle) on the same barrier.
