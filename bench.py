@@ -183,6 +183,15 @@ class ClockSampler:
             self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
         except Exception:  # NVML missing: no clock record
             self._nv = None
+        if self._nv is not None:
+            # the first queries of a process can take longer than a short timed
+            # region; pay for them here, before it starts
+            try:
+                self._nv.nvmlDeviceGetClockInfo(self._h, self._nv.NVML_CLOCK_SM)
+                self._nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+            except Exception:
+                pass
+        self.after_region = False
 
     def _run(self):
         nv = self._nv
@@ -205,8 +214,11 @@ class ClockSampler:
         if self._thread is not None:
             self._thread.join()
         if self._nv is not None and not self.samples:
+            # nothing landed inside the region: one read right after it, flagged
             try:
                 self.samples.append(self._nv.nvmlDeviceGetClockInfo(self._h, self._nv.NVML_CLOCK_SM))
+                self.reasons |= self._nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                self.after_region = True
             except Exception:
                 pass
 
@@ -214,8 +226,11 @@ class ClockSampler:
         if self._nv is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
         names = [k for k, bit in self.HW.items() if self.reasons & bit]
-        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
-                "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples)}
+        out = {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+               "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples)}
+        if self.after_region:
+            out["sampled"] = "once, right after the timed region (no sample landed inside it)"
+        return out
 
 
 # ----------------------------------------------------------------------------- distributed

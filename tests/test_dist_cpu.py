@@ -142,3 +142,74 @@ def test_traffic_record_tracks_its_kernel_sources(tmp_path, monkeypatch):
     assert bench.measured_traffic("single_request") == before["single_request"]
     assert bench.measured_traffic("batched") == before["batched"]
     assert bench.measured_traffic("tiny") is None          # never captured
+
+
+class _FakeNvml:
+    """Stands in for pynvml: a fixed SM clock and throttle-reason mask; while
+    `failing` is set the per-sample queries raise, as a busy driver can."""
+    NVML_CLOCK_SM = 1
+
+    def __init__(self, mhz, reasons):
+        self.mhz, self.mask, self.failing, self.calls = mhz, reasons, False, []
+
+    def nvmlInit(self):
+        self.calls.append("init")
+
+    def nvmlDeviceGetHandleByIndex(self, i):
+        return ("dev", i)
+
+    def nvmlDeviceGetMaxClockInfo(self, h, kind):
+        return 1965
+
+    def nvmlDeviceGetClockInfo(self, h, kind):
+        self.calls.append("clock")
+        if self.failing:
+            raise RuntimeError("busy")
+        return self.mhz
+
+    def nvmlDeviceGetCurrentClocksEventReasons(self, h):
+        self.calls.append("reasons")
+        if self.failing:
+            raise RuntimeError("busy")
+        return self.mask
+
+
+def test_clock_sampler_reads_inside_the_region_and_names_reasons(monkeypatch):
+    """The sampler's first NVML queries run when it is made (before the timed
+    region); inside the region it samples the SM clock and ORs the throttle
+    reasons, which it names."""
+    import time
+    sys.path.insert(0, ROOT)
+    import bench
+    fake = _FakeNvml(1800, bench.ClockSampler.HW["sw_power_cap"] | bench.ClockSampler.HW["hw_slowdown"])
+    monkeypatch.setitem(sys.modules, "pynvml", fake)
+    s = bench.ClockSampler(0, period_s=0.001)
+    assert fake.calls[:3] == ["init", "clock", "reasons"]
+    n_before = len(fake.calls)
+    with s:
+        time.sleep(0.05)
+    assert len(fake.calls) > n_before
+    out = s.summary()
+    assert out["sm_mhz"] == 1800 and out["sm_max_mhz"] == 1965 and out["samples"] >= 2
+    assert sorted(out["reasons"]) == ["hw_slowdown", "sw_power_cap"]
+    assert "sampled" not in out
+
+
+def test_clock_sampler_flags_a_read_taken_after_the_region(monkeypatch):
+    """When no sample lands inside the region, the one read taken right after
+    it is reported as such, never as a sample from inside."""
+    import time
+    sys.path.insert(0, ROOT)
+    import bench
+    fake = _FakeNvml(1965, 0)
+    monkeypatch.setitem(sys.modules, "pynvml", fake)
+    s = bench.ClockSampler(0, period_s=0.001)
+    fake.failing = True
+    with s:
+        time.sleep(0.01)
+        s._stop.set()             # the region's sampling ends with nothing read
+        s._thread.join()
+        fake.failing = False      # the driver answers again only after it
+    out = s.summary()
+    assert out["samples"] == 1 and out["sm_mhz"] == 1965 and out["reasons"] == []
+    assert out["sampled"].startswith("once, right after the timed region")
