@@ -57,6 +57,15 @@
  *    query token at most 64; num_pages at most SMLA_MAX_PAGES.  Otherwise
  *    SMLA_ERR_UNSUPPORTED.
  *  - B, T, H or K equal to 0 are legal (K = 0: every o = 0, lse = -inf).
+ *  - K (an index list's width, the dense variant's longest visible length,
+ *    the indexer's selection width) must be at most SMLA_MAX_K: the host's
+ *    split arithmetic (ceil(K / nsplit), rounded up to whole pages, plus K)
+ *    and the kernels' fill loops are 32-bit.  This is a precondition the
+ *    library does not check; the Python binding refuses larger K.
+ *  - Output buffers are the caller's and must hold the element counts each
+ *    entry point lists (o [B, T, H, 512], lse [B, T, H], the partials
+ *    [B, T, H, nsplit(, 512)], the indexer's [B, T, K] and [B, T, max_n]);
+ *    the library writes through the pointers without knowing their extent.
  *  - A CUDA error at launch returns SMLA_ERR_CUDA; smla_last_error() gives
  *    its text.  No entry point throws, aborts or exits.
  *  - Entry points may be called from several host threads on different
@@ -79,6 +88,7 @@ extern "C" {
 #define SMLA_MAX_HEADS 64
 #define SMLA_MAX_NSPLIT 1024
 #define SMLA_MAX_PAGES 33554431 /* cache rows must be addressable as int32 */
+#define SMLA_MAX_K 1073741760   /* 2^30 - 64: largest K (a precondition, see below) */
 
 typedef enum {
     SMLA_OK = 0,

@@ -18,6 +18,11 @@ LIB_PATH = os.path.join(_PKG, "libsmla.so")
 DC, DR, D, PAGE_SIZE = 512, 64, 576, 64
 MAX_HEADS, MAX_NSPLIT = 64, 1024
 NOALLOC_SCRATCH_BYTES = 16 << 20
+# Largest K (index-list width, dense longest visible length, indexer selection
+# width): the library's split arithmetic (ceil(K / nsplit) rounded up to whole
+# pages, then K + that split length) and its fill loops are 32-bit.  The
+# library does not check this bound itself.
+MAX_K = 2**30 - 64
 
 STATUS = {
     0: "SMLA_OK", 1: "SMLA_ERR_INVALID_ARG", 2: "SMLA_ERR_UNSUPPORTED", 3: "SMLA_ERR_MISALIGNED",
@@ -91,6 +96,12 @@ def lib():
     return _lib
 
 
+def _k_in_range(K: int) -> int:
+    if K > MAX_K:
+        raise ValueError(f"K = {K} is above the library's limit {MAX_K}")
+    return K
+
+
 def _check(status: int, where: str):
     if status != 0:
         raise SmlaError(status, where)
@@ -106,19 +117,27 @@ def _ptr(t: Optional[torch.Tensor]):
     return None if t is None else t.data_ptr()
 
 
-def _need(t, dtype, name, device=None):
+def _need(t, dtype, name, device=None, shape=None):
+    """Type, dtype, contiguity, shape (when given: the library reads or writes
+    exactly that many elements through the pointer) and device of a tensor."""
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor")
     if t.dtype != dtype:
         raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {list(shape)}, got {list(t.shape)}")
+    _on_device(t, name, device)
+
+
+def _on_device(t, name, device):
     if not t.is_cuda or (device is not None and t.device != device):
         raise ValueError(f"{name} must be a CUDA tensor on {device}")
 
 
 def choose_nsplit(B: int, T: int, H: int, K: int, sm_count: int = 0) -> int:
-    return int(lib().smla_choose_nsplit(B, T, H, K, sm_count))
+    return int(lib().smla_choose_nsplit(B, T, H, _k_in_range(K), sm_count))
 
 
 def workspace_bytes(B: int, T: int, H: int, nsplit: int) -> int:
@@ -141,7 +160,7 @@ def _decode_args(q, cache, page_table, idx):
     if cache.numel() % (PAGE_SIZE * D):
         raise ValueError("cache must be [num_pages, 64, 576]")
     num_pages = cache.numel() // (PAGE_SIZE * D)
-    return B, T, H, idx.shape[2], page_table.shape[1], num_pages
+    return B, T, H, _k_in_range(idx.shape[2]), page_table.shape[1], num_pages
 
 
 def decode_partial(q, cache, page_table, idx, scale: float, nsplit: int, *, part_o=None,
@@ -155,8 +174,9 @@ def decode_partial(q, cache, page_table, idx, scale: float, nsplit: int, *, part
         part_m = torch.empty((B, T, H, nsplit), dtype=torch.float32, device=dev)
     if part_lse is None:
         part_lse = torch.empty((B, T, H, nsplit), dtype=torch.float32, device=dev)
-    for t, n in ((part_o, "part_o"), (part_m, "part_m"), (part_lse, "part_lse")):
-        _need(t, torch.float32, n, dev)
+    _need(part_o, torch.float32, "part_o", dev, (B, T, H, nsplit, DC))
+    _need(part_m, torch.float32, "part_m", dev, (B, T, H, nsplit))
+    _need(part_lse, torch.float32, "part_lse", dev, (B, T, H, nsplit))
     _check(lib().smla_decode_partial(_ptr(q), _ptr(cache), num_pages, _ptr(page_table), pt_stride,
                                      _ptr(idx), B, T, H, K, PAGE_SIZE, float(scale), int(nsplit),
                                      _ptr(part_o), _ptr(part_m), _ptr(part_lse),
@@ -179,8 +199,8 @@ def lse_combine(part_o, part_m, part_lse, *, o=None, lse=None, stream=None):
         o = torch.empty((B, T, H, DC), dtype=torch.bfloat16, device=dev)
     if lse is None:
         lse = torch.empty((B, T, H), dtype=torch.float32, device=dev)
-    _need(o, torch.bfloat16, "o", dev)
-    _need(lse, torch.float32, "lse", dev)
+    _need(o, torch.bfloat16, "o", dev, (B, T, H, DC))
+    _need(lse, torch.float32, "lse", dev, (B, T, H))
     _check(lib().smla_lse_combine(_ptr(part_o), _ptr(part_m), _ptr(part_lse), B, T, H, S, _ptr(o),
                                   _ptr(lse), _stream(stream)), "smla_lse_combine")
     return o, lse
@@ -205,8 +225,8 @@ def decode(q, cache, page_table, idx, scale: float, nsplit: int = 0, *, workspac
         o = torch.empty((B, T, H, DC), dtype=torch.bfloat16, device=dev)
     if lse is None:
         lse = torch.empty((B, T, H), dtype=torch.float32, device=dev)
-    _need(o, torch.bfloat16, "o", dev)
-    _need(lse, torch.float32, "lse", dev)
+    _need(o, torch.bfloat16, "o", dev, (B, T, H, DC))
+    _need(lse, torch.float32, "lse", dev, (B, T, H))
     _check(lib().smla_decode(_ptr(q), _ptr(cache), num_pages, _ptr(page_table), pt_stride,
                              _ptr(idx), B, T, H, K, PAGE_SIZE, float(scale), int(nsplit),
                              _ptr(workspace), workspace.numel(), _ptr(o), _ptr(lse),
@@ -222,8 +242,8 @@ def decode_noalloc(q, cache, page_table, idx, scale: float, nsplit: int = 0, *, 
     decode, so o and lse must be given.  Calls that overlap on the GPU race on
     the shared scratch."""
     B, T, H, K, pt_stride, num_pages = _decode_args(q, cache, page_table, idx)
-    _need(o, torch.bfloat16, "o", q.device)
-    _need(lse, torch.float32, "lse", q.device)
+    _need(o, torch.bfloat16, "o", q.device, (B, T, H, DC))
+    _need(lse, torch.float32, "lse", q.device, (B, T, H))
     _check(lib().smla_decode_noalloc(_ptr(q), _ptr(cache), num_pages, _ptr(page_table),
                                      pt_stride, _ptr(idx), B, T, H, K, PAGE_SIZE, float(scale),
                                      int(nsplit), _ptr(o), _ptr(lse), _stream(stream)),
@@ -232,7 +252,7 @@ def decode_noalloc(q, cache, page_table, idx, scale: float, nsplit: int = 0, *, 
 
 
 def dense_nsplit(B: int, T: int, H: int, K: int) -> int:
-    return int(lib().smla_dense_nsplit(B, T, H, K))
+    return int(lib().smla_dense_nsplit(B, T, H, _k_in_range(K)))
 
 
 def dense_workspace_bytes(B: int, T: int, H: int, K: int, nsplit: int) -> int:
@@ -256,7 +276,7 @@ def _dense_args(q, cache, page_table, seq_lens, K):
         raise ValueError("cache must be [num_pages, 64, 576]")
     if K is None:
         K = int(seq_lens.max().item()) if seq_lens.numel() else 0
-    return B, T, H, int(K), page_table.shape[1], cache.numel() // (PAGE_SIZE * D)
+    return B, T, H, _k_in_range(int(K)), page_table.shape[1], cache.numel() // (PAGE_SIZE * D)
 
 
 def decode_dense(q, cache, page_table, seq_lens, scale: float, nsplit: int = 0, *, K=None,
@@ -277,8 +297,8 @@ def decode_dense(q, cache, page_table, seq_lens, scale: float, nsplit: int = 0, 
         o = torch.empty((B, T, H, DC), dtype=torch.bfloat16, device=dev)
     if lse is None:
         lse = torch.empty((B, T, H), dtype=torch.float32, device=dev)
-    _need(o, torch.bfloat16, "o", dev)
-    _need(lse, torch.float32, "lse", dev)
+    _need(o, torch.bfloat16, "o", dev, (B, T, H, DC))
+    _need(lse, torch.float32, "lse", dev, (B, T, H))
     _check(lib().smla_decode_dense(_ptr(q), _ptr(cache), num_pages, _ptr(page_table), pt_stride,
                                    _ptr(seq_lens), B, T, H, K, PAGE_SIZE, float(scale),
                                    int(nsplit), _ptr(workspace), workspace.numel(), _ptr(o),
@@ -298,8 +318,9 @@ def decode_dense_partial(q, cache, page_table, seq_lens, scale: float, nsplit: i
         part_m = torch.empty((B, T, H, nsplit), dtype=torch.float32, device=dev)
     if part_lse is None:
         part_lse = torch.empty((B, T, H, nsplit), dtype=torch.float32, device=dev)
-    for t, n in ((part_o, "part_o"), (part_m, "part_m"), (part_lse, "part_lse")):
-        _need(t, torch.float32, n, dev)
+    _need(part_o, torch.float32, "part_o", dev, (B, T, H, nsplit, DC))
+    _need(part_m, torch.float32, "part_m", dev, (B, T, H, nsplit))
+    _need(part_lse, torch.float32, "part_lse", dev, (B, T, H, nsplit))
     _check(lib().smla_decode_dense_partial(_ptr(q), _ptr(cache), num_pages, _ptr(page_table),
                                            pt_stride, _ptr(seq_lens), B, T, H, K, PAGE_SIZE,
                                            float(scale), int(nsplit), _ptr(part_o), _ptr(part_m),
@@ -330,7 +351,15 @@ def decode_host(q, cache, page_table, idx, scale: float, nsplit: int = 0, *, o, 
     if q.dim() != 4 or q.shape[-1] != D:
         raise ValueError(f"q must be [B,T,H,{D}]")
     B, T, H, _ = q.shape
-    K, pt_stride = idx.shape[2], page_table.shape[1]
+    if idx.dim() != 3 or tuple(idx.shape[:2]) != (B, T):
+        raise ValueError("idx must be [B,T,K]")
+    if page_table.dim() != 2 or page_table.shape[0] != B:
+        raise ValueError("page_table must be [B, pt_stride]")
+    K, pt_stride = _k_in_range(idx.shape[2]), page_table.shape[1]
+    if tuple(o.shape) != (B, T, H, DC) or tuple(lse.shape) != (B, T, H):
+        raise ValueError(f"o must be [{B}, {T}, {H}, {DC}] and lse [{B}, {T}, {H}]")
+    if cache.numel() % (PAGE_SIZE * D):
+        raise ValueError("cache must be [num_pages, 64, 576]")
     num_pages = cache.numel() // (PAGE_SIZE * D)
     if nsplit == 0:
         nsplit = choose_nsplit(B, T, H, K, 0)
@@ -382,9 +411,10 @@ def indexer_topk(q_index, w, k_index, page_table, n_vis, K: int, max_n: int, *, 
     n_vis (it sizes the work and the score buffer)."""
     B, T, HI, pt_stride, num_pages = _indexer_args(q_index, w, k_index, page_table, n_vis)
     dev = q_index.device
+    K = _k_in_range(int(K))
     if out is None:
         out = torch.empty((B, T, K), dtype=torch.int32, device=dev)
-    _need(out, torch.int32, "out", dev)
+    _need(out, torch.int32, "out", dev, (B, T, K))
     if workspace is None:
         workspace = torch.empty(max(16, indexer_workspace_bytes(B, T, max_n)), dtype=torch.uint8,
                                 device=dev)
@@ -404,7 +434,8 @@ def indexer_scores(q_index, w, k_index, page_table, n_vis, max_n: int, *, scores
     dev = q_index.device
     if scores is None:
         scores = torch.full((B, T, max(max_n, 1)), float("nan"), dtype=torch.float32, device=dev)
-    _need(scores, torch.float32, "scores", dev)
+    # rows of max_n scores, one per query token (nothing is written when max_n is 0)
+    _need(scores, torch.float32, "scores", dev, (B, T, max_n) if max_n > 0 else None)
     if workspace is None:
         workspace = torch.empty(max(16, indexer_workspace_bytes(B, T, 0)), dtype=torch.uint8,
                                 device=dev)
@@ -420,11 +451,14 @@ def indexer_select(scores, n_vis, K: int, *, out=None, workspace=None, stream=No
     """The indexer's selection rule on given scores fp32 [B, T, max_n]."""
     _need(scores, torch.float32, "scores")
     dev = scores.device
-    _need(n_vis, torch.int32, "n_vis", dev)
+    if scores.dim() != 3:
+        raise ValueError("scores must be [B, T, max_n]")
     B, T, max_n = scores.shape
+    _need(n_vis, torch.int32, "n_vis", dev, (B, T))
+    K = _k_in_range(int(K))
     if out is None:
         out = torch.empty((B, T, K), dtype=torch.int32, device=dev)
-    _need(out, torch.int32, "out", dev)
+    _need(out, torch.int32, "out", dev, (B, T, K))
     if workspace is None:
         workspace = torch.empty(max(16, indexer_select_workspace_bytes(B, T, max_n)),
                                 dtype=torch.uint8, device=dev)

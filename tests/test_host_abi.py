@@ -55,6 +55,7 @@ def test_binding_constants_match_the_header():
     assert want["SMLA_INDEXER_DIM"] == binding.INDEXER_DIM
     assert want["SMLA_INDEXER_MAX_HEADS"] == binding.INDEXER_MAX_HEADS
     assert want["SMLA_INDEXER_MAX_N"] == binding.INDEXER_MAX_N
+    assert want["SMLA_MAX_K"] == binding.MAX_K == 2**30 - 64
 
 
 def test_workspace_bytes_formula(lib):
@@ -298,3 +299,91 @@ def test_workspace_host_bytes_formula(lib):
         assert binding.workspace_host_bytes(B, T, H, K, P, S) == want
     assert binding.workspace_host_bytes(1, 1, 1, 1, 1, 0) == 0
     assert binding.workspace_host_bytes(1, 1, 1, -1, 1, 1) == 0
+
+
+# ------------------------------------------------------------------ binding buffer checks
+def _cpu_as_device(monkeypatch):
+    """Let CPU tensors through the binding's device test, so that its shape
+    checks (which run before any library call) can be exercised here."""
+    monkeypatch.setattr(binding, "_on_device", lambda t, name, device: None)
+
+
+def test_need_checks_shape_before_device():
+    import torch
+    with pytest.raises(ValueError, match="out must have shape"):
+        binding._need(torch.zeros((2, 3), dtype=torch.int32), torch.int32, "out", shape=(2, 4))
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        binding._need(torch.zeros((2, 4), dtype=torch.int32), torch.int32, "out", shape=(2, 4))
+
+
+def _decode_inputs(B=2, T=3, H=16, K=40, P=2):
+    import torch
+    return (torch.zeros((B, T, H, 576), dtype=torch.bfloat16), torch.zeros((P, 64, 576), dtype=torch.bfloat16),
+            torch.zeros((B, 1), dtype=torch.int32), torch.zeros((B, T, K), dtype=torch.int32))
+
+
+def test_binding_rejects_wrong_output_shapes(lib, monkeypatch):
+    """Every caller-supplied buffer the library writes through must have the
+    shape the call implies; a wrong one is refused before anything runs."""
+    import torch
+    _cpu_as_device(monkeypatch)
+    q, cache, pt, idx = _decode_inputs()
+    bf, f32 = torch.bfloat16, torch.float32
+    o_ok, lse_ok = torch.zeros((2, 3, 16, 512), dtype=bf), torch.zeros((2, 3, 16), dtype=f32)
+    o_bad, lse_bad = torch.zeros((2, 3, 8, 512), dtype=bf), torch.zeros((2, 3, 17), dtype=f32)
+    calls = [
+        ("o", lambda: binding.decode(q, cache, pt, idx, 0.1, 2, o=o_bad, lse=lse_ok)),
+        ("lse", lambda: binding.decode(q, cache, pt, idx, 0.1, 2, o=o_ok, lse=lse_bad)),
+        ("o", lambda: binding.decode_noalloc(q, cache, pt, idx, 0.1, 2, o=o_bad, lse=lse_ok)),
+        ("part_o", lambda: binding.decode_partial(q, cache, pt, idx, 0.1, 3,
+                                                  part_o=torch.zeros((2, 3, 16, 2, 512), dtype=f32))),
+        ("part_m", lambda: binding.decode_partial(q, cache, pt, idx, 0.1, 3,
+                                                  part_m=torch.zeros((2, 3, 16, 4), dtype=f32))),
+        ("o", lambda: binding.lse_combine(torch.zeros((2, 3, 16, 4, 512), dtype=f32),
+                                          torch.zeros((2, 3, 16, 4), dtype=f32),
+                                          torch.zeros((2, 3, 16, 4), dtype=f32), o=o_bad)),
+    ]
+    seq_lens = torch.full((2, 3), 30, dtype=torch.int32)
+    calls += [
+        ("lse", lambda: binding.decode_dense(q, cache, pt, seq_lens, 0.1, 2, K=40, o=o_ok,
+                                             lse=lse_bad)),
+        ("part_lse", lambda: binding.decode_dense_partial(
+            q, cache, pt, seq_lens, 0.1, 2, K=40, part_lse=torch.zeros((2, 3, 16, 3), dtype=f32))),
+    ]
+    qi = torch.zeros((2, 3, 4, 128), dtype=bf)
+    wi, ki, nv = torch.zeros((2, 3, 4), dtype=f32), torch.zeros((2, 64, 128), dtype=bf), \
+        torch.zeros((2, 3), dtype=torch.int32)
+    calls += [
+        ("out", lambda: binding.indexer_topk(qi, wi, ki, pt, nv, 16, 100,
+                                             out=torch.zeros((2, 3, 8), dtype=torch.int32))),
+        ("scores", lambda: binding.indexer_scores(qi, wi, ki, pt, nv, 100,
+                                                  scores=torch.zeros((2, 3, 64), dtype=f32))),
+        ("n_vis", lambda: binding.indexer_select(torch.zeros((2, 3, 100), dtype=f32),
+                                                 torch.zeros((6,), dtype=torch.int32), 16)),
+        ("out", lambda: binding.indexer_select(torch.zeros((2, 3, 100), dtype=f32), nv, 16,
+                                               out=torch.zeros((2, 3, 17), dtype=torch.int32))),
+    ]
+    for name, call in calls:
+        with pytest.raises(ValueError, match=f"^{name} must have shape"):
+            call()
+    with pytest.raises(ValueError, match="scores must be"):
+        binding.indexer_select(torch.zeros((6, 100), dtype=f32), nv, 16)
+
+
+def test_binding_enforces_the_k_limit(lib, monkeypatch):
+    """K above the library's 32-bit split arithmetic is refused by the
+    binding; at the limit the host heuristics stay in range."""
+    import torch
+    _cpu_as_device(monkeypatch)
+    monkeypatch.delenv("SMLA_NSPLIT", raising=False)
+    big = binding.MAX_K + 1
+    for call in (lambda: binding.choose_nsplit(1, 1, 16, big, 148),
+                 lambda: binding.dense_nsplit(1, 1, 8, big),
+                 lambda: binding.indexer_select(torch.zeros((1, 1, 8), dtype=torch.float32),
+                                                torch.zeros((1, 1), dtype=torch.int32), big)):
+        with pytest.raises(ValueError, match="above the library's limit"):
+            call()
+    assert 1 <= binding.choose_nsplit(1, 1, 16, binding.MAX_K, 148) <= 1024
+    assert 1 <= binding.dense_nsplit(1, 1, 8, binding.MAX_K) <= 1024
+    ws = binding.dense_workspace_bytes(1, 1, 8, binding.MAX_K, 1)
+    assert ws == 0
