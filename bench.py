@@ -371,6 +371,21 @@ def bench_config(w, workload: str, nsplit_arg: int, world: int) -> dict:
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
 
 
+INDEXER_DATA = "synthetic (seeded index queries, keys and weights)"
+
+
+def indexer_shape(w) -> str:
+    return (f"B{w.B} T{w.T} HI{w.HI} x128 bf16 index keys, top-{w.K}, ctx "
+            f"{min(w.ctx_lens)}..{max(w.ctx_lens)}")
+
+
+def indexer_config(w, world: int) -> dict:
+    """The `config` object of an indexer_mixed line, identical in both arms."""
+    return {"workload": "indexer_mixed", "shape": indexer_shape(w),
+            "l2": "flushed before every step: 256 MB write then 256 MB read",
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
+
+
 class Harness:
     """Device-side timing through the C ABI on one stream: L2 flush before
     every step, CUDA events on the launching stream around each step."""
@@ -559,8 +574,7 @@ def side_indexer(h, steps, warmup, peaks):
     hbm_peak, tc_peak, peak_src = peaks
     key_bytes = nbytes - B * T * K * 4
     flops = 2 * int(w_host.n_vis.clamp(min=0).sum()) * HI * 128
-    rec = {"shape": f"B{B} T{T} HI{HI} x128 bf16 index keys, top-{K}, ctx "
-                    f"{min(w_host.ctx_lens)}..{max(w_host.ctx_lens)}",
+    rec = {"shape": indexer_shape(w_host), "query_tokens": B * T,
            "steps": steps, "us_per_call": round(us, 3),
            "us_per_call_mean": round(statistics.fmean(t_all) * 1e3, 3),
            "q_tok_s": round(B * T / (us * 1e-6), 1),
@@ -586,26 +600,30 @@ def side_indexer(h, steps, warmup, peaks):
 def run_indexer_headline(args, world, rank, local):
     """`--workload indexer_mixed`: the top-k indexer as the timed step (the
     profiling recipe's launch list and captures of the indexer kernels use
-    it); the line carries the indexer record's figures."""
+    it); the line carries the indexer record's figures.  Under torchrun every
+    rank runs the same workload (weak scaling) and the line reports all
+    ranks' query tokens over the slowest rank's time."""
     import torch
     from sparse_mla_decode_partial_b200 import build
     build.build()
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     h = Harness(dev)
+    barrier(world)
+    torch.cuda.synchronize(dev)
     rec = side_indexer(h, args.steps, args.warmup, load_peaks())
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    _, ms_max, value = aggregate(float(rec["query_tokens"]), rec["us_per_call"] * 1e-3, world)
     if rank != 0:
         return None
     from sparse_mla_decode_partial_b200 import workloads
     w = workloads.indexer_mixed()
-    us = rec["us_per_call"]
-    return {"metric": "top-k indexer query-tokens/s", "value": rec["q_tok_s"],
+    return {"metric": "top-k indexer query-tokens/s", "value": round(value, 1),
             "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": round(us * 1e-3, 6), "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded index queries, keys "
-            "and weights)", "config": {"workload": "indexer_mixed", "shape": rec["shape"],
-                                       "l2": "flushed before every step: 256 MB write then 256 MB read",
-                                       "parallelism": "single GPU"},
+            "ms_per_step": round(ms_max, 6), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": INDEXER_DATA,
+            "config": indexer_config(w, world),
             "roofline": rec["roofline"], "clocks": rec["clocks"], "gpu_launches": rec["gpu_launches"],
             "indexer": rec}
 
@@ -798,7 +816,7 @@ def run_ours(args, world, rank, local):
     return line
 
 
-def indexer_cpu_baseline(seconds: float):
+def indexer_cpu_baseline(seconds: float, w=None):
     """The fp64 indexer oracle on this host's cores over the first query
     tokens of the indexer workload (one token at a time until the time is
     spent)."""
@@ -806,7 +824,8 @@ def indexer_cpu_baseline(seconds: float):
     import torch
     from oracle import indexer as ix_oracle
     from sparse_mla_decode_partial_b200 import workloads
-    w = workloads.indexer_mixed()
+    if w is None:
+        w = workloads.indexer_mixed()
     bits = lambda t: t.contiguous().view(torch.int16).numpy().view(np.uint16)
     q, k = bits(w.q_index), bits(w.k_index)
     wt, pt, nv = w.w.numpy(), w.page_table.numpy(), w.n_vis.numpy()
@@ -829,12 +848,13 @@ def run_reference(args, world, rank):
         return None
     from sparse_mla_decode_partial_b200 import workloads
     if args.workload == "indexer_mixed":
-        res = indexer_cpu_baseline(max(2.0, args.cpu_seconds))
+        w = workloads.indexer_mixed()
+        res = indexer_cpu_baseline(max(2.0, args.cpu_seconds), w)
         return {"metric": "top-k indexer query-tokens/s", "value": round(res["value"], 3),
                 "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
                 "ms_per_step": round(1e3 / res["value"], 3), "higher_is_better": True,
-                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-                "config": {"workload": "indexer_mixed"}, "impl": "reference", "cpu_baseline": res,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": INDEXER_DATA,
+                "config": indexer_config(w, world), "impl": "reference", "cpu_baseline": res,
                 "e2e": {"value": round(res["value"], 3), "unit": UNIT, "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}}
     w = workloads.WORKLOADS[args.workload]()

@@ -215,3 +215,46 @@ def test_clock_sampler_flags_a_read_taken_after_the_region(monkeypatch):
     out = s.summary()
     assert out["samples"] == 1 and out["sm_mhz"] == 1965 and out["reasons"] == []
     assert out["sampled"].startswith("once, right after the timed region")
+
+
+def test_reference_arm_indexer_workload_prints_the_same_config():
+    """The indexer's reference line carries the config and data note the
+    GPU arm prints for the same command (one helper builds both)."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from sparse_mla_decode_partial_b200 import workloads
+    env = dict(os.environ, RANK="0", WORLD_SIZE="1")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--workload", "indexer_mixed", "--cpu-seconds", "0.5"],
+                       env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr
+    d = json.loads([l for l in r.stdout.splitlines() if l.strip()][0])
+    w = workloads.indexer_mixed()
+    assert d["impl"] == "reference" and d["config"] == bench.indexer_config(w, 1)
+    assert d["data"] == bench.INDEXER_DATA and d["value"] > 0
+    assert d["config"]["shape"].startswith(f"B{w.B} T{w.T} HI{w.HI} ")
+    assert bench.indexer_config(w, 4)["parallelism"] == "replicas x4"
+
+
+def test_indexer_headline_reports_the_job_from_the_timed_record(monkeypatch):
+    """The indexer line's value is query tokens over the timed call's
+    duration, with the shared config (timing faked: the record the timed
+    region produces is given, CUDA calls are stubbed)."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from sparse_mla_decode_partial_b200 import build, workloads
+    w = workloads.indexer_mixed()
+    rec = {"shape": bench.indexer_shape(w), "query_tokens": w.B * w.T, "us_per_call": 100.0,
+           "roofline": {"frac": 0.8}, "clocks": {"sm_mhz": 1965}, "gpu_launches": 40}
+    monkeypatch.setattr(build, "build", lambda: None)
+    monkeypatch.setattr(bench, "Harness", lambda dev: None)
+    monkeypatch.setattr(bench, "side_indexer", lambda h, steps, warmup, peaks: rec)
+    monkeypatch.setattr(torch.cuda, "set_device", lambda dev: None)
+    monkeypatch.setattr(torch.cuda, "synchronize", lambda dev=None: None)
+
+    class A:
+        steps, warmup = 10, 3
+    line = bench.run_indexer_headline(A(), 1, 0, 0)
+    assert line["value"] == round(w.B * w.T / 100e-6, 1) and line["ms_per_step"] == 0.1
+    assert line["config"] == bench.indexer_config(w, 1) and line["data"] == bench.INDEXER_DATA
+    assert line["n_gpus"] == 1 and line["indexer"] is rec
