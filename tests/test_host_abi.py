@@ -387,3 +387,74 @@ def test_binding_enforces_the_k_limit(lib, monkeypatch):
     assert 1 <= binding.dense_nsplit(1, 1, 8, binding.MAX_K) <= 1024
     ws = binding.dense_workspace_bytes(1, 1, 8, binding.MAX_K, 1)
     assert ws == 0
+
+
+# ------------------------------------------------------------------ indexer entry points
+def call_topk(lib, q=FAKE, w=FAKE, k=FAKE, num_pages=10, pt=FAKE, pt_stride=4, nv=FAKE, B=2, T=1,
+              HI=64, max_n=256, K=64, ps=64, ws=FAKE, ws_bytes=1 << 30, out=FAKE):
+    return lib.smla_indexer_topk(q, w, k, num_pages, pt, pt_stride, nv, B, T, HI, max_n, K, ps,
+                                 ws, ws_bytes, out, None)
+
+
+def call_scores(lib, q=FAKE, w=FAKE, k=FAKE, num_pages=10, pt=FAKE, pt_stride=4, nv=FAKE, B=2,
+                T=1, HI=64, max_n=256, ps=64, ws=FAKE, ws_bytes=1 << 30, scores=FAKE):
+    return lib.smla_indexer_scores(q, w, k, num_pages, pt, pt_stride, nv, B, T, HI, max_n, ps, ws,
+                                   ws_bytes, scores, None)
+
+
+def call_select(lib, scores=FAKE, nv=FAKE, B=2, T=1, max_n=256, K=64, ws=FAKE, ws_bytes=1 << 30,
+                out=FAKE):
+    return lib.smla_indexer_select(scores, nv, B, T, max_n, K, ws, ws_bytes, out, None)
+
+
+# shared by the two entry points that score
+INDEXER_INPUT_ERRORS = [
+    (dict(ps=32), 2), (dict(HI=65), 2), (dict(HI=0), 1), (dict(B=-1), 1), (dict(max_n=-1), 1),
+    (dict(max_n=binding.INDEXER_MAX_N + 1), 2), (dict(B=1048577), 2), (dict(q=0), 1),
+    (dict(w=0), 1), (dict(nv=0), 1), (dict(q=FAKE + 8), 3), (dict(w=FAKE + 2), 3),
+    (dict(nv=FAKE + 2), 3), (dict(k=0), 1), (dict(pt=0), 1), (dict(num_pages=0), 1),
+    (dict(pt_stride=0), 1), (dict(num_pages=33554432), 2), (dict(k=FAKE + 8), 3),
+    (dict(pt=FAKE + 2), 3), (dict(ws_bytes=100), 4), (dict(ws=0), 1), (dict(ws=FAKE + 8), 3),
+]
+
+
+@pytest.mark.parametrize("kw,expect", INDEXER_INPUT_ERRORS + [
+    (dict(K=0), 1), (dict(out=0), 1), (dict(out=FAKE + 2), 3), (dict(B=0), 0), (dict(T=0), 0),
+])
+def test_indexer_topk_rejects_bad_arguments(lib, kw, expect):
+    assert call_topk(lib, **kw) == expect
+
+
+@pytest.mark.parametrize("kw,expect", INDEXER_INPUT_ERRORS + [
+    (dict(scores=0), 1), (dict(scores=FAKE + 2), 3), (dict(B=0), 0), (dict(max_n=0), 0),
+])
+def test_indexer_scores_rejects_bad_arguments(lib, kw, expect):
+    assert call_scores(lib, **kw) == expect
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(K=0), 1), (dict(B=-1), 1), (dict(max_n=-1), 1), (dict(max_n=binding.INDEXER_MAX_N + 1), 2),
+    (dict(B=1048577), 2), (dict(nv=0), 1), (dict(out=0), 1), (dict(scores=0), 1),
+    (dict(nv=FAKE + 2), 3), (dict(out=FAKE + 2), 3), (dict(scores=FAKE + 2), 3),
+    (dict(ws_bytes=100), 4), (dict(ws=0), 1), (dict(ws=FAKE + 8), 3), (dict(B=0), 0),
+    (dict(T=0), 0),
+])
+def test_indexer_select_rejects_bad_arguments(lib, kw, expect):
+    assert call_select(lib, **kw) == expect
+
+
+def test_indexer_workspace_sizes(lib):
+    """The top-k workspace is the tile plan, the fp32 score rows and the
+    selection scratch, each 256-byte rounded; the scratch holds per token a
+    16 KiB digit histogram, a bitmap of max_n positions and max_n candidates
+    of (key, position)."""
+    r = lambda x: (x + 255) // 256 * 256
+    for B, T, n in [(60, 1, 123434), (1, 9, 46089), (3, 2, 1), (512, 8, 700), (1, 1, 0)]:
+        sel = binding.indexer_select_workspace_bytes(B, T, n)
+        assert sel >= B * T * (16384 + -(-n // 32) * 4 + n * 8)
+        assert sel == r(sel)
+        assert binding.indexer_workspace_bytes(B, T, n) == r((B * T + 1) * 4) + r(B * T * n * 4) + sel
+    assert binding.indexer_workspace_bytes(-1, 1, 1) == 0
+    assert binding.indexer_select_workspace_bytes(1, 1, -1) == 0
+    # the scores entry point needs only the plan
+    assert binding.indexer_workspace_bytes(4, 2, 0) >= r(9 * 4)
