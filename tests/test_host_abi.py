@@ -458,3 +458,41 @@ def test_indexer_workspace_sizes(lib):
     assert binding.indexer_select_workspace_bytes(1, 1, -1) == 0
     # the scores entry point needs only the plan
     assert binding.indexer_workspace_bytes(4, 2, 0) >= r(9 * 4)
+
+
+# ------------------------------------------------------------------ the other decode entry points
+def call_noalloc(lib, q=FAKE, cache=FAKE, num_pages=10, pt=FAKE, pt_stride=4, idx=FAKE, B=1, T=1,
+                 H=16, K=64, ps=64, scale=0.1, nsplit=2, o=FAKE, lse=FAKE):
+    return lib.smla_decode_noalloc(q, cache, num_pages, pt, pt_stride, idx, B, T, H, K, ps, scale,
+                                   nsplit, o, lse, None)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(ps=32), 2), (dict(H=65), 2), (dict(B=-1), 1), (dict(q=0), 1), (dict(q=FAKE + 8), 3),
+    (dict(scale=math.nan), 1), (dict(nsplit=-1), 1), (dict(nsplit=1025), 1), (dict(B=0), 0),
+])
+def test_noalloc_rejects_bad_arguments(lib, kw, expect):
+    assert call_noalloc(lib, **kw) == expect
+
+
+def test_noalloc_refuses_partials_beyond_its_scratch_on_the_host(lib):
+    """64 tokens x 64 heads x 8 splits of partials need about 67 MB: refused
+    with a message before the scratch array is even looked up."""
+    assert binding.workspace_bytes(64, 1, 64, 8) > binding.NOALLOC_SCRATCH_BYTES
+    assert call_noalloc(lib, B=64, H=64, K=256, nsplit=8) == 4
+    assert b"scratch" in lib.smla_last_error()
+
+
+def call_host(lib, q=FAKE, cache=FAKE, num_pages=10, pt=FAKE, pt_stride=4, idx=FAKE, B=1, T=1,
+              H=16, K=64, ps=64, scale=0.1, nsplit=2, ws=FAKE, ws_bytes=1 << 30, o=FAKE, lse=FAKE):
+    return lib.smla_decode_host(q, cache, num_pages, pt, pt_stride, idx, B, T, H, K, ps, scale,
+                                nsplit, ws, ws_bytes, o, lse, None)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(ps=32), 2), (dict(H=65), 2), (dict(B=-1), 1), (dict(q=0), 1), (dict(cache=FAKE + 4), 3),
+    (dict(scale=math.inf), 1), (dict(nsplit=-1), 1), (dict(nsplit=1025), 1), (dict(o=0), 1),
+    (dict(lse=0), 1), (dict(num_pages=0), 1), (dict(B=0), 0),
+])
+def test_decode_host_rejects_bad_arguments_before_any_launch(lib, kw, expect):
+    assert call_host(lib, **kw) == expect
