@@ -496,3 +496,14 @@ def call_host(lib, q=FAKE, cache=FAKE, num_pages=10, pt=FAKE, pt_stride=4, idx=F
 ])
 def test_decode_host_rejects_bad_arguments_before_any_launch(lib, kw, expect):
     assert call_host(lib, **kw) == expect
+
+
+def test_nsplit_of_every_bench_workload(lib, monkeypatch):
+    """The split counts the heuristic gives the benchmark's shapes on a
+    148-SM B200 (the values the results tables are measured at)."""
+    monkeypatch.delenv("SMLA_NSPLIT", raising=False)
+    assert binding.choose_nsplit(1, 1, 16, 2048, 148) == 64      # single_request
+    assert binding.choose_nsplit(1, 9, 8, 2048, 148) == 32       # spec_verify
+    assert binding.choose_nsplit(64, 1, 16, 2048, 148) == 4      # batched
+    assert binding.choose_nsplit(60, 1, 64, 2048, 148) == 2      # mixed
+    assert binding.dense_nsplit(1, 9, 8, 46089) == 74            # dense_verify (148 CTAs)
