@@ -258,3 +258,51 @@ def test_indexer_headline_reports_the_job_from_the_timed_record(monkeypatch):
     assert line["value"] == round(w.B * w.T / 100e-6, 1) and line["ms_per_step"] == 0.1
     assert line["config"] == bench.indexer_config(w, 1) and line["data"] == bench.INDEXER_DATA
     assert line["n_gpus"] == 1 and line["indexer"] is rec
+
+
+def test_side_indexer_record_from_fixed_timings(monkeypatch):
+    """The indexer record of the default bench line, built from fixed step
+    times (the harness is a stand-in: every call returns status 0, every
+    timed loop reports 100 / 75 / 30 us per step), so its arithmetic can be
+    checked without a GPU."""
+    sys.path.insert(0, ROOT)
+    import types
+    import bench
+    from sparse_mla_decode_partial_b200 import workloads
+
+    calls = []
+
+    class FakeLib:
+        def __getattr__(self, name):
+            def fn(*args):
+                calls.append(name)
+                return 0
+            return fn
+
+    per_step = {"topk": 0.100, "scores": 0.075, "select": 0.030}
+
+    class FakeHarness:
+        dev = torch.device("cpu")
+        lib, sptr = FakeLib(), 0
+
+        def warm(self, fns, n):
+            for f in fns:
+                assert f()[0] == 0
+
+        def timed(self, step, n):
+            st, nl = step()
+            return [per_step[step.__name__]] * n, nl * n
+
+    monkeypatch.setattr(torch.cuda, "empty_cache", lambda: None)
+    rec = bench.side_indexer(FakeHarness(), 10, 3, (6650.0, 1590.0, "fallback"))
+    w = workloads.indexer_mixed()
+    key_bytes = bench.indexer_bytes(w) - w.B * w.T * w.K * 4
+    assert rec["shape"] == bench.indexer_shape(w) and rec["query_tokens"] == w.B * w.T
+    assert rec["us_per_call"] == 100.0 and rec["scores_us"] == 75.0 and rec["select_us"] == 30.0
+    assert rec["q_tok_s"] == round(w.B * w.T / 100e-6, 1)
+    r = rec["roofline"]
+    assert r["kernel"] == "smla_ix_score_kernel" and r["algorithmic_bytes_per_launch"] == key_bytes
+    assert r["achieved"] == round(key_bytes / 75e-6 / 1e9, 1)
+    assert r["frac"] == round(key_bytes / 75e-6 / 1e9 / 6650.0, 4)
+    assert rec["gpu_launches"] == 40                      # 10 top-k calls x 4 kernels
+    assert {"smla_indexer_topk", "smla_indexer_scores", "smla_indexer_select"} <= set(calls)
